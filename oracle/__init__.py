@@ -1,0 +1,159 @@
+"""Oracle for the causal gated delta-rule recurrence (float64, CPU).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package; the product package
+``gated_delta_rule_97_b200`` never does, and this package never imports it.
+
+Two implementations of the same definition:
+
+* ``gdn_forward`` -- the C recurrence in ``gdn_oracle.c`` (float64, OpenMP
+  over heads), for every size the tests and the benchmark use;
+* ``gdn_forward_np`` -- the same three steps written with NumPy, vectorised
+  over heads, for small cases and to cross-check the compiled one.
+
+Definition (column convention, S in R^{dv x dk}, stored [B,H,dv,dk]):
+``S_t = S_{t-1} Diag(alpha_t)(I - beta_t k_t k_t^T) + beta_t v_t k_t^T``,
+``o_t = S_t q_t``, alpha_t = exp(g_t).  Expanded: decay the columns of S by
+alpha_t, then write (``v k^T`` in the additive/decay modes; ``u k^T`` with
+``u = beta (v - S k)`` in the delta mode), then read ``o = S q``.
+Sources ("Linear Attention, Visualized"): "Naive linear attention",
+"Mamba-2: input-dependent scalar decay", "DeltaNet" / "Recurrent form",
+"Gated DeltaNet (GDN)", "Gated Linear Attention (GLA)",
+"Kimi Delta Attention (KDA)".
+
+Pins (tests/test_oracle_pins.py) tie this definition to closed forms,
+invariants and brute-force constructions that do not reuse it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+UPDATE_IDS = {"additive": 0, "decay": 1, "delta": 2}
+GATE_IDS = {"none": 0, "scalar": 1, "channel": 2}
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99", _SRC, "-o", tmp, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_gdn_forward.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_long, ctypes.c_long,
+                                           ctypes.c_long, ctypes.c_long, dp, dp, dp, dp, dp, dp, dp, dp]
+        lib.oracle_gdn_forward.restype = ctypes.c_int
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """Threads the C oracle's OpenMP region uses."""
+    return int(_load().oracle_num_threads())
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return ctypes.cast(None, ctypes.POINTER(ctypes.c_double))
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _check(update, gate, q, k, v, g, beta):
+    if update not in UPDATE_IDS or gate not in GATE_IDS:
+        raise ValueError("bad mode")
+    if update == "delta" and beta is None:
+        raise ValueError("delta mode needs beta")
+    if (gate != "none") != (g is not None):
+        raise ValueError("g must be given iff gate != 'none'")
+    if q.shape[:-1] != k.shape[:-1] or q.shape[-1] != k.shape[-1] or v.shape[:-1] != q.shape[:-1]:
+        raise ValueError("shape mismatch")
+
+
+def gdn_forward(update, gate, q, k, v, g=None, beta=None, S0=None):
+    """Recurrence over T tokens for every head (C, float64).
+
+    q, k: [..., T, dk]; v: [..., T, dv]; g: [..., T] (scalar) or [..., T, dk]
+    (channel) or None; beta: [..., T] or None; S0: [..., dv, dk] or None.
+    Returns (o [..., T, dv], S_T [..., dv, dk]) as float64.
+    """
+    _check(update, gate, q, k, v, g, beta)
+    lead = q.shape[:-2]
+    T, dk = q.shape[-2], q.shape[-1]
+    dv = v.shape[-1]
+    BH = int(np.prod(lead)) if lead else 1
+    qd, kd, vd = _f64(q), _f64(k), _f64(v)
+    gd, bd, sd = _f64(g), _f64(beta), _f64(S0)
+    o = np.empty(lead + (T, dv), np.float64)
+    ST = np.empty(lead + (dv, dk), np.float64)
+    rc = _load().oracle_gdn_forward(UPDATE_IDS[update], GATE_IDS[gate], BH, T, dk, dv,
+                                    _ptr(qd), _ptr(kd), _ptr(vd), _ptr(gd), _ptr(bd), _ptr(sd),
+                                    _ptr(o), _ptr(ST))
+    if rc != 0:
+        raise RuntimeError("oracle_gdn_forward failed: %d" % rc)
+    return o, ST
+
+
+def gdn_forward_np(update, gate, q, k, v, g=None, beta=None, S0=None):
+    """The same recurrence with NumPy (vectorised over heads; loops over t)."""
+    _check(update, gate, q, k, v, g, beta)
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    g, beta = _f64(g), _f64(beta)
+    lead = q.shape[:-2]
+    T, dk = q.shape[-2], q.shape[-1]
+    dv = v.shape[-1]
+    S = np.zeros(lead + (dv, dk)) if S0 is None else _f64(S0).copy()
+    o = np.empty(lead + (T, dv))
+    for t in range(T):
+        if gate == "scalar":
+            S = S * np.exp(g[..., t])[..., None, None]
+        elif gate == "channel":
+            S = S * np.exp(g[..., t, :])[..., None, :]
+        kt = k[..., t, :]
+        if update == "delta":
+            pred = np.einsum("...ij,...j->...i", S, kt)
+            u = beta[..., t][..., None] * (v[..., t, :] - pred)
+        else:
+            u = v[..., t, :]
+        S = S + u[..., :, None] * kt[..., None, :]
+        o[..., t, :] = np.einsum("...ij,...j->...i", S, q[..., t, :])
+    return o, S
+
+
+def decode_sequence(update, gate, S0, steps):
+    """Oracle for ``len(steps)`` consecutive decode steps on the same state.
+
+    ``steps`` is a list of dicts with q,k [..., 1, d], v [..., 1, dv], beta
+    [..., 1], g [..., 1] or [..., 1, dk].  Consecutive single-token steps are
+    the recurrence over the stacked sequence, so this stacks them along T.
+    Returns (o [..., n_steps, dv], S_final).
+    """
+    def cat(name):
+        if steps[0].get(name) is None:
+            return None
+        return np.concatenate([np.asarray(s[name], dtype=np.float64) for s in steps],
+                              axis=-2 if name in ("q", "k", "v") or (name == "g" and gate == "channel") else -1)
+
+    return gdn_forward(update, gate, cat("q"), cat("k"), cat("v"), cat("g"), cat("beta"), S0)
