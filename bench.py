@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta-rule hot path on B200.
+
+One step = one gdn_chunk_fwd over the Gated DeltaNet prefill workload
+(B=8, H=16, T=8192, dk=dv=128, bf16 q/k/v, fp32 gate/beta/state/output, chunk 64),
+which runs every prefill row of the path (gate prefix, K-Gram, UT solve, W/U,
+state correction, output, state pass).  The line also carries the decode
+workload (256 x 32 heads, 1000 in-place steps) and, unless --quick, the linear
+attention and per-channel (KDA) prefill workloads.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+
+Prints ONE JSON line on rank 0.  Under torchrun (N > 1) every rank runs its own
+full batch (weak scaling, no collective on the data path); timing uses a
+barrier plus device synchronisation on both sides and the max over ranks.
+The reference arm (--impl reference) times the float64 CPU oracle on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, iter_decode_blocks, make_decode_state, make_prefill_inputs  # noqa: E402
+
+HEADLINE = "gdn_prefill_bf16"
+METRIC = "gated-delta prefill tokens/s + % roofline; decode state-update HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work (bytes: each input read once, each output written once)
+# ---------------------------------------------------------------------------
+
+def prefill_bytes(w, out_bytes=4):
+    in_b = 2 if w.dtype == "bf16" else 4
+    per_tok = (2 * w.dk + w.dv) * in_b + w.dv * out_bytes
+    if w.gate == "scalar":
+        per_tok += 4
+    elif w.gate == "channel":
+        per_tok += 4 * w.dk
+    if w.update == "delta":
+        per_tok += 4
+    state = w.dv * w.dk * 4 * ((1 if w.s0_std > 0 else 0) + 1)
+    return w.n_heads * (w.T * per_tok + state)
+
+
+def prefill_flops(w, C=64):
+    d = w.dk
+    per = (10 * C * d + 6 * d * d) if w.update == "delta" else (4 * C * d + 4 * d * d)
+    return w.n_heads * w.T * per
+
+
+def decode_bytes_per_step(w, out_bytes=4):
+    in_b = 2 if w.dtype == "bf16" else 4
+    per_head = 2 * w.dv * w.dk * 4 + (2 * w.dk + w.dv) * in_b + w.dv * out_bytes + 4
+    if w.update == "delta":
+        per_head += 4
+    if w.gate == "channel":
+        per_head += 4 * (w.dk - 1)
+    return w.n_heads * per_head
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [s for s in sm if mx and s > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def to_dev(x, dtype, torch):
+    if x is None:
+        return None
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).cuda().to(dtype).contiguous()
+
+
+def time_prefill(w, x, steps, warmup, torch, gdn, dist=None):
+    """Device-timed steps of gdn_chunk_fwd over the whole batch; returns ms/step (max over ranks)."""
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q, k, v = to_dev(x["q"], dt, torch), to_dev(x["k"], dt, torch), to_dev(x["v"], dt, torch)
+    g, beta, S0 = to_dev(x["g"], torch.float32, torch), to_dev(x["beta"], torch.float32, torch), \
+        to_dev(x["S0"], torch.float32, torch)
+    o = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device="cuda")
+    ST = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device="cuda")
+
+    def step():
+        gdn.chunk_fwd(q, k, v, g, beta, S0, update=w.update, gate=w.gate, o=o, S_T=ST)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if gdn.device_status() != 0:
+        raise RuntimeError("device status after warm-up: %d" % gdn.device_status())
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dist, "cuda")
+    del q, k, v, g, beta, S0, o, ST
+    return ms
+
+
+def time_prefill_e2e(w, x, steps, warmup, torch, gdn):
+    """Same metric through the public API with pinned host buffers: every step
+    copies the inputs host->device, runs gdn_chunk_fwd and reads o and S_T back."""
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def pin(a, dtype):
+        if a is None:
+            return None
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dtype).pin_memory()
+
+    hq, hk, hv = pin(x["q"], dt), pin(x["k"], dt), pin(x["v"], dt)
+    hg, hb, hS = pin(x["g"], torch.float32), pin(x["beta"], torch.float32), pin(x["S0"], torch.float32)
+    ho = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32).pin_memory()
+    hST = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hS) if t is not None)
+    d2h = ho.numel() * 4 + hST.numel() * 4
+
+    def step():
+        dq = hq.to("cuda", non_blocking=True)
+        dk_ = hk.to("cuda", non_blocking=True)
+        dv_ = hv.to("cuda", non_blocking=True)
+        dg = None if hg is None else hg.to("cuda", non_blocking=True)
+        db = None if hb is None else hb.to("cuda", non_blocking=True)
+        dS = None if hS is None else hS.to("cuda", non_blocking=True)
+        o, ST = gdn.chunk_fwd(dq, dk_, dv_, dg, db, dS, update=w.update, gate=w.gate)
+        ho.copy_(o, non_blocking=True)
+        hST.copy_(ST, non_blocking=True)
+
+    for _ in range(max(1, min(warmup, 2))):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def time_decode(w, n_steps, torch, gdn, warmup=3):
+    """Device time of ``n_steps`` consecutive in-place decode steps (inputs of
+    every step resident in HBM before timing); returns ms/step."""
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    S = to_dev(make_decode_state(w), torch.float32, torch)
+    dev_in = []
+    for _, blk in iter_decode_blocks(w, n_steps):
+        dev_in += [{k: to_dev(v, dt if k in ("q", "k", "v") else torch.float32, torch) for k, v in s.items()}
+                   for s in blk]
+    o = torch.empty((w.B, w.H, 1, w.dv), dtype=torch.float32, device="cuda")
+
+    def run(s):
+        gdn.decode_step(s["q"], s["k"], s["v"], s["g"], s["beta"], S, update=w.update, gate=w.gate, o=o)
+
+    for i in range(warmup):
+        run(dev_in[i % len(dev_in)])
+    S.copy_(to_dev(make_decode_state(w), torch.float32, torch))
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in dev_in:
+        run(s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if gdn.device_status() != 0:
+        raise RuntimeError("device status after decode")
+    del dev_in, S
+    return e0.elapsed_time(e1) / n_steps
+
+
+def max_over_ranks(value, dist, device):
+    """Max of a per-rank float over all ranks (timing only; not on the data path)."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([float(value)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(w, budget_s=15.0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole
+    sequences of a few heads, sized to roughly ``budget_s`` of CPU time."""
+    import oracle
+
+    oracle.build()
+    threads = oracle.num_threads()
+    probe_T = min(w.T, 1024)
+    xs = make_prefill_inputs(w.with_(T=probe_T), heads=[(0, 0)])
+    t0 = time.perf_counter()
+    oracle.gdn_forward(w.update, w.gate, xs["q"], xs["k"], xs["v"], g=xs["g"], beta=xs["beta"], S0=xs["S0"])
+    per_tok = (time.perf_counter() - t0) / probe_T
+    n_heads = max(1, min(w.n_heads, int(budget_s * threads / max(per_tok * w.T, 1e-9))))
+    n_heads = min(n_heads, 4 * threads)
+    heads = [(i // w.H, i % w.H) for i in range(n_heads)]
+    xs = make_prefill_inputs(w, heads=heads)
+    t0 = time.perf_counter()
+    oracle.gdn_forward(w.update, w.gate, xs["q"], xs["k"], xs["v"], g=xs["g"], beta=xs["beta"], S0=xs["S0"])
+    dt = time.perf_counter() - t0
+    token_heads = n_heads * w.T
+    return {"value": token_heads / dt / w.H, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "%d of %d heads, full T=%d (%d token-heads), float64 C recurrence, %.1f s"
+                      % (n_heads, w.n_heads, w.T, token_heads, dt)}
+
+
+def run_ours(args):
+    import torch
+
+    import gated_delta_rule_97_b200 as gdn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    gdn.load()
+    gdn.device_status(clear=True)
+    peaks, peak_kind = load_peaks()
+
+    w = WORKLOADS[args.workload]
+    x = make_prefill_inputs(w)
+    with ClockSampler(local) as clk:
+        ms = time_prefill(w, x, args.steps, args.warmup, torch, gdn, dist)
+    clocks = clk.summary()
+    tokens = w.B * w.T
+    value = world * tokens / (ms * 1e-3)
+    nbytes = prefill_bytes(w)
+    flops = prefill_flops(w)
+    achieved_gbs = nbytes / (ms * 1e-3) / 1e9
+    t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    result = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+              "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+              "vs_baseline": None, "dtype": "bf16 in / fp32 state, accumulation, output", "data": "synthetic",
+              "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
+                         "update": w.update, "gate": w.gate, "chunk": w.chunk, "global_batch": w.B * world,
+                         "seq_len": w.T, "parallelism": "replicas x%d (batch per GPU fixed)" % world,
+                         "l2": "inputs (%.2f GB) larger than the 126 MB L2" % (nbytes / 1e9)},
+              "token_heads_per_s": world * w.n_heads * w.T / (ms * 1e-3),
+              "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None,
+                           "peak_source": peak_kind, "algorithmic_bytes_per_launch": nbytes,
+                           "flops_per_launch": flops,
+                           "achieved_tflops": flops / (ms * 1e-3) / 1e12,
+                           "roofline_us": t_roof * 1e6, "frac_of_roofline_time": t_roof / (ms * 1e-3)},
+              "gpu_launches": args.steps, "clocks": clocks}
+
+    ms_e2e, h2d, d2h = time_prefill_e2e(w, x, max(2, min(args.steps, 5)), args.warmup, torch, gdn)
+    result["e2e"] = {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+    del x
+
+    wd = WORKLOADS["decode_gdn_bf16"]
+    n_dec = wd.steps if not args.quick else 100
+    ms_d = max_over_ranks(time_decode(wd, n_dec, torch, gdn), dist, "cuda")
+    dbytes = decode_bytes_per_step(wd)
+    result["decode"] = {"workload": wd.name, "steps": n_dec, "ms_per_step": ms_d,
+                        "value": dbytes / (ms_d * 1e-3) / 1e9, "unit": "GB/s",
+                        "frac": dbytes / (ms_d * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                        "bytes_per_step": dbytes, "tokens_per_s": wd.n_heads / wd.H * world / (ms_d * 1e-3)}
+    result["gpu_launches"] += n_dec
+
+    if not args.quick:
+        others = {}
+        for name in ("linear_attn_bf16", "kda_prefill_bf16"):
+            wo = WORKLOADS[name]
+            xo = make_prefill_inputs(wo)
+            mso = time_prefill(wo, xo, max(3, args.steps // 2), args.warmup, torch, gdn, dist)
+            del xo
+            nb, fl = prefill_bytes(wo), prefill_flops(wo)
+            tr = max(nb / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+            others[name] = {"ms_per_step": mso, "tokens_per_s": wo.B * wo.T * world / (mso * 1e-3),
+                            "achieved_gbs": nb / (mso * 1e-3) / 1e9, "roofline_us": tr * 1e6,
+                            "frac_of_roofline_time": tr / (mso * 1e-3)}
+        result["prefill_workloads"] = others
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_reference(args):
+    """The oracle as the reference arm: float64 CPU recurrence on a bounded
+    sample per step (one whole head sequence per step), on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    w = WORKLOADS[args.workload]
+    threads = oracle.num_threads()
+    heads = [(i // w.H, i % w.H) for i in range(threads)]
+    xs = make_prefill_inputs(w, heads=heads)
+    run = lambda: oracle.gdn_forward(w.update, w.gate, xs["q"], xs["k"], xs["v"], g=xs["g"], beta=xs["beta"],
+                                     S0=xs["S0"])
+    for _ in range(min(args.warmup, 1)):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = len(heads) * w.T / dt / w.H
+    sample = "%d of %d heads per step, full T=%d, float64 C oracle" % (len(heads), w.n_heads, w.T)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "update": w.update,
+                   "gate": w.gate, "chunk": w.chunk},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+        flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=HEADLINE, choices=[k for k, w in WORKLOADS.items() if w.steps == 0])
+    ap.add_argument("--quick", action="store_true", help="skip the extra prefill workloads; 100 decode steps")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

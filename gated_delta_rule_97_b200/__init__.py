@@ -1,0 +1,205 @@
+"""B200 (sm_100a) gated delta-rule library: thin Python binding of libgdn.so.
+
+The compute lives in ``libgdn.so`` (CUDA kernels behind the C ABI declared in
+``include/gdn.h``).  This module only marshals arguments: it checks tensor
+shapes and dtypes, passes raw device pointers and the current CUDA stream to
+the C entry points, and raises ``GDNError`` on a non-zero return code.  There
+is no fallback: if the library is not built, every call raises.
+
+    import gated_delta_rule_97_b200 as gdn
+    o, S_T = gdn.chunk_fwd(q, k, v, g, beta, S0, update="delta", gate="scalar")
+    o = gdn.decode_step(q1, k1, v1, g1, beta1, S, update="delta", gate="scalar")
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["GDNError", "chunk_fwd", "decode_step", "device_status", "strerror", "version", "load",
+           "lib_path", "Desc", "UPDATES", "GATES", "build"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+UPDATES = {"additive": 0, "decay": 1, "delta": 2}
+GATES = {"none": 0, "scalar": 1, "channel": 2}
+ALGOS = {"auto": 0, "simt": 1, "tc": 2}
+F32, BF16 = 0, 1
+
+GDN_OK = 0
+ERRORS = {-1: "GDN_ERR_ARG", -2: "GDN_ERR_ALIGN", -3: "GDN_ERR_UNSUPPORTED", -4: "GDN_ERR_CUDA",
+          -5: "GDN_ERR_TIMEOUT", -6: "GDN_ERR_RANGE"}
+
+
+class GDNError(RuntimeError):
+    def __init__(self, code, what=""):
+        self.code = code
+        super().__init__("%s: %s (%d)%s" % (ERRORS.get(code, "?"), strerror(code) if _lib else "", code,
+                                            (" in " + what) if what else ""))
+
+
+class Desc(ctypes.Structure):
+    """Mirror of gdn_desc_t."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("dk", ctypes.c_int),
+                ("dv", ctypes.c_int), ("update", ctypes.c_int), ("gate", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("algo", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def build(verbose: bool = False, force: bool = False) -> str:
+    """Compiles libgdn.so in-tree (nvcc, sm_100a)."""
+    from .build import build as _build
+
+    return _build(verbose=verbose, force=force)
+
+
+def load():
+    """Loads libgdn.so; raises if it is missing (there is no fallback path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError("libgdn.so is not built (%s); run gated_delta_rule_97_b200.build()" % _LIB_PATH)
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp = ctypes.c_void_p
+    dp = ctypes.POINTER(Desc)
+    lib.gdn_chunk_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gdn_chunk_fwd.restype = ctypes.c_int
+    lib.gdn_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gdn_decode_step.restype = ctypes.c_int
+    lib.gdn_strerror.argtypes = [ctypes.c_int]
+    lib.gdn_strerror.restype = ctypes.c_char_p
+    lib.gdn_device_status.argtypes = [ctypes.c_int]
+    lib.gdn_device_status.restype = ctypes.c_int
+    lib.gdn_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def strerror(code: int) -> str:
+    return load().gdn_strerror(int(code)).decode()
+
+
+def version() -> int:
+    return int(load().gdn_version())
+
+
+def device_status(clear: bool = True) -> int:
+    """The library's device status word (synchronises the device)."""
+    return int(load().gdn_device_status(1 if clear else 0))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(dt):
+    import torch
+
+    if dt == torch.bfloat16:
+        return BF16
+    if dt == torch.float32:
+        return F32
+    raise TypeError("q, k, v, o must be bfloat16 or float32, got %s" % dt)
+
+
+def make_desc(B, H, T, dk, dv, update, gate, dtype, out_dtype, algo="auto", chunk=64) -> Desc:
+    return Desc(B, H, T, dk, dv, UPDATES[update], GATES[gate], dtype, out_dtype, chunk, ALGOS[algo])
+
+
+def _check(t, name, shape, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=None, o=None, S_T=None,
+              return_state=True, algo="auto", stream=None):
+    """Prefill over T tokens (gdn_chunk_fwd).  Returns (o, S_T).
+
+    q, k [B,H,T,dk]; v [B,H,T,dv] (bf16 or fp32, same dtype); g [B,H,T] or
+    [B,H,T,dk] fp32 (log of the gate) or None; beta [B,H,T] fp32 (delta);
+    S0 [B,H,dv,dk] fp32 or None.  o defaults to fp32; S_T may be S0 (in place).
+    """
+    import torch
+
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
+    if gate == "scalar":
+        _check(g, "g", (B, H, T), torch.float32)
+    elif gate == "channel":
+        _check(g, "g", (B, H, T, dk), torch.float32)
+    _check(beta, "beta", (B, H, T), torch.float32)
+    _check(S0, "S0", (B, H, dv, dk), torch.float32)
+    if out_dtype is None:
+        out_dtype = o.dtype if o is not None else torch.float32
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
+    _check(o, "o", (B, H, T, dv), out_dtype)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo)
+    rc = load().gdn_chunk_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                              _ptr(o), _ptr(S_T), _stream(stream))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_chunk_fwd")
+    return o, S_T
+
+
+def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, stream=None):
+    """One decode step (gdn_decode_step); S [B,H,dv,dk] is updated in place.
+
+    q, k [B,H,1,dk]; v [B,H,1,dv]; g [B,H,1] or [B,H,1,dk] or None; beta [B,H,1].
+    Returns o [B,H,1,dv].
+    """
+    import torch
+
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if T != 1:
+        raise ValueError("decode_step takes one token (T == 1)")
+    _check(q, "q", (B, H, 1, dk))
+    _check(k, "k", (B, H, 1, dk), q.dtype)
+    _check(v, "v", (B, H, 1, dv), q.dtype)
+    if gate == "scalar":
+        _check(g, "g", (B, H, 1), torch.float32)
+    elif gate == "channel":
+        _check(g, "g", (B, H, 1, dk), torch.float32)
+    _check(beta, "beta", (B, H, 1), torch.float32)
+    _check(S, "S", (B, H, dv, dk), torch.float32)
+    if out_dtype is None:
+        out_dtype = o.dtype if o is not None else torch.float32
+    if o is None:
+        o = torch.empty((B, H, 1, dv), dtype=out_dtype, device=q.device)
+    _check(o, "o", (B, H, 1, dv), out_dtype)
+    d = make_desc(B, H, 1, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype))
+    rc = load().gdn_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                                _ptr(o), _stream(stream))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_decode_step")
+    return o

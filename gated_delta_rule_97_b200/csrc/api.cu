@@ -1,0 +1,146 @@
+// C ABI of libgdn.so: argument validation and kernel dispatch (see gdn.h).
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/gdn.h"
+#include "common.cuh"
+
+// The library's device status word (first error code any kernel recorded).
+__device__ int g_gdn_status = 0;
+
+namespace {
+
+int *status_ptr() {
+    // The address is per device; looked up on every call (cheap, no allocation).
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gdn_status) != cudaSuccess) return nullptr;
+    return static_cast<int *>(p);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(int dtype) { return dtype == GDN_BF16 ? 2 : 4; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+int validate_common(const gdn_desc_t *d) {
+    if (!d) return GDN_ERR_ARG;
+    if (d->B < 0 || d->H < 0 || d->T < 0) return GDN_ERR_ARG;
+    if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return GDN_ERR_ARG;
+    if (d->update < GDN_ADDITIVE || d->update > GDN_DELTA) return GDN_ERR_ARG;
+    if (d->gate < GDN_GATE_NONE || d->gate > GDN_GATE_CHANNEL) return GDN_ERR_ARG;
+    if (d->update == GDN_ADDITIVE && d->gate != GDN_GATE_NONE) return GDN_ERR_ARG;
+    if (d->update == GDN_DECAY && d->gate == GDN_GATE_NONE) return GDN_ERR_ARG;
+    if ((d->dtype != GDN_F32 && d->dtype != GDN_BF16) || (d->out_dtype != GDN_F32 && d->out_dtype != GDN_BF16))
+        return GDN_ERR_ARG;
+    const long bh = (long)d->B * d->H;
+    if (bh > (1L << 30)) return GDN_ERR_ARG;
+    return GDN_OK;
+}
+
+int from_cuda(int e) { return e == 0 ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" int gdn_version(void) { return GDN_VERSION; }
+
+extern "C" const char *gdn_strerror(int code) {
+    switch (code) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_ARG: return "invalid argument (null pointer, bad enum, size or overlap)";
+        case GDN_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case GDN_ERR_UNSUPPORTED: return "request not supported by this build";
+        case GDN_ERR_CUDA: return "CUDA runtime error";
+        case GDN_ERR_TIMEOUT: return "a bounded wait inside a kernel timed out";
+        case GDN_ERR_RANGE: return "an fp16 tensor-core operand overflowed";
+        default: return "unknown error";
+    }
+}
+
+extern "C" int gdn_device_status(int clear) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_gdn_status, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+    if (clear) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(g_gdn_status, &z, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    return v;
+}
+
+int gdn_tc_supported(const gdn_desc_t *d);
+int gdn_launch_chunk_tc(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
+
+extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *S0, void *o, float *S_T, void *stream) {
+    int rc = validate_common(d);
+    if (rc != GDN_OK) return rc;
+    if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC) return GDN_ERR_ARG;
+    const long BH = (long)d->B * d->H;
+    const size_t n_qk = (size_t)BH * d->T * d->dk, n_v = (size_t)BH * d->T * d->dv;
+    const size_t n_S = (size_t)BH * d->dv * d->dk;
+    const size_t n_g = d->gate == GDN_GATE_CHANNEL ? n_qk : (size_t)BH * d->T;
+    const bool has_tokens = BH > 0 && d->T > 0;
+    if (has_tokens) {
+        if (!q || !k || !v || !o) return GDN_ERR_ARG;
+        if (d->update == GDN_DELTA && !beta) return GDN_ERR_ARG;
+    }
+    if ((d->gate != GDN_GATE_NONE) != (g != nullptr) && has_tokens) return GDN_ERR_ARG;
+    if (d->gate == GDN_GATE_NONE && g != nullptr) return GDN_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, o, S_T};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t es = elem_size(d->dtype), eo = elem_size(d->out_dtype);
+    const size_t no = n_v * eo;
+    if (overlaps(o, no, q, n_qk * es) || overlaps(o, no, k, n_qk * es) || overlaps(o, no, v, n_v * es) ||
+        overlaps(o, no, g, n_g * 4) || overlaps(o, no, beta, (size_t)BH * d->T * 4) ||
+        overlaps(o, no, S0, n_S * 4) || overlaps(o, no, S_T, n_S * 4))
+        return GDN_ERR_ARG;
+    if (S_T && S0 && S_T != S0 && overlaps(S_T, n_S * 4, S0, n_S * 4)) return GDN_ERR_ARG;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (BH == 0) return GDN_OK;
+    if (d->T == 0) return from_cuda(gdn_launch_copy_state(S0, S_T, (long)n_S, st));
+
+    gdn::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
+    a.status = status_ptr();
+    a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
+
+    const bool tc_ok = gdn_tc_supported(d) != 0;
+    if (d->algo == GDN_ALGO_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
+    if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok))
+        return from_cuda(gdn_launch_chunk_tc(a, d, st));
+    return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
+}
+
+extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, float *S, void *o, void *stream) {
+    int rc = validate_common(d);
+    if (rc != GDN_OK) return rc;
+    if (d->T != 1) return GDN_ERR_ARG;
+    const long BH = (long)d->B * d->H;
+    if (BH == 0) return GDN_OK;
+    if (!q || !k || !v || !S || !o) return GDN_ERR_ARG;
+    if (d->update == GDN_DELTA && !beta) return GDN_ERR_ARG;
+    if ((d->gate != GDN_GATE_NONE) != (g != nullptr)) return GDN_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S, o};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t n_S = (size_t)BH * d->dv * d->dk;
+    const size_t no = (size_t)BH * d->dv * elem_size(d->out_dtype);
+    const size_t es = elem_size(d->dtype);
+    if (overlaps(o, no, S, n_S * 4) || overlaps(o, no, q, BH * d->dk * es) || overlaps(o, no, k, BH * d->dk * es) ||
+        overlaps(o, no, v, BH * d->dv * es))
+        return GDN_ERR_ARG;
+    gdn::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.o = o;
+    a.BH = (int)BH; a.dk = d->dk; a.dv = d->dv;
+    return from_cuda(gdn_launch_decode(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16,
+                                       static_cast<cudaStream_t>(stream)));
+}

@@ -1,0 +1,63 @@
+// Shared device helpers for the gated delta-rule kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+enum Update { kAdditive = 0, kDecay = 1, kDelta = 2 };
+enum Gate { kGateNone = 0, kGateScalar = 1, kGateChannel = 2 };
+
+constexpr int kChunk = 64;  // chunk length C of the chunkwise form
+
+// Status codes written to the device status word (mirror gdn.h).
+constexpr int kStatusTimeout = -5;
+constexpr int kStatusRange = -6;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Records the first error code seen by any kernel (0 = none yet).
+__device__ __forceinline__ void record_status(int *status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// Arguments common to the prefill kernels.  All pointers are device pointers.
+struct ChunkArgs {
+    const void *q, *k, *v;   // [BH,T,dk] / [BH,T,dv], input dtype
+    const float *g;          // [BH,T] or [BH,T,dk] or null
+    const float *beta;       // [BH,T] or null
+    const float *S0;         // [BH,dv,dk] or null
+    void *o;                 // [BH,T,dv], output dtype
+    float *ST;               // [BH,dv,dk] or null
+    int *status;             // device status word
+    int BH, T, dk, dv;
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v;   // [BH,dk] / [BH,dv]
+    const float *g;          // [BH] or [BH,dk] or null
+    const float *beta;       // [BH] or null
+    float *S;                // [BH,dv,dk] in/out
+    void *o;                 // [BH,dv]
+    int BH, dk, dv;
+};
+
+}  // namespace gdn
+
+// Launchers (defined in the kernel .cu files).  Return a cudaError_t value.
+int gdn_launch_chunk_simt(const gdn::ChunkArgs &a, int update, int gate, int in_bf16, int out_bf16,
+                          cudaStream_t stream);
+int gdn_launch_decode(const gdn::DecodeArgs &a, int update, int gate, int in_bf16, int out_bf16,
+                      cudaStream_t stream);
+int gdn_launch_copy_state(const float *S0, float *ST, long n, cudaStream_t stream);

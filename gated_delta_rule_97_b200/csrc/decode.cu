@@ -1,0 +1,164 @@
+// Decode: one recurrent step per (b,h), state updated in place.
+//
+// Bandwidth-bound rank-1 update ("Linear Attention, Visualized", "Optional:
+// Linear attention as an RNN"; per-token recurrences of the Mamba-2, DeltaNet,
+// GDN, GLA and KDA sections).  Each warp owns kRowsPerWarp consecutive rows of
+// one head's state; lane l holds columns [l*V, l*V+V) of a row (V = dk/32, one
+// 16-byte load for dk = 128).  Per row i, with a = exp(g):
+//   p_i = sum_j S_ij a_j k_j,  r_i = sum_j S_ij a_j q_j      (two warp sums)
+//   u_i = beta (v_i - p_i) (delta) or v_i,
+//   S_ij <- S_ij a_j + u_i k_j,  o_i = r_i + u_i (k . q).
+// The state is streamed once in and once out with evict-first hints; rows are
+// independent, so there is no inter-warp synchronisation.
+#include "common.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRowsPerWarp = 4;
+
+template <int V>
+struct VecF;
+template <>
+struct VecF<4> {
+    using T = float4;
+    __device__ static void load(const float *p, float *x) {
+        const float4 t = __ldcs(reinterpret_cast<const float4 *>(p));
+        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+    }
+    __device__ static void store(float *p, const float *x) {
+        __stcs(reinterpret_cast<float4 *>(p), make_float4(x[0], x[1], x[2], x[3]));
+    }
+};
+template <>
+struct VecF<2> {
+    using T = float2;
+    __device__ static void load(const float *p, float *x) {
+        const float2 t = __ldcs(reinterpret_cast<const float2 *>(p));
+        x[0] = t.x; x[1] = t.y;
+    }
+    __device__ static void store(float *p, const float *x) {
+        __stcs(reinterpret_cast<float2 *>(p), make_float2(x[0], x[1]));
+    }
+};
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+template <int DK, int UPD, int GATE, typename TIn, typename TOut>
+__global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
+    constexpr int V = DK / 32;
+    const long warp = ((long)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long row0 = warp * kRowsPerWarp;
+    if (row0 >= (long)a.BH * a.dv) return;
+    const long bh = row0 / a.dv;
+    const int i0 = (int)(row0 - bh * a.dv);
+    const int c0 = lane * V;
+
+    float *Srow = a.S + ((size_t)bh * a.dv + i0) * DK + c0;
+    float s[kRowsPerWarp][V];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) VecF<V>::load(Srow + (size_t)r * DK, s[r]);
+
+    const TIn *qp = static_cast<const TIn *>(a.q) + bh * DK + c0;
+    const TIn *kp = static_cast<const TIn *>(a.k) + bh * DK + c0;
+    float qq[V], kk[V], al[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+        qq[e] = to_f32(qp[e]);
+        kk[e] = to_f32(kp[e]);
+        al[e] = 1.f;
+    }
+    if (GATE == kGateScalar) {
+        const float x = __expf(a.g[bh]);
+#pragma unroll
+        for (int e = 0; e < V; ++e) al[e] = x;
+    } else if (GATE == kGateChannel) {
+#pragma unroll
+        for (int e = 0; e < V; ++e) al[e] = __expf(a.g[bh * DK + c0 + e]);
+    }
+    const float bt = (UPD == kDelta) ? a.beta[bh] : 0.f;
+    const TIn *vp = static_cast<const TIn *>(a.v) + bh * a.dv + i0;
+    float vv[kRowsPerWarp];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) vv[r] = to_f32(vp[r]);
+
+    float kq = 0.f;
+#pragma unroll
+    for (int e = 0; e < V; ++e) kq = fmaf(kk[e], qq[e], kq);
+    kq = warp_sum(kq);
+
+    float outv[kRowsPerWarp];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+        float p = 0.f, rr = 0.f;
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            s[r][e] *= al[e];
+            p = fmaf(s[r][e], kk[e], p);
+            rr = fmaf(s[r][e], qq[e], rr);
+        }
+        // two independent butterfly sums, interleaved
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            p += __shfl_xor_sync(0xffffffffu, p, off);
+            rr += __shfl_xor_sync(0xffffffffu, rr, off);
+        }
+        const float u = (UPD == kDelta) ? bt * (vv[r] - p) : vv[r];
+#pragma unroll
+        for (int e = 0; e < V; ++e) s[r][e] = fmaf(u, kk[e], s[r][e]);
+        VecF<V>::store(Srow + (size_t)r * DK, s[r]);
+        outv[r] = fmaf(u, kq, rr);
+    }
+    if (lane < kRowsPerWarp) {
+        float x = outv[0];
+#pragma unroll
+        for (int r = 1; r < kRowsPerWarp; ++r)
+            if (lane == r) x = outv[r];
+        static_cast<TOut *>(a.o)[bh * a.dv + i0 + lane] = from_f32<TOut>(x);
+    }
+}
+
+template <int DK, int UPD, int GATE, typename TIn, typename TOut>
+int launch(const DecodeArgs &a, cudaStream_t stream) {
+    const long rows = (long)a.BH * a.dv;
+    const long warps = rows / kRowsPerWarp;
+    const long blocks = (warps * 32 + kThreads - 1) / kThreads;
+    if (blocks == 0) return 0;
+    decode_kernel<DK, UPD, GATE, TIn, TOut><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+    return (int)cudaGetLastError();
+}
+
+template <int DK, int UPD, int GATE>
+int launch_types(const DecodeArgs &a, int in_bf16, int out_bf16, cudaStream_t s) {
+    if (in_bf16)
+        return out_bf16 ? launch<DK, UPD, GATE, __nv_bfloat16, __nv_bfloat16>(a, s)
+                        : launch<DK, UPD, GATE, __nv_bfloat16, float>(a, s);
+    return out_bf16 ? launch<DK, UPD, GATE, float, __nv_bfloat16>(a, s) : launch<DK, UPD, GATE, float, float>(a, s);
+}
+
+template <int DK>
+int launch_modes(const DecodeArgs &a, int update, int gate, int in_bf16, int out_bf16, cudaStream_t s) {
+    if (update == kAdditive) return launch_types<DK, kAdditive, kGateNone>(a, in_bf16, out_bf16, s);
+    if (update == kDecay) {
+        if (gate == kGateScalar) return launch_types<DK, kDecay, kGateScalar>(a, in_bf16, out_bf16, s);
+        return launch_types<DK, kDecay, kGateChannel>(a, in_bf16, out_bf16, s);
+    }
+    if (gate == kGateNone) return launch_types<DK, kDelta, kGateNone>(a, in_bf16, out_bf16, s);
+    if (gate == kGateScalar) return launch_types<DK, kDelta, kGateScalar>(a, in_bf16, out_bf16, s);
+    return launch_types<DK, kDelta, kGateChannel>(a, in_bf16, out_bf16, s);
+}
+
+}  // namespace
+}  // namespace gdn
+
+int gdn_launch_decode(const gdn::DecodeArgs &a, int update, int gate, int in_bf16, int out_bf16,
+                      cudaStream_t stream) {
+    if (a.dk == 64) return gdn::launch_modes<64>(a, update, gate, in_bf16, out_bf16, stream);
+    return gdn::launch_modes<128>(a, update, gate, in_bf16, out_bf16, stream);
+}

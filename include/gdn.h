@@ -1,0 +1,151 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated delta-rule library (libgdn.so).
+ *
+ * The library computes the causal gated delta-rule recurrence
+ *
+ *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,            alpha_t = exp(g_t),
+ *
+ * with the state S in R^{dv x dk} stored row-major as [B,H,dv,dk] (the column
+ * convention; the pages write the transposed row-vector form S_t = S_{t-1} +
+ * k_t^T v_t, o_t = q_t S_t, which is the same map).  Sources, all on the page
+ * "Linear Attention, Visualized": "Naive linear attention" (additive write),
+ * "RetNet: scalar decay" and "Mamba-2: input-dependent scalar decay" (scalar
+ * gate), "DeltaNet: correcting memory collisions" / "Recurrent form" (delta
+ * write), "Gated DeltaNet (GDN)" (scalar gate + delta), "Gated Linear
+ * Attention (GLA)" and "Kimi Delta Attention (KDA)" (per-channel gate along
+ * the key dimension).  The three write rules are also listed in "Beyond
+ * attention", section "Linear attention: a running sum".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument is a DEVICE pointer (cudaMalloc'd or torch CUDA
+ *    storage) on the current CUDA device, 16-byte aligned, contiguous in the
+ *    layout stated.  The caller owns every buffer; the library allocates no
+ *    device memory and keeps no state between calls except one device status
+ *    word (see gdn_device_status).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously on it; a return value of GDN_OK means the
+ *    launch was accepted, not that it finished.
+ *  - q, k, v, o element type is given by desc->dtype / desc->out_dtype
+ *    (GDN_F32 = float, GDN_BF16 = bfloat16).  g, beta and the state are float.
+ *  - g holds the log-gate log(alpha) (normally <= 0):  [B,H,T] for
+ *    GDN_GATE_SCALAR, [B,H,T,dk] for GDN_GATE_CHANNEL, and must be NULL for
+ *    GDN_GATE_NONE.  beta [B,H,T] is read only for GDN_DELTA (else may be NULL).
+ *  - NaN or Inf in the inputs propagate to the outputs; nothing traps.
+ *  - Errors are negative return codes; nothing is launched when a call fails
+ *    validation.  gdn_strerror() names them.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_VERSION 1
+
+/* Return codes. */
+#define GDN_OK 0
+#define GDN_ERR_ARG (-1)         /* null pointer, bad enum, bad size or overlap */
+#define GDN_ERR_ALIGN (-2)       /* a pointer is not 16-byte aligned */
+#define GDN_ERR_UNSUPPORTED (-3) /* valid request this build does not implement */
+#define GDN_ERR_CUDA (-4)        /* the CUDA runtime refused the launch */
+#define GDN_ERR_TIMEOUT (-5)     /* device status: a bounded wait in a kernel ran out */
+#define GDN_ERR_RANGE (-6)       /* device status: an fp16 tensor-core operand overflowed */
+
+/* Write rule.  ADDITIVE: S += v k^T, no gate ("Naive linear attention").
+ * DECAY: S = S Diag(alpha) + v k^T, gate required (RetNet / Mamba-2 / GLA).
+ * DELTA: the gated delta rule above; any gate (DeltaNet / GDN / KDA). */
+typedef enum { GDN_ADDITIVE = 0, GDN_DECAY = 1, GDN_DELTA = 2 } gdn_update_t;
+
+/* Gate: none (alpha = 1), one scalar per token and head, or one value per key
+ * channel per token and head. */
+typedef enum { GDN_GATE_NONE = 0, GDN_GATE_SCALAR = 1, GDN_GATE_CHANNEL = 2 } gdn_gate_t;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
+
+/* Kernel choice for gdn_chunk_fwd.  AUTO picks the tensor-core kernel when it
+ * supports the request (bf16 inputs, dk = 128) and the fp32 SIMT kernel
+ * otherwise; the two explicit values force one (GDN_ERR_UNSUPPORTED if it
+ * cannot serve the request). */
+typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TC = 2 } gdn_algo_t;
+
+typedef struct {
+    int B, H;      /* batch and heads; B*H >= 0 */
+    int T;         /* tokens per sequence (gdn_chunk_fwd: T >= 0; decode: T == 1) */
+    int dk, dv;    /* key and value head dims, each 64 or 128 */
+    int update;    /* gdn_update_t */
+    int gate;      /* gdn_gate_t */
+    int dtype;     /* gdn_dtype_t of q, k, v */
+    int out_dtype; /* gdn_dtype_t of o */
+    int chunk;     /* chunk length C of the chunkwise form; 0 or 64 (others rejected) */
+    int algo;      /* gdn_algo_t (gdn_chunk_fwd only; ignored by decode) */
+} gdn_desc_t;
+
+/*
+ * gdn_chunk_fwd -- prefill: the recurrence over T tokens for every (b,h), in
+ * chunkwise-parallel form with chunk length C = 64.
+ *
+ * Defined by "Linear Attention, Visualized", section "Chunkwise algorithm"
+ * (history read plus masked local block, then the state update), with the
+ * decayed operands of "Mamba-2 ... Chunkwise form" / the GLA section and the
+ * correction rows Z of "Optional: Use UT to share the triangular transform"
+ * and "Correct the incoming state" (the GDN and KDA tables).  Every chunk
+ * length gives the token recurrence exactly ("Cost").
+ *
+ *   q, k  [B,H,T,dk]   dtype          v  [B,H,T,dv]  dtype
+ *   g     see above    float          beta [B,H,T]   float (DELTA)
+ *   S0    [B,H,dv,dk]  float, or NULL for a zero initial state
+ *   o     [B,H,T,dv]   out_dtype      (written)
+ *   S_T   [B,H,dv,dk]  float, or NULL to skip; may alias S0 (in-place carry)
+ *
+ * o must not overlap any input.  T == 0 is valid (o is empty, S_T <- S0).
+ * Returns GDN_OK or a negative code.
+ */
+int gdn_chunk_fwd(const gdn_desc_t *desc, const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                  void *stream);
+
+/*
+ * gdn_decode_step -- decode: one recurrent step (T == 1) for every (b,h), with
+ * the state updated in place ("Optional: Linear attention as an RNN": fixed
+ * state, constant work per token; the per-token recurrences of the RetNet,
+ * Mamba-2, DeltaNet, GDN, GLA and KDA sections).  A bandwidth-bound rank-1
+ * update: per state row i, with a = alpha_t,
+ *     p_i = sum_j S_ij a_j k_j,  r_i = sum_j S_ij a_j q_j,
+ *     u_i = beta (v_i - p_i)  (DELTA)  or  v_i  (ADDITIVE / DECAY),
+ *     S_ij <- S_ij a_j + u_i k_j,   o_i = r_i + u_i (k . q).
+ *
+ *   q, k  [B,H,1,dk]   dtype          v  [B,H,1,dv]  dtype
+ *   g     [B,H,1] (scalar) or [B,H,1,dk] (channel) or NULL     float
+ *   beta  [B,H,1]      float (DELTA)
+ *   S     [B,H,dv,dk]  float, read and overwritten in place
+ *   o     [B,H,1,dv]   out_dtype      (written)
+ *
+ * desc->T must be 1; desc->chunk and desc->algo are ignored.
+ */
+int gdn_decode_step(const gdn_desc_t *desc, const void *q, const void *k, const void *v,
+                    const float *g, const float *beta, float *S, void *o, void *stream);
+
+/* Static string naming a return code (never NULL). */
+const char *gdn_strerror(int code);
+
+/*
+ * gdn_device_status -- synchronises the current device, then returns the
+ * library's device status word: GDN_OK, GDN_ERR_TIMEOUT or GDN_ERR_RANGE (the
+ * first error any kernel of this library recorded since the last clear), or
+ * GDN_ERR_CUDA if the synchronisation itself failed.  With clear != 0 the word
+ * is reset to GDN_OK afterwards.  Kernels never trap: a kernel that records an
+ * error finishes (possibly with partial results) and leaves the context usable.
+ */
+int gdn_device_status(int clear);
+
+/* GDN_VERSION of the built library. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,102 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+declared in include/gdn.h, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import gated_delta_rule_97_b200 as gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gdn.build()
+    return gdn.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("gdn_chunk_fwd", "gdn_decode_step", "gdn_strerror"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", gdn.lib_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (gdn_[a-z_0-9]+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_strerror_and_version(lib):
+    assert gdn.version() == 1
+    for code in (0, -1, -2, -3, -4, -5, -6, 123):
+        assert isinstance(gdn.strerror(code), str) and gdn.strerror(code)
+
+
+def _desc(**kw):
+    base = dict(B=2, H=3, T=100, dk=128, dv=128, update="delta", gate="scalar", dtype=gdn.BF16,
+                out_dtype=gdn.F32)
+    base.update(kw)
+    return gdn.make_desc(**base)
+
+
+def _call(lib, d, q=0x10000, k=0x20000, v=0x30000, g=0x40000, beta=0x50000, S0=None, o=0x9000000,
+          ST=None):
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdn_chunk_fwd(ctypes.byref(d) if d is not None else None, vp(q), vp(k), vp(v), vp(g), vp(beta),
+                             vp(S0), vp(o), vp(ST), None)
+
+
+def test_rejects_bad_arguments_without_launching(lib):
+    # Every call below fails validation, which happens before any CUDA call.
+    assert _call(lib, None) == -1
+    assert _call(lib, _desc(dk=96)) == -1
+    assert _call(lib, _desc(dv=32)) == -1
+    assert _call(lib, _desc(update=None) if False else gdn.Desc(2, 3, 100, 128, 128, 7, 1, 1, 0, 64, 0)) == -1
+    assert _call(lib, _desc(update="additive", gate="scalar")) == -1       # additive takes no gate
+    assert _call(lib, _desc(update="decay", gate="none"), g=None) == -1   # decay needs a gate
+    assert _call(lib, _desc(gate="none")) == -1                           # g given but gate none
+    assert _call(lib, _desc(), g=None) == -1                              # gate but no g
+    assert _call(lib, _desc(), beta=None) == -1                           # delta needs beta
+    assert _call(lib, _desc(), q=None) == -1
+    assert _call(lib, _desc(T=-1)) == -1
+    assert _call(lib, _desc(chunk=32)) == -3
+    assert _call(lib, _desc(), k=0x20008) == -2                           # misaligned
+    assert _call(lib, _desc(), o=0x10000 + 64) == -1                      # o overlaps q
+
+
+def test_empty_batch_is_a_noop(lib):
+    assert _call(lib, _desc(B=0)) == 0
+    assert _call(lib, _desc(H=0), q=None, k=None, v=None, g=None, beta=None, o=None) == 0
+
+
+def test_decode_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    d = _desc(T=2)
+    assert lib.gdn_decode_step(ctypes.byref(d), vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000),
+                               vp(0x100000), vp(0x6000), None) == -1   # T must be 1
+    d = _desc(T=1)
+    assert lib.gdn_decode_step(ctypes.byref(d), vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000),
+                               vp(0x100004), vp(0x6000), None) == -2   # misaligned state
+    assert lib.gdn_decode_step(ctypes.byref(d), vp(0x1000), vp(0x2000), vp(0x3000), None, vp(0x5000),
+                               vp(0x100000), vp(0x6000), None) == -1   # gate without g
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(gdn, "_lib", None)
+    monkeypatch.setattr(gdn, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        gdn.load()
