@@ -317,8 +317,20 @@ def run_ours(args):
     gdn.device_status(clear=True)
     peaks, peak_kind = load_peaks()
 
+    if args.only == "decode":
+        wd = WORKLOADS["decode_gdn_bf16"]
+        n_dec = wd.steps if not args.quick else 100
+        ms_d = time_decode(wd, n_dec, torch, gdn)
+        if rank == 0:
+            print(json.dumps({"only": "decode", "ms_per_step": ms_d}), flush=True)
+        return
     w = WORKLOADS[args.workload]
     x = make_prefill_inputs(w)
+    if args.only == "prefill":
+        ms = time_prefill(w, x, args.steps, args.warmup, torch, gdn, dist)
+        if rank == 0:
+            print(json.dumps({"only": "prefill", "workload": w.name, "ms_per_step": ms}), flush=True)
+        return
     with ClockSampler(local) as clk:
         ms = time_prefill(w, x, args.steps, args.warmup, torch, gdn, dist)
     clocks = clk.summary()
@@ -426,6 +438,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=[k for k, w in WORKLOADS.items() if w.steps == 0])
     ap.add_argument("--quick", action="store_true", help="skip the extra prefill workloads; 100 decode steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="profiling aid: run one part only (its line is not a benchmark result)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -16,7 +16,7 @@ import ctypes
 import os
 
 __all__ = ["GDNError", "chunk_fwd", "decode_step", "device_status", "strerror", "version", "load",
-           "lib_path", "Desc", "UPDATES", "GATES", "build"]
+           "lib_path", "Desc", "UPDATES", "GATES", "build", "device_diag"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libgdn.so")
@@ -79,6 +79,7 @@ def load():
     lib.gdn_device_status.argtypes = [ctypes.c_int]
     lib.gdn_device_status.restype = ctypes.c_int
     lib.gdn_version.restype = ctypes.c_int
+    lib.gdn_device_diag.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -94,6 +95,11 @@ def version() -> int:
 def device_status(clear: bool = True) -> int:
     """The library's device status word (synchronises the device)."""
     return int(load().gdn_device_status(1 if clear else 0))
+
+
+def device_diag() -> int:
+    """Where the first recorded kernel timeout happened (0 if none)."""
+    return int(load().gdn_device_diag())
 
 
 def _ptr(t):

@@ -5,8 +5,10 @@
 #include "../../include/gdn.h"
 #include "common.cuh"
 
-// The library's device status word (first error code any kernel recorded).
+// The library's device status word (first error code any kernel recorded) and
+// diagnostic word (where the first timeout happened).
 __device__ int g_gdn_status = 0;
+__device__ int g_gdn_diag = 0;
 
 namespace {
 
@@ -14,6 +16,12 @@ int *status_ptr() {
     // The address is per device; looked up on every call (cheap, no allocation).
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_gdn_status) != cudaSuccess) return nullptr;
+    return static_cast<int *>(p);
+}
+
+int *diag_ptr() {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gdn_diag) != cudaSuccess) return nullptr;
     return static_cast<int *>(p);
 }
 
@@ -68,7 +76,15 @@ extern "C" int gdn_device_status(int clear) {
     if (clear) {
         const int z = 0;
         if (cudaMemcpyToSymbol(g_gdn_status, &z, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+        if (cudaMemcpyToSymbol(g_gdn_diag, &z, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
     }
+    return v;
+}
+
+extern "C" int gdn_device_diag(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_gdn_diag, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
     return v;
 }
 
@@ -110,6 +126,7 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     gdn::ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
     a.status = status_ptr();
+    a.diag = diag_ptr();
     a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
 
     const bool tc_ok = gdn_tc_supported(d) != 0;

@@ -41,6 +41,7 @@ struct ChunkArgs {
     void *o;                 // [BH,T,dv], output dtype
     float *ST;               // [BH,dv,dk] or null
     int *status;             // device status word
+    int *diag;               // device diagnostic word (first timeout site)
     int BH, T, dk, dv;
 };
 

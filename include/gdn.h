@@ -141,6 +141,15 @@ const char *gdn_strerror(int code);
  */
 int gdn_device_status(int clear);
 
+/*
+ * gdn_device_diag -- synchronises the current device and returns where the
+ * first recorded timeout happened: 0 if none, else 1 + site * 1000000 + chunk,
+ * where site names the wait (1 input tiles, 2 chunk Gram product, 3 W/U
+ * products, 4 history read, 5 output and state update) and chunk is the chunk
+ * index.  Cleared together with the status word by gdn_device_status(1).
+ */
+int gdn_device_diag(void);
+
 /* GDN_VERSION of the built library. */
 int gdn_version(void);
 

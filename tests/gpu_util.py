@@ -30,7 +30,9 @@ def run_prefill(w, x, algo="auto", out_dtype=torch.float32, S0_dev=None):
                           S0_dev if S0_dev is not None else dev(x["S0"]), update=w.update, gate=w.gate,
                           out_dtype=out_dtype, algo=algo)
     torch.cuda.synchronize()
-    assert gdn.device_status() == 0
+    diag = gdn.device_diag()
+    status = gdn.device_status()
+    assert status == 0, ("device status", status, "diag", diag)
     return o, ST
 
 
