@@ -55,7 +55,7 @@ def lib_path() -> str:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     """Compiles libgdn.so in-tree (nvcc, sm_100a)."""
-    from .build import build as _build
+    from .builder import build as _build
 
     return _build(verbose=verbose, force=force)
 

@@ -1,8 +1,8 @@
 // Tensor-core (tcgen05 / TMEM / TMA) chunkwise prefill for bf16 inputs, dk = 128.
 //
-// One CTA (4 warps, thread t <-> TMEM lane t) owns one (b,h) head and a slice
-// of DVS value rows of its state, and walks the chunks of the sequence in
-// order.  The state is kept TRANSPOSED in TMEM as an fp32 accumulator
+// One CTA (8 warps; warp w reads TMEM lane quarter w%4 and column half w/4)
+// owns one (b,h) head and a slice of DVS value rows of its state, and walks
+// the chunks of the sequence in order.  The state is kept TRANSPOSED in TMEM as an fp32 accumulator
 // D_S = S^T [dk=128 lanes][DVS columns], so the per-key-channel decay
 // S Diag(e^{G_C}) is a per-lane scale and the state update is one MMA.
 //
@@ -17,7 +17,7 @@
 //   a3  T = (I + L)^{-1}: fp32 forward substitution, one column per thread,
 //       written as the fp16 operand T2 = T diag(beta)
 //   a4  D_W = [T2;0] K<,  D_ZO = [T2;0] V                    (MMA)
-//   a5  D_ZO += [-W; Q<] S^T  -> rows 0..63 = Z = U - W S^T   (MMA)
+//   a5  D_ZO -= [W; -Q<] S^T  -> rows 0..63 = Z = U - W S^T   (MMA, A negated)
 //   a6  D_ZO += [0; A'] Z     -> rows 64..127 = O             (MMA)
 //   a7  D_S = e^{G_C} D_S + K>^T Z                            (scale + MMA)
 // Operands that are intermediates (T2, W, Q<, K<, K>, A', Z, S^T) are fp16
@@ -33,12 +33,29 @@
 #include "sm100.cuh"
 #include "tma_host.cuh"
 
+#ifdef GDN_TC_PHASE_TIMING
+// Per-phase cycle totals of CTA 0 (profiling builds only).
+__device__ unsigned long long g_tc_phase[16];
+#define TC_MARK(i)                                                              \
+    do {                                                                       \
+        if (blockIdx.x == 0 && t == 0) {                                       \
+            const long long now_ = clock64();                                  \
+            atomicAdd(&g_tc_phase[i], (unsigned long long)(now_ - mark_prev)); \
+            mark_prev = now_;                                                  \
+        }                                                                      \
+    } while (0)
+#else
+#define TC_MARK(i) \
+    do {           \
+    } while (0)
+#endif
+
 namespace gdn {
 namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 256;
 constexpr int C = kChunk;  // 64
 constexpr int DK = 128;
 // Largest per-channel decay (nats) inside one chunk for which the factored
@@ -83,6 +100,7 @@ struct Misc {
     float gam[64];
     float b[64];
     float beta[64];
+    float ib[64];
     float GC[128];
     int abort_flag;
     int range_flag;
@@ -115,6 +133,13 @@ __device__ __forceinline__ uint4 pack_h8(const float *f) {
     return make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
 }
 
+// Float offset of element (r, c) in a row-major fp32 tile with `ld` columns
+// whose 16-byte slots are XOR-swizzled by (r % 8): conflict-free for one row
+// per thread writing float4s and for float4 reads of a shared row.
+__device__ __forceinline__ int f32_swz(int r, int c, int ld) {
+    return r * ld + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3);
+}
+
 // Marks the CTA aborted and remembers the first wait that gave up (site, chunk).
 template <typename M>
 __device__ __forceinline__ void note_timeout(M &ms, int site, int r) {
@@ -123,24 +148,21 @@ __device__ __forceinline__ void note_timeout(M &ms, int site, int r) {
 
 __device__ __forceinline__ bool out_of_fp16(float x) { return !(fabsf(x) <= 65504.f) && x == x; }
 
-// Loads 64 consecutive TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float *v) {
-#pragma unroll
-    for (int c = 0; c < 64; c += 16) tmem_ld16(taddr + c, v + c);
-    tmem_wait_ld();
-}
-
 template <int DVS, int UPD, int GATE, bool OUT_BF16>
 __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_constant__ TcParams p) {
     using L = TcSmem<DVS, GATE>;
     constexpr bool DELTA = (UPD == kDelta);
     constexpr int NB = DVS / 64;  // 64-wide value blocks
+    constexpr int HV = DVS / 2;   // value columns per column half
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     Misc &ms = *reinterpret_cast<Misc *>(sm + L::MISC);
 
     const int t = threadIdx.x;
-    const int warp = t >> 5;
+    const int warp = t >> 5, lane = t & 31;
+    const int sp = warp & 3;          // TMEM lane quarter this warp may access
+    const int ch = warp >> 2;         // column half handled by this warp
+    const int row = sp * 32 + lane;   // accumulator row (TMEM lane) of this thread
     const int bh = blockIdx.x / p.nslices;
     const int v0 = (blockIdx.x % p.nslices) * DVS;
     const int T = p.T, dv = p.dv;
@@ -166,10 +188,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
         tmem_alloc(&ms.tmem_base, 512);
         tmem_relinquish();
     }
-    // zero block of the [T2 | 0 | A'] tile (rows 0..63 of [0; A'])
+    // T2 block (its upper-right 32x32 block stays zero) and the zero block of [0; A']
     for (int i = t; i < 8192 / 16; i += kTcThreads) {
+        reinterpret_cast<uint4 *>(sm + L::TZA)[i] = make_uint4(0, 0, 0, 0);
         reinterpret_cast<uint4 *>(sm + L::TZA + 8192)[i] = make_uint4(0, 0, 0, 0);
-        if (!DELTA) {  // rows 0..63 of [-W; Q<] are read but unused without the delta write
+        if (!DELTA) {  // the W rows of [W; -Q<] are read but must contribute nothing
             reinterpret_cast<uint4 *>(sm + L::AT)[i] = make_uint4(0, 0, 0, 0);
             reinterpret_cast<uint4 *>(sm + L::AT + 24576)[i] = make_uint4(0, 0, 0, 0);
         }
@@ -177,7 +200,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ms.tmem_base;
-    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t t_lane = tmem + ((uint32_t)(sp * 32) << 16);
     const uint32_t TM_P = 0, TM_W = 64, TM_ZO = 192, TM_S = 192 + DVS;
 
     auto issue_tma = [&](int r) {
@@ -193,37 +216,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
             for (int j = 0; j < 4; ++j) tma_load_3d(sm + L::GCH + j * 8192, &p.g_map, j * 32, t0, bh, &ms.bar_tma);
     };
     if (t == 0 && nchunks > 0) issue_tma(0);
-
-    // initial state: thread t = key channel t holds column t of S (row t of S^T)
-    {
-        float sv[16];
-        for (int j0 = 0; j0 < DVS; j0 += 16) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                sv[i] = p.S0 ? p.S0[((size_t)bh * dv + v0 + j0 + i) * DK + t] : 0.f;
-            __syncwarp();
-            tmem_st16(t_lane + TM_S + j0, sv);
-            // fp16 copy: S^T tile row t, columns j0..j0+15 (blocks of 64)
-#pragma unroll
-            for (int i = 0; i < 16; i += 8) {
-                const int j = j0 + i;
-                *reinterpret_cast<uint4 *>(sm + L::ST16 + (j / 64) * 16384 + sw128_off(t, j % 64)) = pack_h8(sv + i);
-            }
+    // gate and beta of a chunk are loaded one chunk ahead into registers
+    float gpre0 = 0.f, gpre1 = 0.f, bpre = 0.f;
+    auto load_gate_beta = [&](int r) {
+        const int t0 = r * C;
+        if (GATE == kGateScalar && warp == 0) {
+            const int l0 = 2 * lane;
+            gpre0 = (t0 + l0 < T) ? p.g[(size_t)bh * T + t0 + l0] : 0.f;
+            gpre1 = (t0 + l0 + 1 < T) ? p.g[(size_t)bh * T + t0 + l0 + 1] : 0.f;
         }
-        tmem_wait_st();
+        if (DELTA && t < C) bpre = (t0 + t < T) ? p.beta[(size_t)bh * T + t0 + t] : 0.f;
+    };
+    if (nchunks > 0) load_gate_beta(0);
+
+    // initial state: lane `row` = key channel; this warp's column half of S^T
+    for (int j0 = ch * HV; j0 < ch * HV + HV; j0 += 16) {
+        float sv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sv[i] = p.S0 ? p.S0[((size_t)bh * dv + v0 + j0 + i) * DK + row] : 0.f;
+        __syncwarp();
+        tmem_st16(t_lane + TM_S + j0, sv);
+#pragma unroll
+        for (int i = 0; i < 16; i += 8) {
+            const int j = j0 + i;
+            *reinterpret_cast<uint4 *>(sm + L::ST16 + (j >> 6) * 16384 + sw128_off(row, j & 63)) = pack_h8(sv + i);
+        }
     }
+    tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
 
+#ifdef GDN_TC_PHASE_TIMING
+    long long mark_prev = clock64();
+#endif
     bool ok = true;
-    bool range_bad = false;  // this thread produced an operand outside fp16 range
+    float rmax = 0.f;  // largest |value| this thread handed to an fp16 operand (range check)
     for (int r = 0; r < nchunks && ok; ++r) {
         const uint32_t ph = r & 1;
         const int t0 = r * C;
         const int n = min(C, T - t0);
         // ---------------------------------------------------- wait for inputs
+        TC_MARK(0);
         if (!mbar_wait(&ms.bar_tma, ph)) note_timeout(ms, 1, r);
+        TC_MARK(1);
         // scalar / no gate: P = [Q;K] K^T straight from the bf16 tiles
         if (GATE != kGateChannel && t == 0 && !ms.abort_flag) {
             tc_fence_after();
@@ -240,109 +276,130 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
         // ---------------------------------------------------- a1: gate prefix
         if (GATE == kGateScalar) {
             if (warp == 0) {
-                const int l0 = 2 * t;
-                float x0 = (t0 + l0 < T) ? p.g[(size_t)bh * T + t0 + l0] : 0.f;
-                float x1 = (t0 + l0 + 1 < T) ? p.g[(size_t)bh * T + t0 + l0 + 1] : 0.f;
+                const int l0 = 2 * lane;
+                const float x0 = gpre0, x1 = gpre1;
                 float s = x0 + x1;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, s, off);
-                    if (t >= off) s += y;
+                    if (lane >= off) s += y;
                 }
                 const float e = s - (x0 + x1);
                 ms.G[l0] = e + x0;
                 ms.G[l0 + 1] = e + x0 + x1;
             }
         } else if (GATE == kGateChannel) {
-            // thread t = channel t: inclusive prefix over the 64 tokens, in place
-            float *gcol = reinterpret_cast<float *>(sm + L::GCH + (t / 32) * 8192) + (t % 32);
+            // channel c = t & 127, token half hf = t >> 7: prefix over 32 tokens, then join
+            const int c = t & 127, hf = t >> 7;
+            float *gcol = reinterpret_cast<float *>(sm + L::GCH + (c >> 5) * 8192) + (c & 31);
             float s = 0.f;
-            for (int l = 0; l < C; ++l) {
+#pragma unroll 8
+            for (int l = 32 * hf; l < 32 * hf + 32; ++l) {
                 s += gcol[l * 32];
                 gcol[l * 32] = s;
             }
-            ms.GC[t] = s;
+            __syncthreads();
+            if (hf == 1) {
+                const float base = gcol[31 * 32];
+#pragma unroll 8
+                for (int l = 32; l < 64; ++l) gcol[l * 32] += base;
+                ms.GC[c] = s + base;
+            }
         }
-        if (DELTA && t < C) ms.beta[t] = (t < n) ? p.beta[(size_t)bh * T + t0 + t] : 0.f;
+        if (DELTA && t < C) ms.beta[t] = bpre;
+        if (r + 1 < nchunks) load_gate_beta(r + 1);  // consumed next chunk; latency hidden
         __syncthreads();
-        if (GATE == kGateScalar && t < C) {
+        bool fastg = true;  // scalar gate: decay factors as b_l / b_m (chunk decay <= 80 nats)
+        if (GATE == kGateScalar) {
             const float gc = ms.G[C - 1];
-            ms.b[t] = __expf(ms.G[t]);
-            ms.gam[t] = __expf(gc - ms.G[t]);
+            fastg = -gc <= 80.f;
+            if (t < C) {
+                const float G = ms.G[t];
+                ms.b[t] = __expf(G);
+                ms.gam[t] = __expf(gc - G);
+                ms.ib[t] = __expf(-G);
+            }
         }
-        if (GATE == kGateChannel && t == 0) {
+        if (GATE == kGateChannel && warp == 0) {
             float mx = 0.f;
-            for (int c = 0; c < DK; ++c) mx = fmaxf(mx, -ms.GC[c]);
-            ms.slow_chunk = !(mx <= kFactorMaxDecay);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx = fmaxf(mx, -ms.GC[lane + 32 * i]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if (lane == 0) ms.slow_chunk = !(mx <= kFactorMaxDecay);
         }
         // scale the state by the chunk's total decay: D_S <- e^{G_C} D_S (lane = channel)
         if (GATE != kGateNone) {
-            __syncthreads();
-            const float dec = (GATE == kGateScalar) ? __expf(ms.G[C - 1]) : __expf(ms.GC[t]);
-            float sv[16];
-            for (int j0 = 0; j0 < DVS; j0 += 16) {
+            const float dec = (GATE == kGateScalar) ? __expf(ms.G[C - 1]) : __expf(ms.GC[row]);
+#pragma unroll
+            for (int j0 = 0; j0 < HV; j0 += 32) {
+                float sv[32];
                 __syncwarp();
-                tmem_ld16(t_lane + TM_S + j0, sv);
+                tmem_ld32(t_lane + TM_S + ch * HV + j0, sv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) sv[i] *= dec;
-                tmem_st16(t_lane + TM_S + j0, sv);
+                for (int i = 0; i < 32; ++i) sv[i] *= dec;
+                tmem_st16(t_lane + TM_S + ch * HV + j0, sv);
+                tmem_st16(t_lane + TM_S + ch * HV + j0 + 16, sv + 16);
             }
             tmem_wait_st();
         }
         __syncthreads();
 
+        TC_MARK(2);
         // ---------------------------------------------------- operand conversions
         // Each 16-byte chunk of a 128B-swizzled [64][64] box holds 8 consecutive
         // channels of one token row; the same offset addresses the same element in
-        // every tile that shares the layout.
+        // every tile that shares the layout.  Q< is stored negated: the history
+        // MMA negates its A operand [W; -Q<].
+        const bool slow = (GATE == kGateChannel) && ms.slow_chunk;
         for (int i = t; i < 2 * 512; i += kTcThreads) {
             const int h = i >> 9, off = (i & 511) * 16;
             const int l = off >> 7;
             const int c0 = h * 64 + ((((off >> 4) & 7) ^ (l & 7)) << 3);
-            float qf[8], kf[8], ql[8], kl[8], kr[8], kt[8];
+            float qf[8], kf[8], ql[8], kl[8], kr[8];
             unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + off), qf);
             unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + 8192 + off), kf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fmaxf(fabsf(qf[e]), fabsf(kf[e])));
             if (GATE == kGateChannel) {
-                const float *gg = reinterpret_cast<const float *>(sm + L::GCH + (c0 / 32) * 8192) + l * 32 + (c0 % 32);
+                const float *gg = reinterpret_cast<const float *>(sm + L::GCH + (c0 >> 5) * 8192) + l * 32 + (c0 & 31);
+                float kt[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float G = gg[e];
                     const float eg = __expf(G), emg = __expf(-G);
-                    ql[e] = qf[e] * eg;
+                    ql[e] = -qf[e] * eg;
                     kl[e] = kf[e] * eg;
-                    kt[e] = kf[e] * emg;
+                    kt[e] = slow ? 0.f : kf[e] * emg;  // factored fast path only
                     kr[e] = kf[e] * __expf(ms.GC[c0 + e] - G);
+                    rmax = fmaxf(rmax, fabsf(kt[e]));
                 }
+                *reinterpret_cast<uint4 *>(sm + L::KT + h * 8192 + off) = pack_h8(kt);
             } else {
                 const float bl = (GATE == kGateScalar) ? ms.b[l] : 1.f;
                 const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    ql[e] = qf[e] * bl;
+                    ql[e] = -qf[e] * bl;
                     kl[e] = kf[e] * bl;
                     kr[e] = kf[e] * gl;
-                    kt[e] = 0.f;
                 }
             }
             *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(ql);
             if (DELTA) *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
             *reinterpret_cast<uint4 *>(sm + L::KR + h * 8192 + off) = pack_h8(kr);
-            if (GATE == kGateChannel) {
-                *reinterpret_cast<uint4 *>(sm + L::KT + h * 8192 + off) = pack_h8(kt);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    range_bad |= out_of_fp16(kt[e]);
-            }
         }
         for (int i = t; i < NB * 512; i += kTcThreads) {
             float vf[8];
             unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_V + i * 16), vf);
             *reinterpret_cast<uint4 *>(sm + L::V16 + i * 16) = pack_h8(vf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(vf[e]));
         }
         fence_proxy_async_smem();
         __syncthreads();
-        // per-channel gate: P = [Q<; K<] (k e^{-G})^T on fp16 operands
+        // per-channel gate: P = [-Q<; K<] (k e^{-G})^T on fp16 operands
         if (GATE == kGateChannel && t == 0) {
             tc_fence_after();
             const uint32_t at = smem_u32(sm + L::AT), kt = smem_u32(sm + L::KT);
@@ -355,21 +412,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
             }
             mma_commit(&ms.bar_p1);
         }
+        TC_MARK(3);
         if (!mbar_wait(&ms.bar_p1, ph)) note_timeout(ms, 2, r);
+        TC_MARK(4);
         tc_fence_after();
 
         // ---------------------------------------------------- a2: A' and L
         {
-            const int l = t & 63;
-            const bool top = t < 64;
-            float pr[64];
+            const int l = row & 63;
+            const bool top = row < 64;
+            const int m0 = ch * 32;  // this warp's 32 columns
+            float pr[32];
             __syncwarp();
-            tmem_ld64(t_lane + TM_P, pr);
-            const bool slow = (GATE == kGateChannel) && ms.slow_chunk;
-            if (slow) {
+            tmem_ld32(t_lane + TM_P + m0, pr);
+            tmem_wait_ld();
+            TC_MARK(15);
+            if (GATE == kGateChannel && slow) {
                 // exact fp32: sum_c x_lc k_mc e^{G_lc - G_mc}
                 const unsigned char *xrow = sm + L::RAW_QK + (top ? 0 : 8192);
-                for (int m = 0; m < 64; ++m) {
+                for (int e = 0; e < 32; ++e) {
+                    const int m = m0 + e;
                     float acc = 0.f;
                     if (m <= l) {
                         for (int c = 0; c < DK; ++c) {
@@ -378,81 +440,148 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
                             const float xv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xrow + h * 16384 + ox));
                             const float kv = __bfloat162float(
                                 *reinterpret_cast<const __nv_bfloat16 *>(sm + L::RAW_QK + h * 16384 + 8192 + om));
-                            const float *gc = reinterpret_cast<const float *>(sm + L::GCH + (c / 32) * 8192);
-                            acc = fmaf(xv * kv, __expf(gc[l * 32 + (c % 32)] - gc[m * 32 + (c % 32)]), acc);
+                            const float *gc = reinterpret_cast<const float *>(sm + L::GCH + (c >> 5) * 8192);
+                            acc = fmaf(xv * kv, __expf(gc[l * 32 + (c & 31)] - gc[m * 32 + (c & 31)]), acc);
                         }
                     }
-                    pr[m] = acc;
+                    pr[e] = acc;
                 }
+            } else if (GATE == kGateChannel && top) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pr[e] = -pr[e];  // the factored product used -Q<
+            }
+            float dec[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int m = m0 + e;
+                float d = 1.f;
+                if (GATE == kGateScalar) d = fastg ? ms.b[l] * ms.ib[m] : __expf(ms.G[l] - ms.G[m < l ? m : l]);
+                dec[e] = d;
             }
             if (top) {
                 // A'[l][m] (m <= l) -> fp16, row 64+l of [0; A'] (K-major, K = 64)
 #pragma unroll
-                for (int m0 = 0; m0 < 64; m0 += 8) {
+                for (int e0 = 0; e0 < 32; e0 += 8) {
                     float a[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int m = m0 + e;
-                        float x = pr[m];
-                        if (GATE == kGateScalar) x *= __expf(ms.G[l] - ms.G[m < l ? m : l]);
-                        a[e] = (m <= l) ? x : 0.f;
-                        range_bad |= out_of_fp16(a[e]);
+                        const int m = m0 + e0 + e;
+                        a[e] = (m <= l) ? pr[e0 + e] * dec[e0 + e] : 0.f;
+                        rmax = fmaxf(rmax, fabsf(a[e]));
                     }
-                    *reinterpret_cast<uint4 *>(sm + L::TZA + 16384 + sw128_off(l, m0)) = pack_h8(a);
+                    *reinterpret_cast<uint4 *>(sm + L::TZA + 16384 + sw128_off(l, m0 + e0)) = pack_h8(a);
                 }
             } else if (DELTA) {
-                // L[l][m] = beta_l * P[l][m] (m < l), fp32, float4-XOR-swizzled rows
+                // L[l][m] = beta_l * P[l][m] (m < l), fp32, swizzled rows
                 const float bl = ms.beta[l];
                 float *Ls = reinterpret_cast<float *>(sm + L::KT);
 #pragma unroll
-                for (int m0 = 0; m0 < 64; m0 += 4) {
+                for (int e0 = 0; e0 < 32; e0 += 4) {
                     float4 v;
                     float *vv = &v.x;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int m = m0 + e;
-                        float x = pr[m];
-                        if (GATE == kGateScalar) x *= __expf(ms.G[l] - ms.G[m < l ? m : l]);
-                        vv[e] = (m < l) ? bl * x : 0.f;
+                        const int m = m0 + e0 + e;
+                        vv[e] = (m < l) ? bl * pr[e0 + e] * dec[e0 + e] : 0.f;
                     }
-                    *reinterpret_cast<float4 *>(Ls + l * 64 + (((m0 >> 2) ^ (l & 15)) << 2)) = v;
+                    *reinterpret_cast<float4 *>(Ls + f32_swz(l, m0 + e0, 64)) = v;
                 }
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+        TC_MARK(5);
         // the raw stage is consumed (P, conversions, exact path): prefetch the next chunk
         if (t == 0 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
 
         if (DELTA) {
             // ------------------------------------------------ a3: T = (I + L)^{-1}
+            // Two-level block solve.  Stage 1: the inverses of the two 32x32
+            // diagonal blocks by forward substitution, one column per thread
+            // (threads 0..63).  Stage 2: T_BA = -T_BB (L_BA T_AA), 4 outputs per
+            // thread.  T is written as the fp16 operand T2 = T diag(beta); the fp32
+            // blocks T_AA (upper-right block of the L scratch, zero in L), T_BB and
+            // X = L_BA T_AA (Z tile region, idle until the history read) feed stage 2.
+            float *Ls = reinterpret_cast<float *>(sm + L::KT);
+            float *Tbb = reinterpret_cast<float *>(sm + L::ZT);
+            float *Xs = Tbb + 32 * 32;
             if (t < 64) {
-                const float *Ls = reinterpret_cast<const float *>(sm + L::KT);
-                float x[64];
+                const int b = t >> 5, c = t & 31, o = 32 * b;
+                float x[32];
 #pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = (i == t) ? 1.f : 0.f;
+                for (int i = 0; i < 32; ++i) x[i] = (i == c) ? 1.f : 0.f;
 #pragma unroll
-                for (int rr = 1; rr < 64; ++rr) {
-                    float acc = x[rr];
+                for (int rr = 1; rr < 32; ++rr) {
+                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-                    for (int m0 = 0; m0 < rr; m0 += 4) {
-                        const float4 lv = *reinterpret_cast<const float4 *>(Ls + rr * 64 + (((m0 >> 2) ^ (rr & 15)) << 2));
-                        acc = fmaf(-lv.x, x[m0], acc);
-                        if (m0 + 1 < rr) acc = fmaf(-lv.y, x[m0 + 1], acc);
-                        if (m0 + 2 < rr) acc = fmaf(-lv.z, x[m0 + 2], acc);
-                        if (m0 + 3 < rr) acc = fmaf(-lv.w, x[m0 + 3], acc);
+                    for (int mm = 0; mm < rr; mm += 4) {
+                        const float4 lv = *reinterpret_cast<const float4 *>(Ls + f32_swz(o + rr, o + mm, 64));
+                        s0 = fmaf(lv.x, x[mm], s0);
+                        if (mm + 1 < rr) s1 = fmaf(lv.y, x[mm + 1], s1);
+                        if (mm + 2 < rr) s2 = fmaf(lv.z, x[mm + 2], s2);
+                        if (mm + 3 < rr) s3 = fmaf(lv.w, x[mm + 3], s3);
                     }
-                    x[rr] = acc;
+                    x[rr] -= (s0 + s1) + (s2 + s3);
                 }
-                // T2[rr][t] = T[rr][t] * beta_t -> fp16, K-major [64][64]
-                const float bt = ms.beta[t];
+                const float bt = ms.beta[o + c];
 #pragma unroll
-                for (int rr = 0; rr < 64; ++rr)
-                    *reinterpret_cast<__half *>(sm + L::TZA + sw128_off(rr, t)) = __float2half_rn(x[rr] * bt);
+                for (int rr = 0; rr < 32; ++rr) {
+                    const float tv = x[rr] * bt;
+                    rmax = fmaxf(rmax, fabsf(tv));
+                    *reinterpret_cast<__half *>(sm + L::TZA + sw128_off(o + rr, o + c)) = __float2half_rn(tv);
+                    if (b == 0)
+                        Ls[f32_swz(rr, 32 + c, 64)] = x[rr];
+                    else
+                        Tbb[f32_swz(rr, c, 32)] = x[rr];
+                }
+            }
+            __syncthreads();
+            TC_MARK(14);
+            {
+                const int rr = t >> 3, c0 = (t & 7) * 4;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int mm = 0; mm < 32; mm += 4) {
+                    const float4 lv = *reinterpret_cast<const float4 *>(Ls + f32_swz(32 + rr, mm, 64));
+                    const float lm[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 a0 = *reinterpret_cast<const float4 *>(Ls + f32_swz(mm + e, 32 + c0, 64));
+                        acc[0] = fmaf(lm[e], a0.x, acc[0]);
+                        acc[1] = fmaf(lm[e], a0.y, acc[1]);
+                        acc[2] = fmaf(lm[e], a0.z, acc[2]);
+                        acc[3] = fmaf(lm[e], a0.w, acc[3]);
+                    }
+                }
+                *reinterpret_cast<float4 *>(Xs + f32_swz(rr, c0, 32)) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                __syncthreads();
+                acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+                for (int mm = 0; mm < 32; mm += 4) {
+                    const float4 tv = *reinterpret_cast<const float4 *>(Tbb + f32_swz(rr, mm, 32));
+                    const float tm[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 a0 = *reinterpret_cast<const float4 *>(Xs + f32_swz(mm + e, c0, 32));
+                        acc[0] = fmaf(tm[e], a0.x, acc[0]);
+                        acc[1] = fmaf(tm[e], a0.y, acc[1]);
+                        acc[2] = fmaf(tm[e], a0.z, acc[2]);
+                        acc[3] = fmaf(tm[e], a0.w, acc[3]);
+                    }
+                }
+                float tb[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    tb[e] = -acc[e] * ms.beta[c0 + e];
+                    rmax = fmaxf(rmax, fabsf(tb[e]));
+                }
+                *reinterpret_cast<uint2 *>(sm + L::TZA + sw128_off(32 + rr, c0)) =
+                    make_uint2(pack_h2(tb[0], tb[1]), pack_h2(tb[2], tb[3]));
             }
             fence_proxy_async_smem();
             __syncthreads();
+            TC_MARK(6);
             // ------------------------------------------------ a4: W and U
             if (t == 0) {
                 tc_fence_after();
@@ -468,34 +597,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
                 mma_commit(&ms.bar_w);
             }
             if (!mbar_wait(&ms.bar_w, ph)) note_timeout(ms, 3, r);
+            TC_MARK(7);
             tc_fence_after();
-            if (t < 64) {
-                // -W -> rows 0..63 of the [-W | Q< | K<] tile
-                for (int c0 = 0; c0 < 128; c0 += 16) {
-                    float w[16];
+            if (sp < 2) {
+                // W rows (lanes 0..63): this warp's 64-column half -> W slot of that half
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 32) {
+                    float w[32];
                     __syncwarp();
-                    tmem_ld16(t_lane + TM_W + c0, w);
+                    tmem_ld32(t_lane + TM_W + ch * 64 + c0, w);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        w[e] = -w[e];
-                        range_bad |= out_of_fp16(w[e]);
-                    }
-                    const int h = c0 >> 6;
-                    *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + sw128_off(t, c0 & 63)) = pack_h8(w);
-                    *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + sw128_off(t, (c0 & 63) + 8)) = pack_h8(w + 8);
+                    for (int e = 0; e < 32; ++e) rmax = fmaxf(rmax, fabsf(w[e]));
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8)
+                        *reinterpret_cast<uint4 *>(sm + L::AT + ch * 24576 + sw128_off(row, c0 + e)) = pack_h8(w + e);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncthreads();
         }
+        TC_MARK(8);
 
         // ---------------------------------------------------- a5: history read (+ correction)
         if (t == 0 && !ms.abort_flag) {
             tc_fence_after();
             const uint32_t at = smem_u32(sm + L::AT), st = smem_u32(sm + L::ST16);
-            constexpr uint32_t id = idesc_f16(128, DVS, 0, 0, 1);
+            constexpr uint32_t id = idesc_f16(128, DVS, 0, 0, 1, /*negate A*/ 1);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const uint32_t ka = (k >> 2) * 24576 + (k & 3) * 32;
@@ -505,24 +634,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
             mma_commit(&ms.bar_1);
         }
         if (!mbar_wait(&ms.bar_1, ph)) note_timeout(ms, 4, r);
+        TC_MARK(9);
         tc_fence_after();
-        if (DELTA && t < 64) {
-            // Z rows -> fp16 MN-major tile [64 tok][DVS]
-            for (int j0 = 0; j0 < DVS; j0 += 16) {
-                float z[16];
+        if (DELTA && sp < 2) {
+            // Z rows (lanes 0..63), this warp's column half -> fp16 MN-major tile [64 tok][DVS]
+#pragma unroll
+            for (int j0 = 0; j0 < HV; j0 += 32) {
+                float z[32];
                 __syncwarp();
-                tmem_ld16(t_lane + TM_ZO + j0, z);
+                tmem_ld32(t_lane + TM_ZO + ch * HV + j0, z);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) range_bad |= out_of_fp16(z[e]);
-                unsigned char *zb = sm + L::ZT + (j0 >> 6) * 8192;
-                *reinterpret_cast<uint4 *>(zb + sw128_off(t, j0 & 63)) = pack_h8(z);
-                *reinterpret_cast<uint4 *>(zb + sw128_off(t, (j0 & 63) + 8)) = pack_h8(z + 8);
+                for (int e = 0; e < 32; ++e) rmax = fmaxf(rmax, fabsf(z[e]));
+                const int j = ch * HV + j0;
+                unsigned char *zb = sm + L::ZT + (j >> 6) * 8192;
+#pragma unroll
+                for (int e = 0; e < 32; e += 8)
+                    *reinterpret_cast<uint4 *>(zb + sw128_off(row, (j & 63) + e)) = pack_h8(z + e);
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+        TC_MARK(10);
 
         // ---------------------------------------------------- a6 + a7: local output and state update
         if (t == 0 && !ms.abort_flag) {
@@ -540,66 +674,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
             mma_commit(&ms.bar_2);
         }
         if (!mbar_wait(&ms.bar_2, ph)) note_timeout(ms, 5, r);
+        TC_MARK(11);
         tc_fence_after();
-        if (t >= 64) {
-            const int l = t - 64;
+        if (sp >= 2) {
+            // O rows (lanes 64..127), this warp's column half
+            const int l = row - 64;
             const bool valid = l < n;  // tcgen05.ld is warp-collective: every lane loads, valid rows store
-            {
-                const size_t row = ((size_t)bh * T + t0 + (valid ? l : 0)) * dv + v0;
-                for (int j0 = 0; j0 < DVS; j0 += 16) {
-                    float ov[16];
-                    __syncwarp();
-                    tmem_ld16(t_lane + TM_ZO + j0, ov);
-                    tmem_wait_ld();
-                    if (!valid) continue;  // reconverged by the __syncwarp above
+            const size_t orow = ((size_t)bh * T + t0 + (valid ? l : 0)) * dv + v0 + ch * HV;
+#pragma unroll
+            for (int j0 = 0; j0 < HV; j0 += 32) {
+                float ov[32];
+                __syncwarp();
+                tmem_ld32(t_lane + TM_ZO + ch * HV + j0, ov);
+                tmem_wait_ld();
+                if (valid) {
                     if (OUT_BF16) {
-                        uint32_t w[8];
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow + j0);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            __nv_bfloat162 b2 = __floats2bfloat162_rn(ov[2 * e], ov[2 * e + 1]);
-                            w[e] = *reinterpret_cast<uint32_t *>(&b2);
+                        for (int e = 0; e < 4; ++e) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(ov[8 * e + 2 * u], ov[8 * e + 2 * u + 1]);
+                                w[u] = *reinterpret_cast<uint32_t *>(&b2);
+                            }
+                            dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
                         }
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + row + j0);
-                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                     } else {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + row + j0);
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow + j0);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) dst[e] = make_float4(ov[4 * e], ov[4 * e + 1], ov[4 * e + 2], ov[4 * e + 3]);
+                        for (int e = 0; e < 8; ++e) dst[e] = make_float4(ov[4 * e], ov[4 * e + 1], ov[4 * e + 2], ov[4 * e + 3]);
                     }
                 }
             }
         }
-        // new state -> fp16 S^T operand for the next chunk
-        for (int j0 = 0; j0 < DVS; j0 += 16) {
-            float sv[16];
+        TC_MARK(12);
+        // new state -> fp16 S^T operand for the next chunk (lane = channel, this warp's half)
+#pragma unroll
+        for (int j0 = 0; j0 < HV; j0 += 32) {
+            float sv[32];
             __syncwarp();
-            tmem_ld16(t_lane + TM_S + j0, sv);
+            tmem_ld32(t_lane + TM_S + ch * HV + j0, sv);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) range_bad |= out_of_fp16(sv[e]);
-            unsigned char *sb = sm + L::ST16 + (j0 >> 6) * 16384;
-            *reinterpret_cast<uint4 *>(sb + sw128_off(t, j0 & 63)) = pack_h8(sv);
-            *reinterpret_cast<uint4 *>(sb + sw128_off(t, (j0 & 63) + 8)) = pack_h8(sv + 8);
+            for (int e = 0; e < 32; ++e) rmax = fmaxf(rmax, fabsf(sv[e]));
+            const int j = ch * HV + j0;
+            unsigned char *sb = sm + L::ST16 + (j >> 6) * 16384;
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+                *reinterpret_cast<uint4 *>(sb + sw128_off(row, (j & 63) + e)) = pack_h8(sv + e);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         ok = !ms.abort_flag;
+        TC_MARK(13);
     }
 
     // ------------------------------------------------------------ final state
     if (ok && p.ST) {
-        for (int j0 = 0; j0 < DVS; j0 += 16) {
+#pragma unroll
+        for (int j0 = 0; j0 < HV; j0 += 16) {
             float sv[16];
             __syncwarp();
-            tmem_ld16(t_lane + TM_S + j0, sv);
+            tmem_ld16(t_lane + TM_S + ch * HV + j0, sv);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) p.ST[((size_t)bh * dv + v0 + j0 + i) * DK + t] = sv[i];
+            for (int i = 0; i < 16; ++i) p.ST[((size_t)bh * dv + v0 + ch * HV + j0 + i) * DK + row] = sv[i];
         }
     }
-    if (range_bad) ms.range_flag = 1;
+    if (!(rmax <= 65504.f)) ms.range_flag = 1;
     __syncthreads();
     if (t == 0) {
         if (ms.abort_flag) {
@@ -647,6 +791,18 @@ int launch_modes(const TcParams &prm, int grid, int update, int gate, bool ob, c
 
 }  // namespace
 }  // namespace gdn
+
+#ifdef GDN_TC_PHASE_TIMING
+extern "C" int gdn_tc_phase_times(unsigned long long *out, int clear) {
+    cudaDeviceSynchronize();
+    if (cudaMemcpyFromSymbol(out, g_tc_phase, sizeof(unsigned long long) * 16) != cudaSuccess) return -1;
+    if (clear) {
+        unsigned long long z[16] = {0};
+        cudaMemcpyToSymbol(g_tc_phase, z, sizeof(z));
+    }
+    return 0;
+}
+#endif
 
 int gdn_tc_supported(const gdn_desc_t *d) {
     return d->dtype == GDN_BF16 && d->dk == 128 && (d->dv == 64 || d->dv == 128);
