@@ -23,7 +23,7 @@ _LIB_PATH = os.path.join(_HERE, "libgdn.so")
 
 UPDATES = {"additive": 0, "decay": 1, "delta": 2}
 GATES = {"none": 0, "scalar": 1, "channel": 2}
-ALGOS = {"auto": 0, "simt": 1, "tc": 2}
+ALGOS = {"auto": 0, "simt": 1, "tc": 2, "tc_seq": 3}
 F32, BF16 = 0, 1
 
 GDN_OK = 0

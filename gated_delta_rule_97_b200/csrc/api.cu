@@ -90,13 +90,14 @@ extern "C" int gdn_device_diag(void) {
 
 int gdn_tc_supported(const gdn_desc_t *d);
 int gdn_launch_chunk_tc(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
+int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
 
 extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const float *S0, void *o, float *S_T, void *stream) {
     int rc = validate_common(d);
     if (rc != GDN_OK) return rc;
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
-    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC) return GDN_ERR_ARG;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC_SEQ) return GDN_ERR_ARG;
     const long BH = (long)d->B * d->H;
     const size_t n_qk = (size_t)BH * d->T * d->dk, n_v = (size_t)BH * d->T * d->dv;
     const size_t n_S = (size_t)BH * d->dv * d->dk;
@@ -130,9 +131,9 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
 
     const bool tc_ok = gdn_tc_supported(d) != 0;
-    if (d->algo == GDN_ALGO_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
-    if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok))
-        return from_cuda(gdn_launch_chunk_tc(a, d, st));
+    if ((d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) && !tc_ok) return GDN_ERR_UNSUPPORTED;
+    if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
+    if (d->algo == GDN_ALGO_TC_SEQ) return from_cuda(gdn_launch_chunk_tc(a, d, st));
     return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
 }
 

@@ -155,7 +155,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_tc_kernel(const __grid_co
     constexpr int NB = DVS / 64;  // 64-wide value blocks
     constexpr int HV = DVS / 2;   // value columns per column half
     extern __shared__ unsigned char smraw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    // Align by an integer offset from the shared array itself, so that every access
+    // through `sm` stays in the shared address space (LDS/STS, not generic).
+    unsigned char *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
     Misc &ms = *reinterpret_cast<Misc *>(sm + L::MISC);
 
     const int t = threadIdx.x;

@@ -1,0 +1,875 @@
+// Warp-specialised tensor-core chunkwise prefill (bf16 inputs, dk = 128).
+//
+// One CTA owns one (b,h) head and a slice of DVS value rows (64 or 128) and
+// walks its chunks (C = 64) with two warp groups that overlap:
+//
+//   prep group  (warps 0-7) for chunk r+1: TMA of q, k, v (and the channel
+//       gate), P = [Q;K] K^T, the gate prefix, fp16 operands Q<, K<, K>, V,
+//       A' = P_top masked with decay, L = beta P_bottom, the UT transform
+//       T = (I + L)^{-1} (fp32 blocked forward substitution), W = T2 K<.
+//   state group (warps 8-11) for chunk r, every MMA with M = DVS value rows
+//       (the transposed form), so that the state and the correction rows are
+//       A operands held in TMEM:
+//         Z^T  = V^T T2^T - S W^T          (U^T, then the history correction)
+//         O^T  = S Q<^T + Z^T A'^T
+//         S    = S Diag(e^{G_C}) + Z^T K>
+//
+// Same algebra as "Linear Attention, Visualized": "Chunkwise algorithm",
+// "Mamba-2 ... Chunkwise form", "Gated Linear Attention (GLA)", "The triangular
+// correction system", "Optional: Use UT to share the triangular transform",
+// "Correct the incoming state" and the GDN / KDA tables; only the storage is
+// transposed (S is kept [dv x dk] with lane = value row).
+//
+// TMEM (512 columns): prep P/W products [0,128); state: Z^T|O^T [128,256),
+// S fp32 [256,384), S fp16 (A operand) [384,448), Z^T fp16 (A operand) [448,480).
+// Hand-offs: bar_rdy (prep -> state, one phase per chunk), bar_fA (state MMAs
+// that read T2, W, Q<, V completed), bar_fB0/1 (state MMAs that read A', K>
+// of an even / odd chunk completed; A' and K> are double-buffered).  All waits
+// are bounded; intermediates are fp16 with a range flag (see chunk_tc.cu).
+#include <string.h>
+
+#include "../../include/gdn.h"
+#include "common.cuh"
+#include "sm100.cuh"
+#include "tc_util.cuh"
+#include "tma_host.cuh"
+
+#ifdef GDN_TC_PHASE_TIMING
+// Per-phase cycle totals of CTA 0: slots 0..15 prep group, 16..31 state group.
+__device__ unsigned long long g_tc2_phase[32];
+#define TC2_MARK(who, i)                                                           \
+    do {                                                                          \
+        if (blockIdx.x == 0 && t == (who)) {                                      \
+            const long long now_ = clock64();                                     \
+            atomicAdd(&g_tc2_phase[i], (unsigned long long)(now_ - mark_prev));   \
+            mark_prev = now_;                                                     \
+        }                                                                         \
+    } while (0)
+#else
+#define TC2_MARK(who, i) \
+    do {                 \
+    } while (0)
+#endif
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+using namespace tcu;
+
+constexpr int kThreads = 384;  // warps 0-7 prep, 8-11 state
+constexpr int C = kChunk;
+constexpr int DK = 128;
+constexpr float kFactorMaxDecay = 10.0f;
+constexpr int kPrepBar = 1, kStateBar = 2;
+
+struct Params {
+    CUtensorMap q_map, k_map, v_map, g_map, o_map;
+    const float *g;
+    const float *beta;
+    const float *S0;
+    void *o;
+    float *ST;
+    int *status;
+    int *diag;
+    int BH, T, dv, nslices;
+};
+
+template <int DVS, int GATE>
+struct Smem {
+    static constexpr int RAW_QK = 0;                                     // [Q0 K0 | Q1 K1] bf16
+    static constexpr int RAW_V = RAW_QK + 32768;                         // V slice bf16
+    static constexpr int GCH = RAW_V + DVS * 128;                        // channel gate fp32 [64][128]
+    static constexpr int AT = GCH + (GATE == kGateChannel ? 32768 : 0);  // [-W | Q< | K<] x 2 halves
+    static constexpr int KT = AT + 49152;                                // k e^{-G} fp16 / L^T fp32 scratch
+    static constexpr int KR = KT + 16384;                                // K> fp16, 2 buffers
+    static constexpr int V16 = KR + 32768;                               // V fp16
+    static constexpr int TZA = V16 + DVS * 128;                          // [T2 | A'0 | A'1] fp16
+    static constexpr int OST = TZA + 24576;                              // O staging [64 tok][DVS] (TMA store)
+    static constexpr int DEC = OST + DVS * 256;                          // float dec[2][128]
+    static constexpr int MISC = DEC + 1024;
+    static constexpr int TOTAL = MISC + 3072;
+    static constexpr int DYN = TOTAL + 1024;
+};
+
+struct Misc {
+    float G[64];
+    float b[64];
+    float gam[64];
+    float ib[64];
+    float beta[64];
+    float GC[128];
+    int abort_flag, range_flag, slow_chunk, abort_site;
+    int p_abort, s_abort, pad0, pad1;
+    uint32_t tmem_base, pad2[3];
+    uint64_t bar_tma, bar_p1, bar_w, bar_rdy, bar_fA, bar_fB0, bar_fB1, pad3;
+};
+
+template <typename M>
+__device__ __forceinline__ void note_timeout(M &ms, int site, int r) {
+    if (atomicCAS(&ms.abort_flag, 0, 1) == 0) ms.abort_site = site * 1000000 + r;
+}
+
+constexpr uint32_t TP = 0, TZO = 128, TSM = 256, TS16 = 384, TZ16 = 448;
+
+template <int DVS, int UPD, int GATE, bool OUT_BF16>
+__global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_constant__ Params p) {
+    using L = Smem<DVS, GATE>;
+    constexpr bool DELTA = (UPD == kDelta);
+    constexpr int NB = DVS / 64;
+    extern __shared__ unsigned char smraw[];
+    // Align by an integer offset from the shared array itself, so that every access
+    // through `sm` stays in the shared address space (LDS/STS, not generic).
+    unsigned char *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
+    Misc &ms = *reinterpret_cast<Misc *>(sm + L::MISC);
+    float *dec = reinterpret_cast<float *>(sm + L::DEC);
+
+    const int t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int sp = warp & 3;
+    const int bh = blockIdx.x / p.nslices;
+    const int v0 = (blockIdx.x % p.nslices) * DVS;
+    const int T = p.T, dv = p.dv;
+    const int nchunks = (T + C - 1) / C;
+
+    if (t == 0) {
+        mbar_init(&ms.bar_tma, 1);
+        mbar_init(&ms.bar_p1, 1);
+        mbar_init(&ms.bar_w, 1);
+        mbar_init(&ms.bar_rdy, 1);
+        mbar_init(&ms.bar_fA, 1);
+        mbar_init(&ms.bar_fB0, 1);
+        mbar_init(&ms.bar_fB1, 1);
+        fence_mbar_init();
+        ms.abort_flag = 0;
+        ms.range_flag = 0;
+        ms.p_abort = 0;
+        ms.s_abort = 0;
+        tma_prefetch_desc(&p.q_map);
+        tma_prefetch_desc(&p.k_map);
+        tma_prefetch_desc(&p.v_map);
+        if (GATE == kGateChannel) tma_prefetch_desc(&p.g_map);
+        tma_prefetch_desc(&p.o_map);
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tmem_alloc(&ms.tmem_base, 512);
+        tmem_relinquish();
+    }
+    // T2 tile: its upper-right 32x32 block is never written and stays zero
+    for (int i = t; i < 8192 / 16; i += kThreads) reinterpret_cast<uint4 *>(sm + L::TZA)[i] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms.tmem_base;
+    const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
+    float rmax = 0.f;  // largest |value| this thread handed to an fp16 operand
+#ifdef GDN_TC_PHASE_TIMING
+    long long mark_prev = clock64();
+#endif
+
+    if (warp < 8) {
+        // =================================================================== prep group (8 warps)
+        const int ch = warp >> 2;          // column half of a TMEM tile handled by this warp
+        const int row = sp * 32 + lane;    // TMEM lane (product row) read by this thread
+        float gpre0 = 0.f, gpre1 = 0.f, bpre = 0.f;
+        auto load_gate_beta = [&](int r) {
+            const int t0 = r * C;
+            if (GATE == kGateScalar && warp == 0) {
+                const int l0 = 2 * lane;
+                gpre0 = (t0 + l0 < T) ? p.g[(size_t)bh * T + t0 + l0] : 0.f;
+                gpre1 = (t0 + l0 + 1 < T) ? p.g[(size_t)bh * T + t0 + l0 + 1] : 0.f;
+            }
+            if (DELTA && t < C) bpre = (t0 + t < T) ? p.beta[(size_t)bh * T + t0 + t] : 0.f;
+        };
+        auto issue_tma = [&](int r) {
+            const int t0 = r * C;
+            const uint32_t bytes = 32768 + DVS * 128 + (GATE == kGateChannel ? 32768 : 0);
+            mbar_arrive_expect_tx(&ms.bar_tma, bytes);
+            for (int h = 0; h < 2; ++h) {
+                tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, t0, bh, &ms.bar_tma);
+                tma_load_3d(sm + L::RAW_QK + h * 16384 + 8192, &p.k_map, h * 64, t0, bh, &ms.bar_tma);
+            }
+            for (int j = 0; j < NB; ++j)
+                tma_load_3d(sm + L::RAW_V + j * 8192, &p.v_map, v0 + j * 64, t0, bh, &ms.bar_tma);
+            if (GATE == kGateChannel)
+                for (int j = 0; j < 4; ++j) tma_load_3d(sm + L::GCH + j * 8192, &p.g_map, j * 32, t0, bh, &ms.bar_tma);
+        };
+        if (t == 0 && nchunks > 0) issue_tma(0);
+        if (nchunks > 0) load_gate_beta(0);
+
+        for (int r = 0; r < nchunks; ++r) {
+            if (ms.p_abort) break;
+            const uint32_t ph = r & 1;
+            const int buf = r & 1;
+            TC2_MARK(0, 0);
+            if (!mbar_wait(&ms.bar_tma, ph)) note_timeout(ms, 1, r);
+            TC2_MARK(0, 1);
+            if (GATE != kGateChannel && t == 0 && !ms.abort_flag) {
+                tc_fence_after();
+                const uint32_t qk = smem_u32(sm + L::RAW_QK);
+                constexpr uint32_t id = idesc_f16(128, 64, 1, 0, 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_f16(tmem + TP, smem_desc_sw128(qk + ko, 16, 1024), smem_desc_sw128(qk + 8192 + ko, 16, 1024),
+                            id, k > 0);
+                }
+                mma_commit(&ms.bar_p1);
+            }
+            // ---------------------------------------------------- a1: gate prefix
+            if (GATE == kGateScalar) {
+                if (warp == 0) {
+                    // two tokens per lane; the warp also derives b = e^G, gamma = e^{G_C-G}, 1/b
+                    const int l0 = 2 * lane;
+                    const float x0 = gpre0, x1 = gpre1;
+                    float s = x0 + x1;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, s, off);
+                        if (lane >= off) s += y;
+                    }
+                    const float G0 = s - x1, G1 = s;
+                    const float gc = __shfl_sync(0xffffffffu, G1, 31);
+                    ms.G[l0] = G0;
+                    ms.G[l0 + 1] = G1;
+                    ms.b[l0] = __expf(G0);
+                    ms.b[l0 + 1] = __expf(G1);
+                    ms.gam[l0] = __expf(gc - G0);
+                    ms.gam[l0 + 1] = __expf(gc - G1);
+                    ms.ib[l0] = __expf(-G0);
+                    ms.ib[l0 + 1] = __expf(-G1);
+                    if (lane == 0) dec[buf * 128] = __expf(gc);
+                }
+            } else if (GATE == kGateChannel) {
+                // channel c, token half hf: prefix over 32 tokens, then join the halves
+                const int c = t & 127, hf = t >> 7;
+                float *gcol = reinterpret_cast<float *>(sm + L::GCH + (c >> 5) * 8192) + (c & 31);
+                float gv[32];
+#pragma unroll
+                for (int l = 0; l < 32; ++l) gv[l] = gcol[(32 * hf + l) * 32];
+#pragma unroll
+                for (int l = 1; l < 32; ++l) gv[l] += gv[l - 1];
+                if (hf == 0) {
+#pragma unroll
+                    for (int l = 0; l < 32; ++l) gcol[l * 32] = gv[l];
+                }
+                named_bar(kPrepBar, 256);
+                if (hf == 1) {
+                    const float base = gcol[31 * 32];
+#pragma unroll
+                    for (int l = 0; l < 32; ++l) gcol[(32 + l) * 32] = gv[l] + base;
+                    ms.GC[c] = gv[31] + base;
+                    dec[buf * 128 + c] = __expf(gv[31] + base);
+                }
+                named_bar(kPrepBar, 256);
+                if (warp == 0) {
+                    float mx = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) mx = fmaxf(mx, -ms.GC[lane + 32 * i]);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                    if (lane == 0) ms.slow_chunk = !(mx <= kFactorMaxDecay);
+                }
+            }
+            if (DELTA && t < C) ms.beta[t] = bpre;
+            if (r + 1 < nchunks) load_gate_beta(r + 1);
+            named_bar(kPrepBar, 256);
+            const bool fastg = (GATE != kGateScalar) || (-ms.G[C - 1] <= 80.f);
+            TC2_MARK(0, 2);
+            // the state group must be done with the buffers this chunk overwrites
+            if (r >= 1) {
+                if (DELTA) {
+                    if (!mbar_wait(&ms.bar_fA, (r - 1) & 1)) note_timeout(ms, 9, r);
+                } else {
+                    uint64_t *fb = ((r - 1) & 1) ? &ms.bar_fB1 : &ms.bar_fB0;
+                    if (!mbar_wait(fb, ((r - 1) >> 1) & 1)) note_timeout(ms, 10, r);
+                }
+            }
+            if (r >= 2) {
+                uint64_t *fb = buf ? &ms.bar_fB1 : &ms.bar_fB0;
+                if (!mbar_wait(fb, ((r - 2) >> 1) & 1)) note_timeout(ms, 10, r);
+            }
+            TC2_MARK(0, 3);
+            // ---------------------------------------------------- operand conversions
+            const bool slow = (GATE == kGateChannel) && ms.slow_chunk;
+            for (int i = t; i < 2 * 512; i += 256) {
+                const int h = i >> 9, off = (i & 511) * 16;
+                const int l = off >> 7;
+                const int c0 = h * 64 + ((((off >> 4) & 7) ^ (l & 7)) << 3);
+                float qf[8], kf[8], ql[8], kl[8], kr[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + off), qf);
+                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + 8192 + off), kf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fmaxf(fabsf(qf[e]), fabsf(kf[e])));
+                if (GATE == kGateChannel) {
+                    const float *gg = reinterpret_cast<const float *>(sm + L::GCH + (c0 >> 5) * 8192) + l * 32 + (c0 & 31);
+                    float kt[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float G = gg[e];
+                        const float eg = __expf(G), emg = __expf(-G);
+                        ql[e] = qf[e] * eg;
+                        kl[e] = kf[e] * eg;
+                        kt[e] = slow ? 0.f : kf[e] * emg;
+                        kr[e] = kf[e] * __expf(ms.GC[c0 + e] - G);
+                        rmax = fmaxf(rmax, fabsf(kt[e]));
+                    }
+                    *reinterpret_cast<uint4 *>(sm + L::KT + h * 8192 + off) = pack_h8(kt);
+                } else {
+                    const float bl = (GATE == kGateScalar) ? ms.b[l] : 1.f;
+                    const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        ql[e] = qf[e] * bl;
+                        kl[e] = kf[e] * bl;
+                        kr[e] = kf[e] * gl;
+                    }
+                }
+                *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(ql);
+                if (DELTA || GATE == kGateChannel)
+                    *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
+                *reinterpret_cast<uint4 *>(sm + L::KR + buf * 16384 + h * 8192 + off) = pack_h8(kr);
+            }
+            for (int i = t; i < NB * 512; i += 256) {
+                float vf[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_V + i * 16), vf);
+                *reinterpret_cast<uint4 *>(sm + L::V16 + i * 16) = pack_h8(vf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(vf[e]));
+            }
+            fence_proxy_async_smem();
+            named_bar(kPrepBar, 256);
+            if (GATE == kGateChannel && t == 0) {
+                tc_fence_after();
+                const uint32_t at = smem_u32(sm + L::AT), kt = smem_u32(sm + L::KT);
+                constexpr uint32_t id = idesc_f16(128, 64, 0, 0, 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t ka = (k >> 2) * 24576 + 8192 + (k & 3) * 32;
+                    const uint32_t kb = (k >> 2) * 8192 + (k & 3) * 32;
+                    mma_f16(tmem + TP, smem_desc_sw128(at + ka, 16, 1024), smem_desc_sw128(kt + kb, 16, 1024), id,
+                            k > 0);
+                }
+                mma_commit(&ms.bar_p1);
+            }
+            TC2_MARK(0, 4);
+            if (!mbar_wait(&ms.bar_p1, ph)) note_timeout(ms, 2, r);
+            TC2_MARK(0, 5);
+            tc_fence_after();
+
+            // ---------------------------------------------------- a2: A' and L^T (32 columns per thread)
+            {
+                const int l = row & 63;
+                const bool top = row < 64;
+                const int m0 = ch * 32;
+                float pr[32];
+                __syncwarp();
+                tmem_ld32(lane_addr + TP + m0, pr);
+                tmem_wait_ld();
+                if (GATE == kGateChannel && slow) {
+                    const unsigned char *xrow = sm + L::RAW_QK + (top ? 0 : 8192);
+                    for (int e = 0; e < 32; ++e) {
+                        const int m = m0 + e;
+                        float acc = 0.f;
+                        if (m <= l) {
+                            for (int c = 0; c < DK; ++c) {
+                                const int h = c >> 6;
+                                const uint32_t ox = sw128_off(l, c & 63), om = sw128_off(m, c & 63);
+                                const float xv =
+                                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xrow + h * 16384 + ox));
+                                const float kv = __bfloat162float(
+                                    *reinterpret_cast<const __nv_bfloat16 *>(sm + L::RAW_QK + h * 16384 + 8192 + om));
+                                const float *gc = reinterpret_cast<const float *>(sm + L::GCH + (c >> 5) * 8192);
+                                acc = fmaf(xv * kv, __expf(gc[l * 32 + (c & 31)] - gc[m * 32 + (c & 31)]), acc);
+                            }
+                        }
+                        pr[e] = acc;
+                    }
+                }
+                // decay factors e^{G_l - G_m}: all shared loads first, then the stores
+                float dm[32];
+                if (GATE == kGateScalar) {
+                    if (fastg) {
+                        const float bl = ms.b[l];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 x = *reinterpret_cast<const float4 *>(&ms.ib[m0 + e]);
+                            dm[e] = bl * x.x; dm[e + 1] = bl * x.y; dm[e + 2] = bl * x.z; dm[e + 3] = bl * x.w;
+                        }
+                    } else {
+                        const float Gl = ms.G[l];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 x = *reinterpret_cast<const float4 *>(&ms.G[m0 + e]);
+                            dm[e] = __expf(Gl - fmaxf(x.x, Gl)); dm[e + 1] = __expf(Gl - fmaxf(x.y, Gl));
+                            dm[e + 2] = __expf(Gl - fmaxf(x.z, Gl)); dm[e + 3] = __expf(Gl - fmaxf(x.w, Gl));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) dm[e] = 1.f;
+                }
+                if (top) {
+                    unsigned char *ap = sm + L::TZA + 8192 * (1 + buf);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        pr[e] = (m0 + e <= l) ? pr[e] * dm[e] : 0.f;
+                        rmax = fmaxf(rmax, fabsf(pr[e]));
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) *reinterpret_cast<uint4 *>(ap + sw128_off(l, m0 + e)) = pack_h8(pr + e);
+                } else if (DELTA) {
+                    const float bl = ms.beta[l];
+                    float *Lt = reinterpret_cast<float *>(sm + L::KT);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) pr[e] = (m0 + e < l) ? bl * pr[e] * dm[e] : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) Lt[f32_swz(m0 + e, l, 64)] = pr[e];
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(kPrepBar, 256);
+            TC2_MARK(0, 6);
+            if (t == 0 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
+
+            if (DELTA) {
+                // ------------------------------------------------ a3: T = (I + L)^{-1}
+                // L^T is held in the KT scratch ([64][64] fp32, row m = column m of
+                // L).  Stage 1: the two 32x32 diagonal blocks, one column of T per
+                // thread, right-looking (once x_m is final it updates every later
+                // row, so the dependent chain is one FMA per row).  Stage 2:
+                // T_BA = -T_BB (L_BA T_AA).  T_AA goes to the zero block
+                // [32:64, 0:32] of L^T, T_BB over L_AA^T, X = L_BA T_AA over L_BB^T.
+                float *Lt = reinterpret_cast<float *>(sm + L::KT);
+                if (t < 64) {
+                    const int b = t >> 5, c = t & 31, o = 32 * b;
+                    float x[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = (i == c) ? 1.f : 0.f;
+#pragma unroll
+                    for (int m = 0; m < 31; ++m) {
+                        const float xm = x[m];
+#pragma unroll
+                        for (int i0 = (m + 1) & ~3; i0 < 32; i0 += 4) {
+                            const float4 lv = *reinterpret_cast<const float4 *>(Lt + f32_swz(o + m, o + i0, 64));
+                            if (i0 + 0 > m) x[i0 + 0] = fmaf(-lv.x, xm, x[i0 + 0]);
+                            if (i0 + 1 > m) x[i0 + 1] = fmaf(-lv.y, xm, x[i0 + 1]);
+                            if (i0 + 2 > m) x[i0 + 2] = fmaf(-lv.z, xm, x[i0 + 2]);
+                            if (i0 + 3 > m) x[i0 + 3] = fmaf(-lv.w, xm, x[i0 + 3]);
+                        }
+                    }
+                    const float bt = ms.beta[o + c];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float tv = x[i] * bt;
+                        rmax = fmaxf(rmax, fabsf(tv));
+                        *reinterpret_cast<__half *>(sm + L::TZA + sw128_off(o + i, o + c)) = __float2half_rn(tv);
+                        if (b == 0) Lt[f32_swz(32 + i, c, 64)] = x[i];
+                    }
+                    named_bar(kPrepBar, 256);
+                    if (b == 1) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) Lt[f32_swz(i, c, 64)] = x[i];
+                    }
+                } else {
+                    named_bar(kPrepBar, 256);
+                }
+                named_bar(kPrepBar, 256);
+                TC2_MARK(0, 7);
+                {
+                    const int rr = t >> 3, c0 = (t & 7) * 4;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int m = 0; m < 32; ++m) {
+                        const float lm = Lt[f32_swz(m, 32 + rr, 64)];  // L_BA[rr][m]
+                        const float4 a0 = *reinterpret_cast<const float4 *>(Lt + f32_swz(32 + m, c0, 64));
+                        acc[0] = fmaf(lm, a0.x, acc[0]);
+                        acc[1] = fmaf(lm, a0.y, acc[1]);
+                        acc[2] = fmaf(lm, a0.z, acc[2]);
+                        acc[3] = fmaf(lm, a0.w, acc[3]);
+                    }
+                    *reinterpret_cast<float4 *>(Lt + f32_swz(32 + rr, 32 + c0, 64)) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                    named_bar(kPrepBar, 256);
+                    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+                    for (int m0 = 0; m0 < 32; m0 += 4) {
+                        const float4 tv = *reinterpret_cast<const float4 *>(Lt + f32_swz(rr, m0, 64));  // T_BB[rr][m0..]
+                        const float tm[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float4 a0 = *reinterpret_cast<const float4 *>(Lt + f32_swz(32 + m0 + e, 32 + c0, 64));
+                            acc[0] = fmaf(tm[e], a0.x, acc[0]);
+                            acc[1] = fmaf(tm[e], a0.y, acc[1]);
+                            acc[2] = fmaf(tm[e], a0.z, acc[2]);
+                            acc[3] = fmaf(tm[e], a0.w, acc[3]);
+                        }
+                    }
+                    float tb[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        tb[e] = -acc[e] * ms.beta[c0 + e];
+                        rmax = fmaxf(rmax, fabsf(tb[e]));
+                    }
+                    *reinterpret_cast<uint2 *>(sm + L::TZA + sw128_off(32 + rr, c0)) =
+                        make_uint2(pack_h2(tb[0], tb[1]), pack_h2(tb[2], tb[3]));
+                }
+                fence_proxy_async_smem();
+                named_bar(kPrepBar, 256);
+                TC2_MARK(0, 8);
+                // ------------------------------------------------ a4: W = T2 K<
+                if (t == 0 && !ms.abort_flag) {
+                    tc_fence_after();
+                    const uint32_t tza = smem_u32(sm + L::TZA), at = smem_u32(sm + L::AT);
+                    constexpr uint32_t idw = idesc_f16(128, 128, 0, 0, 1);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_f16(tmem + TP, smem_desc_sw128(tza + k * 32, 16, 1024),
+                                smem_desc_sw128(at + 16384 + k * 2048, 24576, 1024), idw, k > 0);
+                    mma_commit(&ms.bar_w);
+                }
+                if (!mbar_wait(&ms.bar_w, ph)) note_timeout(ms, 3, r);
+                TC2_MARK(0, 9);
+                tc_fence_after();
+                if (sp < 2) {
+                    // W rows (lanes 0..63), this warp's 64-column half -> -W slot of that half
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        float w[32];
+                        __syncwarp();
+                        tmem_ld32(lane_addr + TP + ch * 64 + c0, w);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            w[e] = -w[e];
+                            rmax = fmaxf(rmax, fabsf(w[e]));
+                        }
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8)
+                            *reinterpret_cast<uint4 *>(sm + L::AT + ch * 24576 + sw128_off(row, c0 + e)) = pack_h8(w + e);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (t == 0) ms.p_abort = ms.abort_flag;
+            named_bar(kPrepBar, 256);
+            if (t == 0) mbar_arrive(&ms.bar_rdy);
+            TC2_MARK(0, 10);
+        }
+    } else {
+        // =================================================================== state group
+        const int ts = t - 256;
+        const bool has_row = (DVS == 128) || (lane < 16);
+        const int vrow = (DVS == 128) ? ts : (sp * 16 + lane);
+        const size_t srow = ((size_t)bh * dv + v0 + (has_row ? vrow : 0)) * DK;
+        // initial state: fp32 master and fp16 operand copy (lane = value row)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float sv[64];
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) {
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (p.S0 && has_row) x = *reinterpret_cast<const float4 *>(p.S0 + srow + h * 64 + j);
+                sv[j] = x.x; sv[j + 1] = x.y; sv[j + 2] = x.z; sv[j + 3] = x.w;
+            }
+            __syncwarp();
+            tmem_st32f(lane_addr + TSM + h * 64, sv);
+            tmem_st32f(lane_addr + TSM + h * 64 + 32, sv + 32);
+            uint32_t w[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) w[c] = pack_h2(sv[2 * c], sv[2 * c + 1]);
+            tmem_st32(lane_addr + TS16 + h * 32, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        named_bar(kStateBar, 128);
+
+        // the first chunk's decay is applied here; later ones ride on the fp16
+        // write-back at the end of the previous chunk
+        if (nchunks > 0) {
+            if (!mbar_wait(&ms.bar_rdy, 0)) note_timeout(ms, 6, 0);
+            tc_fence_after();
+            if (GATE != kGateNone) {
+#pragma unroll
+                for (int j0 = 0; j0 < 128; j0 += 32) {
+                    float sv[32];
+                    __syncwarp();
+                    tmem_ld32(lane_addr + TSM + j0, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) sv[i] *= (GATE == kGateScalar) ? dec[0] : dec[j0 + i];
+                    tmem_st32f(lane_addr + TSM + j0, sv);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            named_bar(kStateBar, 128);
+        }
+        float *ost = reinterpret_cast<float *>(sm + L::OST);
+        for (int r = 0; r < nchunks; ++r) {
+            if (ms.s_abort) break;
+            const uint32_t ph = r & 1;
+            const int t0 = r * C;
+            const int buf = r & 1;
+            TC2_MARK(256, 17);
+            if (ts == 0 && !ms.abort_flag) {
+                tc_fence_after();
+                const uint32_t at = smem_u32(sm + L::AT);
+                constexpr uint32_t id1 = idesc_f16(DVS, 64, 0, 0, 0);
+                if (DELTA) {
+                    const uint32_t v16 = smem_u32(sm + L::V16), tza = smem_u32(sm + L::TZA);
+                    constexpr uint32_t idu = idesc_f16(DVS, 64, 0, 1, 0);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)  // U^T = V^T T2^T
+                        mma_f16(tmem + TZO, smem_desc_sw128(v16 + k * 2048, 8192, 1024),
+                                smem_desc_sw128(tza + k * 32, 16, 1024), idu, k > 0);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)  // -= S W^T  (the tile holds -W)
+                        mma_f16_ts(tmem + TZO, tmem + TS16 + k * 8,
+                                   smem_desc_sw128(at + (k >> 2) * 24576 + (k & 3) * 32, 16, 1024), id1, 1);
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k)  // O^T = S Q<^T
+                    mma_f16_ts(tmem + TZO + 64, tmem + TS16 + k * 8,
+                               smem_desc_sw128(at + (k >> 2) * 24576 + 8192 + (k & 3) * 32, 16, 1024), id1, k > 0);
+                mma_commit(&ms.bar_fA);
+            }
+            TC2_MARK(256, 18);
+            if (!mbar_wait(&ms.bar_fA, ph)) note_timeout(ms, 7, r);
+            TC2_MARK(256, 19);
+            tc_fence_after();
+            if (DELTA) {
+                // Z^T -> fp16 A operand (tokens 2c, 2c+1 in column c)
+                float z[64];
+                __syncwarp();
+                tmem_ld32(lane_addr + TZO, z);
+                tmem_ld32(lane_addr + TZO + 32, z + 32);
+                tmem_wait_ld();
+                uint32_t w[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    rmax = fmaxf(rmax, fmaxf(fabsf(z[2 * c]), fabsf(z[2 * c + 1])));
+                    w[c] = pack_h2(z[2 * c], z[2 * c + 1]);
+                }
+                tmem_st32(lane_addr + TZ16, w);
+                tmem_wait_st();
+                tc_fence_before();
+                named_bar(kStateBar, 128);
+            }
+            TC2_MARK(256, 20);
+            uint64_t *fb = buf ? &ms.bar_fB1 : &ms.bar_fB0;
+            if (ts == 0 && !ms.abort_flag) {
+                tc_fence_after();
+                const uint32_t tza = smem_u32(sm + L::TZA), kr = smem_u32(sm + L::KR) + buf * 16384;
+                const uint32_t ap = tza + 8192 * (1 + buf);
+                constexpr uint32_t id2 = idesc_f16(DVS, 64, 0, 0, 0);
+                constexpr uint32_t id3 = idesc_f16(DVS, 128, 0, 0, 1);
+                if (DELTA) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t za = tmem + TZ16 + k * 8;
+                        mma_f16_ts(tmem + TZO + 64, za, smem_desc_sw128(ap + k * 32, 16, 1024), id2, 1);
+                        mma_f16_ts(tmem + TSM, za, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3, 1);
+                    }
+                } else {
+                    const uint32_t v16 = smem_u32(sm + L::V16);
+                    constexpr uint32_t id2s = idesc_f16(DVS, 64, 0, 1, 0);
+                    constexpr uint32_t id3s = idesc_f16(DVS, 128, 0, 1, 1);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t va = smem_desc_sw128(v16 + k * 2048, 8192, 1024);
+                        mma_f16(tmem + TZO + 64, va, smem_desc_sw128(ap + k * 32, 16, 1024), id2s, 1);
+                        mma_f16(tmem + TSM, va, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3s, 1);
+                    }
+                }
+                mma_commit(fb);
+            }
+            TC2_MARK(256, 21);
+            if (!mbar_wait(fb, (r >> 1) & 1)) note_timeout(ms, 8, r);
+            TC2_MARK(256, 22);
+            tc_fence_after();
+            {
+                // O^T -> row-major staging [64 tok][DVS] -> one TMA store (rows past T clipped)
+                float ov[64];
+                __syncwarp();
+                tmem_ld32(lane_addr + TZO + 64, ov);
+                tmem_ld32(lane_addr + TZO + 96, ov + 32);
+                tmem_wait_ld();
+                if (ts == 0) bulk_wait_read0();  // the previous chunk's store has read the staging tile
+                named_bar(kStateBar, 128);
+                if (has_row) {
+                    if (OUT_BF16) {
+                        __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(ost);
+#pragma unroll
+                        for (int l = 0; l < 64; ++l) ob[l * DVS + vrow] = __float2bfloat16_rn(ov[l]);
+                    } else {
+#pragma unroll
+                        for (int l = 0; l < 64; ++l) ost[l * DVS + vrow] = ov[l];
+                    }
+                }
+                fence_proxy_async_smem();
+                named_bar(kStateBar, 128);
+                if (ts == 0) {
+                    tma_store_3d(&p.o_map, ost, v0, t0, bh);
+                    bulk_commit();
+                }
+            }
+            TC2_MARK(256, 23);
+            // fp16 copy of the new state for the next chunk's history read; the
+            // next chunk's decay is applied to the fp32 state in the same pass
+            const bool more = r + 1 < nchunks;
+            if (more) {
+                if (!mbar_wait(&ms.bar_rdy, (r + 1) & 1)) note_timeout(ms, 6, r + 1);
+                tc_fence_after();
+            }
+            const int nbuf = buf ^ 1;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float sv[64];
+                __syncwarp();
+                tmem_ld32(lane_addr + TSM + h * 64, sv);
+                tmem_ld32(lane_addr + TSM + h * 64 + 32, sv + 32);
+                tmem_wait_ld();
+                uint32_t w[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    rmax = fmaxf(rmax, fmaxf(fabsf(sv[2 * c]), fabsf(sv[2 * c + 1])));
+                    w[c] = pack_h2(sv[2 * c], sv[2 * c + 1]);
+                }
+                tmem_st32(lane_addr + TS16 + h * 32, w);
+                if (GATE != kGateNone && more) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        sv[i] *= (GATE == kGateScalar) ? dec[nbuf * 128] : dec[nbuf * 128 + h * 64 + i];
+                    tmem_st32f(lane_addr + TSM + h * 64, sv);
+                    tmem_st32f(lane_addr + TSM + h * 64 + 32, sv + 32);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            if (ts == 0) ms.s_abort = ms.abort_flag;
+            named_bar(kStateBar, 128);
+            TC2_MARK(256, 24);
+        }
+        if (ts == 0) bulk_wait0();  // o is in global memory before the kernel ends
+        // final state
+        if (!ms.s_abort && p.ST) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float sv[64];
+                __syncwarp();
+                tmem_ld32(lane_addr + TSM + h * 64, sv);
+                tmem_ld32(lane_addr + TSM + h * 64 + 32, sv + 32);
+                tmem_wait_ld();
+                if (has_row) {
+#pragma unroll
+                    for (int j = 0; j < 64; j += 4)
+                        *reinterpret_cast<float4 *>(p.ST + srow + h * 64 + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+                }
+            }
+        }
+    }
+
+    if (!(rmax <= 65504.f)) ms.range_flag = 1;
+    __syncthreads();
+    if (t == 0) {
+        if (ms.abort_flag) {
+            record_status(p.status, kStatusTimeout);
+            if (p.diag) atomicCAS(p.diag, 0, 1 + ms.abort_site);
+        } else if (ms.range_flag) {
+            record_status(p.status, kStatusRange);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+template <int DVS, int UPD, int GATE, bool OB>
+int launch_one(const Params &prm, int grid, cudaStream_t stream) {
+    using L = Smem<DVS, GATE>;
+    auto kern = chunk_tc2_kernel<DVS, UPD, GATE, OB>;
+    static_assert(L::DYN <= 232448, "shared memory budget");
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN);
+    if (e != cudaSuccess) return (int)e;
+    kern<<<grid, kThreads, L::DYN, stream>>>(prm);
+    return (int)cudaGetLastError();
+}
+
+template <int DVS, int UPD, int GATE>
+int launch_out(const Params &prm, int grid, bool ob, cudaStream_t s) {
+    return ob ? launch_one<DVS, UPD, GATE, true>(prm, grid, s) : launch_one<DVS, UPD, GATE, false>(prm, grid, s);
+}
+
+template <int DVS>
+int launch_modes(const Params &prm, int grid, int update, int gate, bool ob, cudaStream_t s) {
+    if (update == kAdditive) return launch_out<DVS, kAdditive, kGateNone>(prm, grid, ob, s);
+    if (update == kDecay) {
+        if (gate == kGateScalar) return launch_out<DVS, kDecay, kGateScalar>(prm, grid, ob, s);
+        if (DVS == 64) return launch_out<64, kDecay, kGateChannel>(prm, grid, ob, s);
+        return (int)cudaErrorInvalidValue;
+    }
+    if (gate == kGateNone) return launch_out<DVS, kDelta, kGateNone>(prm, grid, ob, s);
+    if (gate == kGateScalar) return launch_out<DVS, kDelta, kGateScalar>(prm, grid, ob, s);
+    if (DVS == 64) return launch_out<64, kDelta, kGateChannel>(prm, grid, ob, s);
+    return (int)cudaErrorInvalidValue;
+}
+
+}  // namespace
+}  // namespace gdn
+
+#ifdef GDN_TC_PHASE_TIMING
+extern "C" int gdn_tc2_phase_times(unsigned long long *out, int clear) {
+    cudaDeviceSynchronize();
+    if (cudaMemcpyFromSymbol(out, g_tc2_phase, sizeof(unsigned long long) * 32) != cudaSuccess) return -1;
+    if (clear) {
+        unsigned long long z[32] = {0};
+        cudaMemcpyToSymbol(g_tc2_phase, z, sizeof(z));
+    }
+    return 0;
+}
+#endif
+
+// Value-slice width: 128 keeps the per-chunk K-side work unduplicated; 64
+// doubles the CTA count when 128-wide slices would leave most SMs idle.
+static int tc2_slice(const gdn_desc_t *d) {
+    const long bh = (long)d->B * d->H;
+    if (d->dv == 64 || d->gate == GDN_GATE_CHANNEL) return 64;
+    return (bh * 2 <= 148) ? 64 : 128;
+}
+
+int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream) {
+    using namespace gdn;
+    Params prm;
+    memset(&prm, 0, sizeof(prm));
+    const uint64_t BH = (uint64_t)a.BH, T = (uint64_t)a.T;
+    if (!make_map_3d(&prm.q_map, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, T, BH, 64, 64, 1, true) ||
+        !make_map_3d(&prm.k_map, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, T, BH, 64, 64, 1, true) ||
+        !make_map_3d(&prm.v_map, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.dv, T, BH, 64, 64, 1, true))
+        return (int)cudaErrorInvalidValue;
+    if (d->gate == GDN_GATE_CHANNEL &&
+        !make_map_3d(&prm.g_map, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, T, BH, 32, 64, 1, false))
+        return (int)cudaErrorInvalidValue;
+    const int dvs = tc2_slice(d);
+    const bool ob = d->out_dtype == GDN_BF16;
+    if (!make_map_3d(&prm.o_map, a.o, ob ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                     ob ? 2 : 4, (uint64_t)a.dv, T, BH, (uint32_t)dvs, 64, 1, false))
+        return (int)cudaErrorInvalidValue;
+    prm.g = a.g;
+    prm.beta = a.beta;
+    prm.S0 = a.S0;
+    prm.o = a.o;
+    prm.ST = a.ST;
+    prm.status = a.status;
+    prm.diag = a.diag;
+    prm.BH = a.BH;
+    prm.T = a.T;
+    prm.dv = a.dv;
+    prm.nslices = a.dv / dvs;
+    const long grid = (long)a.BH * prm.nslices;
+    if (grid == 0) return 0;
+    if (dvs == 64) return launch_modes<64>(prm, (int)grid, d->update, d->gate, ob, stream);
+    return launch_modes<128>(prm, (int)grid, d->update, d->gate, ob, stream);
+}

@@ -65,11 +65,14 @@ typedef enum { GDN_GATE_NONE = 0, GDN_GATE_SCALAR = 1, GDN_GATE_CHANNEL = 2 } gd
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
 
-/* Kernel choice for gdn_chunk_fwd.  AUTO picks the tensor-core kernel when it
+/* Kernel choice for gdn_chunk_fwd.  AUTO picks a tensor-core kernel when one
  * supports the request (bf16 inputs, dk = 128) and the fp32 SIMT kernel
- * otherwise; the two explicit values force one (GDN_ERR_UNSUPPORTED if it
- * cannot serve the request). */
-typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TC = 2 } gdn_algo_t;
+ * otherwise.  TC is the warp-specialised tensor-core kernel (prep of the next
+ * chunk overlapping the state update of the current one); TC_SEQ the
+ * single-group tensor-core kernel that runs the phases of a chunk in sequence.
+ * An explicit value forces that kernel (GDN_ERR_UNSUPPORTED if it cannot serve
+ * the request). */
+typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TC = 2, GDN_ALGO_TC_SEQ = 3 } gdn_algo_t;
 
 typedef struct {
     int B, H;      /* batch and heads; B*H >= 0 */
