@@ -6,13 +6,16 @@
 //   prep group  (warps 0-7) for chunk r+1: TMA of q, k, v (and the channel
 //       gate), P = [Q;K] K^T, the gate prefix, fp16 operands Q<, K<, K>, V,
 //       A' = P_top masked with decay, L = beta P_bottom, the UT transform
-//       T = (I + L)^{-1} (fp32 blocked forward substitution), W = T2 K<.
+//       T = (I + L)^{-1} (fp32: 16x16 diagonal blocks by forward substitution,
+//       then two block merges), W = T2 K<.
 //   state group (warps 8-11) for chunk r, every MMA with M = DVS value rows
 //       (the transposed form), so that the state and the correction rows are
 //       A operands held in TMEM:
 //         Z^T  = V^T T2^T - S W^T          (U^T, then the history correction)
 //         O^T  = S Q<^T + Z^T A'^T
 //         S    = S Diag(e^{G_C}) + Z^T K>
+//       S [-W ; Q<]^T is one N = 128 MMA chain; O leaves through a staging
+//       tile and a TMA store.
 //
 // Same algebra as "Linear Attention, Visualized": "Chunkwise algorithm",
 // "Mamba-2 ... Chunkwise form", "Gated Linear Attention (GLA)", "The triangular
@@ -61,7 +64,7 @@ constexpr int kThreads = 384;  // warps 0-7 prep, 8-11 state
 constexpr int C = kChunk;
 constexpr int DK = 128;
 constexpr float kFactorMaxDecay = 10.0f;
-constexpr int kPrepBar = 1, kStateBar = 2;
+constexpr int kPrepBar = 1, kStateBar = 2, kSolveBar = 3;
 
 struct Params {
     CUtensorMap q_map, k_map, v_map, g_map, o_map;
@@ -216,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 }
                 mma_commit(&ms.bar_p1);
             }
+            TC2_MARK(0, 11);
             // ---------------------------------------------------- a1: gate prefix
             if (GATE == kGateScalar) {
                 if (warp == 0) {
@@ -292,50 +296,68 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             TC2_MARK(0, 3);
             // ---------------------------------------------------- operand conversions
             const bool slow = (GATE == kGateChannel) && ms.slow_chunk;
-            for (int i = t; i < 2 * 512; i += 256) {
-                const int h = i >> 9, off = (i & 511) * 16;
-                const int l = off >> 7;
-                const int c0 = h * 64 + ((((off >> 4) & 7) ^ (l & 7)) << 3);
-                float qf[8], kf[8], ql[8], kl[8], kr[8];
-                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + off), qf);
-                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + 8192 + off), kf);
+            {
+                // every raw load of this thread first: a shared store would otherwise
+                // hold each later load behind it (the compiler cannot rule out aliasing)
+                uint4 rq[4], rk[4], rv[2 * NB];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fmaxf(fabsf(qf[e]), fabsf(kf[e])));
-                if (GATE == kGateChannel) {
-                    const float *gg = reinterpret_cast<const float *>(sm + L::GCH + (c0 >> 5) * 8192) + l * 32 + (c0 & 31);
-                    float kt[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float G = gg[e];
-                        const float eg = __expf(G), emg = __expf(-G);
-                        ql[e] = qf[e] * eg;
-                        kl[e] = kf[e] * eg;
-                        kt[e] = slow ? 0.f : kf[e] * emg;
-                        kr[e] = kf[e] * __expf(ms.GC[c0 + e] - G);
-                        rmax = fmaxf(rmax, fabsf(kt[e]));
-                    }
-                    *reinterpret_cast<uint4 *>(sm + L::KT + h * 8192 + off) = pack_h8(kt);
-                } else {
-                    const float bl = (GATE == kGateScalar) ? ms.b[l] : 1.f;
-                    const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        ql[e] = qf[e] * bl;
-                        kl[e] = kf[e] * bl;
-                        kr[e] = kf[e] * gl;
-                    }
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const int i = t + 256 * s4;
+                    const int h = i >> 9, off = (i & 511) * 16;
+                    rq[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + off);
+                    rk[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + 8192 + off);
                 }
-                *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(ql);
-                if (DELTA || GATE == kGateChannel)
-                    *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
-                *reinterpret_cast<uint4 *>(sm + L::KR + buf * 16384 + h * 8192 + off) = pack_h8(kr);
-            }
-            for (int i = t; i < NB * 512; i += 256) {
-                float vf[8];
-                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::RAW_V + i * 16), vf);
-                *reinterpret_cast<uint4 *>(sm + L::V16 + i * 16) = pack_h8(vf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(vf[e]));
+                for (int s4 = 0; s4 < 2 * NB; ++s4)
+                    rv[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_V + (t + 256 * s4) * 16);
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const int i = t + 256 * s4;
+                    const int h = i >> 9, off = (i & 511) * 16;
+                    const int l = off >> 7;
+                    const int c0 = h * 64 + ((((off >> 4) & 7) ^ (l & 7)) << 3);
+                    float qf[8], kf[8], ql[8], kl[8], kr[8];
+                    unpack_bf16x8(rq[s4], qf);
+                    unpack_bf16x8(rk[s4], kf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fmaxf(fabsf(qf[e]), fabsf(kf[e])));
+                    if (GATE == kGateChannel) {
+                        const float *gg = reinterpret_cast<const float *>(sm + L::GCH + (c0 >> 5) * 8192) + l * 32 + (c0 & 31);
+                        float kt[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float G = gg[e];
+                            const float eg = __expf(G), emg = __expf(-G);
+                            ql[e] = qf[e] * eg;
+                            kl[e] = kf[e] * eg;
+                            kt[e] = slow ? 0.f : kf[e] * emg;
+                            kr[e] = kf[e] * __expf(ms.GC[c0 + e] - G);
+                            rmax = fmaxf(rmax, fabsf(kt[e]));
+                        }
+                        *reinterpret_cast<uint4 *>(sm + L::KT + h * 8192 + off) = pack_h8(kt);
+                    } else {
+                        const float bl = (GATE == kGateScalar) ? ms.b[l] : 1.f;
+                        const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            ql[e] = qf[e] * bl;
+                            kl[e] = kf[e] * bl;
+                            kr[e] = kf[e] * gl;
+                        }
+                    }
+                    *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(ql);
+                    if (DELTA || GATE == kGateChannel)
+                        *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
+                    *reinterpret_cast<uint4 *>(sm + L::KR + buf * 16384 + h * 8192 + off) = pack_h8(kr);
+                }
+#pragma unroll
+                for (int s4 = 0; s4 < 2 * NB; ++s4) {
+                    float vf[8];
+                    unpack_bf16x8(rv[s4], vf);
+                    *reinterpret_cast<uint4 *>(sm + L::V16 + (t + 256 * s4) * 16) = pack_h8(vf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(vf[e]));
+                }
             }
             fence_proxy_async_smem();
             named_bar(kPrepBar, 256);
@@ -431,92 +453,161 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             tc_fence_before();
             named_bar(kPrepBar, 256);
             TC2_MARK(0, 6);
-            if (t == 0 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
+            // warp 7 has no share of the diagonal solve: it issues the next chunk's loads
+            if (t == 224 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
 
             if (DELTA) {
                 // ------------------------------------------------ a3: T = (I + L)^{-1}
-                // L^T is held in the KT scratch ([64][64] fp32, row m = column m of
-                // L).  Stage 1: the two 32x32 diagonal blocks, one column of T per
-                // thread, right-looking (once x_m is final it updates every later
-                // row, so the dependent chain is one FMA per row).  Stage 2:
-                // T_BA = -T_BB (L_BA T_AA).  T_AA goes to the zero block
-                // [32:64, 0:32] of L^T, T_BB over L_AA^T, X = L_BA T_AA over L_BB^T.
-                float *Lt = reinterpret_cast<float *>(sm + L::KT);
-                if (t < 64) {
-                    const int b = t >> 5, c = t & 31, o = 32 * b;
-                    float x[32];
+                // The fp32 scratch Ls holds L^T (Ls[m][l] = L[l][m], m < l).  The
+                // inverse of a unit lower-triangular matrix is built from its 16x16
+                // diagonal blocks (forward substitution, one column per lane), then
+                // merged twice, 16 -> 32 -> 64, with T_IJ = -T_II (L_IJ T_JJ) on the
+                // warp-level tf32 tensor-core path.  fp32 T blocks go to the diagonal
+                // and lower blocks of Ls (its upper blocks keep L^T, which the merges
+                // skip); T2 = T diag(beta) goes to the fp16 tile, whose upper blocks
+                // stay zero.
+                float *Ls = reinterpret_cast<float *>(sm + L::KT);
+                unsigned char *t2 = sm + L::TZA;
+                if (warp < 2) {
+                    // lanes 0-15: block 2w, lanes 16-31: block 2w+1
+                    const int o = 16 * (2 * warp + (lane >> 4)), c = lane & 15;
+                    float x[16];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] = (i == c) ? 1.f : 0.f;
+                    for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
 #pragma unroll
-                    for (int m = 0; m < 31; ++m) {
+                    for (int m = 0; m < 15; ++m) {
                         const float xm = x[m];
 #pragma unroll
-                        for (int i0 = (m + 1) & ~3; i0 < 32; i0 += 4) {
-                            const float4 lv = *reinterpret_cast<const float4 *>(Lt + f32_swz(o + m, o + i0, 64));
+                        for (int i0 = (m + 1) & ~3; i0 < 16; i0 += 4) {
+                            const float4 lv = *reinterpret_cast<const float4 *>(Ls + f32_swz(o + m, o + i0, 64));
                             if (i0 + 0 > m) x[i0 + 0] = fmaf(-lv.x, xm, x[i0 + 0]);
                             if (i0 + 1 > m) x[i0 + 1] = fmaf(-lv.y, xm, x[i0 + 1]);
                             if (i0 + 2 > m) x[i0 + 2] = fmaf(-lv.z, xm, x[i0 + 2]);
                             if (i0 + 3 > m) x[i0 + 3] = fmaf(-lv.w, xm, x[i0 + 3]);
                         }
                     }
+                    __syncwarp();
                     const float bt = ms.beta[o + c];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < 16; ++i) {
                         const float tv = x[i] * bt;
                         rmax = fmaxf(rmax, fabsf(tv));
-                        *reinterpret_cast<__half *>(sm + L::TZA + sw128_off(o + i, o + c)) = __float2half_rn(tv);
-                        if (b == 0) Lt[f32_swz(32 + i, c, 64)] = x[i];
+                        Ls[f32_swz(o + i, o + c, 64)] = x[i];
+                        *reinterpret_cast<__half *>(t2 + sw128_off(o + i, o + c)) = __float2half_rn(tv);
                     }
-                    named_bar(kPrepBar, 256);
-                    if (b == 1) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) Lt[f32_swz(i, c, 64)] = x[i];
-                    }
-                } else {
-                    named_bar(kPrepBar, 256);
                 }
                 named_bar(kPrepBar, 256);
                 TC2_MARK(0, 7);
-                {
-                    const int rr = t >> 3, c0 = (t & 7) * 4;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const int g = lane >> 2, tq = lane & 3;  // mma fragment coordinates
+                if (warp < 4) {
+                    // 16 -> 32 for the block pairs (1,0) and (3,2); warp = (pair, 8-column tile)
+                    const int pr = warp >> 1, j = warp & 1;
+                    const int oJ = 32 * pr, oI = oJ + 16, xr = 32 + 16 * pr;
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int m = 0; m < 32; ++m) {
-                        const float lm = Lt[f32_swz(m, 32 + rr, 64)];  // L_BA[rr][m]
-                        const float4 a0 = *reinterpret_cast<const float4 *>(Lt + f32_swz(32 + m, c0, 64));
-                        acc[0] = fmaf(lm, a0.x, acc[0]);
-                        acc[1] = fmaf(lm, a0.y, acc[1]);
-                        acc[2] = fmaf(lm, a0.z, acc[2]);
-                        acc[3] = fmaf(lm, a0.w, acc[3]);
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const int k0 = oJ + 8 * ks;
+                        uint32_t a[4], b[2];
+                        a[0] = f2tf32(Ls[f32_swz(k0 + tq, oI + g, 64)]);  // L_IJ[i][k] = Ls[oJ+k][oI+i]
+                        a[1] = f2tf32(Ls[f32_swz(k0 + tq, oI + g + 8, 64)]);
+                        a[2] = f2tf32(Ls[f32_swz(k0 + tq + 4, oI + g, 64)]);
+                        a[3] = f2tf32(Ls[f32_swz(k0 + tq + 4, oI + g + 8, 64)]);
+                        b[0] = f2tf32(Ls[f32_swz(k0 + tq, oJ + 8 * j + g, 64)]);  // T_JJ
+                        b[1] = f2tf32(Ls[f32_swz(k0 + tq + 4, oJ + 8 * j + g, 64)]);
+                        mma_tf32_16x8x8(d, a, b);
                     }
-                    *reinterpret_cast<float4 *>(Lt + f32_swz(32 + rr, 32 + c0, 64)) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                    named_bar(kPrepBar, 256);
-                    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                    // X = L_IJ T_JJ waits in rows 32..63, columns 0..15 (free until the next level)
+                    *reinterpret_cast<float2 *>(Ls + f32_swz(xr + g, 8 * j + 2 * tq, 64)) = make_float2(d[0], d[1]);
+                    *reinterpret_cast<float2 *>(Ls + f32_swz(xr + g + 8, 8 * j + 2 * tq, 64)) = make_float2(d[2], d[3]);
+                    __syncwarp();
+                    float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int m0 = 0; m0 < 32; m0 += 4) {
-                        const float4 tv = *reinterpret_cast<const float4 *>(Lt + f32_swz(rr, m0, 64));  // T_BB[rr][m0..]
-                        const float tm[4] = {tv.x, tv.y, tv.z, tv.w};
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const int k0 = 8 * ks;
+                        uint32_t a[4], b[2];
+                        a[0] = f2tf32(Ls[f32_swz(oI + g, oI + k0 + tq, 64)]);  // T_II
+                        a[1] = f2tf32(Ls[f32_swz(oI + g + 8, oI + k0 + tq, 64)]);
+                        a[2] = f2tf32(Ls[f32_swz(oI + g, oI + k0 + tq + 4, 64)]);
+                        a[3] = f2tf32(Ls[f32_swz(oI + g + 8, oI + k0 + tq + 4, 64)]);
+                        b[0] = f2tf32(Ls[f32_swz(xr + k0 + tq, 8 * j + g, 64)]);
+                        b[1] = f2tf32(Ls[f32_swz(xr + k0 + tq + 4, 8 * j + g, 64)]);
+                        mma_tf32_16x8x8(e, a, b);
+                    }
+                    const int c = oJ + 8 * j + 2 * tq;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float4 a0 = *reinterpret_cast<const float4 *>(Lt + f32_swz(32 + m0 + e, 32 + c0, 64));
-                            acc[0] = fmaf(tm[e], a0.x, acc[0]);
-                            acc[1] = fmaf(tm[e], a0.y, acc[1]);
-                            acc[2] = fmaf(tm[e], a0.z, acc[2]);
-                            acc[3] = fmaf(tm[e], a0.w, acc[3]);
+                    for (int h = 0; h < 2; ++h) {
+                        const float v0 = -e[2 * h], v1 = -e[2 * h + 1];
+                        const int row = oI + g + 8 * h;
+                        *reinterpret_cast<float2 *>(Ls + f32_swz(row, c, 64)) = make_float2(v0, v1);
+                        const float b0 = v0 * ms.beta[c], b1 = v1 * ms.beta[c + 1];
+                        rmax = fmaxf(rmax, fmaxf(fabsf(b0), fabsf(b1)));
+                        *reinterpret_cast<uint32_t *>(t2 + sw128_off(row, c)) = pack_h2(b0, b1);
+                    }
+                    named_bar(kSolveBar, 128);
+                    TC2_MARK(0, 8);
+                    // 32 -> 64: 8-column tile j = warp of T_BA = -T_BB (L_BA T_AA)
+                    const int jj = warp;
+                    float dx[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        if (jj >= 2 && ks < 2) continue;  // T_AA[k < 16][c >= 16] = 0
+                        const int k0 = 8 * ks;
+                        uint32_t b[2];
+                        b[0] = f2tf32(Ls[f32_swz(k0 + tq, 8 * jj + g, 64)]);
+                        b[1] = f2tf32(Ls[f32_swz(k0 + tq + 4, 8 * jj + g, 64)]);
+#pragma unroll
+                        for (int mt = 0; mt < 2; ++mt) {
+                            const int i0 = 32 + 16 * mt;  // L[i0+i][k] = Ls[k][i0+i]
+                            uint32_t a[4];
+                            a[0] = f2tf32(Ls[f32_swz(k0 + tq, i0 + g, 64)]);
+                            a[1] = f2tf32(Ls[f32_swz(k0 + tq, i0 + g + 8, 64)]);
+                            a[2] = f2tf32(Ls[f32_swz(k0 + tq + 4, i0 + g, 64)]);
+                            a[3] = f2tf32(Ls[f32_swz(k0 + tq + 4, i0 + g + 8, 64)]);
+                            mma_tf32_16x8x8(dx[mt], a, b);
                         }
                     }
-                    float tb[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        tb[e] = -acc[e] * ms.beta[c0 + e];
-                        rmax = fmaxf(rmax, fabsf(tb[e]));
+                    for (int mt = 0; mt < 2; ++mt) {
+                        *reinterpret_cast<float2 *>(Ls + f32_swz(32 + 16 * mt + g, 8 * jj + 2 * tq, 64)) =
+                            make_float2(dx[mt][0], dx[mt][1]);
+                        *reinterpret_cast<float2 *>(Ls + f32_swz(32 + 16 * mt + g + 8, 8 * jj + 2 * tq, 64)) =
+                            make_float2(dx[mt][2], dx[mt][3]);
                     }
-                    *reinterpret_cast<uint2 *>(sm + L::TZA + sw128_off(32 + rr, c0)) =
-                        make_uint2(pack_h2(tb[0], tb[1]), pack_h2(tb[2], tb[3]));
+                    __syncwarp();
+                    float ex[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const int k0 = 8 * ks;
+                        uint32_t b[2];
+                        b[0] = f2tf32(Ls[f32_swz(32 + k0 + tq, 8 * jj + g, 64)]);
+                        b[1] = f2tf32(Ls[f32_swz(32 + k0 + tq + 4, 8 * jj + g, 64)]);
+#pragma unroll
+                        for (int mt = 0; mt < 2; ++mt) {
+                            if (mt == 0 && ks >= 2) continue;  // T_BB[i < 16][k >= 16] = 0
+                            const int i0 = 32 + 16 * mt;
+                            uint32_t a[4];
+                            a[0] = f2tf32(Ls[f32_swz(i0 + g, 32 + k0 + tq, 64)]);
+                            a[1] = f2tf32(Ls[f32_swz(i0 + g + 8, 32 + k0 + tq, 64)]);
+                            a[2] = f2tf32(Ls[f32_swz(i0 + g, 32 + k0 + tq + 4, 64)]);
+                            a[3] = f2tf32(Ls[f32_swz(i0 + g + 8, 32 + k0 + tq + 4, 64)]);
+                            mma_tf32_16x8x8(ex[mt], a, b);
+                        }
+                    }
+                    const int cc = 8 * jj + 2 * tq;
+                    const float bc0 = ms.beta[cc], bc1 = ms.beta[cc + 1];
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int row = 32 + 16 * mt + g + 8 * h;
+                            const float b0 = -ex[mt][2 * h] * bc0, b1 = -ex[mt][2 * h + 1] * bc1;
+                            rmax = fmaxf(rmax, fmaxf(fabsf(b0), fabsf(b1)));
+                            *reinterpret_cast<uint32_t *>(t2 + sw128_off(row, cc)) = pack_h2(b0, b1);
+                        }
                 }
                 fence_proxy_async_smem();
                 named_bar(kPrepBar, 256);
-                TC2_MARK(0, 8);
+                TC2_MARK(0, 9);
                 // ------------------------------------------------ a4: W = T2 K<
                 if (t == 0 && !ms.abort_flag) {
                     tc_fence_after();
@@ -529,7 +620,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     mma_commit(&ms.bar_w);
                 }
                 if (!mbar_wait(&ms.bar_w, ph)) note_timeout(ms, 3, r);
-                TC2_MARK(0, 9);
                 tc_fence_after();
                 if (sp < 2) {
                     // W rows (lanes 0..63), this warp's 64-column half -> -W slot of that half
@@ -616,23 +706,28 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             if (ts == 0 && !ms.abort_flag) {
                 tc_fence_after();
                 const uint32_t at = smem_u32(sm + L::AT);
-                constexpr uint32_t id1 = idesc_f16(DVS, 64, 0, 0, 0);
                 if (DELTA) {
+                    // [Z^T | O^T] = S [-W ; Q<]^T in one N = 128 chain (the two B tiles are
+                    // adjacent in each K half), then Z^T += V^T T2^T
                     const uint32_t v16 = smem_u32(sm + L::V16), tza = smem_u32(sm + L::TZA);
+                    constexpr uint32_t id1w = idesc_f16(DVS, 128, 0, 0, 0);
                     constexpr uint32_t idu = idesc_f16(DVS, 64, 0, 1, 0);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)  // U^T = V^T T2^T
-                        mma_f16(tmem + TZO, smem_desc_sw128(v16 + k * 2048, 8192, 1024),
-                                smem_desc_sw128(tza + k * 32, 16, 1024), idu, k > 0);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)  // -= S W^T  (the tile holds -W)
+                    for (int k = 0; k < 8; ++k)
                         mma_f16_ts(tmem + TZO, tmem + TS16 + k * 8,
-                                   smem_desc_sw128(at + (k >> 2) * 24576 + (k & 3) * 32, 16, 1024), id1, 1);
-                }
+                                   smem_desc_sw128(at + (k >> 2) * 24576 + (k & 3) * 32, 16, 1024), id1w, k > 0);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)  // O^T = S Q<^T
-                    mma_f16_ts(tmem + TZO + 64, tmem + TS16 + k * 8,
-                               smem_desc_sw128(at + (k >> 2) * 24576 + 8192 + (k & 3) * 32, 16, 1024), id1, k > 0);
+                    for (int k = 0; k < 4; ++k)
+                        mma_f16(tmem + TZO, smem_desc_sw128(v16 + k * 2048, 8192, 1024),
+                                smem_desc_sw128(tza + k * 32, 16, 1024), idu, 1);
+                } else {
+                    constexpr uint32_t id1 = idesc_f16(DVS, 64, 0, 0, 0);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)  // O^T = S Q<^T
+                        mma_f16_ts(tmem + TZO + 64, tmem + TS16 + k * 8,
+                                   smem_desc_sw128(at + (k >> 2) * 24576 + 8192 + (k & 3) * 32, 16, 1024), id1,
+                                   k > 0);
+                }
                 mma_commit(&ms.bar_fA);
             }
             TC2_MARK(256, 18);
@@ -690,7 +785,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             TC2_MARK(256, 22);
             tc_fence_after();
             {
-                // O^T -> row-major staging [64 tok][DVS] -> one TMA store (rows past T clipped)
+                // O^T -> row-major staging [64 tok][DVS] -> one TMA store (rows past T
+                // clipped).  Stores issued straight from registers were measured slower:
+                // they queue behind the prep group's shared-memory traffic.
                 float ov[64];
                 __syncwarp();
                 tmem_ld32(lane_addr + TZO + 64, ov);
@@ -723,6 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 if (!mbar_wait(&ms.bar_rdy, (r + 1) & 1)) note_timeout(ms, 6, r + 1);
                 tc_fence_after();
             }
+            TC2_MARK(256, 25);
             const int nbuf = buf ^ 1;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {

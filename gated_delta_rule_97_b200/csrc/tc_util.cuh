@@ -32,5 +32,24 @@ __device__ __forceinline__ int f32_swz(int r, int c, int ld) {
     return r * ld + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3);
 }
 
+// fp32 -> tf32 (round to nearest, ties away), as a 32-bit operand register.
+__device__ __forceinline__ uint32_t f2tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// Warp-level D += A B, A 16x8 (row), B 8x8 (col), tf32 in, fp32 accumulate.
+// Fragments (g = lane / 4, q = lane % 4):
+//   a = {A[g][q], A[g+8][q], A[g][q+4], A[g+8][q+4]},  b = {B[q][g], B[q+4][g]},
+//   d = {D[g][2q], D[g][2q+1], D[g+8][2q], D[g+8][2q+1]}.
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 }  // namespace tcu
 }  // namespace gdn
