@@ -64,7 +64,7 @@ constexpr int kThreads = 384;  // warps 0-7 prep, 8-11 state
 constexpr int C = kChunk;
 constexpr int DK = 128;
 constexpr float kFactorMaxDecay = 10.0f;
-constexpr int kPrepBar = 1, kStateBar = 2, kSolveBar = 3;
+constexpr int kPrepBar = 1, kStateBar = 2, kSolveBar = 3, kConvBar = 4;
 
 struct Params {
     CUtensorMap q_map, k_map, v_map, g_map, o_map;
@@ -100,7 +100,7 @@ struct Misc {
     float b[64];
     float gam[64];
     float ib[64];
-    float beta[64];
+    float beta[2][64];  // by chunk parity: the solve of chunk r overlaps the gate pass of r+1
     float GC[128];
     int abort_flag, range_flag, slow_chunk, abort_site;
     int p_abort, s_abort, pad0, pad1;
@@ -114,6 +114,14 @@ __device__ __forceinline__ void note_timeout(M &ms, int site, int r) {
 }
 
 constexpr uint32_t TP = 0, TZO = 128, TSM = 256, TS16 = 384, TZ16 = 448;
+
+// Shared offset of chunk parity `buf`'s fp16 V tile.  Without the delta rule V is
+// an operand of the state's last MMAs, so it is double-buffered, the second copy in
+// the L^T scratch that those modes leave unused.
+template <typename L, int UPD, int GATE>
+__device__ __forceinline__ int v16_slot(int buf) {
+    return (UPD != kDelta && GATE != kGateChannel && buf) ? L::KT : L::V16;
+}
 
 template <int DVS, int UPD, int GATE, bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_constant__ Params p) {
@@ -175,14 +183,44 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         const int ch = warp >> 2;          // column half of a TMEM tile handled by this warp
         const int row = sp * 32 + lane;    // TMEM lane (product row) read by this thread
         float gpre0 = 0.f, gpre1 = 0.f, bpre = 0.f;
+        // raw gates (warp 4, two tokens a lane) and betas (warps 4-5) of chunk r into registers
         auto load_gate_beta = [&](int r) {
             const int t0 = r * C;
-            if (GATE == kGateScalar && warp == 0) {
+            if (GATE == kGateScalar && warp == 4) {
                 const int l0 = 2 * lane;
                 gpre0 = (t0 + l0 < T) ? p.g[(size_t)bh * T + t0 + l0] : 0.f;
                 gpre1 = (t0 + l0 + 1 < T) ? p.g[(size_t)bh * T + t0 + l0 + 1] : 0.f;
             }
-            if (DELTA && t < C) bpre = (t0 + t < T) ? p.beta[(size_t)bh * T + t0 + t] : 0.f;
+            if (DELTA && t >= 128 && t < 128 + C) {
+                const int l = t - 128;
+                bpre = (t0 + l < T) ? p.beta[(size_t)bh * T + t0 + l] : 0.f;
+            }
+        };
+        // scalar gate prefix of chunk r and its factors b = e^G, gamma = e^{G_C-G},
+        // 1/b, e^{G_C}; beta of chunk r into its parity slot (warps 4-5)
+        auto gate_pass = [&](int r) {
+            if (GATE == kGateScalar && warp == 4) {
+                const int l0 = 2 * lane;
+                const float x0 = gpre0, x1 = gpre1;
+                float s = x0 + x1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, s, off);
+                    if (lane >= off) s += y;
+                }
+                const float G0 = s - x1, G1 = s;
+                const float gc = __shfl_sync(0xffffffffu, G1, 31);
+                ms.G[l0] = G0;
+                ms.G[l0 + 1] = G1;
+                ms.b[l0] = __expf(G0);
+                ms.b[l0 + 1] = __expf(G1);
+                ms.gam[l0] = __expf(gc - G0);
+                ms.gam[l0 + 1] = __expf(gc - G1);
+                ms.ib[l0] = __expf(-G0);
+                ms.ib[l0 + 1] = __expf(-G1);
+                if (lane == 0) dec[(r & 1) * 128] = __expf(gc);
+            }
+            if (DELTA && t >= 128 && t < 128 + C) ms.beta[r & 1][t - 128] = bpre;
         };
         auto issue_tma = [&](int r) {
             const int t0 = r * C;
@@ -198,53 +236,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 for (int j = 0; j < 4; ++j) tma_load_3d(sm + L::GCH + j * 8192, &p.g_map, j * 32, t0, bh, &ms.bar_tma);
         };
         if (t == 0 && nchunks > 0) issue_tma(0);
-        if (nchunks > 0) load_gate_beta(0);
+        if (nchunks > 0) {
+            load_gate_beta(0);
+            if (GATE != kGateChannel) {
+                gate_pass(0);
+                if (nchunks > 1) load_gate_beta(1);
+            }
+        }
+        named_bar(kPrepBar, 256);
 
         for (int r = 0; r < nchunks; ++r) {
             if (ms.p_abort) break;
             const uint32_t ph = r & 1;
             const int buf = r & 1;
+            const float *bet = ms.beta[buf];
             TC2_MARK(0, 0);
             if (!mbar_wait(&ms.bar_tma, ph)) note_timeout(ms, 1, r);
             TC2_MARK(0, 1);
-            if (GATE != kGateChannel && t == 0 && !ms.abort_flag) {
-                tc_fence_after();
-                const uint32_t qk = smem_u32(sm + L::RAW_QK);
-                constexpr uint32_t id = idesc_f16(128, 64, 1, 0, 0);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_f16(tmem + TP, smem_desc_sw128(qk + ko, 16, 1024), smem_desc_sw128(qk + 8192 + ko, 16, 1024),
-                            id, k > 0);
-                }
-                mma_commit(&ms.bar_p1);
-            }
-            TC2_MARK(0, 11);
-            // ---------------------------------------------------- a1: gate prefix
-            if (GATE == kGateScalar) {
-                if (warp == 0) {
-                    // two tokens per lane; the warp also derives b = e^G, gamma = e^{G_C-G}, 1/b
-                    const int l0 = 2 * lane;
-                    const float x0 = gpre0, x1 = gpre1;
-                    float s = x0 + x1;
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const float y = __shfl_up_sync(0xffffffffu, s, off);
-                        if (lane >= off) s += y;
-                    }
-                    const float G0 = s - x1, G1 = s;
-                    const float gc = __shfl_sync(0xffffffffu, G1, 31);
-                    ms.G[l0] = G0;
-                    ms.G[l0 + 1] = G1;
-                    ms.b[l0] = __expf(G0);
-                    ms.b[l0 + 1] = __expf(G1);
-                    ms.gam[l0] = __expf(gc - G0);
-                    ms.gam[l0 + 1] = __expf(gc - G1);
-                    ms.ib[l0] = __expf(-G0);
-                    ms.ib[l0 + 1] = __expf(-G1);
-                    if (lane == 0) dec[buf * 128] = __expf(gc);
-                }
-            } else if (GATE == kGateChannel) {
+            if (GATE == kGateChannel) {
+                // ------------------------------------------------ a1: channel gate prefix
                 // channel c, token half hf: prefix over 32 tokens, then join the halves
                 const int c = t & 127, hf = t >> 7;
                 float *gcol = reinterpret_cast<float *>(sm + L::GCH + (c >> 5) * 8192) + (c & 31);
@@ -274,93 +284,130 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
                     if (lane == 0) ms.slow_chunk = !(mx <= kFactorMaxDecay);
                 }
+                gate_pass(r);
+                if (r + 1 < nchunks) load_gate_beta(r + 1);
+                named_bar(kPrepBar, 256);
             }
-            if (DELTA && t < C) ms.beta[t] = bpre;
-            if (r + 1 < nchunks) load_gate_beta(r + 1);
-            named_bar(kPrepBar, 256);
             const bool fastg = (GATE != kGateScalar) || (-ms.G[C - 1] <= 80.f);
             TC2_MARK(0, 2);
-            // the state group must be done with the buffers this chunk overwrites
-            if (r >= 1) {
-                if (DELTA) {
-                    if (!mbar_wait(&ms.bar_fA, (r - 1) & 1)) note_timeout(ms, 9, r);
-                } else {
-                    uint64_t *fb = ((r - 1) & 1) ? &ms.bar_fB1 : &ms.bar_fB0;
-                    if (!mbar_wait(fb, ((r - 1) >> 1) & 1)) note_timeout(ms, 10, r);
-                }
-            }
+            // A'[buf] and K>[buf] were last read by the state's chunk r-2
             if (r >= 2) {
                 uint64_t *fb = buf ? &ms.bar_fB1 : &ms.bar_fB0;
                 if (!mbar_wait(fb, ((r - 2) >> 1) & 1)) note_timeout(ms, 10, r);
             }
+            // the history operands (Q<, V, T2, -W) were last read by the state's chunk r-1:
+            // its first MMAs (fA), or its last ones where the single V tile feeds them
+            auto wait_history = [&]() {
+                if (r >= 1) {
+                    if (DELTA || GATE != kGateChannel) {
+                        if (!mbar_wait(&ms.bar_fA, (r - 1) & 1)) note_timeout(ms, 9, r);
+                    } else {
+                        uint64_t *fb = ((r - 1) & 1) ? &ms.bar_fB1 : &ms.bar_fB0;
+                        if (!mbar_wait(fb, ((r - 1) >> 1) & 1)) note_timeout(ms, 10, r);
+                    }
+                }
+            };
             TC2_MARK(0, 3);
             // ---------------------------------------------------- operand conversions
             const bool slow = (GATE == kGateChannel) && ms.slow_chunk;
-            {
-                // every raw load of this thread first: a shared store would otherwise
-                // hold each later load behind it (the compiler cannot rule out aliasing)
-                uint4 rq[4], rk[4], rv[2 * NB];
+            if (GATE == kGateChannel) {
+                wait_history();
+                {
+                    // every raw load of this thread first: a shared store would otherwise
+                    // hold each later load behind it (the compiler cannot rule out aliasing)
+                    uint4 rq[4], rk[4], rv[2 * NB];
+#pragma unroll
+                    for (int s4 = 0; s4 < 4; ++s4) {
+                        const int i = t + 256 * s4;
+                        const int h = i >> 9, off = (i & 511) * 16;
+                        rq[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + off);
+                        rk[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + 8192 + off);
+                    }
+#pragma unroll
+                    for (int s4 = 0; s4 < 2 * NB; ++s4)
+                        rv[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_V + (t + 256 * s4) * 16);
+#pragma unroll
+                    for (int s4 = 0; s4 < 4; ++s4) {
+                        const int i = t + 256 * s4;
+                        const int h = i >> 9, off = (i & 511) * 16;
+                        const int l = off >> 7;
+                        const int c0 = h * 64 + ((((off >> 4) & 7) ^ (l & 7)) << 3);
+                        float qf[8], kf[8], ql[8], kl[8], kr[8];
+                        unpack_bf16x8(rq[s4], qf);
+                        unpack_bf16x8(rk[s4], kf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fmaxf(fabsf(qf[e]), fabsf(kf[e])));
+                        if (GATE == kGateChannel) {
+                            const float *gg = reinterpret_cast<const float *>(sm + L::GCH + (c0 >> 5) * 8192) + l * 32 + (c0 & 31);
+                            float kt[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float G = gg[e];
+                                const float eg = __expf(G), emg = __expf(-G);
+                                ql[e] = qf[e] * eg;
+                                kl[e] = kf[e] * eg;
+                                kt[e] = slow ? 0.f : kf[e] * emg;
+                                kr[e] = kf[e] * __expf(ms.GC[c0 + e] - G);
+                                rmax = fmaxf(rmax, fabsf(kt[e]));
+                            }
+                            *reinterpret_cast<uint4 *>(sm + L::KT + h * 8192 + off) = pack_h8(kt);
+                        } else {
+                            const float bl = (GATE == kGateScalar) ? ms.b[l] : 1.f;
+                            const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                ql[e] = qf[e] * bl;
+                                kl[e] = kf[e] * bl;
+                                kr[e] = kf[e] * gl;
+                            }
+                        }
+                        *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(ql);
+                        if (DELTA || GATE == kGateChannel)
+                            *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
+                        *reinterpret_cast<uint4 *>(sm + L::KR + buf * 16384 + h * 8192 + off) = pack_h8(kr);
+                    }
+#pragma unroll
+                    for (int s4 = 0; s4 < 2 * NB; ++s4) {
+                        float vf[8];
+                        unpack_bf16x8(rv[s4], vf);
+                        *reinterpret_cast<uint4 *>(sm + L::V16 + (t + 256 * s4) * 16) = pack_h8(vf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(vf[e]));
+                    }
+                }
+            } else {
+                // K< (the W product) and K> (the state update) first: no MMA in flight reads
+                // their slots, so this overlaps the state's history MMAs of chunk r-1
+                uint4 rk[4];
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
                     const int i = t + 256 * s4;
-                    const int h = i >> 9, off = (i & 511) * 16;
-                    rq[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + off);
-                    rk[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + 8192 + off);
+                    rk[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + (i >> 9) * 16384 + 8192 + (i & 511) * 16);
                 }
-#pragma unroll
-                for (int s4 = 0; s4 < 2 * NB; ++s4)
-                    rv[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_V + (t + 256 * s4) * 16);
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
                     const int i = t + 256 * s4;
                     const int h = i >> 9, off = (i & 511) * 16;
                     const int l = off >> 7;
-                    const int c0 = h * 64 + ((((off >> 4) & 7) ^ (l & 7)) << 3);
-                    float qf[8], kf[8], ql[8], kl[8], kr[8];
-                    unpack_bf16x8(rq[s4], qf);
+                    float kf[8], kl[8], kr[8];
                     unpack_bf16x8(rk[s4], kf);
+                    const float bl = (GATE == kGateScalar) ? ms.b[l] : 1.f;
+                    const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fmaxf(fabsf(qf[e]), fabsf(kf[e])));
-                    if (GATE == kGateChannel) {
-                        const float *gg = reinterpret_cast<const float *>(sm + L::GCH + (c0 >> 5) * 8192) + l * 32 + (c0 & 31);
-                        float kt[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float G = gg[e];
-                            const float eg = __expf(G), emg = __expf(-G);
-                            ql[e] = qf[e] * eg;
-                            kl[e] = kf[e] * eg;
-                            kt[e] = slow ? 0.f : kf[e] * emg;
-                            kr[e] = kf[e] * __expf(ms.GC[c0 + e] - G);
-                            rmax = fmaxf(rmax, fabsf(kt[e]));
-                        }
-                        *reinterpret_cast<uint4 *>(sm + L::KT + h * 8192 + off) = pack_h8(kt);
-                    } else {
-                        const float bl = (GATE == kGateScalar) ? ms.b[l] : 1.f;
-                        const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            ql[e] = qf[e] * bl;
-                            kl[e] = kf[e] * bl;
-                            kr[e] = kf[e] * gl;
-                        }
+                    for (int e = 0; e < 8; ++e) {
+                        rmax = fmaxf(rmax, fabsf(kf[e]));
+                        kl[e] = kf[e] * bl;
+                        kr[e] = kf[e] * gl;
                     }
-                    *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(ql);
-                    if (DELTA || GATE == kGateChannel)
-                        *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
+                    if (DELTA) *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
                     *reinterpret_cast<uint4 *>(sm + L::KR + buf * 16384 + h * 8192 + off) = pack_h8(kr);
                 }
-#pragma unroll
-                for (int s4 = 0; s4 < 2 * NB; ++s4) {
-                    float vf[8];
-                    unpack_bf16x8(rv[s4], vf);
-                    *reinterpret_cast<uint4 *>(sm + L::V16 + (t + 256 * s4) * 16) = pack_h8(vf);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(vf[e]));
-                }
             }
-            fence_proxy_async_smem();
-            named_bar(kPrepBar, 256);
+            if (GATE == kGateChannel) {
+                // the channel-gate products take the converted operands: P = [Q<;K<] (k e^{-G})^T
+                fence_proxy_async_smem();
+                named_bar(kPrepBar, 256);
+            }
             if (GATE == kGateChannel && t == 0) {
                 tc_fence_after();
                 const uint32_t at = smem_u32(sm + L::AT), kt = smem_u32(sm + L::KT);
@@ -390,10 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 tmem_wait_ld();
                 if (GATE == kGateChannel && slow) {
                     const unsigned char *xrow = sm + L::RAW_QK + (top ? 0 : 8192);
+#pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int m = m0 + e;
                         float acc = 0.f;
                         if (m <= l) {
+#pragma unroll 1
                             for (int c = 0; c < DK; ++c) {
                                 const int h = c >> 6;
                                 const uint32_t ox = sw128_off(l, c & 63), om = sw128_off(m, c & 63);
@@ -441,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) *reinterpret_cast<uint4 *>(ap + sw128_off(l, m0 + e)) = pack_h8(pr + e);
                 } else if (DELTA) {
-                    const float bl = ms.beta[l];
+                    const float bl = bet[l];
                     float *Lt = reinterpret_cast<float *>(sm + L::KT);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) pr[e] = (m0 + e < l) ? bl * pr[e] * dm[e] : 0.f;
@@ -453,8 +502,54 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             tc_fence_before();
             named_bar(kPrepBar, 256);
             TC2_MARK(0, 6);
-            // warp 7 has no share of the diagonal solve: it issues the next chunk's loads
-            if (t == 224 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
+            if (GATE == kGateChannel) {
+                if (t == 224 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
+            } else if (!DELTA || warp >= 2) {
+                // Q< and V16 (history operands) on warps 2-7 while warps 0-1 run the
+                // diagonal solve; then the next chunk's loads (the raw tiles are consumed)
+                // and its gate pass (this chunk's factors are no longer read)
+                wait_history();
+                {
+                    constexpr int NW = DELTA ? 192 : 256;
+                    constexpr int NQV = 1024 + 512 * NB;
+                    constexpr int IT = (NQV + NW - 1) / NW;
+                    const int wt = DELTA ? t - 64 : t;
+                    uint4 raw[IT];
+#pragma unroll
+                    for (int s4 = 0; s4 < IT; ++s4) {
+                        const int i = wt + NW * s4;
+                        raw[s4] = make_uint4(0, 0, 0, 0);
+                        if (i < 1024)
+                            raw[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + (i >> 9) * 16384 + (i & 511) * 16);
+                        else if (i < NQV)
+                            raw[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_V + (i - 1024) * 16);
+                    }
+#pragma unroll
+                    for (int s4 = 0; s4 < IT; ++s4) {
+                        const int i = wt + NW * s4;
+                        float f[8];
+                        unpack_bf16x8(raw[s4], f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(f[e]));
+                        if (i < 1024) {
+                            const int h = i >> 9, off = (i & 511) * 16;
+                            const float bl = (GATE == kGateScalar) ? ms.b[off >> 7] : 1.f;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) f[e] *= bl;
+                            *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(f);
+                        } else if (i < NQV) {
+                            *reinterpret_cast<uint4 *>(sm + v16_slot<L, UPD, GATE>(buf) + (i - 1024) * 16) = pack_h8(f);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                named_bar(kConvBar, DELTA ? 192 : 256);
+                if (t == 224 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
+                if (!DELTA && r + 1 < nchunks) {
+                    gate_pass(r + 1);
+                    if (r + 2 < nchunks) load_gate_beta(r + 2);
+                }
+            }
 
             if (DELTA) {
                 // ------------------------------------------------ a3: T = (I + L)^{-1}
@@ -486,8 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                             if (i0 + 3 > m) x[i0 + 3] = fmaf(-lv.w, xm, x[i0 + 3]);
                         }
                     }
+                    if (GATE != kGateChannel) wait_history();  // T2 of chunk r-1 has been read
                     __syncwarp();
-                    const float bt = ms.beta[o + c];
+                    const float bt = bet[o + c];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const float tv = x[i] * bt;
@@ -499,6 +595,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 named_bar(kPrepBar, 256);
                 TC2_MARK(0, 7);
                 const int g = lane >> 2, tq = lane & 3;  // mma fragment coordinates
+                if (GATE != kGateChannel && warp >= 4 && r + 1 < nchunks) {
+                    // next chunk's gate pass (this chunk's factors were last read by the
+                    // conversions before the barrier above)
+                    gate_pass(r + 1);
+                    if (r + 2 < nchunks) load_gate_beta(r + 2);
+                }
                 if (warp < 4) {
                     // 16 -> 32 for the block pairs (1,0) and (3,2); warp = (pair, 8-column tile)
                     const int pr = warp >> 1, j = warp & 1;
@@ -539,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         const float v0 = -e[2 * h], v1 = -e[2 * h + 1];
                         const int row = oI + g + 8 * h;
                         *reinterpret_cast<float2 *>(Ls + f32_swz(row, c, 64)) = make_float2(v0, v1);
-                        const float b0 = v0 * ms.beta[c], b1 = v1 * ms.beta[c + 1];
+                        const float b0 = v0 * bet[c], b1 = v1 * bet[c + 1];
                         rmax = fmaxf(rmax, fmaxf(fabsf(b0), fabsf(b1)));
                         *reinterpret_cast<uint32_t *>(t2 + sw128_off(row, c)) = pack_h2(b0, b1);
                     }
@@ -594,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         }
                     }
                     const int cc = 8 * jj + 2 * tq;
-                    const float bc0 = ms.beta[cc], bc1 = ms.beta[cc + 1];
+                    const float bc0 = bet[cc], bc1 = bet[cc + 1];
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -651,6 +753,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         // =================================================================== state group
         const int ts = t - 256;
         const bool has_row = (DVS == 128) || (lane < 16);
+        // P = [Q;K] K^T of chunk r from the raw bf16 tiles, issued by this group's MMA
+        // thread (the prep group's threads then never stall on the tensor pipe's queue)
+        auto issue_p1 = [&](int r) {
+            if (!mbar_wait(&ms.bar_tma, r & 1)) note_timeout(ms, 11, r);
+            tc_fence_after();
+            const uint32_t qk = smem_u32(sm + L::RAW_QK);
+            constexpr uint32_t id = idesc_f16(128, 64, 1, 0, 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32;
+                mma_f16(tmem + TP, smem_desc_sw128(qk + ko, 16, 1024), smem_desc_sw128(qk + 8192 + ko, 16, 1024), id,
+                        k > 0);
+            }
+            mma_commit(&ms.bar_p1);
+        };
+        if (GATE != kGateChannel && ts == 0 && nchunks > 0) issue_p1(0);
         const int vrow = (DVS == 128) ? ts : (sp * 16 + lane);
         const size_t srow = ((size_t)bh * dv + v0 + (has_row ? vrow : 0)) * DK;
         // initial state: fp32 master and fp16 operand copy (lane = value row)
@@ -702,9 +820,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             const uint32_t ph = r & 1;
             const int t0 = r * C;
             const int buf = r & 1;
+            if (GATE != kGateChannel && r > 0) {
+                if (!mbar_wait(&ms.bar_rdy, ph)) note_timeout(ms, 6, r);
+                tc_fence_after();
+            }
             TC2_MARK(256, 17);
             if (ts == 0 && !ms.abort_flag) {
                 tc_fence_after();
+                // P1 of the next chunk goes to the tensor pipe first: the prep group
+                // released TP with rdy(r) and waits on P1 before its A'/L pass
+                if (GATE != kGateChannel && r + 1 < nchunks) issue_p1(r + 1);
                 const uint32_t at = smem_u32(sm + L::AT);
                 if (DELTA) {
                     // [Z^T | O^T] = S [-W ; Q<]^T in one N = 128 chain (the two B tiles are
@@ -768,7 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         mma_f16_ts(tmem + TSM, za, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3, 1);
                     }
                 } else {
-                    const uint32_t v16 = smem_u32(sm + L::V16);
+                    const uint32_t v16 = smem_u32(sm + v16_slot<L, UPD, GATE>(buf));
                     constexpr uint32_t id2s = idesc_f16(DVS, 64, 0, 1, 0);
                     constexpr uint32_t id3s = idesc_f16(DVS, 128, 0, 1, 1);
 #pragma unroll
@@ -816,7 +941,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             // fp16 copy of the new state for the next chunk's history read; the
             // next chunk's decay is applied to the fp32 state in the same pass
             const bool more = r + 1 < nchunks;
-            if (more) {
+            // the channel gate's decay of chunk r+1 comes from that chunk's prep; the
+            // scalar gate's was published with rdy(r) (the prep group runs a chunk's
+            // gate pass one chunk early), so S16 and the decay need not wait
+            if (GATE == kGateChannel && more) {
                 if (!mbar_wait(&ms.bar_rdy, (r + 1) & 1)) note_timeout(ms, 6, r + 1);
                 tc_fence_after();
             }
