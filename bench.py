@@ -43,6 +43,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Algorithmic work (bytes: each input read once, each output written once)
 # ---------------------------------------------------------------------------
 
+def measured_traffic(workload):
+    """DRAM bytes of one launch from the committed ncu capture, or None when the
+    kernel source has changed since that capture (the figure would be stale)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        rec = json.load(open(path))[workload]
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, KeyError, ValueError):
+        return None
+    if hashlib.sha256(src).hexdigest() != rec["source_sha256"]:
+        return None
+    return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+
+
 def prefill_bytes(w, out_bytes=4):
     in_b = 2 if w.dtype == "bf16" else 4
     per_tok = (2 * w.dk + w.dv) * in_b + w.dv * out_bytes
@@ -349,7 +364,7 @@ def run_ours(args):
                          "l2": "inputs (%.2f GB) larger than the 126 MB L2" % (nbytes / 1e9)},
               "token_heads_per_s": world * w.n_heads * w.T / (ms * 1e-3),
               "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None,
+                           "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": measured_traffic(w.name),
                            "peak_source": peak_kind, "algorithmic_bytes_per_launch": nbytes,
                            "flops_per_launch": flops,
                            "achieved_tflops": flops / (ms * 1e-3) / 1e12,
