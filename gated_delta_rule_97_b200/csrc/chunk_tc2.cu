@@ -4,29 +4,31 @@
 // walks its chunks (C = 64) with two warp groups that overlap:
 //
 //   prep group  (warps 0-7) for chunk r+1: TMA of q, k, v (and the channel
-//       gate), P = [Q;K] K^T, the gate prefix, fp16 operands Q<, K<, K>, V,
-//       A' = P_top masked with decay, L = beta P_bottom, the UT transform
-//       T = (I + L)^{-1} (fp32: 16x16 diagonal blocks by forward substitution,
-//       then two block merges), W = T2 K<.
+//       gate), the gate prefix, fp16 operands Q<, K<, K>, V, A' = P_top
+//       masked with decay and L = beta P_bottom from P = [Q;K] K^T, and the UT
+//       transform T = (I + L)^{-1} (fp32: 16x16 diagonal blocks by forward
+//       substitution, then two block merges on tf32 warp MMAs) as T2 = T diag(beta).
 //   state group (warps 8-11) for chunk r, every MMA with M = DVS value rows
 //       (the transposed form), so that the state and the correction rows are
 //       A operands held in TMEM:
-//         Z^T  = V^T T2^T - S W^T          (U^T, then the history correction)
-//         O^T  = S Q<^T + Z^T A'^T
+//         [O^T | X^T] = S [Q< ; K<]^T        (one N = 128 chain)
+//         Z^T  = V^T T2^T - X^T T2^T         (U^T minus the history correction)
+//         O^T += Z^T A'^T
 //         S    = S Diag(e^{G_C}) + Z^T K>
-//       S [-W ; Q<]^T is one N = 128 MMA chain; O leaves through a staging
-//       tile and a TMA store.
+//       Its MMA thread also issues the next chunk's P.  O leaves through a
+//       staging tile and a TMA store.
 //
 // Same algebra as "Linear Attention, Visualized": "Chunkwise algorithm",
 // "Mamba-2 ... Chunkwise form", "Gated Linear Attention (GLA)", "The triangular
 // correction system", "Optional: Use UT to share the triangular transform",
-// "Correct the incoming state" and the GDN / KDA tables; only the storage is
-// transposed (S is kept [dv x dk] with lane = value row).
+// "Correct the incoming state" and the GDN / KDA tables (W S^T = T2 (K< S^T) is
+// evaluated as (S K<^T) T2^T); only the storage is transposed (S is kept
+// [dv x dk] with lane = value row).
 //
-// TMEM (512 columns): prep P/W products [0,128); state: Z^T|O^T [128,256),
-// S fp32 [256,384), S fp16 (A operand) [384,448), Z^T fp16 (A operand) [448,480).
+// TMEM (512 columns): P [0,64), Z^T [64,128), O^T|X^T [128,256), S fp32
+// [256,384), S fp16 (A operand) [384,448), -X^T / Z^T fp16 (A operand) [448,480).
 // Hand-offs: bar_rdy (prep -> state, one phase per chunk), bar_fA (state MMAs
-// that read T2, W, Q<, V completed), bar_fB0/1 (state MMAs that read A', K>
+// that read Q<, K<, V, T2 completed), bar_fB0/1 (state MMAs that read A', K>
 // of an even / odd chunk completed; A' and K> are double-buffered).  All waits
 // are bounded; intermediates are fp16 with a range flag (see chunk_tc.cu).
 #include <string.h>
@@ -64,7 +66,7 @@ constexpr int kThreads = 384;  // warps 0-7 prep, 8-11 state
 constexpr int C = kChunk;
 constexpr int DK = 128;
 constexpr float kFactorMaxDecay = 10.0f;
-constexpr int kPrepBar = 1, kStateBar = 2, kSolveBar = 3, kConvBar = 4;
+constexpr int kPrepBar = 1, kStateBar = 2, kConvBar = 4, kPairBar = 5;  // kPairBar..kPairBar+3
 
 struct Params {
     CUtensorMap q_map, k_map, v_map, g_map, o_map;
@@ -83,8 +85,8 @@ struct Smem {
     static constexpr int RAW_QK = 0;                                     // [Q0 K0 | Q1 K1] bf16
     static constexpr int RAW_V = RAW_QK + 32768;                         // V slice bf16
     static constexpr int GCH = RAW_V + DVS * 128;                        // channel gate fp32 [64][128]
-    static constexpr int AT = GCH + (GATE == kGateChannel ? 32768 : 0);  // [-W | Q< | K<] x 2 halves
-    static constexpr int KT = AT + 49152;                                // k e^{-G} fp16 / L^T fp32 scratch
+    static constexpr int AT = GCH + (GATE == kGateChannel ? 32768 : 0);  // [Q< | K<] x 2 key halves
+    static constexpr int KT = AT + 32768;                                // k e^{-G} fp16 / L^T fp32 scratch
     static constexpr int KR = KT + 16384;                                // K> fp16, 2 buffers
     static constexpr int V16 = KR + 32768;                               // V fp16
     static constexpr int TZA = V16 + DVS * 128;                          // [T2 | A'0 | A'1] fp16
@@ -105,7 +107,7 @@ struct Misc {
     int abort_flag, range_flag, slow_chunk, abort_site;
     int p_abort, s_abort, pad0, pad1;
     uint32_t tmem_base, pad2[3];
-    uint64_t bar_tma, bar_p1, bar_w, bar_rdy, bar_fA, bar_fB0, bar_fB1, pad3;
+    uint64_t bar_tma, bar_p1, bar_x, bar_rdy, bar_fA, bar_fB0, bar_fB1, pad3;
 };
 
 template <typename M>
@@ -113,7 +115,7 @@ __device__ __forceinline__ void note_timeout(M &ms, int site, int r) {
     if (atomicCAS(&ms.abort_flag, 0, 1) == 0) ms.abort_site = site * 1000000 + r;
 }
 
-constexpr uint32_t TP = 0, TZO = 128, TSM = 256, TS16 = 384, TZ16 = 448;
+constexpr uint32_t TP = 0, TZ = 64, TOX = 128, TSM = 256, TS16 = 384, TZ16 = 448;
 
 // Shared offset of chunk parity `buf`'s fp16 V tile.  Without the delta rule V is
 // an operand of the state's last MMAs, so it is double-buffered, the second copy in
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     if (t == 0) {
         mbar_init(&ms.bar_tma, 1);
         mbar_init(&ms.bar_p1, 1);
-        mbar_init(&ms.bar_w, 1);
+        mbar_init(&ms.bar_x, 1);
         mbar_init(&ms.bar_rdy, 1);
         mbar_init(&ms.bar_fA, 1);
         mbar_init(&ms.bar_fB0, 1);
@@ -295,8 +297,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 uint64_t *fb = buf ? &ms.bar_fB1 : &ms.bar_fB0;
                 if (!mbar_wait(fb, ((r - 2) >> 1) & 1)) note_timeout(ms, 10, r);
             }
-            // the history operands (Q<, V, T2, -W) were last read by the state's chunk r-1:
-            // its first MMAs (fA), or its last ones where the single V tile feeds them
+            // the history operands were last read by the state's chunk r-1: Q<, K<, V by
+            // its first MMA group (bar_x; fA without the delta rule), T2 also by the
+            // correction MMA (fA), the single V tile of the channel modes by its last MMAs
+            auto wait_first_mmas = [&]() {
+                if (DELTA && r >= 1) {
+                    if (!mbar_wait(&ms.bar_x, (r - 1) & 1)) note_timeout(ms, 12, r);
+                }
+            };
             auto wait_history = [&]() {
                 if (r >= 1) {
                     if (DELTA || GATE != kGateChannel) {
@@ -311,7 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             // ---------------------------------------------------- operand conversions
             const bool slow = (GATE == kGateChannel) && ms.slow_chunk;
             if (GATE == kGateChannel) {
-                wait_history();
+                if (DELTA)
+                    wait_first_mmas();
+                else
+                    wait_history();
                 {
                     // every raw load of this thread first: a shared store would otherwise
                     // hold each later load behind it (the compiler cannot rule out aliasing)
@@ -361,9 +372,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                                 kr[e] = kf[e] * gl;
                             }
                         }
-                        *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(ql);
+                        *reinterpret_cast<uint4 *>(sm + L::AT + h * 16384 + off) = pack_h8(ql);
                         if (DELTA || GATE == kGateChannel)
-                            *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
+                            *reinterpret_cast<uint4 *>(sm + L::AT + h * 16384 + 8192 + off) = pack_h8(kl);
                         *reinterpret_cast<uint4 *>(sm + L::KR + buf * 16384 + h * 8192 + off) = pack_h8(kr);
                     }
 #pragma unroll
@@ -376,8 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     }
                 }
             } else {
-                // K< (the W product) and K> (the state update) first: no MMA in flight reads
-                // their slots, so this overlaps the state's history MMAs of chunk r-1
+                // K> (the state update) first: no MMA in flight reads its slot, so this
+                // overlaps the state's history MMAs of chunk r-1
                 uint4 rk[4];
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
@@ -389,17 +400,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     const int i = t + 256 * s4;
                     const int h = i >> 9, off = (i & 511) * 16;
                     const int l = off >> 7;
-                    float kf[8], kl[8], kr[8];
+                    float kf[8], kr[8];
                     unpack_bf16x8(rk[s4], kf);
-                    const float bl = (GATE == kGateScalar) ? ms.b[l] : 1.f;
                     const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         rmax = fmaxf(rmax, fabsf(kf[e]));
-                        kl[e] = kf[e] * bl;
                         kr[e] = kf[e] * gl;
                     }
-                    if (DELTA) *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 16384 + off) = pack_h8(kl);
                     *reinterpret_cast<uint4 *>(sm + L::KR + buf * 16384 + h * 8192 + off) = pack_h8(kr);
                 }
             }
@@ -414,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 constexpr uint32_t id = idesc_f16(128, 64, 0, 0, 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint32_t ka = (k >> 2) * 24576 + 8192 + (k & 3) * 32;
+                    const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
                     const uint32_t kb = (k >> 2) * 8192 + (k & 3) * 32;
                     mma_f16(tmem + TP, smem_desc_sw128(at + ka, 16, 1024), smem_desc_sw128(kt + kb, 16, 1024), id,
                             k > 0);
@@ -505,40 +513,48 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             if (GATE == kGateChannel) {
                 if (t == 224 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
             } else if (!DELTA || warp >= 2) {
-                // Q< and V16 (history operands) on warps 2-7 while warps 0-1 run the
+                // Q<, K< and V16 (history operands) on warps 2-7 while warps 0-1 run the
                 // diagonal solve; then the next chunk's loads (the raw tiles are consumed)
                 // and its gate pass (this chunk's factors are no longer read)
-                wait_history();
+                if (DELTA)
+                    wait_first_mmas();
+                else
+                    wait_history();
                 {
                     constexpr int NW = DELTA ? 192 : 256;
-                    constexpr int NQV = 1024 + 512 * NB;
+                    constexpr int NQK = DELTA ? 2048 : 1024;  // q chunks, then (delta) k chunks
+                    constexpr int NQV = NQK + 512 * NB;
                     constexpr int IT = (NQV + NW - 1) / NW;
                     const int wt = DELTA ? t - 64 : t;
                     uint4 raw[IT];
 #pragma unroll
                     for (int s4 = 0; s4 < IT; ++s4) {
                         const int i = wt + NW * s4;
+                        const int j = i & 1023;  // chunk of the q or k tile
                         raw[s4] = make_uint4(0, 0, 0, 0);
-                        if (i < 1024)
-                            raw[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + (i >> 9) * 16384 + (i & 511) * 16);
+                        if (i < NQK)
+                            raw[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + (j >> 9) * 16384 +
+                                                                       (i >> 10) * 8192 + (j & 511) * 16);
                         else if (i < NQV)
-                            raw[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_V + (i - 1024) * 16);
+                            raw[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_V + (i - NQK) * 16);
                     }
 #pragma unroll
                     for (int s4 = 0; s4 < IT; ++s4) {
                         const int i = wt + NW * s4;
+                        const int j = i & 1023;
                         float f[8];
                         unpack_bf16x8(raw[s4], f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(f[e]));
-                        if (i < 1024) {
-                            const int h = i >> 9, off = (i & 511) * 16;
+                        if (i < NQK) {
+                            // q -> Q< (i < 1024), k -> K< (delta): row l scaled by b_l = e^{G_l}
+                            const int h = j >> 9, off = (j & 511) * 16;
                             const float bl = (GATE == kGateScalar) ? ms.b[off >> 7] : 1.f;
 #pragma unroll
                             for (int e = 0; e < 8; ++e) f[e] *= bl;
-                            *reinterpret_cast<uint4 *>(sm + L::AT + h * 24576 + 8192 + off) = pack_h8(f);
+                            *reinterpret_cast<uint4 *>(sm + L::AT + h * 16384 + (i >> 10) * 8192 + off) = pack_h8(f);
                         } else if (i < NQV) {
-                            *reinterpret_cast<uint4 *>(sm + v16_slot<L, UPD, GATE>(buf) + (i - 1024) * 16) = pack_h8(f);
+                            *reinterpret_cast<uint4 *>(sm + v16_slot<L, UPD, GATE>(buf) + (i - NQK) * 16) = pack_h8(f);
                         }
                     }
                 }
@@ -581,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                             if (i0 + 3 > m) x[i0 + 3] = fmaf(-lv.w, xm, x[i0 + 3]);
                         }
                     }
-                    if (GATE != kGateChannel) wait_history();  // T2 of chunk r-1 has been read
+                    wait_history();  // T2 of chunk r-1 has been read
                     __syncwarp();
                     const float bt = bet[o + c];
 #pragma unroll
@@ -645,102 +661,57 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         rmax = fmaxf(rmax, fmaxf(fabsf(b0), fabsf(b1)));
                         *reinterpret_cast<uint32_t *>(t2 + sw128_off(row, c)) = pack_h2(b0, b1);
                     }
-                    named_bar(kSolveBar, 128);
-                    TC2_MARK(0, 8);
-                    // 32 -> 64: 8-column tile j = warp of T_BA = -T_BB (L_BA T_AA)
-                    const int jj = warp;
-                    float dx[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                }
+                named_bar(kPrepBar, 256);  // T_10 and T_32 are in Ls
+                TC2_MARK(0, 8);
+                {
+                    // 32 -> 64 on all eight warps: warp = (16-row tile mt, 8-column tile jj) of
+                    // T_BA = -T_BB (L_BA T_AA); the two warps of a column tile meet at a
+                    // 64-thread barrier to exchange their halves of X = L_BA T_AA
+                    const int mt = warp >> 2, jj = warp & 3;
+                    const int i0 = 32 + 16 * mt;
+                    float dx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         if (jj >= 2 && ks < 2) continue;  // T_AA[k < 16][c >= 16] = 0
                         const int k0 = 8 * ks;
-                        uint32_t b[2];
+                        uint32_t a[4], b[2];
                         b[0] = f2tf32(Ls[f32_swz(k0 + tq, 8 * jj + g, 64)]);
                         b[1] = f2tf32(Ls[f32_swz(k0 + tq + 4, 8 * jj + g, 64)]);
-#pragma unroll
-                        for (int mt = 0; mt < 2; ++mt) {
-                            const int i0 = 32 + 16 * mt;  // L[i0+i][k] = Ls[k][i0+i]
-                            uint32_t a[4];
-                            a[0] = f2tf32(Ls[f32_swz(k0 + tq, i0 + g, 64)]);
-                            a[1] = f2tf32(Ls[f32_swz(k0 + tq, i0 + g + 8, 64)]);
-                            a[2] = f2tf32(Ls[f32_swz(k0 + tq + 4, i0 + g, 64)]);
-                            a[3] = f2tf32(Ls[f32_swz(k0 + tq + 4, i0 + g + 8, 64)]);
-                            mma_tf32_16x8x8(dx[mt], a, b);
-                        }
+                        a[0] = f2tf32(Ls[f32_swz(k0 + tq, i0 + g, 64)]);  // L[i0+i][k] = Ls[k][i0+i]
+                        a[1] = f2tf32(Ls[f32_swz(k0 + tq, i0 + g + 8, 64)]);
+                        a[2] = f2tf32(Ls[f32_swz(k0 + tq + 4, i0 + g, 64)]);
+                        a[3] = f2tf32(Ls[f32_swz(k0 + tq + 4, i0 + g + 8, 64)]);
+                        mma_tf32_16x8x8(dx, a, b);
                     }
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        *reinterpret_cast<float2 *>(Ls + f32_swz(32 + 16 * mt + g, 8 * jj + 2 * tq, 64)) =
-                            make_float2(dx[mt][0], dx[mt][1]);
-                        *reinterpret_cast<float2 *>(Ls + f32_swz(32 + 16 * mt + g + 8, 8 * jj + 2 * tq, 64)) =
-                            make_float2(dx[mt][2], dx[mt][3]);
-                    }
-                    __syncwarp();
-                    float ex[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                    *reinterpret_cast<float2 *>(Ls + f32_swz(i0 + g, 8 * jj + 2 * tq, 64)) = make_float2(dx[0], dx[1]);
+                    *reinterpret_cast<float2 *>(Ls + f32_swz(i0 + g + 8, 8 * jj + 2 * tq, 64)) = make_float2(dx[2], dx[3]);
+                    named_bar(kPairBar + jj, 64);
+                    float ex[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
+                        if (mt == 0 && ks >= 2) continue;  // T_BB[i < 16][k >= 16] = 0
                         const int k0 = 8 * ks;
-                        uint32_t b[2];
+                        uint32_t a[4], b[2];
                         b[0] = f2tf32(Ls[f32_swz(32 + k0 + tq, 8 * jj + g, 64)]);
                         b[1] = f2tf32(Ls[f32_swz(32 + k0 + tq + 4, 8 * jj + g, 64)]);
-#pragma unroll
-                        for (int mt = 0; mt < 2; ++mt) {
-                            if (mt == 0 && ks >= 2) continue;  // T_BB[i < 16][k >= 16] = 0
-                            const int i0 = 32 + 16 * mt;
-                            uint32_t a[4];
-                            a[0] = f2tf32(Ls[f32_swz(i0 + g, 32 + k0 + tq, 64)]);
-                            a[1] = f2tf32(Ls[f32_swz(i0 + g + 8, 32 + k0 + tq, 64)]);
-                            a[2] = f2tf32(Ls[f32_swz(i0 + g, 32 + k0 + tq + 4, 64)]);
-                            a[3] = f2tf32(Ls[f32_swz(i0 + g + 8, 32 + k0 + tq + 4, 64)]);
-                            mma_tf32_16x8x8(ex[mt], a, b);
-                        }
+                        a[0] = f2tf32(Ls[f32_swz(i0 + g, 32 + k0 + tq, 64)]);
+                        a[1] = f2tf32(Ls[f32_swz(i0 + g + 8, 32 + k0 + tq, 64)]);
+                        a[2] = f2tf32(Ls[f32_swz(i0 + g, 32 + k0 + tq + 4, 64)]);
+                        a[3] = f2tf32(Ls[f32_swz(i0 + g + 8, 32 + k0 + tq + 4, 64)]);
+                        mma_tf32_16x8x8(ex, a, b);
                     }
                     const int cc = 8 * jj + 2 * tq;
                     const float bc0 = bet[cc], bc1 = bet[cc + 1];
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int row = 32 + 16 * mt + g + 8 * h;
-                            const float b0 = -ex[mt][2 * h] * bc0, b1 = -ex[mt][2 * h + 1] * bc1;
-                            rmax = fmaxf(rmax, fmaxf(fabsf(b0), fabsf(b1)));
-                            *reinterpret_cast<uint32_t *>(t2 + sw128_off(row, cc)) = pack_h2(b0, b1);
-                        }
-                }
-                fence_proxy_async_smem();
-                named_bar(kPrepBar, 256);
-                TC2_MARK(0, 9);
-                // ------------------------------------------------ a4: W = T2 K<
-                if (t == 0 && !ms.abort_flag) {
-                    tc_fence_after();
-                    const uint32_t tza = smem_u32(sm + L::TZA), at = smem_u32(sm + L::AT);
-                    constexpr uint32_t idw = idesc_f16(128, 128, 0, 0, 1);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_f16(tmem + TP, smem_desc_sw128(tza + k * 32, 16, 1024),
-                                smem_desc_sw128(at + 16384 + k * 2048, 24576, 1024), idw, k > 0);
-                    mma_commit(&ms.bar_w);
-                }
-                if (!mbar_wait(&ms.bar_w, ph)) note_timeout(ms, 3, r);
-                tc_fence_after();
-                if (sp < 2) {
-                    // W rows (lanes 0..63), this warp's 64-column half -> -W slot of that half
-#pragma unroll
-                    for (int c0 = 0; c0 < 64; c0 += 32) {
-                        float w[32];
-                        __syncwarp();
-                        tmem_ld32(lane_addr + TP + ch * 64 + c0, w);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            w[e] = -w[e];
-                            rmax = fmaxf(rmax, fabsf(w[e]));
-                        }
-#pragma unroll
-                        for (int e = 0; e < 32; e += 8)
-                            *reinterpret_cast<uint4 *>(sm + L::AT + ch * 24576 + sw128_off(row, c0 + e)) = pack_h8(w + e);
+                    for (int h = 0; h < 2; ++h) {
+                        const int row = i0 + g + 8 * h;
+                        const float b0 = -ex[2 * h] * bc0, b1 = -ex[2 * h + 1] * bc1;
+                        rmax = fmaxf(rmax, fmaxf(fabsf(b0), fabsf(b1)));
+                        *reinterpret_cast<uint32_t *>(t2 + sw128_off(row, cc)) = pack_h2(b0, b1);
                     }
                 }
+                TC2_MARK(0, 9);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -832,30 +803,62 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 if (GATE != kGateChannel && r + 1 < nchunks) issue_p1(r + 1);
                 const uint32_t at = smem_u32(sm + L::AT);
                 if (DELTA) {
-                    // [Z^T | O^T] = S [-W ; Q<]^T in one N = 128 chain (the two B tiles are
-                    // adjacent in each K half), then Z^T += V^T T2^T
+                    // [O^T | X^T] = S [Q< ; K<]^T in one N = 128 chain (the two B tiles are
+                    // adjacent in each key half); Z^T = V^T T2^T (U^T) alongside
                     const uint32_t v16 = smem_u32(sm + L::V16), tza = smem_u32(sm + L::TZA);
                     constexpr uint32_t id1w = idesc_f16(DVS, 128, 0, 0, 0);
                     constexpr uint32_t idu = idesc_f16(DVS, 64, 0, 1, 0);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_f16_ts(tmem + TZO, tmem + TS16 + k * 8,
-                                   smem_desc_sw128(at + (k >> 2) * 24576 + (k & 3) * 32, 16, 1024), id1w, k > 0);
+                        mma_f16_ts(tmem + TOX, tmem + TS16 + k * 8,
+                                   smem_desc_sw128(at + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024), id1w, k > 0);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_f16(tmem + TZO, smem_desc_sw128(v16 + k * 2048, 8192, 1024),
-                                smem_desc_sw128(tza + k * 32, 16, 1024), idu, 1);
+                        mma_f16(tmem + TZ, smem_desc_sw128(v16 + k * 2048, 8192, 1024),
+                                smem_desc_sw128(tza + k * 32, 16, 1024), idu, k > 0);
+                    mma_commit(&ms.bar_x);
                 } else {
                     constexpr uint32_t id1 = idesc_f16(DVS, 64, 0, 0, 0);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)  // O^T = S Q<^T
-                        mma_f16_ts(tmem + TZO + 64, tmem + TS16 + k * 8,
-                                   smem_desc_sw128(at + (k >> 2) * 24576 + 8192 + (k & 3) * 32, 16, 1024), id1,
-                                   k > 0);
+                        mma_f16_ts(tmem + TOX, tmem + TS16 + k * 8,
+                                   smem_desc_sw128(at + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024), id1, k > 0);
+                    mma_commit(&ms.bar_fA);
                 }
-                mma_commit(&ms.bar_fA);
             }
             TC2_MARK(256, 18);
+            if (DELTA) {
+                // history correction Z^T = U^T - (S K<^T) T2^T: X^T = S K<^T leaves TMEM as
+                // -X^T in fp16 (the A operand of the product with T2)
+                if (!mbar_wait(&ms.bar_x, ph)) note_timeout(ms, 3, r);
+                tc_fence_after();
+                {
+                    float x[64];
+                    __syncwarp();
+                    tmem_ld32(lane_addr + TOX + 64, x);
+                    tmem_ld32(lane_addr + TOX + 96, x + 32);
+                    tmem_wait_ld();
+                    uint32_t w[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        rmax = fmaxf(rmax, fmaxf(fabsf(x[2 * c]), fabsf(x[2 * c + 1])));
+                        w[c] = pack_h2(-x[2 * c], -x[2 * c + 1]);
+                    }
+                    tmem_st32(lane_addr + TZ16, w);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                named_bar(kStateBar, 128);
+                if (ts == 0 && !ms.abort_flag) {
+                    tc_fence_after();
+                    const uint32_t tza = smem_u32(sm + L::TZA);
+                    constexpr uint32_t idz = idesc_f16(DVS, 64, 0, 0, 0);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_f16_ts(tmem + TZ, tmem + TZ16 + k * 8, smem_desc_sw128(tza + k * 32, 16, 1024), idz, 1);
+                    mma_commit(&ms.bar_fA);
+                }
+            }
             if (!mbar_wait(&ms.bar_fA, ph)) note_timeout(ms, 7, r);
             TC2_MARK(256, 19);
             tc_fence_after();
@@ -863,8 +866,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 // Z^T -> fp16 A operand (tokens 2c, 2c+1 in column c)
                 float z[64];
                 __syncwarp();
-                tmem_ld32(lane_addr + TZO, z);
-                tmem_ld32(lane_addr + TZO + 32, z + 32);
+                tmem_ld32(lane_addr + TZ, z);
+                tmem_ld32(lane_addr + TZ + 32, z + 32);
                 tmem_wait_ld();
                 uint32_t w[32];
 #pragma unroll
@@ -889,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t za = tmem + TZ16 + k * 8;
-                        mma_f16_ts(tmem + TZO + 64, za, smem_desc_sw128(ap + k * 32, 16, 1024), id2, 1);
+                        mma_f16_ts(tmem + TOX, za, smem_desc_sw128(ap + k * 32, 16, 1024), id2, 1);
                         mma_f16_ts(tmem + TSM, za, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3, 1);
                     }
                 } else {
@@ -899,7 +902,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint64_t va = smem_desc_sw128(v16 + k * 2048, 8192, 1024);
-                        mma_f16(tmem + TZO + 64, va, smem_desc_sw128(ap + k * 32, 16, 1024), id2s, 1);
+                        mma_f16(tmem + TOX, va, smem_desc_sw128(ap + k * 32, 16, 1024), id2s, 1);
                         mma_f16(tmem + TSM, va, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3s, 1);
                     }
                 }
@@ -915,8 +918,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 // they queue behind the prep group's shared-memory traffic.
                 float ov[64];
                 __syncwarp();
-                tmem_ld32(lane_addr + TZO + 64, ov);
-                tmem_ld32(lane_addr + TZO + 96, ov + 32);
+                tmem_ld32(lane_addr + TOX, ov);
+                tmem_ld32(lane_addr + TOX + 32, ov + 32);
                 tmem_wait_ld();
                 if (ts == 0) bulk_wait_read0();  // the previous chunk's store has read the staging tile
                 named_bar(kStateBar, 128);
