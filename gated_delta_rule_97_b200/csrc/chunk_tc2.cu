@@ -66,7 +66,7 @@ constexpr int kThreads = 384;  // warps 0-7 prep, 8-11 state
 constexpr int C = kChunk;
 constexpr int DK = 128;
 constexpr float kFactorMaxDecay = 10.0f;
-constexpr int kPrepBar = 1, kStateBar = 2, kConvBar = 4, kPairBar = 5;  // kPairBar..kPairBar+3
+constexpr int kPrepBar = 1, kStateBar = 2, kConvBar = 4, kPairBar = 5, kVBar = 9;  // kPairBar..kPairBar+3
 
 struct Params {
     CUtensorMap q_map, k_map, v_map, g_map, o_map;
@@ -84,7 +84,7 @@ template <int DVS, int GATE>
 struct Smem {
     static constexpr int RAW_QK = 0;                                     // [Q0 K0 | Q1 K1] bf16
     static constexpr int RAW_V = RAW_QK + 32768;                         // V slice bf16
-    static constexpr int GCH = RAW_V + DVS * 128;                        // channel gate fp32 [64][128]
+    static constexpr int GCH = RAW_V + DVS * 128;                        // channel gate: 4 x [64][32] fp32, swizzled
     static constexpr int AT = GCH + (GATE == kGateChannel ? 32768 : 0);  // [Q< | K<] x 2 key halves
     static constexpr int KT = AT + 32768;                                // k e^{-G} fp16 / L^T fp32 scratch
     static constexpr int KR = KT + 16384;                                // K> fp16, 2 buffers
@@ -107,7 +107,7 @@ struct Misc {
     int abort_flag, range_flag, slow_chunk, abort_site;
     int p_abort, s_abort, pad0, pad1;
     uint32_t tmem_base, pad2[3];
-    uint64_t bar_tma, bar_p1, bar_x, bar_rdy, bar_fA, bar_fB0, bar_fB1, pad3;
+    uint64_t bar_tma, bar_p1, bar_x, bar_rdy, bar_fA, bar_fB0, bar_fB1, bar_tv;
 };
 
 template <typename M>
@@ -116,6 +116,13 @@ __device__ __forceinline__ void note_timeout(M &ms, int site, int r) {
 }
 
 constexpr uint32_t TP = 0, TZ = 64, TOX = 128, TSM = 256, TS16 = 384, TZ16 = 448;
+
+// Float index of gate element (token l, channel c) in the channel-gate tile: four
+// [64][32] fp32 sub-tiles loaded by TMA with the 128-byte swizzle (16-byte slot
+// XOR token % 8), so reads of one channel group across tokens spread over banks.
+__device__ __forceinline__ int gch_idx(int l, int c) {
+    return (c >> 5) * 2048 + l * 32 + ((((c & 31) >> 2) ^ (l & 7)) << 2) + (c & 3);
+}
 
 // Shared offset of chunk parity `buf`'s fp16 V tile.  Without the delta rule V is
 // an operand of the state's last MMAs, so it is double-buffered, the second copy in
@@ -129,6 +136,14 @@ template <int DVS, int UPD, int GATE, bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_constant__ Params p) {
     using L = Smem<DVS, GATE>;
     constexpr bool DELTA = (UPD == kDelta);
+    // P = [Q;K]K^T of a chunk is issued by the state group's MMA thread right after
+    // rdy when the prep group is the longer side (delta rule, scalar / no gate), else
+    // by the prep group itself (it then has slack; the channel gate's P also needs
+    // the converted operands)
+    constexpr bool kStateP1 = DELTA && GATE != kGateChannel;
+    // In the same modes the V tile has its own TMA barrier (bar_tv): its fp16
+    // conversion runs during the 16 -> 32 merge, after the q / k conversion window
+    constexpr bool kSplitV = DELTA && GATE != kGateChannel;
     constexpr int NB = DVS / 64;
     extern __shared__ unsigned char smraw[];
     // Align by an integer offset from the shared array itself, so that every access
@@ -147,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 
     if (t == 0) {
         mbar_init(&ms.bar_tma, 1);
+        mbar_init(&ms.bar_tv, 1);
         mbar_init(&ms.bar_p1, 1);
         mbar_init(&ms.bar_x, 1);
         mbar_init(&ms.bar_rdy, 1);
@@ -224,20 +240,31 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             }
             if (DELTA && t >= 128 && t < 128 + C) ms.beta[r & 1][t - 128] = bpre;
         };
+        // q, k (+ the channel gate tile) on bar_tma; v on bar_tv when split, else also on bar_tma
+        auto issue_tma_v = [&](int r, uint64_t *bar) {
+            for (int j = 0; j < NB; ++j)
+                tma_load_3d(sm + L::RAW_V + j * 8192, &p.v_map, v0 + j * 64, r * C, bh, bar);
+        };
         auto issue_tma = [&](int r) {
             const int t0 = r * C;
-            const uint32_t bytes = 32768 + DVS * 128 + (GATE == kGateChannel ? 32768 : 0);
+            const uint32_t bytes = 32768 + (kSplitV ? 0 : DVS * 128) + (GATE == kGateChannel ? 32768 : 0);
             mbar_arrive_expect_tx(&ms.bar_tma, bytes);
             for (int h = 0; h < 2; ++h) {
                 tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, t0, bh, &ms.bar_tma);
                 tma_load_3d(sm + L::RAW_QK + h * 16384 + 8192, &p.k_map, h * 64, t0, bh, &ms.bar_tma);
             }
-            for (int j = 0; j < NB; ++j)
-                tma_load_3d(sm + L::RAW_V + j * 8192, &p.v_map, v0 + j * 64, t0, bh, &ms.bar_tma);
+            if (!kSplitV) issue_tma_v(r, &ms.bar_tma);
             if (GATE == kGateChannel)
                 for (int j = 0; j < 4; ++j) tma_load_3d(sm + L::GCH + j * 8192, &p.g_map, j * 32, t0, bh, &ms.bar_tma);
         };
-        if (t == 0 && nchunks > 0) issue_tma(0);
+        auto issue_tma_split_v = [&](int r) {
+            mbar_arrive_expect_tx(&ms.bar_tv, DVS * 128);
+            issue_tma_v(r, &ms.bar_tv);
+        };
+        if (t == 0 && nchunks > 0) {
+            issue_tma(0);
+            if (kSplitV) issue_tma_split_v(0);
+        }
         if (nchunks > 0) {
             load_gate_beta(0);
             if (GATE != kGateChannel) {
@@ -255,25 +282,37 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             TC2_MARK(0, 0);
             if (!mbar_wait(&ms.bar_tma, ph)) note_timeout(ms, 1, r);
             TC2_MARK(0, 1);
+            if (!kStateP1 && GATE != kGateChannel && t == 0 && !ms.abort_flag) {
+                tc_fence_after();
+                const uint32_t qk = smem_u32(sm + L::RAW_QK);
+                constexpr uint32_t id = idesc_f16(128, 64, 1, 0, 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_f16(tmem + TP, smem_desc_sw128(qk + ko, 16, 1024), smem_desc_sw128(qk + 8192 + ko, 16, 1024),
+                            id, k > 0);
+                }
+                mma_commit(&ms.bar_p1);
+            }
             if (GATE == kGateChannel) {
                 // ------------------------------------------------ a1: channel gate prefix
                 // channel c, token half hf: prefix over 32 tokens, then join the halves
                 const int c = t & 127, hf = t >> 7;
-                float *gcol = reinterpret_cast<float *>(sm + L::GCH + (c >> 5) * 8192) + (c & 31);
+                float *gt = reinterpret_cast<float *>(sm + L::GCH);
                 float gv[32];
 #pragma unroll
-                for (int l = 0; l < 32; ++l) gv[l] = gcol[(32 * hf + l) * 32];
+                for (int l = 0; l < 32; ++l) gv[l] = gt[gch_idx(32 * hf + l, c)];
 #pragma unroll
                 for (int l = 1; l < 32; ++l) gv[l] += gv[l - 1];
                 if (hf == 0) {
 #pragma unroll
-                    for (int l = 0; l < 32; ++l) gcol[l * 32] = gv[l];
+                    for (int l = 0; l < 32; ++l) gt[gch_idx(l, c)] = gv[l];
                 }
                 named_bar(kPrepBar, 256);
                 if (hf == 1) {
-                    const float base = gcol[31 * 32];
+                    const float base = gt[gch_idx(31, c)];
 #pragma unroll
-                    for (int l = 0; l < 32; ++l) gcol[(32 + l) * 32] = gv[l] + base;
+                    for (int l = 0; l < 32; ++l) gt[gch_idx(32 + l, c)] = gv[l] + base;
                     ms.GC[c] = gv[31] + base;
                     dec[buf * 128 + c] = __expf(gv[31] + base);
                 }
@@ -349,17 +388,39 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
                         for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fmaxf(fabsf(qf[e]), fabsf(kf[e])));
                         if (GATE == kGateChannel) {
-                            const float *gg = reinterpret_cast<const float *>(sm + L::GCH + (c0 >> 5) * 8192) + l * 32 + (c0 & 31);
+                            const float *gt = reinterpret_cast<const float *>(sm + L::GCH);
+                            const float4 g0 = *reinterpret_cast<const float4 *>(gt + gch_idx(l, c0));
+                            const float4 g1 = *reinterpret_cast<const float4 *>(gt + gch_idx(l, c0 + 4));
+                            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
                             float kt[8];
+                            if (!slow) {
+                                // e^{G_C} per channel was stored by the prefix pass; here
+                                // e^{G_C - G} = e^{G_C} e^{-G} (e^{-G} <= e^{10})
+                                const float4 d0 = *reinterpret_cast<const float4 *>(dec + buf * 128 + c0);
+                                const float4 d1 = *reinterpret_cast<const float4 *>(dec + buf * 128 + c0 + 4);
+                                const float egc[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const float G = gg[e];
-                                const float eg = __expf(G), emg = __expf(-G);
-                                ql[e] = qf[e] * eg;
-                                kl[e] = kf[e] * eg;
-                                kt[e] = slow ? 0.f : kf[e] * emg;
-                                kr[e] = kf[e] * __expf(ms.GC[c0 + e] - G);
-                                rmax = fmaxf(rmax, fabsf(kt[e]));
+                                for (int e = 0; e < 8; ++e) {
+                                    const float x = gg[e] * 1.4426950408889634f;  // log2(e)
+                                    const float eg = ex2_approx(x), emg = ex2_approx(-x);
+                                    ql[e] = qf[e] * eg;
+                                    kl[e] = kf[e] * eg;
+                                    kt[e] = kf[e] * emg;
+                                    kr[e] = kt[e] * egc[e];
+                                    rmax = fmaxf(rmax, fabsf(kt[e]));
+                                }
+                            } else {
+                                // strong decay in this chunk: no k e^{-G} operand (the exact
+                                // fp32 path evaluates P), e^{G_C - G} directly
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    const float G = gg[e];
+                                    const float eg = __expf(G);
+                                    ql[e] = qf[e] * eg;
+                                    kl[e] = kf[e] * eg;
+                                    kt[e] = 0.f;
+                                    kr[e] = kf[e] * __expf(ms.GC[c0 + e] - G);
+                                }
                             }
                             *reinterpret_cast<uint4 *>(sm + L::KT + h * 8192 + off) = pack_h8(kt);
                         } else {
@@ -458,8 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                                     __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xrow + h * 16384 + ox));
                                 const float kv = __bfloat162float(
                                     *reinterpret_cast<const __nv_bfloat16 *>(sm + L::RAW_QK + h * 16384 + 8192 + om));
-                                const float *gc = reinterpret_cast<const float *>(sm + L::GCH + (c >> 5) * 8192);
-                                acc = fmaf(xv * kv, __expf(gc[l * 32 + (c & 31)] - gc[m * 32 + (c & 31)]), acc);
+                                const float *gt = reinterpret_cast<const float *>(sm + L::GCH);
+                                acc = fmaf(xv * kv, __expf(gt[gch_idx(l, c)] - gt[gch_idx(m, c)]), acc);
                             }
                         }
                         pr[e] = acc;
@@ -520,10 +581,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     wait_first_mmas();
                 else
                     wait_history();
+                TC2_MARK(64, 11);
                 {
                     constexpr int NW = DELTA ? 192 : 256;
                     constexpr int NQK = DELTA ? 2048 : 1024;  // q chunks, then (delta) k chunks
-                    constexpr int NQV = NQK + 512 * NB;
+                    constexpr int NQV = NQK + (kSplitV ? 0 : 512 * NB);
                     constexpr int IT = (NQV + NW - 1) / NW;
                     const int wt = DELTA ? t - 64 : t;
                     uint4 raw[IT];
@@ -558,8 +620,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         }
                     }
                 }
+                TC2_MARK(64, 12);
                 fence_proxy_async_smem();
                 named_bar(kConvBar, DELTA ? 192 : 256);
+                TC2_MARK(64, 13);
                 if (t == 224 && r + 1 < nchunks && !ms.abort_flag) issue_tma(r + 1);
                 if (!DELTA && r + 1 < nchunks) {
                     gate_pass(r + 1);
@@ -597,6 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                             if (i0 + 3 > m) x[i0 + 3] = fmaf(-lv.w, xm, x[i0 + 3]);
                         }
                     }
+                    TC2_MARK(0, 14);
                     wait_history();  // T2 of chunk r-1 has been read
                     __syncwarp();
                     const float bt = bet[o + c];
@@ -611,11 +676,35 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 named_bar(kPrepBar, 256);
                 TC2_MARK(0, 7);
                 const int g = lane >> 2, tq = lane & 3;  // mma fragment coordinates
-                if (GATE != kGateChannel && warp >= 4 && r + 1 < nchunks) {
+                if (GATE != kGateChannel && warp >= 4) {
                     // next chunk's gate pass (this chunk's factors were last read by the
                     // conversions before the barrier above)
-                    gate_pass(r + 1);
-                    if (r + 2 < nchunks) load_gate_beta(r + 2);
+                    if (r + 1 < nchunks) {
+                        gate_pass(r + 1);
+                        if (r + 2 < nchunks) load_gate_beta(r + 2);
+                    }
+                    if (kSplitV) {
+                        // V -> fp16 (its slot was released with bar_x(r-1), waited in the
+                        // window), then the next chunk's v load
+                        if (!mbar_wait(&ms.bar_tv, ph)) note_timeout(ms, 13, r);
+                        constexpr int NV = 512 * NB, ITV = NV / 128;
+                        const int wt = t - 128;
+                        uint4 raw[ITV];
+#pragma unroll
+                        for (int s4 = 0; s4 < ITV; ++s4)
+                            raw[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_V + (wt + 128 * s4) * 16);
+#pragma unroll
+                        for (int s4 = 0; s4 < ITV; ++s4) {
+                            float f[8];
+                            unpack_bf16x8(raw[s4], f);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(f[e]));
+                            *reinterpret_cast<uint4 *>(sm + L::V16 + (wt + 128 * s4) * 16) = pack_h8(f);
+                        }
+                        fence_proxy_async_smem();
+                        named_bar(kVBar, 128);
+                        if (t == 224 && r + 1 < nchunks && !ms.abort_flag) issue_tma_split_v(r + 1);
+                    }
                 }
                 if (warp < 4) {
                     // 16 -> 32 for the block pairs (1,0) and (3,2); warp = (pair, 8-column tile)
@@ -739,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             }
             mma_commit(&ms.bar_p1);
         };
-        if (GATE != kGateChannel && ts == 0 && nchunks > 0) issue_p1(0);
+        if (kStateP1 && ts == 0 && nchunks > 0) issue_p1(0);
         const int vrow = (DVS == 128) ? ts : (sp * 16 + lane);
         const size_t srow = ((size_t)bh * dv + v0 + (has_row ? vrow : 0)) * DK;
         // initial state: fp32 master and fp16 operand copy (lane = value row)
@@ -800,7 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 tc_fence_after();
                 // P1 of the next chunk goes to the tensor pipe first: the prep group
                 // released TP with rdy(r) and waits on P1 before its A'/L pass
-                if (GATE != kGateChannel && r + 1 < nchunks) issue_p1(r + 1);
+                if (kStateP1 && r + 1 < nchunks) issue_p1(r + 1);
                 const uint32_t at = smem_u32(sm + L::AT);
                 if (DELTA) {
                     // [O^T | X^T] = S [Q< ; K<]^T in one N = 128 chain (the two B tiles are
@@ -824,6 +913,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         mma_f16_ts(tmem + TOX, tmem + TS16 + k * 8,
                                    smem_desc_sw128(at + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024), id1, k > 0);
                     mma_commit(&ms.bar_fA);
+                    // without the delta rule nothing sits between: O^T += V^T A'^T and
+                    // S += V^T K> follow at once (S is read from its fp16 copy above)
+                    const uint32_t tza = smem_u32(sm + L::TZA), kr = smem_u32(sm + L::KR) + buf * 16384;
+                    const uint32_t ap = tza + 8192 * (1 + buf);
+                    const uint32_t v16 = smem_u32(sm + v16_slot<L, UPD, GATE>(buf));
+                    constexpr uint32_t id2s = idesc_f16(DVS, 64, 0, 1, 0);
+                    constexpr uint32_t id3s = idesc_f16(DVS, 128, 0, 1, 1);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t va = smem_desc_sw128(v16 + k * 2048, 8192, 1024);
+                        mma_f16(tmem + TOX, va, smem_desc_sw128(ap + k * 32, 16, 1024), id2s, 1);
+                        mma_f16(tmem + TSM, va, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3s, 1);
+                    }
+                    mma_commit(buf ? &ms.bar_fB1 : &ms.bar_fB0);
                 }
             }
             TC2_MARK(256, 18);
@@ -859,7 +962,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     mma_commit(&ms.bar_fA);
                 }
             }
-            if (!mbar_wait(&ms.bar_fA, ph)) note_timeout(ms, 7, r);
+            if (DELTA) {
+                if (!mbar_wait(&ms.bar_fA, ph)) note_timeout(ms, 7, r);
+            }
             TC2_MARK(256, 19);
             tc_fence_after();
             if (DELTA) {
@@ -882,29 +987,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             }
             TC2_MARK(256, 20);
             uint64_t *fb = buf ? &ms.bar_fB1 : &ms.bar_fB0;
-            if (ts == 0 && !ms.abort_flag) {
+            if (DELTA && ts == 0 && !ms.abort_flag) {
                 tc_fence_after();
                 const uint32_t tza = smem_u32(sm + L::TZA), kr = smem_u32(sm + L::KR) + buf * 16384;
                 const uint32_t ap = tza + 8192 * (1 + buf);
                 constexpr uint32_t id2 = idesc_f16(DVS, 64, 0, 0, 0);
                 constexpr uint32_t id3 = idesc_f16(DVS, 128, 0, 0, 1);
-                if (DELTA) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t za = tmem + TZ16 + k * 8;
-                        mma_f16_ts(tmem + TOX, za, smem_desc_sw128(ap + k * 32, 16, 1024), id2, 1);
-                        mma_f16_ts(tmem + TSM, za, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3, 1);
-                    }
-                } else {
-                    const uint32_t v16 = smem_u32(sm + v16_slot<L, UPD, GATE>(buf));
-                    constexpr uint32_t id2s = idesc_f16(DVS, 64, 0, 1, 0);
-                    constexpr uint32_t id3s = idesc_f16(DVS, 128, 0, 1, 1);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t va = smem_desc_sw128(v16 + k * 2048, 8192, 1024);
-                        mma_f16(tmem + TOX, va, smem_desc_sw128(ap + k * 32, 16, 1024), id2s, 1);
-                        mma_f16(tmem + TSM, va, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3s, 1);
-                    }
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t za = tmem + TZ16 + k * 8;
+                    mma_f16_ts(tmem + TOX, za, smem_desc_sw128(ap + k * 32, 16, 1024), id2, 1);
+                    mma_f16_ts(tmem + TSM, za, smem_desc_sw128(kr + k * 2048, 8192, 1024), id3, 1);
                 }
                 mma_commit(fb);
             }
@@ -1079,7 +1172,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
         !make_map_3d(&prm.v_map, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.dv, T, BH, 64, 64, 1, true))
         return (int)cudaErrorInvalidValue;
     if (d->gate == GDN_GATE_CHANNEL &&
-        !make_map_3d(&prm.g_map, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, T, BH, 32, 64, 1, false))
+        !make_map_3d(&prm.g_map, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, T, BH, 32, 64, 1, true))
         return (int)cudaErrorInvalidValue;
     const int dvs = tc2_slice(d);
     const bool ob = d->out_dtype == GDN_BF16;

@@ -32,6 +32,14 @@ __device__ __forceinline__ int f32_swz(int r, int c, int ld) {
     return r * ld + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3);
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32; relative error near
+// the fp32 ulp, flushes subnormal results to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // fp32 -> tf32 (round to nearest, ties away), as a 32-bit operand register.
 __device__ __forceinline__ uint32_t f2tf32(float x) {
     uint32_t r;
