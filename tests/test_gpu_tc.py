@@ -57,6 +57,17 @@ def test_tc_ragged_lengths(T):
     check(w, make_prefill_inputs(w))
 
 
+@pytest.mark.parametrize("update,gate", MODES)
+@pytest.mark.parametrize("dv", [64, 128])
+@pytest.mark.parametrize("T", [1, 65, 129])
+def test_tc_short_and_ragged_all_modes(update, gate, dv, T):
+    # one, two and three chunks: the pipeline's prologue, the chunk-parity buffers
+    # (A', K>, beta, the decay factors, V without the delta rule) and the separate v
+    # load all start from their first phases here
+    w = workload(update, gate, T=T, B=1, H=2, dv=dv, seed=11)
+    check(w, make_prefill_inputs(w))
+
+
 @pytest.mark.parametrize("update,gate", [("delta", "scalar"), ("additive", "none"), ("delta", "none")])
 def test_tc_wide_value_slice(update, gate):
     """Enough heads that each CTA takes all 128 value rows of its head."""
