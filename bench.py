@@ -273,6 +273,41 @@ def time_decode(w, n_steps, torch, gdn, warmup=3):
     return e0.elapsed_time(e1) / n_steps
 
 
+def time_decode_multi(w, T, n_calls, torch, gdn, warmup=3):
+    """Device time of ``n_calls`` in-place decode calls of ``T`` tokens each (the
+    state is read and written once per call); returns ms/call."""
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    S = to_dev(make_decode_state(w), torch.float32, torch)
+    flat = []
+    for _, blk in iter_decode_blocks(w, n_calls * T):
+        flat += blk
+    dev_in = []
+    for c in range(n_calls):
+        grp = flat[c * T:(c + 1) * T]
+        dev_in.append({k: (None if grp[0][k] is None else
+                           to_dev(np.concatenate([s[k] for s in grp], axis=2),
+                                  dt if k in ("q", "k", "v") else torch.float32, torch)) for k in grp[0]})
+    o = torch.empty((w.B, w.H, T, w.dv), dtype=torch.float32, device="cuda")
+
+    def run(s):
+        gdn.decode_step(s["q"], s["k"], s["v"], s["g"], s["beta"], S, update=w.update, gate=w.gate, o=o)
+
+    for i in range(warmup):
+        run(dev_in[i % len(dev_in)])
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in dev_in:
+        run(s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if gdn.device_status() != 0:
+        raise RuntimeError("device status after multi-token decode")
+    del dev_in, S
+    return e0.elapsed_time(e1) / n_calls
+
+
 def max_over_ranks(value, dist, device):
     """Max of a per-rank float over all ranks (timing only; not on the data path)."""
     if dist is None:
@@ -385,6 +420,18 @@ def run_ours(args):
                         "frac": dbytes / (ms_d * 1e-3) / 1e9 / peaks["hbm_gbs"],
                         "bytes_per_step": dbytes, "tokens_per_s": wd.n_heads / wd.H * world / (ms_d * 1e-3)}
     result["gpu_launches"] += n_dec
+    # T = 4 tokens per call through the same entry point (state read / written once per call)
+    T_mt, n_mt = 4, (25 if args.quick else 100)
+    ms_mt = max_over_ranks(time_decode_multi(wd, T_mt, n_mt, torch, gdn), dist, "cuda")
+    in_b = 2 if wd.dtype == "bf16" else 4
+    per_tok = wd.n_heads * ((2 * wd.dk + wd.dv) * in_b + 4 * wd.dv + 8)
+    mt_bytes = wd.n_heads * wd.dv * wd.dk * 4 * 2 + T_mt * per_tok
+    result["decode"]["multi_token"] = {"tokens_per_call": T_mt, "calls": n_mt, "ms_per_call": ms_mt,
+                                       "value": mt_bytes / (ms_mt * 1e-3) / 1e9, "unit": "GB/s",
+                                       "frac": mt_bytes / (ms_mt * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                       "bytes_per_call": mt_bytes,
+                                       "tokens_per_s": wd.B * T_mt * world / (ms_mt * 1e-3)}
+    result["gpu_launches"] += n_mt
 
     if not args.quick:
         others = {}

@@ -26,6 +26,7 @@ GATES = {"none": 0, "scalar": 1, "channel": 2}
 ALGOS = {"auto": 0, "simt": 1, "tc": 2, "tc_seq": 3}
 F32, BF16 = 0, 1
 
+DECODE_MAX_T = 16  # GDN_DECODE_MAX_T
 GDN_OK = 0
 ERRORS = {-1: "GDN_ERR_ARG", -2: "GDN_ERR_ALIGN", -3: "GDN_ERR_UNSUPPORTED", -4: "GDN_ERR_CUDA",
           -5: "GDN_ERR_TIMEOUT", -6: "GDN_ERR_RANGE"}
@@ -178,32 +179,33 @@ def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=No
 
 
 def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, stream=None):
-    """One decode step (gdn_decode_step); S [B,H,dv,dk] is updated in place.
+    """T decode steps (gdn_decode_step, 1 <= T <= DECODE_MAX_T, usually 1); S
+    [B,H,dv,dk] is updated in place and read / written once for the T tokens.
 
-    q, k [B,H,1,dk]; v [B,H,1,dv]; g [B,H,1] or [B,H,1,dk] or None; beta [B,H,1].
-    Returns o [B,H,1,dv].
+    q, k [B,H,T,dk]; v [B,H,T,dv]; g [B,H,T] or [B,H,T,dk] or None; beta [B,H,T].
+    Returns o [B,H,T,dv].
     """
     import torch
 
     B, H, T, dk = q.shape
     dv = v.shape[-1]
-    if T != 1:
-        raise ValueError("decode_step takes one token (T == 1)")
-    _check(q, "q", (B, H, 1, dk))
-    _check(k, "k", (B, H, 1, dk), q.dtype)
-    _check(v, "v", (B, H, 1, dv), q.dtype)
+    if not 1 <= T <= DECODE_MAX_T:
+        raise ValueError("decode_step takes 1..%d tokens (gdn_chunk_fwd for longer runs)" % DECODE_MAX_T)
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
     if gate == "scalar":
-        _check(g, "g", (B, H, 1), torch.float32)
+        _check(g, "g", (B, H, T), torch.float32)
     elif gate == "channel":
-        _check(g, "g", (B, H, 1, dk), torch.float32)
-    _check(beta, "beta", (B, H, 1), torch.float32)
+        _check(g, "g", (B, H, T, dk), torch.float32)
+    _check(beta, "beta", (B, H, T), torch.float32)
     _check(S, "S", (B, H, dv, dk), torch.float32)
     if out_dtype is None:
         out_dtype = o.dtype if o is not None else torch.float32
     if o is None:
-        o = torch.empty((B, H, 1, dv), dtype=out_dtype, device=q.device)
-    _check(o, "o", (B, H, 1, dv), out_dtype)
-    d = make_desc(B, H, 1, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype))
+        o = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
+    _check(o, "o", (B, H, T, dv), out_dtype)
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype))
     rc = load().gdn_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
                                 _ptr(o), _stream(stream))
     if rc != GDN_OK:

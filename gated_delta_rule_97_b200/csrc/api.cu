@@ -141,9 +141,10 @@ extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k
                                const float *beta, float *S, void *o, void *stream) {
     int rc = validate_common(d);
     if (rc != GDN_OK) return rc;
-    if (d->T != 1) return GDN_ERR_ARG;
+    if (d->T < 0) return GDN_ERR_ARG;
+    if (d->T > GDN_DECODE_MAX_T) return GDN_ERR_UNSUPPORTED;
     const long BH = (long)d->B * d->H;
-    if (BH == 0) return GDN_OK;
+    if (BH == 0 || d->T == 0) return GDN_OK;
     if (!q || !k || !v || !S || !o) return GDN_ERR_ARG;
     if (d->update == GDN_DELTA && !beta) return GDN_ERR_ARG;
     if ((d->gate != GDN_GATE_NONE) != (g != nullptr)) return GDN_ERR_ARG;
@@ -151,14 +152,15 @@ extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     const size_t n_S = (size_t)BH * d->dv * d->dk;
-    const size_t no = (size_t)BH * d->dv * elem_size(d->out_dtype);
+    const size_t BT = (size_t)BH * d->T;
+    const size_t no = BT * d->dv * elem_size(d->out_dtype);
     const size_t es = elem_size(d->dtype);
-    if (overlaps(o, no, S, n_S * 4) || overlaps(o, no, q, BH * d->dk * es) || overlaps(o, no, k, BH * d->dk * es) ||
-        overlaps(o, no, v, BH * d->dv * es))
+    if (overlaps(o, no, S, n_S * 4) || overlaps(o, no, q, BT * d->dk * es) || overlaps(o, no, k, BT * d->dk * es) ||
+        overlaps(o, no, v, BT * d->dv * es))
         return GDN_ERR_ARG;
     gdn::DecodeArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.o = o;
-    a.BH = (int)BH; a.dk = d->dk; a.dv = d->dv;
+    a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
     return from_cuda(gdn_launch_decode(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16,
                                        static_cast<cudaStream_t>(stream)));
 }

@@ -46,12 +46,12 @@ struct ChunkArgs {
 };
 
 struct DecodeArgs {
-    const void *q, *k, *v;   // [BH,dk] / [BH,dv]
-    const float *g;          // [BH] or [BH,dk] or null
-    const float *beta;       // [BH] or null
+    const void *q, *k, *v;   // [BH,T,dk] / [BH,T,dv]
+    const float *g;          // [BH,T] or [BH,T,dk] or null
+    const float *beta;       // [BH,T] or null
     float *S;                // [BH,dv,dk] in/out
-    void *o;                 // [BH,dv]
-    int BH, dk, dv;
+    void *o;                 // [BH,T,dv]
+    int BH, T, dk, dv;
 };
 
 }  // namespace gdn

@@ -1,4 +1,4 @@
-// Decode: one recurrent step per (b,h), state updated in place.
+// Decode: T (>= 1, small) recurrent steps per (b,h), state updated in place.
 //
 // Bandwidth-bound rank-1 update ("Linear Attention, Visualized", "Optional:
 // Linear attention as an RNN"; per-token recurrences of the Mamba-2, DeltaNet,
@@ -49,6 +49,38 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+template <int DK, int UPD, int GATE, typename TIn>
+struct StepIn {
+    static constexpr int V = DK / 32;
+    float qq[V], kk[V], al[V], bt, vv[kRowsPerWarp];
+    __device__ void load(const DecodeArgs &a, long bh, int t, int c0, int i0) {
+        const long tok = bh * a.T + t;
+        const TIn *qp = static_cast<const TIn *>(a.q) + tok * DK + c0;
+        const TIn *kp = static_cast<const TIn *>(a.k) + tok * DK + c0;
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            qq[e] = to_f32(qp[e]);
+            kk[e] = to_f32(kp[e]);
+            al[e] = 1.f;
+        }
+        if (GATE == kGateScalar) {
+            const float x = __expf(a.g[tok]);
+#pragma unroll
+            for (int e = 0; e < V; ++e) al[e] = x;
+        } else if (GATE == kGateChannel) {
+#pragma unroll
+            for (int e = 0; e < V; ++e) al[e] = __expf(a.g[tok * DK + c0 + e]);
+        }
+        bt = (UPD == kDelta) ? a.beta[tok] : 0.f;
+        const TIn *vp = static_cast<const TIn *>(a.v) + tok * a.dv + i0;
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) vv[r] = to_f32(vp[r]);
+    }
+};
+
+// T >= 1 tokens per call: the state rows stay in registers across the tokens
+// (read and written once); the next token's inputs are loaded while the current
+// one is applied.
 template <int DK, int UPD, int GATE, typename TIn, typename TOut>
 __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
     constexpr int V = DK / 32;
@@ -65,63 +97,48 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r) VecF<V>::load(Srow + (size_t)r * DK, s[r]);
 
-    const TIn *qp = static_cast<const TIn *>(a.q) + bh * DK + c0;
-    const TIn *kp = static_cast<const TIn *>(a.k) + bh * DK + c0;
-    float qq[V], kk[V], al[V];
+    StepIn<DK, UPD, GATE, TIn> cur, nxt;
+    cur.load(a, bh, 0, c0, i0);
+#pragma unroll 1
+    for (int t = 0; t < a.T; ++t) {
+        if (t + 1 < a.T) nxt.load(a, bh, t + 1, c0, i0);
+        float kq = 0.f;
 #pragma unroll
-    for (int e = 0; e < V; ++e) {
-        qq[e] = to_f32(qp[e]);
-        kk[e] = to_f32(kp[e]);
-        al[e] = 1.f;
-    }
-    if (GATE == kGateScalar) {
-        const float x = __expf(a.g[bh]);
-#pragma unroll
-        for (int e = 0; e < V; ++e) al[e] = x;
-    } else if (GATE == kGateChannel) {
-#pragma unroll
-        for (int e = 0; e < V; ++e) al[e] = __expf(a.g[bh * DK + c0 + e]);
-    }
-    const float bt = (UPD == kDelta) ? a.beta[bh] : 0.f;
-    const TIn *vp = static_cast<const TIn *>(a.v) + bh * a.dv + i0;
-    float vv[kRowsPerWarp];
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) vv[r] = to_f32(vp[r]);
+        for (int e = 0; e < V; ++e) kq = fmaf(cur.kk[e], cur.qq[e], kq);
+        kq = warp_sum(kq);
 
-    float kq = 0.f;
+        float outv[kRowsPerWarp];
 #pragma unroll
-    for (int e = 0; e < V; ++e) kq = fmaf(kk[e], qq[e], kq);
-    kq = warp_sum(kq);
-
-    float outv[kRowsPerWarp];
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            float p = 0.f, rr = 0.f;
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        float p = 0.f, rr = 0.f;
+            for (int e = 0; e < V; ++e) {
+                s[r][e] *= cur.al[e];
+                p = fmaf(s[r][e], cur.kk[e], p);
+                rr = fmaf(s[r][e], cur.qq[e], rr);
+            }
+            // two independent butterfly sums, interleaved
 #pragma unroll
-        for (int e = 0; e < V; ++e) {
-            s[r][e] *= al[e];
-            p = fmaf(s[r][e], kk[e], p);
-            rr = fmaf(s[r][e], qq[e], rr);
+            for (int off = 16; off > 0; off >>= 1) {
+                p += __shfl_xor_sync(0xffffffffu, p, off);
+                rr += __shfl_xor_sync(0xffffffffu, rr, off);
+            }
+            const float u = (UPD == kDelta) ? cur.bt * (cur.vv[r] - p) : cur.vv[r];
+#pragma unroll
+            for (int e = 0; e < V; ++e) s[r][e] = fmaf(u, cur.kk[e], s[r][e]);
+            outv[r] = fmaf(u, kq, rr);
         }
-        // two independent butterfly sums, interleaved
+        if (lane < kRowsPerWarp) {
+            float x = outv[0];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            p += __shfl_xor_sync(0xffffffffu, p, off);
-            rr += __shfl_xor_sync(0xffffffffu, rr, off);
+            for (int r = 1; r < kRowsPerWarp; ++r)
+                if (lane == r) x = outv[r];
+            static_cast<TOut *>(a.o)[(bh * a.T + t) * a.dv + i0 + lane] = from_f32<TOut>(x);
         }
-        const float u = (UPD == kDelta) ? bt * (vv[r] - p) : vv[r];
-#pragma unroll
-        for (int e = 0; e < V; ++e) s[r][e] = fmaf(u, kk[e], s[r][e]);
-        VecF<V>::store(Srow + (size_t)r * DK, s[r]);
-        outv[r] = fmaf(u, kq, rr);
+        cur = nxt;
     }
-    if (lane < kRowsPerWarp) {
-        float x = outv[0];
 #pragma unroll
-        for (int r = 1; r < kRowsPerWarp; ++r)
-            if (lane == r) x = outv[r];
-        static_cast<TOut *>(a.o)[bh * a.dv + i0 + lane] = from_f32<TOut>(x);
-    }
+    for (int r = 0; r < kRowsPerWarp; ++r) VecF<V>::store(Srow + (size_t)r * DK, s[r]);
 }
 
 template <int DK, int UPD, int GATE, typename TIn, typename TOut>

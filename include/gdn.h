@@ -54,6 +54,9 @@ extern "C" {
 #define GDN_ERR_TIMEOUT (-5)     /* device status: a bounded wait in a kernel ran out */
 #define GDN_ERR_RANGE (-6)       /* device status: an fp16 tensor-core operand overflowed */
 
+/* Largest token count of one gdn_decode_step call (longer runs: gdn_chunk_fwd). */
+#define GDN_DECODE_MAX_T 16
+
 /* Write rule.  ADDITIVE: S += v k^T, no gate ("Naive linear attention").
  * DECAY: S = S Diag(alpha) + v k^T, gate required (RetNet / Mamba-2 / GLA).
  * DELTA: the gated delta rule above; any gate (DeltaNet / GDN / KDA). */
@@ -111,22 +114,26 @@ int gdn_chunk_fwd(const gdn_desc_t *desc, const void *q, const void *k, const vo
                   void *stream);
 
 /*
- * gdn_decode_step -- decode: one recurrent step (T == 1) for every (b,h), with
- * the state updated in place ("Optional: Linear attention as an RNN": fixed
- * state, constant work per token; the per-token recurrences of the RetNet,
- * Mamba-2, DeltaNet, GDN, GLA and KDA sections).  A bandwidth-bound rank-1
- * update: per state row i, with a = alpha_t,
+ * gdn_decode_step -- decode: T recurrent steps (1 <= T <= GDN_DECODE_MAX_T,
+ * usually 1) for every (b,h), with the state updated in place ("Optional:
+ * Linear attention as an RNN": fixed state, constant work per token; the
+ * per-token recurrences of the RetNet, Mamba-2, DeltaNet, GDN, GLA and KDA
+ * sections).  A bandwidth-bound rank-1 update per token: per state row i,
+ * with a = alpha_t,
  *     p_i = sum_j S_ij a_j k_j,  r_i = sum_j S_ij a_j q_j,
  *     u_i = beta (v_i - p_i)  (DELTA)  or  v_i  (ADDITIVE / DECAY),
  *     S_ij <- S_ij a_j + u_i k_j,   o_i = r_i + u_i (k . q).
+ * The T tokens are applied in order with the state held on chip, so the state
+ * is read and written once per call, not once per token.
  *
- *   q, k  [B,H,1,dk]   dtype          v  [B,H,1,dv]  dtype
- *   g     [B,H,1] (scalar) or [B,H,1,dk] (channel) or NULL     float
- *   beta  [B,H,1]      float (DELTA)
+ *   q, k  [B,H,T,dk]   dtype          v  [B,H,T,dv]  dtype
+ *   g     [B,H,T] (scalar) or [B,H,T,dk] (channel) or NULL     float
+ *   beta  [B,H,T]      float (DELTA)
  *   S     [B,H,dv,dk]  float, read and overwritten in place
- *   o     [B,H,1,dv]   out_dtype      (written)
+ *   o     [B,H,T,dv]   out_dtype      (written)
  *
- * desc->T must be 1; desc->chunk and desc->algo are ignored.
+ * T == 0 is a no-op; T > GDN_DECODE_MAX_T returns GDN_ERR_UNSUPPORTED.
+ * desc->chunk and desc->algo are ignored.
  */
 int gdn_decode_step(const gdn_desc_t *desc, const void *q, const void *k, const void *v,
                     const float *g, const float *beta, float *S, void *o, void *stream);

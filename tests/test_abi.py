@@ -85,9 +85,15 @@ def test_empty_batch_is_a_noop(lib):
 
 def test_decode_rejects_bad_arguments(lib):
     vp = ctypes.c_void_p
-    d = _desc(T=2)
+    d = _desc(T=17)
     assert lib.gdn_decode_step(ctypes.byref(d), vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000),
-                               vp(0x100000), vp(0x6000), None) == -1   # T must be 1
+                               vp(0x100000), vp(0x6000), None) == -3   # T > GDN_DECODE_MAX_T
+    d = _desc(T=-1)
+    assert lib.gdn_decode_step(ctypes.byref(d), vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000),
+                               vp(0x100000), vp(0x6000), None) == -1   # negative T
+    d = _desc(T=0)
+    assert lib.gdn_decode_step(ctypes.byref(d), vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000),
+                               vp(0x100000), vp(0x6000), None) == 0    # no tokens: no-op, no launch
     d = _desc(T=1)
     assert lib.gdn_decode_step(ctypes.byref(d), vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000),
                                vp(0x100004), vp(0x6000), None) == -2   # misaligned state

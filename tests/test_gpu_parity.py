@@ -139,6 +139,55 @@ def test_decode_small_all_modes(update, gate, dtype, dk):
     assert rel_err(og, ro) <= TOL[dtype] and rel_err(np64(S), rS) <= TOL[dtype]
 
 
+def _stack_steps(steps):
+    """List of single-token step inputs -> one [B,H,T,...] input of T tokens."""
+    out = {}
+    for key in steps[0]:
+        out[key] = None if steps[0][key] is None else np.concatenate([s[key] for s in steps], axis=2)
+    return out
+
+
+@pytest.mark.parametrize("update,gate", MODES)
+@pytest.mark.parametrize("T", [2, 5, 16])
+def test_decode_multi_token_all_modes(update, gate, T):
+    # T tokens in one call: the state stays on chip between them
+    w = small_workload(update, gate, "bf16", T=1, dk=128, dv=128, B=3, H=5).with_(steps=T, q_map="none")
+    steps = make_decode_inputs(w, T)
+    x = _stack_steps(steps)
+    S0 = np.random.default_rng(2).standard_normal((3, 5, 128, 128)).astype(np.float32) * 0.05
+    S = dev(S0)
+    d = {k_: (None if v_ is None else dev(v_, torch.bfloat16 if k_ in ("q", "k", "v") else torch.float32))
+         for k_, v_ in x.items()}
+    o = gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], S, update=update, gate=gate)
+    ro, rS = oracle.decode_sequence(update, gate, S0, steps)
+    assert rel_err(np64(o), ro) <= TOL["bf16"] and rel_err(np64(S), rS) <= TOL["bf16"]
+
+
+def test_decode_multi_token_equals_single_steps():
+    w = small_workload("delta", "channel", "f32", T=1, dk=128, dv=128, B=2, H=3).with_(steps=8, q_map="none")
+    steps = make_decode_inputs(w, 8)
+    S0 = np.random.default_rng(4).standard_normal((2, 3, 128, 128)).astype(np.float32) * 0.05
+    S1, S8 = dev(S0), dev(S0)
+    singles = []
+    for s in steps:
+        d = {k_: (None if v_ is None else dev(v_)) for k_, v_ in s.items()}
+        singles.append(gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], S1, update="delta",
+                                       gate="channel"))
+    x = {k_: (None if v_ is None else dev(v_)) for k_, v_ in _stack_steps(steps).items()}
+    o8 = gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S8, update="delta", gate="channel")
+    torch.cuda.synchronize()
+    # the same per-token arithmetic in the same order
+    assert rel_err(np64(o8), np64(torch.cat(singles, dim=2))) < 1e-6
+    assert rel_err(np64(S8), np64(S1)) < 1e-6
+
+
+def test_decode_token_count_limits():
+    q = torch.zeros((1, 1, gdn.DECODE_MAX_T + 1, 64), device="cuda")
+    S = torch.zeros((1, 1, 64, 64), device="cuda")
+    with pytest.raises(ValueError):
+        gdn.decode_step(q, q, q, None, None, S, update="additive", gate="none")
+
+
 # ---------------------------------------------------------------------------
 # Edge cases and consistency
 # ---------------------------------------------------------------------------
