@@ -9,7 +9,8 @@ Two implementations of the same definition:
 * ``gdn_forward`` -- the C recurrence in ``gdn_oracle.c`` (float64, OpenMP
   over heads), for every size the tests and the benchmark use;
 * ``gdn_forward_np`` -- the same three steps written with NumPy, vectorised
-  over heads, for small cases and to cross-check the compiled one.
+  over heads, for small cases and to cross-check the compiled one;
+* ``gdp_forward`` -- Gated DeltaProduct (n_h delta substeps per token), NumPy.
 
 Definition (column convention, S in R^{dv x dk}, stored [B,H,dv,dk]):
 ``S_t = S_{t-1} Diag(alpha_t)(I - beta_t k_t k_t^T) + beta_t v_t k_t^T``,
@@ -138,6 +139,38 @@ def gdn_forward_np(update, gate, q, k, v, g=None, beta=None, S0=None):
         else:
             u = v[..., t, :]
         S = S + u[..., :, None] * kt[..., None, :]
+        o[..., t, :] = np.einsum("...ij,...j->...i", S, q[..., t, :])
+    return o, S
+
+
+def gdp_forward(gate, q, k, v, g=None, beta=None, S0=None):
+    """Gated DeltaProduct, token by token ("Linear Attention, Visualized",
+    "Gated Delta Product (GDP)"): for each real token t the state decays once by
+    a_t = exp(g_t), then takes n_h delta-rule substeps j = 1..n_h, each with its
+    own key k_{t,j}, value v_{t,j} and write strength beta_{t,j}, and only then
+    is read, o_t = S q_t.
+
+    q [...,T,dk]; k [...,T,nh,dk]; v [...,T,nh,dv]; beta [...,T,nh];
+    g [...,T] (scalar) or [...,T,dk] (channel) or None.  Returns (o, S_T).
+    """
+    q, k, v, g, beta = _f64(q), _f64(k), _f64(v), _f64(g), _f64(beta)
+    lead = q.shape[:-2]
+    T, dk = q.shape[-2], q.shape[-1]
+    nh, dv = k.shape[-2], v.shape[-1]
+    if (gate == "none") != (g is None) or beta is None:
+        raise ValueError("gate / g mismatch or missing beta")
+    S = np.zeros(lead + (dv, dk)) if S0 is None else _f64(S0).copy()
+    o = np.empty(lead + (T, dv))
+    for t in range(T):
+        if gate == "scalar":
+            S = S * np.exp(g[..., t])[..., None, None]
+        elif gate == "channel":
+            S = S * np.exp(g[..., t, :])[..., None, :]
+        for j in range(nh):
+            kj = k[..., t, j, :]
+            pred = np.einsum("...ij,...j->...i", S, kj)
+            u = beta[..., t, j][..., None] * (v[..., t, j, :] - pred)
+            S = S + u[..., :, None] * kj[..., None, :]
         o[..., t, :] = np.einsum("...ij,...j->...i", S, q[..., t, :])
     return o, S
 

@@ -234,6 +234,25 @@ def make_prefill_inputs(w: Workload, heads=None) -> dict:
     return {"q": rs(q), "k": rs(k), "v": rs(v), "beta": rs(beta), "g": rs(g), "S0": rs(S0)}
 
 
+def make_product_inputs(w: Workload, nh: int, heads=None) -> dict:
+    """Inputs of a Gated DeltaProduct run with ``nh`` substeps per token.
+
+    q [B,H,T,dk] and g ([B,H,T] or [B,H,T,dk]) per real token (the streams of
+    ``make_prefill_inputs``); k [B,H,T,nh,dk], v [B,H,T,nh,dv] and beta
+    [B,H,T,nh] per substep, drawn as one sequence of T*nh positions from streams
+    keyed additionally by nh; S0 as in ``make_prefill_inputs``.
+    """
+    base = make_prefill_inputs(w, heads)
+    wv = w.with_(T=w.T * nh, seed=w.seed + 7919 * nh)
+    sub = make_prefill_inputs(wv, heads)
+    lead = base["q"].shape[:2]
+    out = {"q": base["q"], "g": base["g"], "S0": base["S0"]}
+    out["k"] = sub["k"].reshape(lead + (w.T, nh, w.dk))
+    out["v"] = sub["v"].reshape(lead + (w.T, nh, w.dv))
+    out["beta"] = None if sub["beta"] is None else sub["beta"].reshape(lead + (w.T, nh))
+    return out
+
+
 def make_decode_state(w: Workload, heads=None) -> np.ndarray:
     """Initial decode state S [B,H,dv,dk] float32 (or [n,1,dv,dk] for ``heads``)."""
     if heads is None:

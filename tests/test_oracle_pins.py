@@ -413,3 +413,81 @@ def test_planted_mistakes_are_caught(oracle_mod, kind):
         if rel_err(o[0], ro) > 1e-6 or rel_err(ST[0], rS) > 1e-6:
             failures += 1
     assert failures > 0, "planted mistake %s was not caught" % kind
+
+
+# ---------------------------------------------------------------------------
+# Gated DeltaProduct ("Gated Delta Product (GDP)", "GDP as GDN over a virtual
+# sequence")
+# ---------------------------------------------------------------------------
+
+def gdp_inputs(seed, BH=3, T=12, nh=3, dk=8, dv=6, gate="scalar"):
+    r = np.random.default_rng(seed)
+    q = r.standard_normal((BH, T, dk))
+    k = r.standard_normal((BH, T, nh, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = r.standard_normal((BH, T, nh, dv))
+    beta = r.uniform(0.1, 1.0, (BH, T, nh))
+    g = None
+    if gate == "scalar":
+        g = r.uniform(-0.3, 0.0, (BH, T))
+    elif gate == "channel":
+        g = r.uniform(-0.3, 0.0, (BH, T, dk))
+    S0 = 0.3 * r.standard_normal((BH, dv, dk))
+    return q, k, v, g, beta, S0
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+def test_gdp_with_one_substep_is_gdn(oracle_mod, gate):
+    q, k, v, g, beta, S0 = gdp_inputs(31, nh=1, gate=gate)
+    o, S = oracle.gdp_forward(gate, q, k, v, g, beta, S0)
+    ro, rS = oracle.gdn_forward("delta", gate, q, k[:, :, 0], v[:, :, 0], g, beta[:, :, 0], S0)
+    assert rel_err(o, ro) < TOL and rel_err(S, rS) < TOL
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+@pytest.mark.parametrize("nh", [2, 3])
+def test_gdp_is_gdn_over_the_virtual_sequence(oracle_mod, gate, nh):
+    # the page's table: substep (t, j) is virtual step t*nh + j; the decay sits on
+    # the first substep of a token, the query on the last, and every nh-th output
+    # is kept
+    q, k, v, g, beta, S0 = gdp_inputs(32, nh=nh, gate=gate)
+    BH, T, dk = q.shape
+    Tv = T * nh
+    qv = np.zeros((BH, Tv, dk))
+    qv[:, nh - 1::nh] = q
+    gv = None
+    if gate == "scalar":
+        gv = np.zeros((BH, Tv))
+        gv[:, 0::nh] = g
+    elif gate == "channel":
+        gv = np.zeros((BH, Tv, dk))
+        gv[:, 0::nh] = g
+    ov, Sv = oracle.gdn_forward("delta", gate, qv, k.reshape(BH, Tv, dk), v.reshape(BH, Tv, -1), gv,
+                                beta.reshape(BH, Tv), S0)
+    o, S = oracle.gdp_forward(gate, q, k, v, g, beta, S0)
+    assert rel_err(o, ov[:, nh - 1::nh]) < TOL and rel_err(S, Sv) < TOL
+
+
+def test_gdp_brute_force_products(oracle_mod):
+    # per token: S <- S Diag(a_t) H_1 ... H_nh + (write terms), each substep the
+    # explicit matrix map S -> S (I - beta k k^T) + beta v k^T
+    q, k, v, g, beta, S0 = gdp_inputs(33, BH=1, T=5, nh=3, dk=4, dv=3, gate="channel")
+    S = S0[0].copy()
+    outs = []
+    for t in range(5):
+        S = S @ np.diag(np.exp(g[0, t]))
+        for j in range(3):
+            kk = k[0, t, j][:, None]
+            S = S @ (np.eye(4) - beta[0, t, j] * kk @ kk.T) + beta[0, t, j] * v[0, t, j][:, None] @ kk.T
+        outs.append(S @ q[0, t])
+    o, Sf = oracle.gdp_forward("channel", q, k, v, g, beta, S0)
+    assert rel_err(o[0], np.array(outs)) < TOL and rel_err(Sf[0], S) < TOL
+
+
+def test_gdp_zero_write_strength_only_decays(oracle_mod):
+    q, k, v, g, beta, S0 = gdp_inputs(34, gate="scalar")
+    beta[:] = 0.0
+    o, S = oracle.gdp_forward("scalar", q, k, v, g, beta, S0)
+    G = np.cumsum(g, axis=1)
+    expect = np.einsum("bij,btj->bti", S0, q) * np.exp(G)[..., None]
+    assert rel_err(o, expect) < TOL and rel_err(S, S0 * np.exp(G[:, -1])[:, None, None]) < TOL
