@@ -27,6 +27,7 @@ ALGOS = {"auto": 0, "simt": 1, "tc": 2, "tc_seq": 3}
 F32, BF16 = 0, 1
 
 DECODE_MAX_T = 16  # GDN_DECODE_MAX_T
+PRODUCT_MAX_NH = 16  # GDN_PRODUCT_MAX_NH
 GDN_OK = 0
 ERRORS = {-1: "GDN_ERR_ARG", -2: "GDN_ERR_ALIGN", -3: "GDN_ERR_UNSUPPORTED", -4: "GDN_ERR_CUDA",
           -5: "GDN_ERR_TIMEOUT", -6: "GDN_ERR_RANGE"}
@@ -75,6 +76,8 @@ def load():
     lib.gdn_chunk_fwd.restype = ctypes.c_int
     lib.gdn_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.gdn_decode_step.restype = ctypes.c_int
+    lib.gdn_product_fwd.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gdn_product_fwd.restype = ctypes.c_int
     lib.gdn_strerror.argtypes = [ctypes.c_int]
     lib.gdn_strerror.restype = ctypes.c_char_p
     lib.gdn_device_status.argtypes = [ctypes.c_int]
@@ -175,6 +178,45 @@ def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=No
                               _ptr(o), _ptr(S_T), _stream(stream))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_chunk_fwd")
+    return o, S_T
+
+
+def product_fwd(q, k, v, g=None, beta=None, S0=None, *, gate, out_dtype=None, o=None, S_T=None,
+                return_state=True, algo="auto", stream=None):
+    """Gated DeltaProduct prefill (gdn_product_fwd): nh = k.shape[-2] delta-rule
+    substeps per token.  Returns (o, S_T).
+
+    q [B,H,T,dk]; k [B,H,T,nh,dk]; v [B,H,T,nh,dv] (same dtype); beta [B,H,T,nh]
+    fp32; g [B,H,T] or [B,H,T,dk] fp32 or None; S0 [B,H,dv,dk] fp32 or None.
+    """
+    import torch
+
+    B, H, T, dk = q.shape
+    nh, dv = k.shape[-2], v.shape[-1]
+    if not 1 <= nh <= PRODUCT_MAX_NH:
+        raise ValueError("1..%d substeps per token" % PRODUCT_MAX_NH)
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, nh, dk), q.dtype)
+    _check(v, "v", (B, H, T, nh, dv), q.dtype)
+    if gate == "scalar":
+        _check(g, "g", (B, H, T), torch.float32)
+    elif gate == "channel":
+        _check(g, "g", (B, H, T, dk), torch.float32)
+    _check(beta, "beta", (B, H, T, nh), torch.float32)
+    _check(S0, "S0", (B, H, dv, dk), torch.float32)
+    if out_dtype is None:
+        out_dtype = o.dtype if o is not None else torch.float32
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
+    _check(o, "o", (B, H, T, dv), out_dtype)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
+    d = make_desc(B, H, T, dk, dv, "delta", gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo)
+    rc = load().gdn_product_fwd(ctypes.byref(d), ctypes.c_int(nh), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_product_fwd")
     return o, S_T
 
 

@@ -129,11 +129,56 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     a.status = status_ptr();
     a.diag = diag_ptr();
     a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
+    a.nh = 1;
 
     const bool tc_ok = gdn_tc_supported(d) != 0;
     if ((d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) && !tc_ok) return GDN_ERR_UNSUPPORTED;
     if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
     if (d->algo == GDN_ALGO_TC_SEQ) return from_cuda(gdn_launch_chunk_tc(a, d, st));
+    return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
+}
+
+extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const void *k, const void *v,
+                               const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                               void *stream) {
+    int rc = validate_common(d);
+    if (rc != GDN_OK) return rc;
+    if (d->update != GDN_DELTA) return GDN_ERR_ARG;  // a product of delta-rule transitions
+    if (nh < 1) return GDN_ERR_ARG;
+    if (nh > GDN_PRODUCT_MAX_NH) return GDN_ERR_UNSUPPORTED;
+    if (nh == 1) return gdn_chunk_fwd(d, q, k, v, g, beta, S0, o, S_T, stream);
+    if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC_SEQ) return GDN_ERR_ARG;
+    if (d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) return GDN_ERR_UNSUPPORTED;
+    if ((long)d->T * nh > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
+    const long BH = (long)d->B * d->H;
+    const size_t Tr = (size_t)d->T, Tv = Tr * nh;
+    const size_t n_q = (size_t)BH * Tr * d->dk, n_k = (size_t)BH * Tv * d->dk, n_v = (size_t)BH * Tv * d->dv;
+    const size_t n_o = (size_t)BH * Tr * d->dv, n_S = (size_t)BH * d->dv * d->dk;
+    const size_t n_g = d->gate == GDN_GATE_CHANNEL ? n_q : (size_t)BH * Tr;
+    const bool has_tokens = BH > 0 && d->T > 0;
+    if (has_tokens && (!q || !k || !v || !o || !beta)) return GDN_ERR_ARG;
+    if ((d->gate != GDN_GATE_NONE) != (g != nullptr) && has_tokens) return GDN_ERR_ARG;
+    if (d->gate == GDN_GATE_NONE && g != nullptr) return GDN_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, o, S_T};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t es = elem_size(d->dtype), no = n_o * elem_size(d->out_dtype);
+    if (overlaps(o, no, q, n_q * es) || overlaps(o, no, k, n_k * es) || overlaps(o, no, v, n_v * es) ||
+        overlaps(o, no, g, n_g * 4) || overlaps(o, no, beta, (size_t)BH * Tv * 4) ||
+        overlaps(o, no, S0, n_S * 4) || overlaps(o, no, S_T, n_S * 4))
+        return GDN_ERR_ARG;
+    if (S_T && S0 && S_T != S0 && overlaps(S_T, n_S * 4, S0, n_S * 4)) return GDN_ERR_ARG;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (BH == 0) return GDN_OK;
+    if (d->T == 0) return from_cuda(gdn_launch_copy_state(S0, S_T, (long)n_S, st));
+    gdn::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
+    a.status = status_ptr();
+    a.diag = diag_ptr();
+    a.BH = (int)BH; a.T = (int)Tv; a.dk = d->dk; a.dv = d->dv;
+    a.nh = nh;
     return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
 }
 

@@ -61,14 +61,16 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
     const int bh = blockIdx.x / nslices;
     const int v0 = (blockIdx.x % nslices) * kDvs;
     const int T = a.T, dv = a.dv;
-    const TIn *q = static_cast<const TIn *>(a.q) + (size_t)bh * T * DK;
+    // virtual steps (k, v, beta) vs real tokens (q, g, o); nh = 1 makes them the same
+    const int nh = a.nh, Tr = T / nh;
+    const TIn *q = static_cast<const TIn *>(a.q) + (size_t)bh * Tr * DK;
     const TIn *k = static_cast<const TIn *>(a.k) + (size_t)bh * T * DK;
     const TIn *v = static_cast<const TIn *>(a.v) + (size_t)bh * T * dv;
     const float *g = nullptr;
-    if (GATE == kGateScalar) g = a.g + (size_t)bh * T;
-    if (GATE == kGateChannel) g = a.g + (size_t)bh * T * DK;
+    if (GATE == kGateScalar) g = a.g + (size_t)bh * Tr;
+    if (GATE == kGateChannel) g = a.g + (size_t)bh * Tr * DK;
     const float *beta = (UPD == kDelta) ? a.beta + (size_t)bh * T : nullptr;
-    TOut *o = static_cast<TOut *>(a.o) + (size_t)bh * T * dv;
+    TOut *o = static_cast<TOut *>(a.o) + (size_t)bh * Tr * dv;
 
     for (int i = tid; i < kDvs * DK; i += kThreads) {
         const int vv = i / DK, j = i % DK;
@@ -83,9 +85,10 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
             const int l = i / DK, j = i % DK;
             float qv = 0.f, kv = 0.f, gv = 0.f;
             if (l < n) {
-                qv = to_f32(q[(size_t)(t0 + l) * DK + j]);
-                kv = to_f32(k[(size_t)(t0 + l) * DK + j]);
-                if (GATE == kGateChannel) gv = g[(size_t)(t0 + l) * DK + j];
+                const int m = t0 + l, tr = m / nh, sub = m - tr * nh;
+                if (sub == nh - 1) qv = to_f32(q[(size_t)tr * DK + j]);
+                kv = to_f32(k[(size_t)m * DK + j]);
+                if (GATE == kGateChannel && sub == 0) gv = g[(size_t)tr * DK + j];
             }
             sQ[l * LDK + j] = qv;
             sK[l * LDK + j] = kv;
@@ -96,7 +99,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
             sV[l * LDV + c] = (l < n) ? to_f32(v[(size_t)(t0 + l) * dv + v0 + c]) : 0.f;
         }
         if (tid < C) {
-            if (GATE == kGateScalar) sG[tid] = (tid < n) ? g[t0 + tid] : 0.f;
+            if (GATE == kGateScalar) sG[tid] = (tid < n && (t0 + tid) % nh == 0) ? g[(t0 + tid) / nh] : 0.f;
             if (UPD == kDelta) sB[tid] = (tid < n) ? beta[t0 + tid] : 0.f;
         }
         __syncthreads();
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
             if (GATE == kGateScalar) hist *= __expf(sG[l]);
             float loc = 0.f;
             for (int m = 0; m <= l; ++m) loc = fmaf(sA[l * LDC + m], sV[m * LDV + vv], loc);
-            if (l < n) o[(size_t)(t0 + l) * dv + v0 + vv] = from_f32<TOut>(hist + loc);
+            if (l < n && (t0 + l) % nh == nh - 1) o[(size_t)((t0 + l) / nh) * dv + v0 + vv] = from_f32<TOut>(hist + loc);
         }
         __syncthreads();
 

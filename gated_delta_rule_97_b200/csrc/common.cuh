@@ -43,6 +43,11 @@ struct ChunkArgs {
     int *status;             // device status word
     int *diag;               // device diagnostic word (first timeout site)
     int BH, T, dk, dv;
+    // Substeps per real token (Gated DeltaProduct; 1 otherwise).  T counts the
+    // virtual steps (real tokens x nh): k, v, beta are laid out per virtual step,
+    // q, g and o per real token; a token's q sits on its last substep, its gate
+    // on its first, and only the last substep's output is written.
+    int nh;
 };
 
 struct DecodeArgs {

@@ -57,6 +57,9 @@ extern "C" {
 /* Largest token count of one gdn_decode_step call (longer runs: gdn_chunk_fwd). */
 #define GDN_DECODE_MAX_T 16
 
+/* Largest number of substeps per token of gdn_product_fwd. */
+#define GDN_PRODUCT_MAX_NH 16
+
 /* Write rule.  ADDITIVE: S += v k^T, no gate ("Naive linear attention").
  * DECAY: S = S Diag(alpha) + v k^T, gate required (RetNet / Mamba-2 / GLA).
  * DELTA: the gated delta rule above; any gate (DeltaNet / GDN / KDA). */
@@ -112,6 +115,29 @@ typedef struct {
 int gdn_chunk_fwd(const gdn_desc_t *desc, const void *q, const void *k, const void *v,
                   const float *g, const float *beta, const float *S0, void *o, float *S_T,
                   void *stream);
+
+/*
+ * gdn_product_fwd -- prefill of Gated DeltaProduct: every real token applies
+ * nh delta-rule transitions in order, each with its own key, value and write
+ * strength, after one decay by the token's gate, and is read after the last
+ * ("Linear Attention, Visualized", "Gated Delta Product (GDP)").  Computed, as
+ * "GDP as GDN over a virtual sequence" describes, by the chunkwise GDN path over
+ * T * nh virtual steps: substep j of token t is step t * nh + j, the gate sits on
+ * the first substep and the query on the last, and every nh-th output is kept.
+ *
+ *   q     [B,H,T,dk]      dtype       k  [B,H,T,nh,dk]  dtype
+ *   v     [B,H,T,nh,dv]   dtype       beta [B,H,T,nh]   float
+ *   g     [B,H,T] (scalar) or [B,H,T,dk] (channel) or NULL        float
+ *   S0, S_T, o            as in gdn_chunk_fwd (o is [B,H,T,dv])
+ *
+ * desc->update must be GDN_DELTA and desc->T counts real tokens.  nh == 1 is
+ * gdn_chunk_fwd; for nh > 1 the fp32 SIMT kernel runs (GDN_ALGO_AUTO or
+ * GDN_ALGO_SIMT; the tensor-core choices return GDN_ERR_UNSUPPORTED).  The
+ * caller owns every buffer; nothing is allocated.
+ */
+int gdn_product_fwd(const gdn_desc_t *desc, int nh, const void *q, const void *k, const void *v,
+                    const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                    void *stream);
 
 /*
  * gdn_decode_step -- decode: T recurrent steps (1 <= T <= GDN_DECODE_MAX_T,

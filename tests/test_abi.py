@@ -101,6 +101,21 @@ def test_decode_rejects_bad_arguments(lib):
                                vp(0x100000), vp(0x6000), None) == -1   # gate without g
 
 
+def test_product_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    args = (vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000), None, vp(0x100000), None, None)
+    lib.gdn_product_fwd.argtypes = [ctypes.c_void_p, ctypes.c_int] + [ctypes.c_void_p] * 9
+    d = _desc()
+    assert lib.gdn_product_fwd(ctypes.byref(d), 0, *args) == -1      # nh < 1
+    assert lib.gdn_product_fwd(ctypes.byref(d), 17, *args) == -3     # nh > GDN_PRODUCT_MAX_NH
+    d = _desc(update="additive", gate="none")
+    assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -1      # only the delta rule has substeps
+    d = _desc(algo="tc")
+    assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -3      # tensor-core kernel: not for nh > 1
+    d = _desc(B=0)
+    assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == 0       # empty batch: no-op
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(gdn, "_lib", None)
     monkeypatch.setattr(gdn, "_LIB_PATH", str(tmp_path / "missing.so"))
