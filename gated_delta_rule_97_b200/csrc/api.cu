@@ -149,7 +149,11 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     if (nh == 1) return gdn_chunk_fwd(d, q, k, v, g, beta, S0, o, S_T, stream);
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
     if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC_SEQ) return GDN_ERR_ARG;
-    if (d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) return GDN_ERR_UNSUPPORTED;
+    // the pipelined tensor-core kernel takes whole tokens per chunk: nh a power of
+    // two (it divides the chunk), scalar or no gate
+    const bool pow2 = (nh & (nh - 1)) == 0;
+    const bool tc_ok = gdn_tc_supported(d) != 0 && pow2 && d->gate != GDN_GATE_CHANNEL;
+    if (d->algo == GDN_ALGO_TC_SEQ || (d->algo == GDN_ALGO_TC && !tc_ok)) return GDN_ERR_UNSUPPORTED;
     if ((long)d->T * nh > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
     const long BH = (long)d->B * d->H;
     const size_t Tr = (size_t)d->T, Tv = Tr * nh;
@@ -179,6 +183,7 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     a.diag = diag_ptr();
     a.BH = (int)BH; a.T = (int)Tv; a.dk = d->dk; a.dv = d->dv;
     a.nh = nh;
+    if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
     return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
 }
 

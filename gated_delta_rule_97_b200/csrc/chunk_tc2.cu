@@ -78,6 +78,7 @@ struct Params {
     int *status;
     int *diag;
     int BH, T, dv, nslices;
+    int lnh;  // log2 of the substeps per token (Gated DeltaProduct), else 0
 };
 
 template <int DVS, int GATE>
@@ -132,7 +133,13 @@ __device__ __forceinline__ int v16_slot(int buf) {
     return (UPD != kDelta && GATE != kGateChannel && buf) ? L::KT : L::V16;
 }
 
-template <int DVS, int UPD, int GATE, bool OUT_BF16>
+// PROD: Gated DeltaProduct with 2^lnh substeps per token ("GDP as GDN over a
+// virtual sequence"): T counts virtual steps; k, v, beta are per virtual step,
+// while q, g and o are per token.  A chunk covers 64 >> lnh whole tokens: their q
+// rows arrive compact and are moved to each token's last substep (zeros
+// elsewhere), the gate sits on each token's first substep, and only each
+// token's last substep is written out.
+template <int DVS, int UPD, int GATE, bool OUT_BF16, bool PROD>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_constant__ Params p) {
     using L = Smem<DVS, GATE>;
     constexpr bool DELTA = (UPD == kDelta);
@@ -140,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     // rdy when the prep group is the longer side (delta rule, scalar / no gate), else
     // by the prep group itself (it then has slack; the channel gate's P also needs
     // the converted operands)
-    constexpr bool kStateP1 = DELTA && GATE != kGateChannel;
+    constexpr bool kStateP1 = DELTA && GATE != kGateChannel && !PROD;
     // In the same modes the V tile has its own TMA barrier (bar_tv): its fp16
     // conversion runs during the 16 -> 32 merge, after the q / k conversion window
     constexpr bool kSplitV = DELTA && GATE != kGateChannel;
@@ -206,8 +213,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             const int t0 = r * C;
             if (GATE == kGateScalar && warp == 4) {
                 const int l0 = 2 * lane;
-                gpre0 = (t0 + l0 < T) ? p.g[(size_t)bh * T + t0 + l0] : 0.f;
-                gpre1 = (t0 + l0 + 1 < T) ? p.g[(size_t)bh * T + t0 + l0 + 1] : 0.f;
+                if (PROD) {
+                    // the token's gate on its first substep, 1 (g = 0) on the others
+                    const int m0 = t0 + l0, m1 = m0 + 1, msk = (1 << p.lnh) - 1;
+                    const size_t gb = (size_t)bh * (T >> p.lnh);
+                    gpre0 = (m0 < T && (m0 & msk) == 0) ? p.g[gb + (m0 >> p.lnh)] : 0.f;
+                    gpre1 = (m1 < T && (m1 & msk) == 0) ? p.g[gb + (m1 >> p.lnh)] : 0.f;
+                } else {
+                    gpre0 = (t0 + l0 < T) ? p.g[(size_t)bh * T + t0 + l0] : 0.f;
+                    gpre1 = (t0 + l0 + 1 < T) ? p.g[(size_t)bh * T + t0 + l0 + 1] : 0.f;
+                }
             }
             if (DELTA && t >= 128 && t < 128 + C) {
                 const int l = t - 128;
@@ -247,10 +262,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         };
         auto issue_tma = [&](int r) {
             const int t0 = r * C;
-            const uint32_t bytes = 32768 + (kSplitV ? 0 : DVS * 128) + (GATE == kGateChannel ? 32768 : 0);
+            const uint32_t qbytes = PROD ? 2u * (64u >> p.lnh) * 128u : 16384u;
+            const uint32_t bytes = qbytes + 16384 + (kSplitV ? 0 : DVS * 128) + (GATE == kGateChannel ? 32768 : 0);
             mbar_arrive_expect_tx(&ms.bar_tma, bytes);
             for (int h = 0; h < 2; ++h) {
-                tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, t0, bh, &ms.bar_tma);
+                tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, PROD ? (t0 >> p.lnh) : t0, bh,
+                            &ms.bar_tma);
                 tma_load_3d(sm + L::RAW_QK + h * 16384 + 8192, &p.k_map, h * 64, t0, bh, &ms.bar_tma);
             }
             if (!kSplitV) issue_tma_v(r, &ms.bar_tma);
@@ -281,6 +298,29 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             const float *bet = ms.beta[buf];
             TC2_MARK(0, 0);
             if (!mbar_wait(&ms.bar_tma, ph)) note_timeout(ms, 1, r);
+            if (PROD) {
+                // compact q rows j -> row (j + 1) * nh - 1, the rest zero (both key halves)
+                const int lnh = p.lnh, msk = (1 << lnh) - 1;
+                uint4 qv[4];
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const int i = t + 256 * s4, h = i >> 9, d = (i & 511) >> 3, c = i & 7;
+                    qv[s4] = make_uint4(0, 0, 0, 0);
+                    if ((d & msk) == msk) {
+                        const int j = d >> lnh;
+                        qv[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + j * 128 +
+                                                                   ((c ^ (j & 7)) << 4));
+                    }
+                }
+                named_bar(kPrepBar, 256);
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const int i = t + 256 * s4, h = i >> 9, d = (i & 511) >> 3, c = i & 7;
+                    *reinterpret_cast<uint4 *>(sm + L::RAW_QK + h * 16384 + d * 128 + ((c ^ (d & 7)) << 4)) = qv[s4];
+                }
+                fence_proxy_async_smem();
+                named_bar(kPrepBar, 256);
+            }
             TC2_MARK(0, 1);
             if (!kStateP1 && GATE != kGateChannel && t == 0 && !ms.abort_flag) {
                 tc_fence_after();
@@ -1016,7 +1056,19 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 tmem_wait_ld();
                 if (ts == 0) bulk_wait_read0();  // the previous chunk's store has read the staging tile
                 named_bar(kStateBar, 128);
-                if (has_row) {
+                if (has_row && PROD) {
+                    // each token's last substep, compacted to one row per token
+                    const int msk = (1 << p.lnh) - 1;
+#pragma unroll
+                    for (int l = 0; l < 64; ++l) {
+                        if ((l & msk) != msk) continue;
+                        const int row = l >> p.lnh;
+                        if (OUT_BF16)
+                            reinterpret_cast<__nv_bfloat16 *>(ost)[row * DVS + vrow] = __float2bfloat16_rn(ov[l]);
+                        else
+                            ost[row * DVS + vrow] = ov[l];
+                    }
+                } else if (has_row) {
                     if (OUT_BF16) {
                         __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(ost);
 #pragma unroll
@@ -1029,7 +1081,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 fence_proxy_async_smem();
                 named_bar(kStateBar, 128);
                 if (ts == 0) {
-                    tma_store_3d(&p.o_map, ost, v0, t0, bh);
+                    tma_store_3d(&p.o_map, ost, v0, PROD ? (t0 >> p.lnh) : t0, bh);
                     bulk_commit();
                 }
             }
@@ -1109,10 +1161,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DVS, int UPD, int GATE, bool OB>
+template <int DVS, int UPD, int GATE, bool OB, bool PROD = false>
 int launch_one(const Params &prm, int grid, cudaStream_t stream) {
     using L = Smem<DVS, GATE>;
-    auto kern = chunk_tc2_kernel<DVS, UPD, GATE, OB>;
+    auto kern = chunk_tc2_kernel<DVS, UPD, GATE, OB, PROD>;
     static_assert(L::DYN <= 232448, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN);
     if (e != cudaSuccess) return (int)e;
@@ -1123,6 +1175,12 @@ int launch_one(const Params &prm, int grid, cudaStream_t stream) {
 template <int DVS, int UPD, int GATE>
 int launch_out(const Params &prm, int grid, bool ob, cudaStream_t s) {
     return ob ? launch_one<DVS, UPD, GATE, true>(prm, grid, s) : launch_one<DVS, UPD, GATE, false>(prm, grid, s);
+}
+
+template <int DVS, int GATE>
+int launch_prod(const Params &prm, int grid, bool ob, cudaStream_t s) {
+    return ob ? launch_one<DVS, kDelta, GATE, true, true>(prm, grid, s)
+              : launch_one<DVS, kDelta, GATE, false, true>(prm, grid, s);
 }
 
 template <int DVS>
@@ -1167,7 +1225,13 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     Params prm;
     memset(&prm, 0, sizeof(prm));
     const uint64_t BH = (uint64_t)a.BH, T = (uint64_t)a.T;
-    if (!make_map_3d(&prm.q_map, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, T, BH, 64, 64, 1, true) ||
+    // Gated DeltaProduct: T counts virtual steps; q and o have T / nh token rows
+    int lnh = 0;
+    while ((1 << lnh) < a.nh) ++lnh;
+    if ((1 << lnh) != a.nh || lnh > 6 || d->gate == GDN_GATE_CHANNEL && lnh > 0) return (int)cudaErrorInvalidValue;
+    const uint64_t Tr = T >> lnh;
+    const uint32_t rows = 64u >> lnh;
+    if (!make_map_3d(&prm.q_map, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, Tr, BH, 64, rows, 1, true) ||
         !make_map_3d(&prm.k_map, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, T, BH, 64, 64, 1, true) ||
         !make_map_3d(&prm.v_map, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.dv, T, BH, 64, 64, 1, true))
         return (int)cudaErrorInvalidValue;
@@ -1177,7 +1241,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     const int dvs = tc2_slice(d);
     const bool ob = d->out_dtype == GDN_BF16;
     if (!make_map_3d(&prm.o_map, a.o, ob ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                     ob ? 2 : 4, (uint64_t)a.dv, T, BH, (uint32_t)dvs, 64, 1, false))
+                     ob ? 2 : 4, (uint64_t)a.dv, Tr, BH, (uint32_t)dvs, rows, 1, false))
         return (int)cudaErrorInvalidValue;
     prm.g = a.g;
     prm.beta = a.beta;
@@ -1190,8 +1254,16 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     prm.T = a.T;
     prm.dv = a.dv;
     prm.nslices = a.dv / dvs;
+    prm.lnh = lnh;
     const long grid = (long)a.BH * prm.nslices;
     if (grid == 0) return 0;
+    if (lnh > 0) {
+        if (dvs == 64)
+            return d->gate == GDN_GATE_SCALAR ? launch_prod<64, kGateScalar>(prm, (int)grid, ob, stream)
+                                              : launch_prod<64, kGateNone>(prm, (int)grid, ob, stream);
+        return d->gate == GDN_GATE_SCALAR ? launch_prod<128, kGateScalar>(prm, (int)grid, ob, stream)
+                                          : launch_prod<128, kGateNone>(prm, (int)grid, ob, stream);
+    }
     if (dvs == 64) return launch_modes<64>(prm, (int)grid, d->update, d->gate, ob, stream);
     return launch_modes<128>(prm, (int)grid, d->update, d->gate, ob, stream);
 }

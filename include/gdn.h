@@ -131,9 +131,12 @@ int gdn_chunk_fwd(const gdn_desc_t *desc, const void *q, const void *k, const vo
  *   S0, S_T, o            as in gdn_chunk_fwd (o is [B,H,T,dv])
  *
  * desc->update must be GDN_DELTA and desc->T counts real tokens.  nh == 1 is
- * gdn_chunk_fwd; for nh > 1 the fp32 SIMT kernel runs (GDN_ALGO_AUTO or
- * GDN_ALGO_SIMT; the tensor-core choices return GDN_ERR_UNSUPPORTED).  The
- * caller owns every buffer; nothing is allocated.
+ * gdn_chunk_fwd.  For nh > 1, GDN_ALGO_AUTO takes the pipelined tensor-core
+ * kernel when it serves the shape (bf16, dk = 128, dv in {64, 128}, scalar or no
+ * gate, nh a power of two, so that a chunk holds whole tokens) and the fp32 SIMT
+ * kernel otherwise; GDN_ALGO_TC demands the former, GDN_ALGO_SIMT the latter,
+ * GDN_ALGO_TC_SEQ returns GDN_ERR_UNSUPPORTED.  The caller owns every buffer;
+ * nothing is allocated.
  */
 int gdn_product_fwd(const gdn_desc_t *desc, int nh, const void *q, const void *k, const void *v,
                     const float *g, const float *beta, const float *S0, void *o, float *S_T,

@@ -111,7 +111,9 @@ def test_product_rejects_bad_arguments(lib):
     d = _desc(update="additive", gate="none")
     assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -1      # only the delta rule has substeps
     d = _desc(algo="tc")
-    assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -3      # tensor-core kernel: not for nh > 1
+    assert lib.gdn_product_fwd(ctypes.byref(d), 3, *args) == -3      # tensor-core kernel: whole tokens per chunk
+    d = _desc(algo="tc_seq")
+    assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -3      # the sequential kernel has no remap
     d = _desc(B=0)
     assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == 0       # empty batch: no-op
 

@@ -77,8 +77,29 @@ def test_product_empty_sequence_copies_state():
     assert o.shape == (2, 2, 0, 64) and torch.equal(ST, S0)
 
 
-def test_product_rejects_tensor_core_choice():
-    w = workload("scalar", "bf16", T=8)
-    x = make_product_inputs(w, 2)
+def test_product_rejects_tensor_core_choice_without_whole_tokens():
+    w = workload("scalar", "bf16", T=8, d=128)
+    x = make_product_inputs(w, 3)
     with pytest.raises(gdn.GDNError):
-        run(w, x, 2, algo="tc")
+        run(w, x, 3, algo="tc")
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar"])
+@pytest.mark.parametrize("nh", [2, 4, 8, 16])
+@pytest.mark.parametrize("dv,T", [(128, 37), (128, 200), (64, 100)])
+def test_product_tensor_core_matches_oracle(gate, nh, dv, T):
+    # a chunk holds 64 / nh whole tokens; T ragged in tokens
+    w = workload(gate, "bf16", T=T, d=128).with_(dv=dv)
+    x = make_product_inputs(w, nh)
+    o, ST = run(w, x, nh, algo="tc")
+    ro, rS = oracle.gdp_forward(gate, x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
+    eo, es = rel_err(np64(o), ro), rel_err(np64(ST), rS)
+    assert eo <= TOL["bf16"] and es <= TOL["bf16"], (eo, es)
+
+
+def test_product_tensor_core_matches_simt():
+    w = workload("scalar", "bf16", T=300, d=128, B=1, H=4)
+    x = make_product_inputs(w, 4)
+    o_tc, S_tc = run(w, x, 4, algo="tc")
+    o_s, S_s = run(w, x, 4, algo="simt")
+    assert rel_err(np64(o_tc), np64(o_s)) <= TOL["bf16"] and rel_err(np64(S_tc), np64(S_s)) <= TOL["bf16"]
