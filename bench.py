@@ -201,6 +201,42 @@ def time_prefill(w, x, steps, warmup, torch, gdn, dist=None):
     return ms
 
 
+def time_product(w, nh, steps, warmup, torch, gdn):
+    """Device-timed gdn_product_fwd (Gated DeltaProduct, nh substeps per token)
+    over workload ``w``'s shape; returns ms/step."""
+    from synth import make_product_inputs
+
+    x = make_product_inputs(w, nh)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    t = {k: (None if v is None else to_dev(v, dt if k in ("q", "k", "v") else torch.float32, torch))
+         for k, v in x.items()}
+    o = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device="cuda")
+    ST = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device="cuda")
+
+    def step():
+        gdn.product_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], gate=w.gate, o=o, S_T=ST)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(torch.cuda.current_stream())
+    for _ in range(steps):
+        step()
+    e1.record(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    if gdn.device_status() != 0:
+        raise RuntimeError("device status after product prefill")
+    return e0.elapsed_time(e1) / steps
+
+
+def product_bytes(w, nh, out_bytes=4):
+    in_b = 2 if w.dtype == "bf16" else 4
+    per_tok = w.dk * in_b + nh * (w.dk + w.dv) * in_b + w.dv * out_bytes + 4 + 4 * nh
+    state = w.dv * w.dk * 4 * ((1 if w.s0_std > 0 else 0) + 1)
+    return w.n_heads * (w.T * per_tok + state)
+
+
 def time_prefill_e2e(w, x, steps, warmup, torch, gdn):
     """Same metric through the public API with pinned host buffers: every step
     copies the inputs host->device, runs gdn_chunk_fwd and reads o and S_T back."""
@@ -439,12 +475,25 @@ def run_ours(args):
             wo = WORKLOADS[name]
             xo = make_prefill_inputs(wo)
             mso = time_prefill(wo, xo, max(3, args.steps // 2), args.warmup, torch, gdn, dist)
+            result["gpu_launches"] += max(3, args.steps // 2)
             del xo
             nb, fl = prefill_bytes(wo), prefill_flops(wo)
             tr = max(nb / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
             others[name] = {"ms_per_step": mso, "tokens_per_s": wo.B * wo.T * world / (mso * 1e-3),
                             "achieved_gbs": nb / (mso * 1e-3) / 1e9, "roofline_us": tr * 1e6,
                             "frac_of_roofline_time": tr / (mso * 1e-3)}
+        # Gated DeltaProduct, 2 substeps per token, on the GDN workload's heads and
+        # 4096 tokens (8192 virtual steps, the GDN workload's length)
+        wp, nh = WORKLOADS["gdn_prefill_bf16"].with_(T=4096, name="gdp_prefill_bf16"), 2
+        msp = max_over_ranks(time_product(wp, nh, max(3, args.steps // 2), args.warmup, torch, gdn), dist, "cuda")
+        nb = product_bytes(wp, nh)
+        fl = prefill_flops(wp.with_(T=wp.T * nh))
+        tr = max(nb / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+        others["gdp_prefill_bf16"] = {"substeps": nh, "B": wp.B, "H": wp.H, "T": wp.T, "ms_per_step": msp,
+                                      "tokens_per_s": wp.B * wp.T * world / (msp * 1e-3),
+                                      "achieved_gbs": nb / (msp * 1e-3) / 1e9, "roofline_us": tr * 1e6,
+                                      "frac_of_roofline_time": tr / (msp * 1e-3)}
+        result["gpu_launches"] += max(3, args.steps // 2)
         result["prefill_workloads"] = others
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
