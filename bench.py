@@ -367,8 +367,9 @@ def cpu_baseline(w, budget_s=15.0):
     t0 = time.perf_counter()
     oracle.gdn_forward(w.update, w.gate, xs["q"], xs["k"], xs["v"], g=xs["g"], beta=xs["beta"], S0=xs["S0"])
     per_tok = (time.perf_counter() - t0) / probe_T
+    # as many whole heads as fit the budget on this host's cores (all of them when
+    # the whole workload does)
     n_heads = max(1, min(w.n_heads, int(budget_s * threads / max(per_tok * w.T, 1e-9))))
-    n_heads = min(n_heads, 4 * threads)
     heads = [(i // w.H, i % w.H) for i in range(n_heads)]
     xs = make_prefill_inputs(w, heads=heads)
     t0 = time.perf_counter()
