@@ -45,7 +45,7 @@ class Desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("dk", ctypes.c_int),
                 ("dv", ctypes.c_int), ("update", ctypes.c_int), ("gate", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("chunk", ctypes.c_int),
-                ("algo", ctypes.c_int)]
+                ("algo", ctypes.c_int), ("prologue", ctypes.c_int)]
 
 
 _lib = None
@@ -127,8 +127,12 @@ def _dtype_code(dt):
     raise TypeError("q, k, v, o must be bfloat16 or float32, got %s" % dt)
 
 
-def make_desc(B, H, T, dk, dv, update, gate, dtype, out_dtype, algo="auto", chunk=64) -> Desc:
-    return Desc(B, H, T, dk, dv, UPDATES[update], GATES[gate], dtype, out_dtype, chunk, ALGOS[algo])
+# Input prologue bits (GDN_PRO_*): maps applied in-kernel to the raw inputs
+PRO_QK_ELU1, PRO_QK_L2, PRO_BETA_SIGMOID, PRO_G_NEG_SOFTPLUS = 1, 2, 4, 8
+
+
+def make_desc(B, H, T, dk, dv, update, gate, dtype, out_dtype, algo="auto", chunk=64, prologue=0) -> Desc:
+    return Desc(B, H, T, dk, dv, UPDATES[update], GATES[gate], dtype, out_dtype, chunk, ALGOS[algo], prologue)
 
 
 def _check(t, name, shape, dtype=None):
@@ -145,7 +149,7 @@ def _check(t, name, shape, dtype=None):
 
 
 def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=None, o=None, S_T=None,
-              return_state=True, algo="auto", stream=None):
+              return_state=True, algo="auto", prologue=0, stream=None):
     """Prefill over T tokens (gdn_chunk_fwd).  Returns (o, S_T).
 
     q, k [B,H,T,dk]; v [B,H,T,dv] (bf16 or fp32, same dtype); g [B,H,T] or
@@ -173,7 +177,8 @@ def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=No
     if S_T is None and return_state:
         S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
     _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
-    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo)
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
+                  prologue=prologue)
     rc = load().gdn_chunk_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
                               _ptr(o), _ptr(S_T), _stream(stream))
     if rc != GDN_OK:
@@ -182,7 +187,7 @@ def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=No
 
 
 def product_fwd(q, k, v, g=None, beta=None, S0=None, *, gate, out_dtype=None, o=None, S_T=None,
-                return_state=True, algo="auto", stream=None):
+                return_state=True, algo="auto", prologue=0, stream=None):
     """Gated DeltaProduct prefill (gdn_product_fwd): nh = k.shape[-2] delta-rule
     substeps per token.  Returns (o, S_T).
 
@@ -212,7 +217,8 @@ def product_fwd(q, k, v, g=None, beta=None, S0=None, *, gate, out_dtype=None, o=
     if S_T is None and return_state:
         S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
     _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
-    d = make_desc(B, H, T, dk, dv, "delta", gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo)
+    d = make_desc(B, H, T, dk, dv, "delta", gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
+                  prologue=prologue)
     rc = load().gdn_product_fwd(ctypes.byref(d), ctypes.c_int(nh), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                 _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream))
     if rc != GDN_OK:
@@ -220,7 +226,7 @@ def product_fwd(q, k, v, g=None, beta=None, S0=None, *, gate, out_dtype=None, o=
     return o, S_T
 
 
-def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, stream=None):
+def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, prologue=0, stream=None):
     """T decode steps (gdn_decode_step, 1 <= T <= DECODE_MAX_T, usually 1); S
     [B,H,dv,dk] is updated in place and read / written once for the T tokens.
 
@@ -247,7 +253,7 @@ def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, st
     if o is None:
         o = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
     _check(o, "o", (B, H, T, dv), out_dtype)
-    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype))
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), prologue=prologue)
     rc = load().gdn_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
                                 _ptr(o), _stream(stream))
     if rc != GDN_OK:

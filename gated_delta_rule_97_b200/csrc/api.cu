@@ -47,10 +47,15 @@ int validate_common(const gdn_desc_t *d) {
         return GDN_ERR_ARG;
     const long bh = (long)d->B * d->H;
     if (bh > (1L << 30)) return GDN_ERR_ARG;
+    if (d->prologue & ~(GDN_PRO_QK_ELU1 | GDN_PRO_QK_L2 | GDN_PRO_BETA_SIGMOID | GDN_PRO_G_NEG_SOFTPLUS))
+        return GDN_ERR_ARG;
     return GDN_OK;
 }
 
 int from_cuda(int e) { return e == 0 ? GDN_OK : GDN_ERR_CUDA; }
+
+// Which input prologue maps the pipelined tensor-core kernel applies itself.
+bool tc2_prologue_ok(const gdn_desc_t *d) { return d->prologue == 0; }
 
 }  // namespace
 
@@ -130,8 +135,11 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     a.diag = diag_ptr();
     a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
     a.nh = 1;
+    a.pro = d->prologue;
 
-    const bool tc_ok = gdn_tc_supported(d) != 0;
+    // the input prologue runs in the SIMT kernel and the pipelined tensor-core kernel
+    const bool tc_ok = gdn_tc_supported(d) != 0 && (d->prologue == 0 || d->algo != GDN_ALGO_TC_SEQ) &&
+                       tc2_prologue_ok(d);
     if ((d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) && !tc_ok) return GDN_ERR_UNSUPPORTED;
     if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
     if (d->algo == GDN_ALGO_TC_SEQ) return from_cuda(gdn_launch_chunk_tc(a, d, st));
@@ -152,7 +160,7 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     // the pipelined tensor-core kernel takes whole tokens per chunk: nh a power of
     // two (it divides the chunk), scalar or no gate
     const bool pow2 = (nh & (nh - 1)) == 0;
-    const bool tc_ok = gdn_tc_supported(d) != 0 && pow2 && d->gate != GDN_GATE_CHANNEL;
+    const bool tc_ok = gdn_tc_supported(d) != 0 && pow2 && d->gate != GDN_GATE_CHANNEL && tc2_prologue_ok(d);
     if (d->algo == GDN_ALGO_TC_SEQ || (d->algo == GDN_ALGO_TC && !tc_ok)) return GDN_ERR_UNSUPPORTED;
     if ((long)d->T * nh > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
     const long BH = (long)d->B * d->H;
@@ -183,6 +191,7 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     a.diag = diag_ptr();
     a.BH = (int)BH; a.T = (int)Tv; a.dk = d->dk; a.dv = d->dv;
     a.nh = nh;
+    a.pro = d->prologue;
     if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
     return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
 }
@@ -211,6 +220,7 @@ extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k
     gdn::DecodeArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.o = o;
     a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
+    a.pro = d->prologue;
     return from_cuda(gdn_launch_decode(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16,
                                        static_cast<cudaStream_t>(stream)));
 }

@@ -86,9 +86,9 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
             float qv = 0.f, kv = 0.f, gv = 0.f;
             if (l < n) {
                 const int m = t0 + l, tr = m / nh, sub = m - tr * nh;
-                if (sub == nh - 1) qv = to_f32(q[(size_t)tr * DK + j]);
-                kv = to_f32(k[(size_t)m * DK + j]);
-                if (GATE == kGateChannel && sub == 0) gv = g[(size_t)tr * DK + j];
+                if (sub == nh - 1) qv = pro_feature(to_f32(q[(size_t)tr * DK + j]), a.pro);
+                kv = pro_feature(to_f32(k[(size_t)m * DK + j]), a.pro);
+                if (GATE == kGateChannel && sub == 0) gv = pro_gate(g[(size_t)tr * DK + j], a.pro);
             }
             sQ[l * LDK + j] = qv;
             sK[l * LDK + j] = kv;
@@ -99,10 +99,28 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
             sV[l * LDV + c] = (l < n) ? to_f32(v[(size_t)(t0 + l) * dv + v0 + c]) : 0.f;
         }
         if (tid < C) {
-            if (GATE == kGateScalar) sG[tid] = (tid < n && (t0 + tid) % nh == 0) ? g[(t0 + tid) / nh] : 0.f;
-            if (UPD == kDelta) sB[tid] = (tid < n) ? beta[t0 + tid] : 0.f;
+            if (GATE == kGateScalar)
+                sG[tid] = (tid < n && (t0 + tid) % nh == 0) ? pro_gate(g[(t0 + tid) / nh], a.pro) : 0.f;
+            if (UPD == kDelta) sB[tid] = (tid < n) ? pro_beta(beta[t0 + tid], a.pro) : 0.f;
         }
         __syncthreads();
+        if (a.pro & kProL2) {
+            // unit rows of q and k (the A scratch is free until a2); zero rows stay zero
+            float *inv = sA;
+            if (tid < 2 * C) {
+                const float *row = (tid < C ? sQ : sK) + (tid % C) * LDK;
+                float ss = 0.f;
+                for (int j = 0; j < DK; ++j) ss = fmaf(row[j], row[j], ss);
+                inv[tid] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+            }
+            __syncthreads();
+            for (int i = tid; i < C * DK; i += kThreads) {
+                const int l = i / DK, j = i % DK;
+                sQ[l * LDK + j] *= inv[l];
+                sK[l * LDK + j] *= inv[C + l];
+            }
+            __syncthreads();
+        }
 
         // ---- a1: inclusive prefix of the log-gate ----
         if (GATE == kGateScalar) {

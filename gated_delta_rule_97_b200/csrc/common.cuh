@@ -48,6 +48,7 @@ struct ChunkArgs {
     // q, g and o per real token; a token's q sits on its last substep, its gate
     // on its first, and only the last substep's output is written.
     int nh;
+    int pro;  // GDN_PRO_* input maps
 };
 
 struct DecodeArgs {
@@ -57,7 +58,22 @@ struct DecodeArgs {
     float *S;                // [BH,dv,dk] in/out
     void *o;                 // [BH,T,dv]
     int BH, T, dk, dv;
+    int pro;                 // GDN_PRO_* input maps
 };
+
+// Input prologue maps (GDN_PRO_* bits, mirrored here for device code).
+constexpr int kProElu1 = 1, kProL2 = 2, kProBetaSigmoid = 4, kProGNegSoftplus = 8;
+
+__device__ __forceinline__ float pro_feature(float x, int pro) {
+    return (pro & kProElu1) ? (x > 0.f ? x + 1.f : __expf(x)) : x;
+}
+__device__ __forceinline__ float pro_beta(float x, int pro) {
+    return (pro & kProBetaSigmoid) ? 1.f / (1.f + __expf(-x)) : x;
+}
+__device__ __forceinline__ float pro_gate(float x, int pro) {
+    // -softplus(x) = -(max(x, 0) + log(1 + e^{-|x|}))
+    return (pro & kProGNegSoftplus) ? -(fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x)))) : x;
+}
 
 }  // namespace gdn
 

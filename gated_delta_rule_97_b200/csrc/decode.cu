@@ -59,19 +59,39 @@ struct StepIn {
         const TIn *kp = static_cast<const TIn *>(a.k) + tok * DK + c0;
 #pragma unroll
         for (int e = 0; e < V; ++e) {
-            qq[e] = to_f32(qp[e]);
-            kk[e] = to_f32(kp[e]);
+            qq[e] = pro_feature(to_f32(qp[e]), a.pro);
+            kk[e] = pro_feature(to_f32(kp[e]), a.pro);
             al[e] = 1.f;
         }
+        if (a.pro & kProL2) {
+            // unit q and k rows (a zero row stays zero); every lane gets both sums
+            float sq = 0.f, sk = 0.f;
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                sq = fmaf(qq[e], qq[e], sq);
+                sk = fmaf(kk[e], kk[e], sk);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            }
+            const float iq = sq > 0.f ? 1.f / sqrtf(sq) : 0.f, ik = sk > 0.f ? 1.f / sqrtf(sk) : 0.f;
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                qq[e] *= iq;
+                kk[e] *= ik;
+            }
+        }
         if (GATE == kGateScalar) {
-            const float x = __expf(a.g[tok]);
+            const float x = __expf(pro_gate(a.g[tok], a.pro));
 #pragma unroll
             for (int e = 0; e < V; ++e) al[e] = x;
         } else if (GATE == kGateChannel) {
 #pragma unroll
-            for (int e = 0; e < V; ++e) al[e] = __expf(a.g[tok * DK + c0 + e]);
+            for (int e = 0; e < V; ++e) al[e] = __expf(pro_gate(a.g[tok * DK + c0 + e], a.pro));
         }
-        bt = (UPD == kDelta) ? a.beta[tok] : 0.f;
+        bt = (UPD == kDelta) ? pro_beta(a.beta[tok], a.pro) : 0.f;
         const TIn *vp = static_cast<const TIn *>(a.v) + tok * a.dv + i0;
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) vv[r] = to_f32(vp[r]);

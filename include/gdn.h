@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define GDN_VERSION 1
+#define GDN_VERSION 2
 
 /* Return codes. */
 #define GDN_OK 0
@@ -80,6 +80,23 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
  * the request). */
 typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TC = 2, GDN_ALGO_TC_SEQ = 3 } gdn_algo_t;
 
+/* Input prologue (bits of gdn_desc_t.prologue): maps the kernels apply to their
+ * inputs as they load them, so that raw projections can be passed directly.
+ *   QK_ELU1        q, k <- elu(x) + 1 elementwise, the feature map of linear
+ *                  attention ("Linear attention: a running sum" code; "Beyond
+ *                  attention" linear-attention forward)
+ *   QK_L2          each q and k row <- x / |x|_2 (after QK_ELU1 when both are
+ *                  set; a zero row stays zero), the normalised keys and queries
+ *                  of the DeltaNet forward
+ *   BETA_SIGMOID   beta <- 1 / (1 + e^{-beta}) (write strength from a logit)
+ *   G_NEG_SOFTPLUS g <- -softplus(g) = -log(1 + e^{g}) (log-gate from a logit,
+ *                  the softplus step of "Optional: Constructing the decay gate")
+ * The oracle applies the same maps in float64 before the recurrence. */
+#define GDN_PRO_QK_ELU1 1
+#define GDN_PRO_QK_L2 2
+#define GDN_PRO_BETA_SIGMOID 4
+#define GDN_PRO_G_NEG_SOFTPLUS 8
+
 typedef struct {
     int B, H;      /* batch and heads; B*H >= 0 */
     int T;         /* tokens per sequence (gdn_chunk_fwd: T >= 0; decode: T == 1) */
@@ -90,6 +107,7 @@ typedef struct {
     int out_dtype; /* gdn_dtype_t of o */
     int chunk;     /* chunk length C of the chunkwise form; 0 or 64 (others rejected) */
     int algo;      /* gdn_algo_t (gdn_chunk_fwd only; ignored by decode) */
+    int prologue;  /* GDN_PRO_* bits, 0 = inputs used as given */
 } gdn_desc_t;
 
 /*

@@ -10,7 +10,9 @@ Two implementations of the same definition:
   over heads), for every size the tests and the benchmark use;
 * ``gdn_forward_np`` -- the same three steps written with NumPy, vectorised
   over heads, for small cases and to cross-check the compiled one;
-* ``gdp_forward`` -- Gated DeltaProduct (n_h delta substeps per token), NumPy.
+* ``gdp_forward`` -- Gated DeltaProduct (n_h delta substeps per token), NumPy;
+* ``prologue`` -- the optional input maps (feature map, L2 rows, sigmoid,
+  -softplus) applied before the recurrence.
 
 Definition (column convention, S in R^{dv x dk}, stored [B,H,dv,dk]):
 ``S_t = S_{t-1} Diag(alpha_t)(I - beta_t k_t k_t^T) + beta_t v_t k_t^T``,
@@ -173,6 +175,34 @@ def gdp_forward(gate, q, k, v, g=None, beta=None, S0=None):
             S = S + u[..., :, None] * kj[..., None, :]
         o[..., t, :] = np.einsum("...ij,...j->...i", S, q[..., t, :])
     return o, S
+
+
+PRO_QK_ELU1, PRO_QK_L2, PRO_BETA_SIGMOID, PRO_G_NEG_SOFTPLUS = 1, 2, 4, 8
+
+
+def prologue(flags, q=None, k=None, beta=None, g=None):
+    """The input maps of the prologue bits, in float64, applied before the
+    recurrence: q, k <- elu(x) + 1 ("Linear attention: a running sum"); q, k rows
+    <- x / |x|_2, a zero row kept zero (the DeltaNet forward's normalised q, k);
+    beta <- sigmoid(beta); g <- -softplus(g) ("Optional: Constructing the decay
+    gate").  Returns (q, k, beta, g)."""
+    def feat(x):
+        if x is None:
+            return None
+        x = _f64(x)
+        if flags & PRO_QK_ELU1:
+            x = np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+        if flags & PRO_QK_L2:
+            n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+            x = np.where(n > 0, x / np.where(n > 0, n, 1.0), 0.0)
+        return x
+    q, k = feat(q), feat(k)
+    beta, g = _f64(beta), _f64(g)
+    if beta is not None and flags & PRO_BETA_SIGMOID:
+        beta = 1.0 / (1.0 + np.exp(-beta))
+    if g is not None and flags & PRO_G_NEG_SOFTPLUS:
+        g = -(np.maximum(g, 0.0) + np.log1p(np.exp(-np.abs(g))))
+    return q, k, beta, g
 
 
 def decode_sequence(update, gate, S0, steps):

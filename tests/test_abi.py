@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_strerror_and_version(lib):
-    assert gdn.version() == 1
+    assert gdn.version() == 2  # gdn_desc_t gained the prologue field
     for code in (0, -1, -2, -3, -4, -5, -6, 123):
         assert isinstance(gdn.strerror(code), str) and gdn.strerror(code)
 
@@ -81,6 +81,13 @@ def test_rejects_bad_arguments_without_launching(lib):
 def test_empty_batch_is_a_noop(lib):
     assert _call(lib, _desc(B=0)) == 0
     assert _call(lib, _desc(H=0), q=None, k=None, v=None, g=None, beta=None, o=None) == 0
+
+
+def test_unknown_prologue_bits_are_rejected(lib):
+    d = _desc(prologue=16)
+    assert _call(lib, d) == -1
+    d = _desc(prologue=1 | 2 | 4 | 8, B=0)
+    assert _call(lib, d) == 0
 
 
 def test_decode_rejects_bad_arguments(lib):

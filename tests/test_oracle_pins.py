@@ -491,3 +491,36 @@ def test_gdp_zero_write_strength_only_decays(oracle_mod):
     G = np.cumsum(g, axis=1)
     expect = np.einsum("bij,btj->bti", S0, q) * np.exp(G)[..., None]
     assert rel_err(o, expect) < TOL and rel_err(S, S0 * np.exp(G[:, -1])[:, None, None]) < TOL
+
+
+# ---------------------------------------------------------------------------
+# Input prologue maps: values fixed by the definitions of elu, the 2-norm,
+# the logistic function and softplus
+# ---------------------------------------------------------------------------
+
+def test_prologue_closed_forms():
+    x = np.array([[-np.inf, -1.0, 0.0, 2.0]])
+    q, _, _, _ = oracle.prologue(oracle.PRO_QK_ELU1, q=x)
+    assert np.allclose(q, [[0.0, np.exp(-1.0), 1.0, 3.0]], rtol=0, atol=1e-15)
+    b = np.array([0.0, np.log(3.0), -np.log(3.0)])
+    _, _, beta, _ = oracle.prologue(oracle.PRO_BETA_SIGMOID, beta=b)
+    assert np.allclose(beta, [0.5, 0.75, 0.25], rtol=0, atol=1e-15)
+    gx = np.array([0.0, np.log(np.e - 1.0), -50.0, 50.0])
+    _, _, _, g = oracle.prologue(oracle.PRO_G_NEG_SOFTPLUS, g=gx)
+    assert np.allclose(g, [-np.log(2.0), -1.0, -np.exp(-50.0), -50.0 - np.exp(-50.0)], rtol=1e-14, atol=1e-300)
+
+
+def test_prologue_l2_rows():
+    r = np.random.default_rng(41)
+    x = r.standard_normal((3, 7, 16)) * r.uniform(0.1, 10.0, (3, 7, 1))
+    x[1, 2] = 0.0
+    q, k, _, _ = oracle.prologue(oracle.PRO_QK_L2, q=x, k=3.0 * x)
+    n = np.linalg.norm(q, axis=-1)
+    mask = np.ones((3, 7), bool)
+    mask[1, 2] = False
+    assert np.allclose(n[mask], 1.0, atol=1e-14) and np.all(q[1, 2] == 0.0)
+    assert np.allclose(q, k, atol=1e-15)  # scale-free
+    # feature map first, then the norm
+    q2, _, _, _ = oracle.prologue(oracle.PRO_QK_ELU1 | oracle.PRO_QK_L2, q=x)
+    e = np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+    assert np.allclose(q2, e / np.linalg.norm(e, axis=-1, keepdims=True), atol=1e-15)
