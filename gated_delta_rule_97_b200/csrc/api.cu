@@ -54,8 +54,8 @@ int validate_common(const gdn_desc_t *d) {
 
 int from_cuda(int e) { return e == 0 ? GDN_OK : GDN_ERR_CUDA; }
 
-// Which input prologue maps the pipelined tensor-core kernel applies itself.
-bool tc2_prologue_ok(const gdn_desc_t *d) { return d->prologue == 0; }
+// The pipelined tensor-core kernel applies every input prologue map itself.
+bool tc2_prologue_ok(const gdn_desc_t *) { return true; }
 
 }  // namespace
 
@@ -137,7 +137,8 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     a.nh = 1;
     a.pro = d->prologue;
 
-    // the input prologue runs in the SIMT kernel and the pipelined tensor-core kernel
+    // the input prologue runs in the SIMT kernel and the pipelined tensor-core
+    // kernel, not in the sequential one
     const bool tc_ok = gdn_tc_supported(d) != 0 && (d->prologue == 0 || d->algo != GDN_ALGO_TC_SEQ) &&
                        tc2_prologue_ok(d);
     if ((d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) && !tc_ok) return GDN_ERR_UNSUPPORTED;

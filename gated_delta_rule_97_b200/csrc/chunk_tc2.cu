@@ -79,6 +79,7 @@ struct Params {
     int *diag;
     int BH, T, dv, nslices;
     int lnh;  // log2 of the substeps per token (Gated DeltaProduct), else 0
+    int pro;  // GDN_PRO_* input maps
 };
 
 template <int DVS, int GATE>
@@ -103,6 +104,8 @@ struct Misc {
     float b[64];
     float gam[64];
     float ib[64];
+    float iq[64], ik[64];  // unit-row factors 1/|q_l|, 1/|k_l| (input map, unit rows only)
+    float ibk[64];         // ib * ik
     float beta[2][64];  // by chunk parity: the solve of chunk r overlaps the gate pass of r+1
     float GC[128];
     int abort_flag, range_flag, slow_chunk, abort_site;
@@ -111,12 +114,29 @@ struct Misc {
     uint64_t bar_tma, bar_p1, bar_x, bar_rdy, bar_fA, bar_fB0, bar_fB1, bar_tv;
 };
 
+static_assert(sizeof(Misc) <= 3072, "the Misc block has 3 KB of shared memory");
+
 template <typename M>
 __device__ __forceinline__ void note_timeout(M &ms, int site, int r) {
     if (atomicCAS(&ms.abort_flag, 0, 1) == 0) ms.abort_site = site * 1000000 + r;
 }
 
 constexpr uint32_t TP = 0, TZ = 64, TOX = 128, TSM = 256, TS16 = 384, TZ16 = 448;
+
+// Eight raw q / k elements as fp32: bf16 as loaded, fp16 once the input map has run.
+__device__ __forceinline__ void unpack_qk8(uint4 u, float *f, bool f16) {
+    if (f16) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+            f[2 * i] = x.x;
+            f[2 * i + 1] = x.y;
+        }
+    } else {
+        unpack_bf16x8(u, f);
+    }
+}
 
 // Float index of gate element (token l, channel c) in the channel-gate tile: four
 // [64][32] fp32 sub-tiles loaded by TMA with the 128-byte swizzle (16-byte slot
@@ -147,7 +167,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     // rdy when the prep group is the longer side (delta rule, scalar / no gate), else
     // by the prep group itself (it then has slack; the channel gate's P also needs
     // the converted operands)
-    constexpr bool kStateP1 = DELTA && GATE != kGateChannel && !PROD;
+    // With the elu+1 input map (alone or before unit rows) the raw tiles are mapped
+    // in place to fp16 after they land, so P follows that pass and is issued by the
+    // prep group.  Unit rows alone leave the tiles as they are: the row norms
+    // become factors on P (rows and columns) and on the converted operands.
+    const bool qkmap = (p.pro & kProElu1) != 0;
+    const bool l2scale = (p.pro & kProL2) != 0 && !qkmap;
+    const bool kStateP1 = DELTA && GATE != kGateChannel && !PROD && !qkmap;
     // In the same modes the V tile has its own TMA barrier (bar_tv): its fp16
     // conversion runs during the 16 -> 32 merge, after the q / k conversion window
     constexpr bool kSplitV = DELTA && GATE != kGateChannel;
@@ -217,16 +243,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     // the token's gate on its first substep, 1 (g = 0) on the others
                     const int m0 = t0 + l0, m1 = m0 + 1, msk = (1 << p.lnh) - 1;
                     const size_t gb = (size_t)bh * (T >> p.lnh);
-                    gpre0 = (m0 < T && (m0 & msk) == 0) ? p.g[gb + (m0 >> p.lnh)] : 0.f;
-                    gpre1 = (m1 < T && (m1 & msk) == 0) ? p.g[gb + (m1 >> p.lnh)] : 0.f;
+                    gpre0 = (m0 < T && (m0 & msk) == 0) ? pro_gate(p.g[gb + (m0 >> p.lnh)], p.pro) : 0.f;
+                    gpre1 = (m1 < T && (m1 & msk) == 0) ? pro_gate(p.g[gb + (m1 >> p.lnh)], p.pro) : 0.f;
                 } else {
-                    gpre0 = (t0 + l0 < T) ? p.g[(size_t)bh * T + t0 + l0] : 0.f;
-                    gpre1 = (t0 + l0 + 1 < T) ? p.g[(size_t)bh * T + t0 + l0 + 1] : 0.f;
+                    gpre0 = (t0 + l0 < T) ? pro_gate(p.g[(size_t)bh * T + t0 + l0], p.pro) : 0.f;
+                    gpre1 = (t0 + l0 + 1 < T) ? pro_gate(p.g[(size_t)bh * T + t0 + l0 + 1], p.pro) : 0.f;
                 }
             }
             if (DELTA && t >= 128 && t < 128 + C) {
                 const int l = t - 128;
-                bpre = (t0 + l < T) ? p.beta[(size_t)bh * T + t0 + l] : 0.f;
+                bpre = (t0 + l < T) ? pro_beta(p.beta[(size_t)bh * T + t0 + l], p.pro) : 0.f;
             }
         };
         // scalar gate prefix of chunk r and its factors b = e^G, gamma = e^{G_C-G},
@@ -321,11 +347,69 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 fence_proxy_async_smem();
                 named_bar(kPrepBar, 256);
             }
+            if (qkmap) {
+                // q / k input map in place: thread = (tensor, row, key half); the two
+                // halves of a row are adjacent lanes.  Rows past T and, for the
+                // product, q rows that are not a token's last substep stay zero.
+                const int ten = t >> 7, row = (t >> 1) & 63, hk = t & 1;
+                const int m = r * C + row;
+                bool valid = m < T;
+                if (PROD && ten == 0) valid = valid && ((row & ((1 << p.lnh) - 1)) == (1 << p.lnh) - 1);
+                unsigned char *base = sm + L::RAW_QK + hk * 16384 + ten * 8192 + row * 128;
+                float f[64];
+                float ss = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(base + ((c ^ (row & 7)) << 4)), f + 8 * c);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        f[8 * c + e] = valid ? pro_feature(f[8 * c + e], p.pro) : 0.f;
+                        ss = fmaf(f[8 * c + e], f[8 * c + e], ss);
+                    }
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                const float sc = (p.pro & kProL2) ? (ss > 0.f ? 1.f / sqrtf(ss) : 0.f) : 1.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        f[8 * c + e] *= sc;
+                        rmax = fmaxf(rmax, fabsf(f[8 * c + e]));
+                    }
+                    *reinterpret_cast<uint4 *>(base + ((c ^ (row & 7)) << 4)) = pack_h8(f + 8 * c);
+                }
+                fence_proxy_async_smem();
+                named_bar(kPrepBar, 256);
+            }
+            if (l2scale) {
+                // 1 / |row| of every q and k row (thread = tensor, row, key half)
+                const int ten = t >> 7, row = (t >> 1) & 63, hk = t & 1;
+                const unsigned char *base = sm + L::RAW_QK + hk * 16384 + ten * 8192 + row * 128;
+                float ss = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float f[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(base + ((c ^ (row & 7)) << 4)), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+                if (hk == 0) {
+                    if (ten == 0) {
+                        ms.iq[row] = inv;
+                    } else {
+                        ms.ik[row] = inv;
+                        ms.ibk[row] = (GATE == kGateScalar ? ms.ib[row] : 1.f) * inv;
+                    }
+                }
+                named_bar(kPrepBar, 256);
+            }
             TC2_MARK(0, 1);
             if (!kStateP1 && GATE != kGateChannel && t == 0 && !ms.abort_flag) {
                 tc_fence_after();
                 const uint32_t qk = smem_u32(sm + L::RAW_QK);
-                constexpr uint32_t id = idesc_f16(128, 64, 1, 0, 0);
+                const uint32_t id = qkmap ? idesc_f16(128, 64, 0, 0, 0) : idesc_f16(128, 64, 1, 0, 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32;
@@ -341,7 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 float *gt = reinterpret_cast<float *>(sm + L::GCH);
                 float gv[32];
 #pragma unroll
-                for (int l = 0; l < 32; ++l) gv[l] = gt[gch_idx(32 * hf + l, c)];
+                for (int l = 0; l < 32; ++l) {
+                    gv[l] = gt[gch_idx(32 * hf + l, c)];
+                    if (r * C + 32 * hf + l < T) gv[l] = pro_gate(gv[l], p.pro);  // padding stays g = 0
+                }
 #pragma unroll
                 for (int l = 1; l < 32; ++l) gv[l] += gv[l - 1];
                 if (hf == 0) {
@@ -423,8 +510,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         const int l = off >> 7;
                         const int c0 = h * 64 + ((((off >> 4) & 7) ^ (l & 7)) << 3);
                         float qf[8], kf[8], ql[8], kl[8], kr[8];
-                        unpack_bf16x8(rq[s4], qf);
-                        unpack_bf16x8(rk[s4], kf);
+                        unpack_qk8(rq[s4], qf, qkmap);
+                        unpack_qk8(rk[s4], kf, qkmap);
+                        if (l2scale) {
+                            const float fq = ms.iq[l], fk = ms.ik[l];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                qf[e] *= fq;
+                                kf[e] *= fk;
+                            }
+                        }
 #pragma unroll
                         for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fmaxf(fabsf(qf[e]), fabsf(kf[e])));
                         if (GATE == kGateChannel) {
@@ -502,8 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     const int h = i >> 9, off = (i & 511) * 16;
                     const int l = off >> 7;
                     float kf[8], kr[8];
-                    unpack_bf16x8(rk[s4], kf);
-                    const float gl = (GATE == kGateScalar) ? ms.gam[l] : 1.f;
+                    unpack_qk8(rk[s4], kf, qkmap);
+                    const float gl = ((GATE == kGateScalar) ? ms.gam[l] : 1.f) * (l2scale ? ms.ik[l] : 1.f);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         rmax = fmaxf(rmax, fabsf(kf[e]));
@@ -555,25 +650,29 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                             for (int c = 0; c < DK; ++c) {
                                 const int h = c >> 6;
                                 const uint32_t ox = sw128_off(l, c & 63), om = sw128_off(m, c & 63);
-                                const float xv =
-                                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xrow + h * 16384 + ox));
-                                const float kv = __bfloat162float(
-                                    *reinterpret_cast<const __nv_bfloat16 *>(sm + L::RAW_QK + h * 16384 + 8192 + om));
+                                const void *xp = xrow + h * 16384 + ox, *kp = sm + L::RAW_QK + h * 16384 + 8192 + om;
+                                const float xv = qkmap ? __half2float(*reinterpret_cast<const __half *>(xp))
+                                                       : __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xp));
+                                const float kv = qkmap ? __half2float(*reinterpret_cast<const __half *>(kp))
+                                                       : __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kp));
                                 const float *gt = reinterpret_cast<const float *>(sm + L::GCH);
                                 acc = fmaf(xv * kv, __expf(gt[gch_idx(l, c)] - gt[gch_idx(m, c)]), acc);
                             }
                         }
-                        pr[e] = acc;
+                        pr[e] = l2scale ? acc * (top ? ms.iq[l] : ms.ik[l]) * ms.ik[m] : acc;
                     }
                 }
                 // decay factors e^{G_l - G_m}: all shared loads first, then the stores
                 float dm[32];
                 if (GATE == kGateScalar) {
                     if (fastg) {
-                        const float bl = ms.b[l];
+                        // b_l / b_m (times 1 / |k_m| and the row's 1 / |q_l| or 1 / |k_l|
+                        // when rows are made unit)
+                        const float bl = ms.b[l] * (l2scale ? (top ? ms.iq[l] : ms.ik[l]) : 1.f);
+                        const float *ibm = l2scale ? ms.ibk : ms.ib;
 #pragma unroll
                         for (int e = 0; e < 32; e += 4) {
-                            const float4 x = *reinterpret_cast<const float4 *>(&ms.ib[m0 + e]);
+                            const float4 x = *reinterpret_cast<const float4 *>(&ibm[m0 + e]);
                             dm[e] = bl * x.x; dm[e + 1] = bl * x.y; dm[e + 2] = bl * x.z; dm[e + 3] = bl * x.w;
                         }
                     } else {
@@ -584,7 +683,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                             dm[e] = __expf(Gl - fmaxf(x.x, Gl)); dm[e + 1] = __expf(Gl - fmaxf(x.y, Gl));
                             dm[e + 2] = __expf(Gl - fmaxf(x.z, Gl)); dm[e + 3] = __expf(Gl - fmaxf(x.w, Gl));
                         }
+                        if (l2scale) {
+                            const float fl = top ? ms.iq[l] : ms.ik[l];
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) dm[e] *= fl * ms.ik[m0 + e];
+                        }
                     }
+                } else if (GATE == kGateNone && l2scale) {
+                    const float fl = top ? ms.iq[l] : ms.ik[l];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) dm[e] = fl * ms.ik[m0 + e];
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) dm[e] = 1.f;
@@ -645,13 +753,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         const int i = wt + NW * s4;
                         const int j = i & 1023;
                         float f[8];
-                        unpack_bf16x8(raw[s4], f);
+                        unpack_qk8(raw[s4], f, qkmap && i < NQK);  // v stays bf16
 #pragma unroll
                         for (int e = 0; e < 8; ++e) rmax = fmaxf(rmax, fabsf(f[e]));
                         if (i < NQK) {
                             // q -> Q< (i < 1024), k -> K< (delta): row l scaled by b_l = e^{G_l}
                             const int h = j >> 9, off = (j & 511) * 16;
-                            const float bl = (GATE == kGateScalar) ? ms.b[off >> 7] : 1.f;
+                            float bl = (GATE == kGateScalar) ? ms.b[off >> 7] : 1.f;
+                            if (l2scale) bl *= (i < 1024) ? ms.iq[off >> 7] : ms.ik[off >> 7];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) f[e] *= bl;
                             *reinterpret_cast<uint4 *>(sm + L::AT + h * 16384 + (i >> 10) * 8192 + off) = pack_h8(f);
@@ -1255,6 +1364,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     prm.dv = a.dv;
     prm.nslices = a.dv / dvs;
     prm.lnh = lnh;
+    prm.pro = a.pro;
     const long grid = (long)a.BH * prm.nslices;
     if (grid == 0) return 0;
     if (lnh > 0) {
