@@ -78,6 +78,10 @@ def load():
     lib.gdn_decode_step.restype = ctypes.c_int
     lib.gdn_product_fwd.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.gdn_product_fwd.restype = ctypes.c_int
+    lib.gdn_segmented_workspace_bytes.argtypes = [dp, ctypes.c_int]
+    lib.gdn_segmented_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_chunk_fwd_segmented.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.gdn_chunk_fwd_segmented.restype = ctypes.c_int
     lib.gdn_strerror.argtypes = [ctypes.c_int]
     lib.gdn_strerror.restype = ctypes.c_char_p
     lib.gdn_device_status.argtypes = [ctypes.c_int]
@@ -224,6 +228,53 @@ def product_fwd(q, k, v, g=None, beta=None, S0=None, *, gate, out_dtype=None, o=
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_product_fwd")
     return o, S_T
+
+
+def chunk_fwd_segmented(q, k, v, g=None, beta=None, S0=None, *, update, gate, nseg, out_dtype=None, o=None,
+                        S_T=None, return_state=True, algo="auto", prologue=0, workspace=None, stream=None):
+    """gdn_chunk_fwd_segmented: the prefill with each sequence cut into ``nseg``
+    segments that run in parallel.  Same tensors as chunk_fwd; ``workspace`` is a
+    CUDA uint8 tensor of at least segmented_workspace_bytes(...) bytes (allocated
+    here through PyTorch when None).  Returns (o, S_T)."""
+    import torch
+
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
+    if gate == "scalar":
+        _check(g, "g", (B, H, T), torch.float32)
+    elif gate == "channel":
+        _check(g, "g", (B, H, T, dk), torch.float32)
+    _check(beta, "beta", (B, H, T), torch.float32)
+    _check(S0, "S0", (B, H, dv, dk), torch.float32)
+    if out_dtype is None:
+        out_dtype = o.dtype if o is not None else torch.float32
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
+    _check(o, "o", (B, H, T, dv), out_dtype)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
+                  prologue=prologue)
+    need = load().gdn_segmented_workspace_bytes(ctypes.byref(d), int(nseg))
+    if workspace is None:
+        workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous() or workspace.numel() * workspace.element_size() < need:
+        raise ValueError("workspace needs %d contiguous CUDA bytes" % need)
+    rc = load().gdn_chunk_fwd_segmented(ctypes.byref(d), int(nseg), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                        _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                                        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_chunk_fwd_segmented")
+    return o, S_T
+
+
+def segmented_workspace_bytes(B, H, T, dk, dv, nseg) -> int:
+    d = make_desc(B, H, T, dk, dv, "delta", "scalar", BF16, F32)
+    return int(load().gdn_segmented_workspace_bytes(ctypes.byref(d), int(nseg)))
 
 
 def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, prologue=0, stream=None):

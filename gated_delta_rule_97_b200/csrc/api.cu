@@ -10,6 +10,11 @@
 __device__ int g_gdn_status = 0;
 __device__ int g_gdn_diag = 0;
 
+// tensor-core launchers (chunk_tc.cu, chunk_tc2.cu)
+int gdn_tc_supported(const gdn_desc_t *d);
+int gdn_launch_chunk_tc(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
+int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
+
 namespace {
 
 int *status_ptr() {
@@ -54,6 +59,22 @@ int validate_common(const gdn_desc_t *d) {
 
 int from_cuda(int e) { return e == 0 ? GDN_OK : GDN_ERR_CUDA; }
 
+bool tc2_prologue_ok(const gdn_desc_t *d);
+
+// Kernel choice of gdn_chunk_fwd (and of the passes of the segmented prefill):
+// the requested kernel, or for AUTO the pipelined tensor-core kernel when it
+// serves the request and the SIMT kernel otherwise.  The input prologue runs in
+// the SIMT kernel and the pipelined tensor-core kernel, not in the sequential one.
+int dispatch_chunk(const gdn_desc_t *d, gdn::ChunkArgs &a, cudaStream_t st) {
+    const bool tc_ok = gdn_tc_supported(d) != 0 && (d->prologue == 0 || d->algo != GDN_ALGO_TC_SEQ) &&
+                       tc2_prologue_ok(d);
+    if ((d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) && !tc_ok) return GDN_ERR_UNSUPPORTED;
+    if (a.mode != 0 && d->algo == GDN_ALGO_TC_SEQ) return GDN_ERR_UNSUPPORTED;
+    if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
+    if (d->algo == GDN_ALGO_TC_SEQ) return from_cuda(gdn_launch_chunk_tc(a, d, st));
+    return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
+}
+
 // The pipelined tensor-core kernel applies every input prologue map itself.
 bool tc2_prologue_ok(const gdn_desc_t *) { return true; }
 
@@ -93,12 +114,10 @@ extern "C" int gdn_device_diag(void) {
     return v;
 }
 
-int gdn_tc_supported(const gdn_desc_t *d);
-int gdn_launch_chunk_tc(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
-int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
 
-extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
-                             const float *beta, const float *S0, void *o, float *S_T, void *stream) {
+// Argument rules of gdn_chunk_fwd (sizes, pointers, alignment, overlaps).
+static int chunk_fwd_check(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const float *S0, const void *o, const float *S_T) {
     int rc = validate_common(d);
     if (rc != GDN_OK) return rc;
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
@@ -125,6 +144,15 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
         return GDN_ERR_ARG;
     if (S_T && S0 && S_T != S0 && overlaps(S_T, n_S * 4, S0, n_S * 4)) return GDN_ERR_ARG;
 
+    return GDN_OK;
+}
+
+extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *S0, void *o, float *S_T, void *stream) {
+    const int rc = chunk_fwd_check(d, q, k, v, g, beta, S0, o, S_T);
+    if (rc != GDN_OK) return rc;
+    const long BH = (long)d->B * d->H;
+    const size_t n_S = (size_t)BH * d->dv * d->dk;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (BH == 0) return GDN_OK;
     if (d->T == 0) return from_cuda(gdn_launch_copy_state(S0, S_T, (long)n_S, st));
@@ -136,15 +164,8 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
     a.nh = 1;
     a.pro = d->prologue;
-
-    // the input prologue runs in the SIMT kernel and the pipelined tensor-core
-    // kernel, not in the sequential one
-    const bool tc_ok = gdn_tc_supported(d) != 0 && (d->prologue == 0 || d->algo != GDN_ALGO_TC_SEQ) &&
-                       tc2_prologue_ok(d);
-    if ((d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) && !tc_ok) return GDN_ERR_UNSUPPORTED;
-    if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
-    if (d->algo == GDN_ALGO_TC_SEQ) return from_cuda(gdn_launch_chunk_tc(a, d, st));
-    return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
+    a.mode = 0;
+    return dispatch_chunk(d, a, st);
 }
 
 extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const void *k, const void *v,
@@ -193,8 +214,83 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     a.BH = (int)BH; a.T = (int)Tv; a.dk = d->dk; a.dv = d->dv;
     a.nh = nh;
     a.pro = d->prologue;
+    a.mode = 0;
     if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
     return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
+}
+
+extern "C" size_t gdn_segmented_workspace_bytes(const gdn_desc_t *d, int nseg) {
+    if (!d || nseg < 1) return 0;
+    const size_t segs = (size_t)d->B * d->H * nseg;
+    return segs * ((size_t)2 * d->dv * d->dk + (size_t)d->dk * d->dk) * sizeof(float);
+}
+
+extern "C" int gdn_chunk_fwd_segmented(const gdn_desc_t *d, int nseg, const void *q, const void *k, const void *v,
+                                       const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = validate_common(d);
+    if (rc != GDN_OK) return rc;
+    if (nseg < 1) return GDN_ERR_ARG;
+    if (nseg == 1) return gdn_chunk_fwd(d, q, k, v, g, beta, S0, o, S_T, stream);
+    if (d->T % nseg != 0) return GDN_ERR_ARG;
+    if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC_SEQ) return GDN_ERR_ARG;
+    const long BH = (long)d->B * d->H;
+    if (BH * nseg > (1L << 30)) return GDN_ERR_ARG;
+    const size_t need = gdn_segmented_workspace_bytes(d, nseg);
+    if (BH > 0 && d->T > 0) {
+        if (!workspace || workspace_bytes < need) return GDN_ERR_ARG;
+        if (!aligned16(workspace)) return GDN_ERR_ALIGN;
+    }
+    // the same argument rules as gdn_chunk_fwd, checked on the whole request
+    rc = chunk_fwd_check(d, q, k, v, g, beta, S0, o, S_T);
+    if (rc != GDN_OK) return rc;
+    const size_t n_o = (size_t)BH * d->T * d->dv * elem_size(d->out_dtype);
+    if (overlaps(workspace, need, o, n_o) || overlaps(workspace, need, S_T, (size_t)BH * d->dv * d->dk * 4) ||
+        overlaps(workspace, need, S0, (size_t)BH * d->dv * d->dk * 4))
+        return GDN_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (BH == 0) return GDN_OK;
+    if (d->T == 0) return from_cuda(gdn_launch_copy_state(S0, S_T, (long)BH * d->dv * d->dk, st));
+
+    // segments of one sequence are consecutive runs of T / nseg tokens, so the
+    // [B,H,T,d] tensors are [B*H*nseg, T/nseg, d] tensors of shorter "heads"
+    const int segs = (int)(BH * nseg);
+    float *H = static_cast<float *>(workspace);
+    float *Sstart = H + (size_t)segs * d->dv * d->dk;
+    float *Lam = Sstart + (size_t)segs * d->dv * d->dk;
+    gdn_desc_t sd = *d;
+    sd.B = (int)BH;
+    sd.H = nseg;
+    sd.T = d->T / nseg;
+    gdn::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o;
+    a.status = status_ptr();
+    a.diag = diag_ptr();
+    a.BH = segs; a.T = sd.T; a.dk = d->dk; a.dv = d->dv;
+    a.nh = 1;
+    a.pro = d->prologue;
+    // 1. every segment from a zero state: H_i (the outputs are rewritten in pass 3)
+    a.S0 = nullptr; a.ST = H; a.mode = 0;
+    if ((rc = dispatch_chunk(&sd, a, st)) != GDN_OK) return rc;
+    // 2. every segment's transition Lambda_i: zero values from the identity state
+    //    (with the additive write and no gate the transition is the identity)
+    const bool identity = d->update == GDN_ADDITIVE;
+    if (!identity) {
+        gdn_desc_t ld = sd;
+        ld.dv = d->dk;
+        gdn::ChunkArgs b = a;
+        b.v = nullptr; b.o = nullptr; b.S0 = nullptr; b.ST = Lam; b.dv = d->dk;
+        b.mode = gdn::kModeZeroV | gdn::kModeNoOut | gdn::kModeS0Eye;
+        if ((rc = dispatch_chunk(&ld, b, st)) != GDN_OK) return rc;
+    }
+    // 3. the state entering each segment, and the final state
+    if ((rc = from_cuda(gdn_launch_compose(S0, H, identity ? nullptr : Lam, Sstart, S_T, (int)BH, nseg, d->dk,
+                                           d->dv, st))) != GDN_OK)
+        return rc;
+    // 4. every segment from its true incoming state: the outputs
+    a.S0 = Sstart; a.ST = nullptr; a.mode = 0;
+    return dispatch_chunk(&sd, a, st);
 }
 
 extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,

@@ -74,7 +74,8 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
 
     for (int i = tid; i < kDvs * DK; i += kThreads) {
         const int vv = i / DK, j = i % DK;
-        sS[vv * LDK + j] = a.S0 ? a.S0[((size_t)bh * dv + v0 + vv) * DK + j] : 0.f;
+        sS[vv * LDK + j] = (a.mode & kModeS0Eye) ? (v0 + vv == j ? 1.f : 0.f)
+                           : a.S0 ? a.S0[((size_t)bh * dv + v0 + vv) * DK + j] : 0.f;
     }
 
     for (int t0 = 0; t0 < T; t0 += C) {
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         }
         for (int i = tid; i < C * kDvs; i += kThreads) {
             const int l = i / kDvs, c = i % kDvs;
-            sV[l * LDV + c] = (l < n) ? to_f32(v[(size_t)(t0 + l) * dv + v0 + c]) : 0.f;
+            sV[l * LDV + c] = (l < n && !(a.mode & kModeZeroV)) ? to_f32(v[(size_t)(t0 + l) * dv + v0 + c]) : 0.f;
         }
         if (tid < C) {
             if (GATE == kGateScalar)
@@ -229,7 +230,8 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
             if (GATE == kGateScalar) hist *= __expf(sG[l]);
             float loc = 0.f;
             for (int m = 0; m <= l; ++m) loc = fmaf(sA[l * LDC + m], sV[m * LDV + vv], loc);
-            if (l < n && (t0 + l) % nh == nh - 1) o[(size_t)((t0 + l) / nh) * dv + v0 + vv] = from_f32<TOut>(hist + loc);
+            if (l < n && (t0 + l) % nh == nh - 1 && !(a.mode & kModeNoOut))
+                o[(size_t)((t0 + l) / nh) * dv + v0 + vv] = from_f32<TOut>(hist + loc);
         }
         __syncthreads();
 

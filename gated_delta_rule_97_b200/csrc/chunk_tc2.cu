@@ -79,7 +79,8 @@ struct Params {
     int *diag;
     int BH, T, dv, nslices;
     int lnh;  // log2 of the substeps per token (Gated DeltaProduct), else 0
-    int pro;  // GDN_PRO_* input maps
+    int pro;   // GDN_PRO_* input maps
+    int mode;  // kMode* bits (internal passes of the segmented prefill)
 };
 
 template <int DVS, int GATE>
@@ -209,9 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         ms.s_abort = 0;
         tma_prefetch_desc(&p.q_map);
         tma_prefetch_desc(&p.k_map);
-        tma_prefetch_desc(&p.v_map);
+        if (!(p.mode & kModeZeroV)) tma_prefetch_desc(&p.v_map);
         if (GATE == kGateChannel) tma_prefetch_desc(&p.g_map);
-        tma_prefetch_desc(&p.o_map);
+        if (!(p.mode & kModeNoOut)) tma_prefetch_desc(&p.o_map);
     }
     __syncwarp();
     if (warp == 0) {
@@ -220,6 +221,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     }
     // T2 tile: its upper-right 32x32 block is never written and stays zero
     for (int i = t; i < 8192 / 16; i += kThreads) reinterpret_cast<uint4 *>(sm + L::TZA)[i] = make_uint4(0, 0, 0, 0);
+    const bool zeroV = (p.mode & kModeZeroV) != 0;
+    if (zeroV) {
+        // values taken as zero: the fp16 V tiles are cleared once and never loaded
+        for (int i = t; i < DVS * 128 / 16; i += kThreads) {
+            reinterpret_cast<uint4 *>(sm + L::V16)[i] = make_uint4(0, 0, 0, 0);
+            if (!DELTA && GATE != kGateChannel) reinterpret_cast<uint4 *>(sm + L::KT)[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ms.tmem_base;
@@ -289,14 +298,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         auto issue_tma = [&](int r) {
             const int t0 = r * C;
             const uint32_t qbytes = PROD ? 2u * (64u >> p.lnh) * 128u : 16384u;
-            const uint32_t bytes = qbytes + 16384 + (kSplitV ? 0 : DVS * 128) + (GATE == kGateChannel ? 32768 : 0);
+            const uint32_t bytes =
+                qbytes + 16384 + ((kSplitV || zeroV) ? 0 : DVS * 128) + (GATE == kGateChannel ? 32768 : 0);
             mbar_arrive_expect_tx(&ms.bar_tma, bytes);
             for (int h = 0; h < 2; ++h) {
                 tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, PROD ? (t0 >> p.lnh) : t0, bh,
                             &ms.bar_tma);
                 tma_load_3d(sm + L::RAW_QK + h * 16384 + 8192, &p.k_map, h * 64, t0, bh, &ms.bar_tma);
             }
-            if (!kSplitV) issue_tma_v(r, &ms.bar_tma);
+            if (!kSplitV && !zeroV) issue_tma_v(r, &ms.bar_tma);
             if (GATE == kGateChannel)
                 for (int j = 0; j < 4; ++j) tma_load_3d(sm + L::GCH + j * 8192, &p.g_map, j * 32, t0, bh, &ms.bar_tma);
         };
@@ -306,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         };
         if (t == 0 && nchunks > 0) {
             issue_tma(0);
-            if (kSplitV) issue_tma_split_v(0);
+            if (kSplitV && !zeroV) issue_tma_split_v(0);
         }
         if (nchunks > 0) {
             load_gate_beta(0);
@@ -575,6 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     }
 #pragma unroll
                     for (int s4 = 0; s4 < 2 * NB; ++s4) {
+                        if (zeroV) break;
                         float vf[8];
                         unpack_bf16x8(rv[s4], vf);
                         *reinterpret_cast<uint4 *>(sm + L::V16 + (t + 256 * s4) * 16) = pack_h8(vf);
@@ -764,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
                             for (int e = 0; e < 8; ++e) f[e] *= bl;
                             *reinterpret_cast<uint4 *>(sm + L::AT + h * 16384 + (i >> 10) * 8192 + off) = pack_h8(f);
-                        } else if (i < NQV) {
+                        } else if (i < NQV && !zeroV) {
                             *reinterpret_cast<uint4 *>(sm + v16_slot<L, UPD, GATE>(buf) + (i - NQK) * 16) = pack_h8(f);
                         }
                     }
@@ -832,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                         gate_pass(r + 1);
                         if (r + 2 < nchunks) load_gate_beta(r + 2);
                     }
-                    if (kSplitV) {
+                    if (kSplitV && !zeroV) {
                         // V -> fp16 (its slot was released with bar_x(r-1), waited in the
                         // window), then the next chunk's v load
                         if (!mbar_wait(&ms.bar_tv, ph)) note_timeout(ms, 13, r);
@@ -987,7 +998,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
             for (int j = 0; j < 64; j += 4) {
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (p.S0 && has_row) x = *reinterpret_cast<const float4 *>(p.S0 + srow + h * 64 + j);
+                if (p.mode & kModeS0Eye) {
+                    const int c = h * 64 + j - (v0 + vrow);  // S0 = I: one 1 per row, at column v0 + vrow
+                    x = make_float4(c == 0 ? 1.f : 0.f, c == -1 ? 1.f : 0.f, c == -2 ? 1.f : 0.f, c == -3 ? 1.f : 0.f);
+                    if (!has_row) x = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else if (p.S0 && has_row) {
+                    x = *reinterpret_cast<const float4 *>(p.S0 + srow + h * 64 + j);
+                }
                 sv[j] = x.x; sv[j + 1] = x.y; sv[j + 2] = x.z; sv[j + 3] = x.w;
             }
             __syncwarp();
@@ -1154,7 +1171,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             if (!mbar_wait(fb, (r >> 1) & 1)) note_timeout(ms, 8, r);
             TC2_MARK(256, 22);
             tc_fence_after();
-            {
+            if (!(p.mode & kModeNoOut)) {
                 // O^T -> row-major staging [64 tok][DVS] -> one TMA store (rows past T
                 // clipped).  Stores issued straight from registers were measured slower:
                 // they queue behind the prep group's shared-memory traffic.
@@ -1341,7 +1358,9 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     const uint64_t Tr = T >> lnh;
     const uint32_t rows = 64u >> lnh;
     if (!make_map_3d(&prm.q_map, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, Tr, BH, 64, rows, 1, true) ||
-        !make_map_3d(&prm.k_map, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, T, BH, 64, 64, 1, true) ||
+        !make_map_3d(&prm.k_map, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, T, BH, 64, 64, 1, true))
+        return (int)cudaErrorInvalidValue;
+    if (!(a.mode & kModeZeroV) &&
         !make_map_3d(&prm.v_map, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.dv, T, BH, 64, 64, 1, true))
         return (int)cudaErrorInvalidValue;
     if (d->gate == GDN_GATE_CHANNEL &&
@@ -1349,7 +1368,8 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
         return (int)cudaErrorInvalidValue;
     const int dvs = tc2_slice(d);
     const bool ob = d->out_dtype == GDN_BF16;
-    if (!make_map_3d(&prm.o_map, a.o, ob ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+    if (!(a.mode & kModeNoOut) &&
+        !make_map_3d(&prm.o_map, a.o, ob ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                      ob ? 2 : 4, (uint64_t)a.dv, Tr, BH, (uint32_t)dvs, rows, 1, false))
         return (int)cudaErrorInvalidValue;
     prm.g = a.g;
@@ -1365,6 +1385,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     prm.nslices = a.dv / dvs;
     prm.lnh = lnh;
     prm.pro = a.pro;
+    prm.mode = a.mode;
     const long grid = (long)a.BH * prm.nslices;
     if (grid == 0) return 0;
     if (lnh > 0) {

@@ -48,8 +48,14 @@ struct ChunkArgs {
     // q, g and o per real token; a token's q sits on its last substep, its gate
     // on its first, and only the last substep's output is written.
     int nh;
-    int pro;  // GDN_PRO_* input maps
+    int pro;   // GDN_PRO_* input maps
+    int mode;  // kMode* bits (internal passes of the segmented prefill), 0 = plain
 };
+
+// Internal pass modes: values taken as zero (v not read), no output written,
+// initial state the identity (dv == dk); with all three the pass yields the
+// transition of the sequence (S_T = S0 Lambda with S0 = I).
+constexpr int kModeZeroV = 1, kModeNoOut = 2, kModeS0Eye = 4;
 
 struct DecodeArgs {
     const void *q, *k, *v;   // [BH,T,dk] / [BH,T,dv]
@@ -83,3 +89,5 @@ int gdn_launch_chunk_simt(const gdn::ChunkArgs &a, int update, int gate, int in_
 int gdn_launch_decode(const gdn::DecodeArgs &a, int update, int gate, int in_bf16, int out_bf16,
                       cudaStream_t stream);
 int gdn_launch_copy_state(const float *S0, float *ST, long n, cudaStream_t stream);
+int gdn_launch_compose(const float *S0, const float *H, const float *Lam, float *Sstart, float *ST, int BH, int nseg,
+                       int dk, int dv, cudaStream_t stream);

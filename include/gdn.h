@@ -39,6 +39,8 @@
 #ifndef GDN_H_
 #define GDN_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -159,6 +161,28 @@ int gdn_chunk_fwd(const gdn_desc_t *desc, const void *q, const void *k, const vo
 int gdn_product_fwd(const gdn_desc_t *desc, int nh, const void *q, const void *k, const void *v,
                     const float *g, const float *beta, const float *S0, void *o, float *S_T,
                     void *stream);
+
+/*
+ * gdn_chunk_fwd_segmented -- the prefill of gdn_chunk_fwd with each sequence
+ * cut into nseg segments of T / nseg tokens that run in parallel (more CTAs
+ * when B*H alone would leave the GPU idle).  A segment acts on its incoming
+ * state as an affine map, S_out = S_in Lambda + H ("One chunk as an affine
+ * recurrence", "Update the state"), so the call runs: every segment from a zero
+ * state (H), every segment's transition (zero values from the identity state;
+ * skipped for the additive write, whose transition is the identity), an
+ * in-order composition S_{i+1} = S_i Lambda_i + H_i, and every segment again
+ * from its true incoming state S_i for the outputs.  Same arguments and results
+ * as gdn_chunk_fwd, about three times its arithmetic; T must be a multiple of
+ * nseg (nseg == 1 is gdn_chunk_fwd).
+ *
+ *   workspace  device buffer of at least gdn_segmented_workspace_bytes(desc,
+ *              nseg) bytes, 16-byte aligned, owned by the caller; it must not
+ *              overlap o, S0 or S_T.  Its contents on return are unspecified.
+ */
+size_t gdn_segmented_workspace_bytes(const gdn_desc_t *desc, int nseg);
+int gdn_chunk_fwd_segmented(const gdn_desc_t *desc, int nseg, const void *q, const void *k, const void *v,
+                            const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * gdn_decode_step -- decode: T recurrent steps (1 <= T <= GDN_DECODE_MAX_T,

@@ -125,6 +125,23 @@ def test_product_rejects_bad_arguments(lib):
     assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == 0       # empty batch: no-op
 
 
+def test_segmented_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    lib.gdn_chunk_fwd_segmented.argtypes = [ctypes.c_void_p, ctypes.c_int] + [ctypes.c_void_p] * 9 + \
+        [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gdn_segmented_workspace_bytes.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    lib.gdn_segmented_workspace_bytes.restype = ctypes.c_size_t
+    d = _desc(T=96)
+    need = lib.gdn_segmented_workspace_bytes(ctypes.byref(d), 3)
+    assert need == 2 * 3 * 3 * (2 * 128 * 128 + 128 * 128) * 4
+    args = (vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000), None, vp(0x100000), None)
+    assert lib.gdn_chunk_fwd_segmented(ctypes.byref(d), 0, *args, vp(0x9000000), need, None) == -1  # nseg < 1
+    assert lib.gdn_chunk_fwd_segmented(ctypes.byref(d), 5, *args, vp(0x9000000), need, None) == -1  # 96 % 5
+    assert lib.gdn_chunk_fwd_segmented(ctypes.byref(d), 3, *args, vp(0x9000000), need - 4, None) == -1  # small
+    assert lib.gdn_chunk_fwd_segmented(ctypes.byref(d), 3, *args, None, need, None) == -1  # no workspace
+    assert lib.gdn_chunk_fwd_segmented(ctypes.byref(d), 3, *args, vp(0x9000008), need, None) == -2  # misaligned
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(gdn, "_lib", None)
     monkeypatch.setattr(gdn, "_LIB_PATH", str(tmp_path / "missing.so"))
