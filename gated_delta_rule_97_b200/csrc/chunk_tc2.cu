@@ -160,10 +160,16 @@ __device__ __forceinline__ int v16_slot(int buf) {
 // rows arrive compact and are moved to each token's last substep (zeros
 // elsewhere), the gate sits on each token's first substep, and only each
 // token's last substep is written out.
-template <int DVS, int UPD, int GATE, bool OUT_BF16, bool PROD>
+//
+// EXT: the input prologue and the segmented prefill's pass modes are compiled
+// in only for calls that use them; the plain path (EXT = false) sees both as
+// constant zero, so it keeps the registers and code it has without them.
+template <int DVS, int UPD, int GATE, bool OUT_BF16, bool PROD, bool EXT>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_constant__ Params p) {
     using L = Smem<DVS, GATE>;
     constexpr bool DELTA = (UPD == kDelta);
+    const int pro = EXT ? p.pro : 0;
+    const int mode = EXT ? p.mode : 0;
     // P = [Q;K]K^T of a chunk is issued by the state group's MMA thread right after
     // rdy when the prep group is the longer side (delta rule, scalar / no gate), else
     // by the prep group itself (it then has slack; the channel gate's P also needs
@@ -172,8 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     // in place to fp16 after they land, so P follows that pass and is issued by the
     // prep group.  Unit rows alone leave the tiles as they are: the row norms
     // become factors on P (rows and columns) and on the converted operands.
-    const bool qkmap = (p.pro & kProElu1) != 0;
-    const bool l2scale = (p.pro & kProL2) != 0 && !qkmap;
+    const bool qkmap = (pro & kProElu1) != 0;
+    const bool l2scale = (pro & kProL2) != 0 && !qkmap;
     const bool kStateP1 = DELTA && GATE != kGateChannel && !PROD && !qkmap;
     // In the same modes the V tile has its own TMA barrier (bar_tv): its fp16
     // conversion runs during the 16 -> 32 merge, after the q / k conversion window
@@ -210,9 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         ms.s_abort = 0;
         tma_prefetch_desc(&p.q_map);
         tma_prefetch_desc(&p.k_map);
-        if (!(p.mode & kModeZeroV)) tma_prefetch_desc(&p.v_map);
+        if (!(mode & kModeZeroV)) tma_prefetch_desc(&p.v_map);
         if (GATE == kGateChannel) tma_prefetch_desc(&p.g_map);
-        if (!(p.mode & kModeNoOut)) tma_prefetch_desc(&p.o_map);
+        if (!(mode & kModeNoOut)) tma_prefetch_desc(&p.o_map);
     }
     __syncwarp();
     if (warp == 0) {
@@ -221,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     }
     // T2 tile: its upper-right 32x32 block is never written and stays zero
     for (int i = t; i < 8192 / 16; i += kThreads) reinterpret_cast<uint4 *>(sm + L::TZA)[i] = make_uint4(0, 0, 0, 0);
-    const bool zeroV = (p.mode & kModeZeroV) != 0;
+    const bool zeroV = (mode & kModeZeroV) != 0;
     if (zeroV) {
         // values taken as zero: the fp16 V tiles are cleared once and never loaded
         for (int i = t; i < DVS * 128 / 16; i += kThreads) {
@@ -252,16 +258,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     // the token's gate on its first substep, 1 (g = 0) on the others
                     const int m0 = t0 + l0, m1 = m0 + 1, msk = (1 << p.lnh) - 1;
                     const size_t gb = (size_t)bh * (T >> p.lnh);
-                    gpre0 = (m0 < T && (m0 & msk) == 0) ? pro_gate(p.g[gb + (m0 >> p.lnh)], p.pro) : 0.f;
-                    gpre1 = (m1 < T && (m1 & msk) == 0) ? pro_gate(p.g[gb + (m1 >> p.lnh)], p.pro) : 0.f;
+                    gpre0 = (m0 < T && (m0 & msk) == 0) ? pro_gate(p.g[gb + (m0 >> p.lnh)], pro) : 0.f;
+                    gpre1 = (m1 < T && (m1 & msk) == 0) ? pro_gate(p.g[gb + (m1 >> p.lnh)], pro) : 0.f;
                 } else {
-                    gpre0 = (t0 + l0 < T) ? pro_gate(p.g[(size_t)bh * T + t0 + l0], p.pro) : 0.f;
-                    gpre1 = (t0 + l0 + 1 < T) ? pro_gate(p.g[(size_t)bh * T + t0 + l0 + 1], p.pro) : 0.f;
+                    gpre0 = (t0 + l0 < T) ? pro_gate(p.g[(size_t)bh * T + t0 + l0], pro) : 0.f;
+                    gpre1 = (t0 + l0 + 1 < T) ? pro_gate(p.g[(size_t)bh * T + t0 + l0 + 1], pro) : 0.f;
                 }
             }
             if (DELTA && t >= 128 && t < 128 + C) {
                 const int l = t - 128;
-                bpre = (t0 + l < T) ? pro_beta(p.beta[(size_t)bh * T + t0 + l], p.pro) : 0.f;
+                bpre = (t0 + l < T) ? pro_beta(p.beta[(size_t)bh * T + t0 + l], pro) : 0.f;
             }
         };
         // scalar gate prefix of chunk r and its factors b = e^G, gamma = e^{G_C-G},
@@ -373,12 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     unpack_bf16x8(*reinterpret_cast<const uint4 *>(base + ((c ^ (row & 7)) << 4)), f + 8 * c);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        f[8 * c + e] = valid ? pro_feature(f[8 * c + e], p.pro) : 0.f;
+                        f[8 * c + e] = valid ? pro_feature(f[8 * c + e], pro) : 0.f;
                         ss = fmaf(f[8 * c + e], f[8 * c + e], ss);
                     }
                 }
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                const float sc = (p.pro & kProL2) ? (ss > 0.f ? 1.f / sqrtf(ss) : 0.f) : 1.f;
+                const float sc = (pro & kProL2) ? (ss > 0.f ? 1.f / sqrtf(ss) : 0.f) : 1.f;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
 #pragma unroll
@@ -437,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
                 for (int l = 0; l < 32; ++l) {
                     gv[l] = gt[gch_idx(32 * hf + l, c)];
-                    if (r * C + 32 * hf + l < T) gv[l] = pro_gate(gv[l], p.pro);  // padding stays g = 0
+                    if (r * C + 32 * hf + l < T) gv[l] = pro_gate(gv[l], pro);  // padding stays g = 0
                 }
 #pragma unroll
                 for (int l = 1; l < 32; ++l) gv[l] += gv[l - 1];
@@ -998,9 +1004,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
             for (int j = 0; j < 64; j += 4) {
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (p.mode & kModeS0Eye) {
-                    const int c = h * 64 + j - (v0 + vrow);  // S0 = I: one 1 per row, at column v0 + vrow
-                    x = make_float4(c == 0 ? 1.f : 0.f, c == -1 ? 1.f : 0.f, c == -2 ? 1.f : 0.f, c == -3 ? 1.f : 0.f);
+                if (mode & kModeS0Eye) {
+                    // S0 = kEyeScale * I: one entry per row, at column v0 + vrow
+                    const int c = h * 64 + j - (v0 + vrow);
+                    constexpr float e = kEyeScale;
+                    x = make_float4(c == 0 ? e : 0.f, c == -1 ? e : 0.f, c == -2 ? e : 0.f, c == -3 ? e : 0.f);
                     if (!has_row) x = make_float4(0.f, 0.f, 0.f, 0.f);
                 } else if (p.S0 && has_row) {
                     x = *reinterpret_cast<const float4 *>(p.S0 + srow + h * 64 + j);
@@ -1171,7 +1179,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             if (!mbar_wait(fb, (r >> 1) & 1)) note_timeout(ms, 8, r);
             TC2_MARK(256, 22);
             tc_fence_after();
-            if (!(p.mode & kModeNoOut)) {
+            if (!(mode & kModeNoOut)) {
                 // O^T -> row-major staging [64 tok][DVS] -> one TMA store (rows past T
                 // clipped).  Stores issued straight from registers were measured slower:
                 // they queue behind the prep group's shared-memory traffic.
@@ -1255,6 +1263,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         if (ts == 0) bulk_wait0();  // o is in global memory before the kernel ends
         // final state
         if (!ms.s_abort && p.ST) {
+            const float osc = (mode & kModeS0Eye) ? 1.f / kEyeScale : 1.f;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float sv[64];
@@ -1265,7 +1274,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 if (has_row) {
 #pragma unroll
                     for (int j = 0; j < 64; j += 4)
-                        *reinterpret_cast<float4 *>(p.ST + srow + h * 64 + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+                        *reinterpret_cast<float4 *>(p.ST + srow + h * 64 + j) =
+                            make_float4(sv[j] * osc, sv[j + 1] * osc, sv[j + 2] * osc, sv[j + 3] * osc);
                 }
             }
         }
@@ -1290,7 +1300,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 template <int DVS, int UPD, int GATE, bool OB, bool PROD = false>
 int launch_one(const Params &prm, int grid, cudaStream_t stream) {
     using L = Smem<DVS, GATE>;
-    auto kern = chunk_tc2_kernel<DVS, UPD, GATE, OB, PROD>;
+    auto kern = (prm.pro != 0 || prm.mode != 0) ? chunk_tc2_kernel<DVS, UPD, GATE, OB, PROD, true>
+                                                : chunk_tc2_kernel<DVS, UPD, GATE, OB, PROD, false>;
     static_assert(L::DYN <= 232448, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN);
     if (e != cudaSuccess) return (int)e;

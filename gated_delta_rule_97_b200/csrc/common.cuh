@@ -56,6 +56,11 @@ struct ChunkArgs {
 // initial state the identity (dv == dk); with all three the pass yields the
 // transition of the sequence (S_T = S0 Lambda with S0 = I).
 constexpr int kModeZeroV = 1, kModeNoOut = 2, kModeS0Eye = 4;
+// The tensor-core kernel runs kModeS0Eye from kEyeScale * I and stores S_T /
+// kEyeScale (exact, a power of two): a transition that decays far below 1 then
+// stays in fp16's normal range in the state's fp16 operand copy, while entries
+// bounded by 1 (products of contractions) stay far below fp16's maximum.
+constexpr float kEyeScale = 1024.f;
 
 struct DecodeArgs {
     const void *q, *k, *v;   // [BH,T,dk] / [BH,T,dv]
@@ -90,4 +95,5 @@ int gdn_launch_decode(const gdn::DecodeArgs &a, int update, int gate, int in_bf1
                       cudaStream_t stream);
 int gdn_launch_copy_state(const float *S0, float *ST, long n, cudaStream_t stream);
 int gdn_launch_compose(const float *S0, const float *H, const float *Lam, float *Sstart, float *ST, int BH, int nseg,
-                       int dk, int dv, cudaStream_t stream);
+                       int dk, int dv, bool segment_major, cudaStream_t stream);
+int gdn_launch_eye(float *L, long BH, int dk, cudaStream_t stream);

@@ -49,21 +49,24 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-template <int DK, int UPD, int GATE, typename TIn>
+// PRO: the input prologue is compiled in only when a call asks for it, so the
+// plain path keeps its registers and straight-line loads.
+template <int DK, int UPD, int GATE, typename TIn, bool PRO>
 struct StepIn {
     static constexpr int V = DK / 32;
     float qq[V], kk[V], al[V], bt, vv[kRowsPerWarp];
     __device__ void load(const DecodeArgs &a, long bh, int t, int c0, int i0) {
+        const int pro = PRO ? a.pro : 0;
         const long tok = bh * a.T + t;
         const TIn *qp = static_cast<const TIn *>(a.q) + tok * DK + c0;
         const TIn *kp = static_cast<const TIn *>(a.k) + tok * DK + c0;
 #pragma unroll
         for (int e = 0; e < V; ++e) {
-            qq[e] = pro_feature(to_f32(qp[e]), a.pro);
-            kk[e] = pro_feature(to_f32(kp[e]), a.pro);
+            qq[e] = pro_feature(to_f32(qp[e]), pro);
+            kk[e] = pro_feature(to_f32(kp[e]), pro);
             al[e] = 1.f;
         }
-        if (a.pro & kProL2) {
+        if (pro & kProL2) {
             // unit q and k rows (a zero row stays zero); every lane gets both sums
             float sq = 0.f, sk = 0.f;
 #pragma unroll
@@ -84,14 +87,14 @@ struct StepIn {
             }
         }
         if (GATE == kGateScalar) {
-            const float x = __expf(pro_gate(a.g[tok], a.pro));
+            const float x = __expf(pro_gate(a.g[tok], pro));
 #pragma unroll
             for (int e = 0; e < V; ++e) al[e] = x;
         } else if (GATE == kGateChannel) {
 #pragma unroll
-            for (int e = 0; e < V; ++e) al[e] = __expf(pro_gate(a.g[tok * DK + c0 + e], a.pro));
+            for (int e = 0; e < V; ++e) al[e] = __expf(pro_gate(a.g[tok * DK + c0 + e], pro));
         }
-        bt = (UPD == kDelta) ? pro_beta(a.beta[tok], a.pro) : 0.f;
+        bt = (UPD == kDelta) ? pro_beta(a.beta[tok], pro) : 0.f;
         const TIn *vp = static_cast<const TIn *>(a.v) + tok * a.dv + i0;
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) vv[r] = to_f32(vp[r]);
@@ -101,7 +104,7 @@ struct StepIn {
 // T >= 1 tokens per call: the state rows stay in registers across the tokens
 // (read and written once); the next token's inputs are loaded while the current
 // one is applied.
-template <int DK, int UPD, int GATE, typename TIn, typename TOut>
+template <int DK, int UPD, int GATE, typename TIn, typename TOut, bool PRO>
 __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
     constexpr int V = DK / 32;
     const long warp = ((long)blockIdx.x * kThreads + threadIdx.x) >> 5;
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r) VecF<V>::load(Srow + (size_t)r * DK, s[r]);
 
-    StepIn<DK, UPD, GATE, TIn> cur, nxt;
+    StepIn<DK, UPD, GATE, TIn, PRO> cur, nxt;
     cur.load(a, bh, 0, c0, i0);
 #pragma unroll 1
     for (int t = 0; t < a.T; ++t) {
@@ -167,7 +170,10 @@ int launch(const DecodeArgs &a, cudaStream_t stream) {
     const long warps = rows / kRowsPerWarp;
     const long blocks = (warps * 32 + kThreads - 1) / kThreads;
     if (blocks == 0) return 0;
-    decode_kernel<DK, UPD, GATE, TIn, TOut><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+    if (a.pro)
+        decode_kernel<DK, UPD, GATE, TIn, TOut, true><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+    else
+        decode_kernel<DK, UPD, GATE, TIn, TOut, false><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
     return (int)cudaGetLastError();
 }
 
