@@ -5,8 +5,9 @@ One step = one gdn_chunk_fwd over the Gated DeltaNet prefill workload
 (B=8, H=16, T=8192, dk=dv=128, bf16 q/k/v, fp32 gate/beta/state/output, chunk 64),
 which runs every prefill row of the path (gate prefix, K-Gram, UT solve, W/U,
 state correction, output, state pass).  The line also carries the decode
-workload (256 x 32 heads, 1000 in-place steps) and, unless --quick, the linear
-attention and per-channel (KDA) prefill workloads.
+workload (256 x 32 heads, 1000 in-place steps, and 4-token calls) and, unless
+--quick, the linear attention, per-channel (KDA), Gated DeltaProduct and
+long-context segmented (1 x 8 heads x 65536 tokens, 16 segments) prefills.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
 
@@ -167,17 +168,27 @@ def to_dev(x, dtype, torch):
     return torch.from_numpy(np.ascontiguousarray(x, np.float32)).cuda().to(dtype).contiguous()
 
 
-def time_prefill(w, x, steps, warmup, torch, gdn, dist=None):
-    """Device-timed steps of gdn_chunk_fwd over the whole batch; returns ms/step (max over ranks)."""
+def time_prefill(w, x, steps, warmup, torch, gdn, dist=None, nseg=1):
+    """Device-timed steps of gdn_chunk_fwd over the whole batch (of
+    gdn_chunk_fwd_segmented with ``nseg`` > 1 segments per sequence, workspace
+    allocated once outside the timed region); returns ms/step (max over ranks)."""
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     q, k, v = to_dev(x["q"], dt, torch), to_dev(x["k"], dt, torch), to_dev(x["v"], dt, torch)
     g, beta, S0 = to_dev(x["g"], torch.float32, torch), to_dev(x["beta"], torch.float32, torch), \
         to_dev(x["S0"], torch.float32, torch)
     o = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device="cuda")
     ST = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device="cuda")
+    ws = None
+    if nseg > 1:
+        ws = torch.empty(gdn.segmented_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, nseg), dtype=torch.uint8,
+                         device="cuda")
 
     def step():
-        gdn.chunk_fwd(q, k, v, g, beta, S0, update=w.update, gate=w.gate, o=o, S_T=ST)
+        if nseg > 1:
+            gdn.chunk_fwd_segmented(q, k, v, g, beta, S0, update=w.update, gate=w.gate, nseg=nseg, o=o, S_T=ST,
+                                    workspace=ws)
+        else:
+            gdn.chunk_fwd(q, k, v, g, beta, S0, update=w.update, gate=w.gate, o=o, S_T=ST)
 
     for _ in range(warmup):
         step()
@@ -197,7 +208,7 @@ def time_prefill(w, x, steps, warmup, torch, gdn, dist=None):
     if dist is not None:
         dist.barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, dist, "cuda")
-    del q, k, v, g, beta, S0, o, ST
+    del q, k, v, g, beta, S0, o, ST, ws
     return ms
 
 
@@ -237,9 +248,15 @@ def product_bytes(w, nh, out_bytes=4):
     return w.n_heads * (w.T * per_tok + state)
 
 
+E2E_SLICES = 8
+
+
 def time_prefill_e2e(w, x, steps, warmup, torch, gdn):
     """Same metric through the public API with pinned host buffers: every step
-    copies the inputs host->device, runs gdn_chunk_fwd and reads o and S_T back."""
+    is one gdn_chunk_fwd_host call, which copies the inputs host->device, runs
+    the prefill and copies o and S_T back, in E2E_SLICES head slices so that
+    the two copy directions and the kernels overlap (device workspace allocated
+    once, outside the timed region)."""
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def pin(a, dtype):
@@ -254,16 +271,13 @@ def time_prefill_e2e(w, x, steps, warmup, torch, gdn):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hS) if t is not None)
     d2h = ho.numel() * 4 + hST.numel() * 4
 
+    ws = torch.empty(gdn.host_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.update, w.gate,
+                                              gdn.BF16 if dt == torch.bfloat16 else gdn.F32, gdn.F32, E2E_SLICES),
+                     dtype=torch.uint8, device="cuda")
+
     def step():
-        dq = hq.to("cuda", non_blocking=True)
-        dk_ = hk.to("cuda", non_blocking=True)
-        dv_ = hv.to("cuda", non_blocking=True)
-        dg = None if hg is None else hg.to("cuda", non_blocking=True)
-        db = None if hb is None else hb.to("cuda", non_blocking=True)
-        dS = None if hS is None else hS.to("cuda", non_blocking=True)
-        o, ST = gdn.chunk_fwd(dq, dk_, dv_, dg, db, dS, update=w.update, gate=w.gate)
-        ho.copy_(o, non_blocking=True)
-        hST.copy_(ST, non_blocking=True)
+        gdn.chunk_fwd_host(hq, hk, hv, hg, hb, hS, update=w.update, gate=w.gate, n_slices=E2E_SLICES, o=ho,
+                           S_T=hST, workspace=ws)
 
     for _ in range(max(1, min(warmup, 2))):
         step()
@@ -445,7 +459,8 @@ def run_ours(args):
 
     ms_e2e, h2d, d2h = time_prefill_e2e(w, x, max(2, min(args.steps, 5)), args.warmup, torch, gdn)
     result["e2e"] = {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+                     "api": "gdn_chunk_fwd_host, %d head slices, pinned host buffers" % E2E_SLICES}
     del x
 
     wd = WORKLOADS["decode_gdn_bf16"]
@@ -495,6 +510,24 @@ def run_ours(args):
                                       "achieved_gbs": nb / (msp * 1e-3) / 1e9, "roofline_us": tr * 1e6,
                                       "frac_of_roofline_time": tr / (msp * 1e-3)}
         result["gpu_launches"] += max(3, args.steps // 2)
+        # Long context, few heads: 8 heads of 65536 tokens occupy 8 of the 148 SMs in
+        # gdn_chunk_fwd; gdn_chunk_fwd_segmented runs 16 segments per sequence in
+        # parallel (4 launches per call: zero-state pass, transition pass,
+        # composition, output pass)
+        wl, nseg = WORKLOADS["gdn_prefill_bf16"].with_(B=1, H=8, T=65536, name="gdn_long_bf16"), 16
+        xl = make_prefill_inputs(wl)
+        ns = max(3, args.steps // 2)
+        ms1 = time_prefill(wl, xl, ns, args.warmup, torch, gdn, dist)
+        msn = time_prefill(wl, xl, ns, args.warmup, torch, gdn, dist, nseg=nseg)
+        del xl
+        result["gpu_launches"] += ns * (1 + 4)
+        nb = prefill_bytes(wl)
+        others["gdn_long_bf16"] = {"B": wl.B, "H": wl.H, "T": wl.T, "nseg": nseg,
+                                   "ms_per_step_unsegmented": ms1, "ms_per_step": msn,
+                                   "tokens_per_s": wl.B * wl.T * world / (msn * 1e-3),
+                                   "speedup_vs_unsegmented": ms1 / msn,
+                                   "achieved_gbs": nb / (msn * 1e-3) / 1e9,
+                                   "frac_of_roofline_time": nb / (peaks["hbm_gbs"] * 1e9) / (msn * 1e-3)}
         result["prefill_workloads"] = others
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

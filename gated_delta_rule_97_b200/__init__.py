@@ -16,7 +16,9 @@ import ctypes
 import os
 
 __all__ = ["GDNError", "chunk_fwd", "decode_step", "device_status", "strerror", "version", "load",
-           "lib_path", "Desc", "UPDATES", "GATES", "build", "device_diag"]
+           "lib_path", "Desc", "UPDATES", "GATES", "build", "device_diag", "product_fwd", "chunk_fwd_segmented",
+           "segmented_workspace_bytes", "segment_maps", "compose_segments", "chunk_fwd_host",
+           "host_workspace_bytes"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libgdn.so")
@@ -82,6 +84,14 @@ def load():
     lib.gdn_segmented_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_chunk_fwd_segmented.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.gdn_chunk_fwd_segmented.restype = ctypes.c_int
+    lib.gdn_host_workspace_bytes.argtypes = [dp, ctypes.c_int]
+    lib.gdn_host_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_chunk_fwd_host.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.gdn_chunk_fwd_host.restype = ctypes.c_int
+    lib.gdn_segment_maps.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gdn_segment_maps.restype = ctypes.c_int
+    lib.gdn_compose_segments.argtypes = [ctypes.c_int] * 4 + [vp] * 6
+    lib.gdn_compose_segments.restype = ctypes.c_int
     lib.gdn_strerror.argtypes = [ctypes.c_int]
     lib.gdn_strerror.restype = ctypes.c_char_p
     lib.gdn_device_status.argtypes = [ctypes.c_int]
@@ -190,6 +200,69 @@ def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=No
     return o, S_T
 
 
+def _check_host(t, name, shape, dtype=None):
+    if t is None:
+        return
+    if t.is_cuda:
+        raise ValueError("%s must be a host (CPU) tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def host_workspace_bytes(B, H, T, dk, dv, update, gate, dtype, out_dtype=F32, n_slices=8) -> int:
+    d = make_desc(B, H, T, dk, dv, update, gate, dtype, out_dtype)
+    return int(load().gdn_host_workspace_bytes(ctypes.byref(d), int(n_slices)))
+
+
+def chunk_fwd_host(q, k, v, g=None, beta=None, S0=None, *, update, gate, n_slices=8, out_dtype=None, o=None,
+                   S_T=None, return_state=True, algo="auto", prologue=0, workspace=None, device=None, stream=None):
+    """gdn_chunk_fwd_host: the prefill on host tensors (pin them for overlap),
+    streamed to the GPU in ``n_slices`` head slices.  ``workspace``: a CUDA
+    uint8 tensor of host_workspace_bytes(...) bytes (allocated here when None).
+    Returns host (o, S_T), complete once ``stream`` (default: the current
+    stream) has synchronised."""
+    import torch
+
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check_host(q, "q", (B, H, T, dk))
+    _check_host(k, "k", (B, H, T, dk), q.dtype)
+    _check_host(v, "v", (B, H, T, dv), q.dtype)
+    if gate == "scalar":
+        _check_host(g, "g", (B, H, T), torch.float32)
+    elif gate == "channel":
+        _check_host(g, "g", (B, H, T, dk), torch.float32)
+    _check_host(beta, "beta", (B, H, T), torch.float32)
+    _check_host(S0, "S0", (B, H, dv, dk), torch.float32)
+    if out_dtype is None:
+        out_dtype = o.dtype if o is not None else torch.float32
+    pin = q.is_pinned()
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=out_dtype, pin_memory=pin)
+    _check_host(o, "o", (B, H, T, dv), out_dtype)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, pin_memory=pin)
+    _check_host(S_T, "S_T", (B, H, dv, dk), torch.float32)
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
+                  prologue=prologue)
+    need = int(load().gdn_host_workspace_bytes(ctypes.byref(d), int(n_slices)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8,
+                                device=device if device is not None else torch.cuda.current_device())
+    if not workspace.is_cuda or not workspace.is_contiguous() or workspace.numel() < need:
+        raise ValueError("workspace needs %d contiguous CUDA bytes" % need)
+    rc = load().gdn_chunk_fwd_host(ctypes.byref(d), int(n_slices), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                   _stream(stream))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_chunk_fwd_host")
+    return o, S_T
+
+
 def product_fwd(q, k, v, g=None, beta=None, S0=None, *, gate, out_dtype=None, o=None, S_T=None,
                 return_state=True, algo="auto", prologue=0, stream=None):
     """Gated DeltaProduct prefill (gdn_product_fwd): nh = k.shape[-2] delta-rule
@@ -275,6 +348,61 @@ def chunk_fwd_segmented(q, k, v, g=None, beta=None, S0=None, *, update, gate, ns
 def segmented_workspace_bytes(B, H, T, dk, dv, nseg) -> int:
     d = make_desc(B, H, T, dk, dv, "delta", "scalar", BF16, F32)
     return int(load().gdn_segmented_workspace_bytes(ctypes.byref(d), int(nseg)))
+
+
+def segment_maps(q, k, v, g=None, beta=None, *, update, gate, H=None, Lam=None, algo="auto", prologue=0,
+                 stream=None):
+    """gdn_segment_maps: the affine map S_in -> S_in Lam + H of the T tokens of
+    every head.  Same inputs as chunk_fwd; returns (H [B,H,dv,dk],
+    Lam [B,H,dk,dk]), both fp32."""
+    import torch
+
+    B, Hh, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, Hh, T, dk))
+    _check(k, "k", (B, Hh, T, dk), q.dtype)
+    _check(v, "v", (B, Hh, T, dv), q.dtype)
+    if gate == "scalar":
+        _check(g, "g", (B, Hh, T), torch.float32)
+    elif gate == "channel":
+        _check(g, "g", (B, Hh, T, dk), torch.float32)
+    _check(beta, "beta", (B, Hh, T), torch.float32)
+    if H is None:
+        H = torch.empty((B, Hh, dv, dk), dtype=torch.float32, device=q.device)
+    if Lam is None:
+        Lam = torch.empty((B, Hh, dk, dk), dtype=torch.float32, device=q.device)
+    _check(H, "H", (B, Hh, dv, dk), torch.float32)
+    _check(Lam, "Lam", (B, Hh, dk, dk), torch.float32)
+    d = make_desc(B, Hh, T, dk, dv, update, gate, _dtype_code(q.dtype), F32, algo, prologue=prologue)
+    rc = load().gdn_segment_maps(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(H),
+                                 _ptr(Lam), _stream(stream))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_segment_maps")
+    return H, Lam
+
+
+def compose_segments(H, Lam=None, S0=None, *, S_in=None, S_T=None, want_inputs=True, stream=None):
+    """gdn_compose_segments: H [nseg,B,H,dv,dk], Lam [nseg,B,H,dk,dk] or None
+    (identity transitions), S0 [B,H,dv,dk] or None.  Returns (S_in
+    [nseg,B,H,dv,dk], the state entering each segment, or None when
+    ``want_inputs`` is false; S_T [B,H,dv,dk], the final state)."""
+    import torch
+
+    nseg, B, Hh, dv, dk = H.shape
+    _check(H, "H", (nseg, B, Hh, dv, dk), torch.float32)
+    _check(Lam, "Lam", (nseg, B, Hh, dk, dk), torch.float32)
+    _check(S0, "S0", (B, Hh, dv, dk), torch.float32)
+    if S_in is None and want_inputs:
+        S_in = torch.empty_like(H)
+    _check(S_in, "S_in", (nseg, B, Hh, dv, dk), torch.float32)
+    if S_T is None:
+        S_T = torch.empty((B, Hh, dv, dk), dtype=torch.float32, device=H.device)
+    _check(S_T, "S_T", (B, Hh, dv, dk), torch.float32)
+    rc = load().gdn_compose_segments(B * Hh, nseg, dk, dv, _ptr(S0), _ptr(H), _ptr(Lam), _ptr(S_in), _ptr(S_T),
+                                     _stream(stream))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_compose_segments")
+    return S_in, S_T
 
 
 def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, prologue=0, stream=None):

@@ -116,8 +116,10 @@ extern "C" int gdn_device_diag(void) {
 
 
 // Argument rules of gdn_chunk_fwd (sizes, pointers, alignment, overlaps).
+// With need_o false (the segment maps) no output rows are read or checked.
 static int chunk_fwd_check(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
-                           const float *beta, const float *S0, const void *o, const float *S_T) {
+                           const float *beta, const float *S0, const void *o, const float *S_T,
+                           bool need_o = true) {
     int rc = validate_common(d);
     if (rc != GDN_OK) return rc;
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
@@ -128,7 +130,7 @@ static int chunk_fwd_check(const gdn_desc_t *d, const void *q, const void *k, co
     const size_t n_g = d->gate == GDN_GATE_CHANNEL ? n_qk : (size_t)BH * d->T;
     const bool has_tokens = BH > 0 && d->T > 0;
     if (has_tokens) {
-        if (!q || !k || !v || !o) return GDN_ERR_ARG;
+        if (!q || !k || !v || (need_o && !o)) return GDN_ERR_ARG;
         if (d->update == GDN_DELTA && !beta) return GDN_ERR_ARG;
     }
     if ((d->gate != GDN_GATE_NONE) != (g != nullptr) && has_tokens) return GDN_ERR_ARG;
@@ -166,6 +168,131 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     a.pro = d->prologue;
     a.mode = 0;
     return dispatch_chunk(d, a, st);
+}
+
+namespace {
+
+// Byte layout of one slot of the host pipeline's device workspace: the inputs
+// and outputs of ``hs`` heads, each tensor on a 256-byte boundary.
+struct SlotLayout {
+    size_t q, k, v, g, beta, S0, o, ST, bytes;
+    size_t nq, nv, ng, nb, nS, no;  // per-head bytes of each tensor
+};
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+SlotLayout slot_layout(const gdn_desc_t *d, long hs) {
+    SlotLayout L;
+    const size_t es = elem_size(d->dtype), T = (size_t)d->T;
+    L.nq = T * d->dk * es;
+    L.nv = T * d->dv * es;
+    L.ng = d->gate == GDN_GATE_NONE ? 0 : (d->gate == GDN_GATE_CHANNEL ? T * d->dk * 4 : T * 4);
+    L.nb = d->update == GDN_DELTA ? T * 4 : 0;
+    L.nS = (size_t)d->dv * d->dk * 4;
+    L.no = T * d->dv * elem_size(d->out_dtype);
+    size_t off = 0;
+    L.q = off; off += up256(hs * L.nq);
+    L.k = off; off += up256(hs * L.nq);
+    L.v = off; off += up256(hs * L.nv);
+    L.g = off; off += up256(hs * L.ng);
+    L.beta = off; off += up256(hs * L.nb);
+    L.S0 = off; off += up256(hs * L.nS);
+    L.o = off; off += up256(hs * L.no);
+    L.ST = off; off += up256(hs * L.nS);
+    L.bytes = off;
+    return L;
+}
+
+long slice_heads(const gdn_desc_t *d, int n_slices) {
+    const long BH = (long)d->B * d->H;
+    const long n = n_slices < BH ? n_slices : BH;
+    return n > 0 ? (BH + n - 1) / n : 0;
+}
+
+int h2d(void *dst, const void *src, size_t n, cudaStream_t s) {
+    if (n == 0 || !src) return GDN_OK;
+    return from_cuda(cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, s));
+}
+
+int d2h(void *dst, const void *src, size_t n, cudaStream_t s) {
+    if (n == 0 || !dst) return GDN_OK;
+    return from_cuda(cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToHost, s));
+}
+
+}  // namespace
+
+extern "C" size_t gdn_host_workspace_bytes(const gdn_desc_t *d, int n_slices) {
+    if (!d || n_slices < 1 || validate_common(d) != GDN_OK) return 0;
+    return 2 * slot_layout(d, slice_heads(d, n_slices)).bytes;
+}
+
+extern "C" int gdn_chunk_fwd_host(const gdn_desc_t *d, int n_slices, const void *q, const void *k, const void *v,
+                                  const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = chunk_fwd_check(d, q, k, v, g, beta, S0, o, S_T);
+    if (rc != GDN_OK) return rc;
+    if (n_slices < 1) return GDN_ERR_ARG;
+    const long BH = (long)d->B * d->H;
+    if (BH == 0) return GDN_OK;
+    const long hs = slice_heads(d, n_slices);
+    const SlotLayout L = slot_layout(d, hs);
+    if (!workspace || workspace_bytes < 2 * L.bytes) return GDN_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_ALIGN;
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[7] = {};  // start, in[2], comp[2], out[2]
+    rc = from_cuda(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking));
+    if (rc == GDN_OK) rc = from_cuda(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking));
+    for (int i = 0; i < 7 && rc == GDN_OK; ++i) rc = from_cuda(cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming));
+    cudaEvent_t &start = ev[0], *in = ev + 1, *comp = ev + 3, *out = ev + 5;
+    if (rc == GDN_OK) rc = from_cuda(cudaEventRecord(start, cs));
+    if (rc == GDN_OK) rc = from_cuda(cudaStreamWaitEvent(s_in, start, 0));
+    if (rc == GDN_OK) rc = from_cuda(cudaStreamWaitEvent(s_out, start, 0));
+
+    const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k);
+    const char *hv = static_cast<const char *>(v), *hg = reinterpret_cast<const char *>(g);
+    const char *hb = reinterpret_cast<const char *>(beta), *hS0 = reinterpret_cast<const char *>(S0);
+    char *ho = static_cast<char *>(o), *hST = reinterpret_cast<char *>(S_T);
+    const long n = (BH + hs - 1) / hs;
+    for (long i = 0; i < n && rc == GDN_OK; ++i) {
+        const int slot = (int)(i & 1);
+        const long h0 = i * hs, nh = (h0 + hs <= BH) ? hs : BH - h0;
+        char *base = static_cast<char *>(workspace) + slot * L.bytes;
+        // the slot is free once the copy-out of slice i - 2 (after its kernel) is done
+        if (i >= 2) rc = from_cuda(cudaStreamWaitEvent(s_in, out[slot], 0));
+        if (rc == GDN_OK) rc = h2d(base + L.q, hq + h0 * L.nq, nh * L.nq, s_in);
+        if (rc == GDN_OK) rc = h2d(base + L.k, hk + h0 * L.nq, nh * L.nq, s_in);
+        if (rc == GDN_OK) rc = h2d(base + L.v, hv + h0 * L.nv, nh * L.nv, s_in);
+        if (rc == GDN_OK && hg) rc = h2d(base + L.g, hg + h0 * L.ng, nh * L.ng, s_in);
+        if (rc == GDN_OK && hb) rc = h2d(base + L.beta, hb + h0 * L.nb, nh * L.nb, s_in);
+        if (rc == GDN_OK && hS0) rc = h2d(base + L.S0, hS0 + h0 * L.nS, nh * L.nS, s_in);
+        if (rc == GDN_OK) rc = from_cuda(cudaEventRecord(in[slot], s_in));
+        if (rc == GDN_OK) rc = from_cuda(cudaStreamWaitEvent(cs, in[slot], 0));
+        if (rc == GDN_OK) {
+            gdn_desc_t sd = *d;
+            sd.B = (int)nh;
+            sd.H = 1;
+            rc = gdn_chunk_fwd(&sd, base + L.q, base + L.k, base + L.v,
+                               hg ? reinterpret_cast<const float *>(base + L.g) : nullptr,
+                               hb ? reinterpret_cast<const float *>(base + L.beta) : nullptr,
+                               hS0 ? reinterpret_cast<const float *>(base + L.S0) : nullptr, base + L.o,
+                               hST ? reinterpret_cast<float *>(base + L.ST) : nullptr, cs);
+        }
+        if (rc == GDN_OK) rc = from_cuda(cudaEventRecord(comp[slot], cs));
+        if (rc == GDN_OK) rc = from_cuda(cudaStreamWaitEvent(s_out, comp[slot], 0));
+        if (rc == GDN_OK) rc = d2h(ho + h0 * L.no, base + L.o, nh * L.no, s_out);
+        if (rc == GDN_OK && hST) rc = d2h(hST + h0 * L.nS, base + L.ST, nh * L.nS, s_out);
+        if (rc == GDN_OK) rc = from_cuda(cudaEventRecord(out[slot], s_out));
+    }
+    // the caller's stream resumes after every copy-out
+    for (int j = 0; j < 2 && rc == GDN_OK && j < n; ++j) rc = from_cuda(cudaStreamWaitEvent(cs, out[j], 0));
+    // streams and events are released once their pending work completes
+    for (int i = 0; i < 7; ++i)
+        if (ev[i]) cudaEventDestroy(ev[i]);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+    return rc;
 }
 
 extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const void *k, const void *v,
@@ -270,8 +397,8 @@ extern "C" int gdn_chunk_fwd_segmented(const gdn_desc_t *d, int nseg, const void
     a.BH = segs; a.T = sd.T; a.dk = d->dk; a.dv = d->dv;
     a.nh = 1;
     a.pro = d->prologue;
-    // 1. every segment from a zero state: H_i (the outputs are rewritten in pass 3)
-    a.S0 = nullptr; a.ST = H; a.mode = 0;
+    // 1. every segment from a zero state: H_i (no outputs)
+    a.S0 = nullptr; a.ST = H; a.mode = gdn::kModeNoOut;
     if ((rc = dispatch_chunk(&sd, a, st)) != GDN_OK) return rc;
     // 2. every segment's transition Lambda_i: zero values from the identity state
     //    (with the additive write and no gate the transition is the identity)
@@ -286,11 +413,78 @@ extern "C" int gdn_chunk_fwd_segmented(const gdn_desc_t *d, int nseg, const void
     }
     // 3. the state entering each segment, and the final state
     if ((rc = from_cuda(gdn_launch_compose(S0, H, identity ? nullptr : Lam, Sstart, S_T, (int)BH, nseg, d->dk,
-                                           d->dv, st))) != GDN_OK)
+                                           d->dv, false, st))) != GDN_OK)
         return rc;
     // 4. every segment from its true incoming state: the outputs
     a.S0 = Sstart; a.ST = nullptr; a.mode = 0;
     return dispatch_chunk(&sd, a, st);
+}
+
+extern "C" int gdn_segment_maps(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *H, float *Lam, void *stream) {
+    int rc = chunk_fwd_check(d, q, k, v, g, beta, nullptr, nullptr, nullptr, false);
+    if (rc != GDN_OK) return rc;
+    const long BH = (long)d->B * d->H;
+    const size_t n_S = (size_t)BH * d->dv * d->dk * 4, n_L = (size_t)BH * d->dk * d->dk * 4;
+    if (BH > 0 && (!H || !Lam)) return GDN_ERR_ARG;
+    if ((H && !aligned16(H)) || (Lam && !aligned16(Lam))) return GDN_ERR_ALIGN;
+    const size_t es = elem_size(d->dtype);
+    const size_t n_qk = (size_t)BH * d->T * d->dk * es, n_v = (size_t)BH * d->T * d->dv * es;
+    const size_t n_g = (d->gate == GDN_GATE_CHANNEL ? (size_t)BH * d->T * d->dk : (size_t)BH * d->T) * 4;
+    const size_t n_b = (size_t)BH * d->T * 4;
+    if (overlaps(H, n_S, Lam, n_L)) return GDN_ERR_ARG;
+    const void *outs[] = {H, Lam};
+    const size_t nouts[] = {n_S, n_L};
+    for (int i = 0; i < 2; ++i)
+        if (overlaps(outs[i], nouts[i], q, n_qk) || overlaps(outs[i], nouts[i], k, n_qk) ||
+            overlaps(outs[i], nouts[i], v, n_v) || overlaps(outs[i], nouts[i], g, n_g) ||
+            overlaps(outs[i], nouts[i], beta, n_b))
+            return GDN_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (BH == 0) return GDN_OK;
+    // the additive write without a gate leaves the transition at the identity
+    const bool identity = d->update == GDN_ADDITIVE || d->T == 0;
+    if (d->T == 0) {
+        if ((rc = from_cuda(gdn_launch_copy_state(nullptr, H, (long)BH * d->dv * d->dk, st))) != GDN_OK) return rc;
+    } else {
+        gdn::ChunkArgs a;
+        a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = nullptr;
+        a.status = status_ptr();
+        a.diag = diag_ptr();
+        a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
+        a.nh = 1;
+        a.pro = d->prologue;
+        a.S0 = nullptr; a.ST = H; a.mode = gdn::kModeNoOut;
+        if ((rc = dispatch_chunk(d, a, st)) != GDN_OK) return rc;
+        if (!identity) {
+            gdn_desc_t ld = *d;
+            ld.dv = d->dk;
+            gdn::ChunkArgs b = a;
+            b.v = nullptr; b.ST = Lam; b.dv = d->dk;
+            b.mode = gdn::kModeZeroV | gdn::kModeNoOut | gdn::kModeS0Eye;
+            return dispatch_chunk(&ld, b, st);
+        }
+    }
+    return from_cuda(gdn_launch_eye(Lam, BH, d->dk, st));
+}
+
+extern "C" int gdn_compose_segments(int BH, int nseg, int dk, int dv, const float *S0, const float *H,
+                                    const float *Lam, float *S_in, float *S_T, void *stream) {
+    if (BH < 0 || nseg < 1 || BH > (1 << 30) || (long)BH * nseg > (1L << 30)) return GDN_ERR_ARG;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return GDN_ERR_ARG;
+    if (BH == 0) return GDN_OK;
+    if (!H) return GDN_ERR_ARG;
+    const void *ptrs[] = {S0, H, Lam, S_in, S_T};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t n_S = (size_t)BH * dv * dk * 4, n_H = n_S * nseg, n_L = (size_t)BH * nseg * dk * dk * 4;
+    // outputs overlap no input (S_T may be S0 itself: each row is read before it is written)
+    if (overlaps(S_in, n_H, S0, n_S) || overlaps(S_in, n_H, H, n_H) || overlaps(S_in, n_H, Lam, n_L) ||
+        overlaps(S_in, n_H, S_T, n_S) || overlaps(S_T, n_S, H, n_H) || overlaps(S_T, n_S, Lam, n_L) ||
+        (S_T != S0 && overlaps(S_T, n_S, S0, n_S)))
+        return GDN_ERR_ARG;
+    return from_cuda(gdn_launch_compose(S0, H, Lam, S_in, S_T, BH, nseg, dk, dv, true,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define GDN_VERSION 2
+#define GDN_VERSION 3
 
 /* Return codes. */
 #define GDN_OK 0
@@ -137,6 +137,32 @@ int gdn_chunk_fwd(const gdn_desc_t *desc, const void *q, const void *k, const vo
                   void *stream);
 
 /*
+ * gdn_chunk_fwd_host -- gdn_chunk_fwd on HOST buffers: the same arguments and
+ * results, with q, k, v, g, beta, S0, o and S_T in host memory (page-locked
+ * for the copies to overlap; pageable memory works, serialised).  The heads are
+ * cut into n_slices contiguous slices; slice i is copied host -> device on an
+ * internal stream, computed by gdn_chunk_fwd on the caller's stream, and copied
+ * device -> host on a second internal stream, alternating between two slots of
+ * the device workspace, so the copies of one slice overlap the kernel of
+ * another and the two copy directions overlap each other.  The call returns
+ * once all work is enqueued; the caller's stream waits for the last copy, so
+ * o and S_T are complete (and the host inputs free) when that stream has
+ * synchronised.  (The pages' prefill has no transfer step; this is the
+ * host-resident use of the same prefill.)
+ *
+ *   workspace  device buffer of gdn_host_workspace_bytes(desc, n_slices)
+ *              bytes, 256-byte aligned, owned by the caller
+ *
+ * n_slices >= 1 (more slices than heads act as one head per slice).  On a
+ * non-zero return some copies may already be in flight: synchronise the device
+ * before reusing the buffers.
+ */
+size_t gdn_host_workspace_bytes(const gdn_desc_t *desc, int n_slices);
+int gdn_chunk_fwd_host(const gdn_desc_t *desc, int n_slices, const void *q, const void *k, const void *v,
+                       const float *g, const float *beta, const float *S0, void *o, float *S_T, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/*
  * gdn_product_fwd -- prefill of Gated DeltaProduct: every real token applies
  * nh delta-rule transitions in order, each with its own key, value and write
  * strength, after one decay by the token's gate, and is read after the last
@@ -183,6 +209,39 @@ size_t gdn_segmented_workspace_bytes(const gdn_desc_t *desc, int nseg);
 int gdn_chunk_fwd_segmented(const gdn_desc_t *desc, int nseg, const void *q, const void *k, const void *v,
                             const float *g, const float *beta, const float *S0, void *o, float *S_T,
                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_segment_maps -- the affine map of a run of tokens taken as one segment
+ * ("One chunk as an affine recurrence", "Update the state"): for every (b,h),
+ * the T tokens send an incoming state S_in to S_in Lambda + H, where
+ *     H       [B,H,dv,dk] float  the state after the T tokens from S = 0,
+ *     Lambda  [B,H,dk,dk] float  the product of the tokens' transitions
+ *                                (Diag(alpha_t)(I - beta_t k_t k_t^T) for DELTA,
+ *                                Diag(alpha_t) for DECAY, I for ADDITIVE),
+ * both written (no outputs o).  Used when the segments of one sequence live on
+ * different devices: each device computes its segment's maps, the maps are
+ * gathered, gdn_compose_segments gives every segment its incoming state, and
+ * gdn_chunk_fwd from that state gives the outputs.  Inputs and their rules as in
+ * gdn_chunk_fwd (q is read though no output is formed); H and Lambda must be
+ * 16-byte aligned and overlap neither each other nor any input.  T == 0 gives
+ * H = 0, Lambda = I.
+ */
+int gdn_segment_maps(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
+                     const float *beta, float *H, float *Lambda, void *stream);
+
+/*
+ * gdn_compose_segments -- thread a state through nseg consecutive segments of
+ * BH sequences given their maps:  S_0 = S0 (zero when NULL),
+ * S_{i+1} = S_i Lambda_i + H_i; fp32 throughout.  Segment-major layouts:
+ *     H      [nseg][BH][dv][dk] float   (from gdn_segment_maps, segment by segment)
+ *     Lambda [nseg][BH][dk][dk] float   (NULL: every transition is the identity)
+ *     S_in   [nseg][BH][dv][dk] float   written: S_i, the state entering segment i (or NULL)
+ *     S_T    [BH][dv][dk]       float   written: S_nseg, the final state (or NULL; may be S0)
+ * dk, dv in {64, 128}; pointers 16-byte aligned; outputs overlap no input
+ * except S_T == S0 exactly.
+ */
+int gdn_compose_segments(int BH, int nseg, int dk, int dv, const float *S0, const float *H, const float *Lambda,
+                         float *S_in, float *S_T, void *stream);
 
 /*
  * gdn_decode_step -- decode: T recurrent steps (1 <= T <= GDN_DECODE_MAX_T,

@@ -12,7 +12,9 @@ Two implementations of the same definition:
   over heads, for small cases and to cross-check the compiled one;
 * ``gdp_forward`` -- Gated DeltaProduct (n_h delta substeps per token), NumPy;
 * ``prologue`` -- the optional input maps (feature map, L2 rows, sigmoid,
-  -softplus) applied before the recurrence.
+  -softplus) applied before the recurrence;
+* ``segment_maps`` -- the affine map (H, Lambda) of a run of tokens, Lambda as
+  the dense product of the per-token transition matrices.
 
 Definition (column convention, S in R^{dv x dk}, stored [B,H,dv,dk]):
 ``S_t = S_{t-1} Diag(alpha_t)(I - beta_t k_t k_t^T) + beta_t v_t k_t^T``,
@@ -175,6 +177,42 @@ def gdp_forward(gate, q, k, v, g=None, beta=None, S0=None):
             S = S + u[..., :, None] * kj[..., None, :]
         o[..., t, :] = np.einsum("...ij,...j->...i", S, q[..., t, :])
     return o, S
+
+
+def segment_maps(update, gate, k, v, g=None, beta=None):
+    """The affine map of a run of tokens ("Linear Attention, Visualized", "One
+    chunk as an affine recurrence" and "Update the state"): for any incoming
+    state, S_out = S_in Lam + H.
+
+    H [..., dv, dk] is the recurrence from the zero state (``gdn_forward`` with
+    S0 = 0).  Lam [..., dk, dk] is the ordered product of the tokens' transition
+    matrices, formed densely one token at a time: M_t = Diag(alpha_t)
+    (I - beta_t k_t k_t^T) for the delta write, Diag(alpha_t) for the decay
+    write, I for the additive write (alpha_t = exp(g_t), a scalar or one per key
+    channel).  Returns (H, Lam) as float64.
+    """
+    _check(update, gate, k, k, v, g, beta)
+    k, g, beta = _f64(k), _f64(g), _f64(beta)
+    lead = k.shape[:-2]
+    T, dk = k.shape[-2], k.shape[-1]
+    _, H = gdn_forward(update, gate, np.zeros_like(k), k, v, g=g, beta=beta)
+    eye = np.eye(dk)
+    Lam = np.broadcast_to(eye, lead + (dk, dk)).copy()
+    for t in range(T):
+        if gate == "scalar":
+            D = np.exp(g[..., t])[..., None, None] * eye
+        elif gate == "channel":
+            D = np.exp(g[..., t, :])[..., None, :] * eye
+        else:
+            D = np.broadcast_to(eye, lead + (dk, dk))
+        if update == "delta":
+            kt = k[..., t, :]
+            P = eye - beta[..., t][..., None, None] * (kt[..., :, None] * kt[..., None, :])
+            M = D @ P
+        else:
+            M = D
+        Lam = Lam @ M
+    return H, Lam
 
 
 PRO_QK_ELU1, PRO_QK_L2, PRO_BETA_SIGMOID, PRO_G_NEG_SOFTPLUS = 1, 2, 4, 8

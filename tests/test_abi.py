@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_strerror_and_version(lib):
-    assert gdn.version() == 2  # gdn_desc_t gained the prologue field
+    assert gdn.version() == 3  # segment maps and their composition joined the boundary
     for code in (0, -1, -2, -3, -4, -5, -6, 123):
         assert isinstance(gdn.strerror(code), str) and gdn.strerror(code)
 
@@ -140,6 +140,63 @@ def test_segmented_rejects_bad_arguments(lib):
     assert lib.gdn_chunk_fwd_segmented(ctypes.byref(d), 3, *args, vp(0x9000000), need - 4, None) == -1  # small
     assert lib.gdn_chunk_fwd_segmented(ctypes.byref(d), 3, *args, None, need, None) == -1  # no workspace
     assert lib.gdn_chunk_fwd_segmented(ctypes.byref(d), 3, *args, vp(0x9000008), need, None) == -2  # misaligned
+
+
+def test_segment_maps_reject_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    lib.gdn_segment_maps.argtypes = [ctypes.c_void_p] + [ctypes.c_void_p] * 8
+    d = _desc(T=96)
+    ins = (vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000))
+    H, L = vp(0x9000000), vp(0xA000000)
+    assert lib.gdn_segment_maps(ctypes.byref(d), *ins, None, L, None) == -1           # no H
+    assert lib.gdn_segment_maps(ctypes.byref(d), *ins, H, None, None) == -1           # no Lambda
+    assert lib.gdn_segment_maps(ctypes.byref(d), *ins, H, vp(0xA000004), None) == -2  # misaligned
+    assert lib.gdn_segment_maps(ctypes.byref(d), *ins, H, vp(0x9000010), None) == -1  # H and Lambda overlap
+    assert lib.gdn_segment_maps(ctypes.byref(d), vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000),
+                                vp(0x3000), L, None) == -1                             # H over v
+    assert lib.gdn_segment_maps(ctypes.byref(d), None, *ins[1:], H, L, None) == -1    # q missing
+    d = _desc(B=0)
+    assert lib.gdn_segment_maps(ctypes.byref(d), *ins, None, None, None) == 0          # empty batch: no-op
+
+
+def test_compose_segments_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    lib.gdn_compose_segments.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 6
+    S0, H, L, Si, ST = vp(0x1000000), vp(0x2000000), vp(0x4000000), vp(0x6000000), vp(0x8000000)
+    f = lib.gdn_compose_segments
+    assert f(4, 0, 128, 128, S0, H, L, Si, ST, None) == -1        # nseg < 1
+    assert f(-1, 2, 128, 128, S0, H, L, Si, ST, None) == -1       # negative count
+    assert f(4, 2, 96, 128, S0, H, L, Si, ST, None) == -1         # unsupported dk
+    assert f(4, 2, 128, 128, S0, None, L, Si, ST, None) == -1     # no H
+    assert f(4, 2, 128, 128, S0, H, L, vp(0x6000008), ST, None) == -2  # misaligned
+    assert f(4, 2, 128, 128, S0, H, L, vp(0x2000000 + 4096), ST, None) == -1  # S_in over H
+    assert f(4, 2, 128, 128, S0, H, L, Si, vp(0x1000000 + 4096), None) == -1  # S_T partly over S0
+    assert f(0, 2, 128, 128, S0, H, L, Si, ST, None) == 0         # no sequences: no-op
+
+
+def test_host_pipeline_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    f = lib.gdn_chunk_fwd_host
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int] + [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gdn_host_workspace_bytes.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    lib.gdn_host_workspace_bytes.restype = ctypes.c_size_t
+    d = _desc(T=96)
+    need = lib.gdn_host_workspace_bytes(ctypes.byref(d), 4)
+    # 6 heads in slices of 2: q, k, v (bf16), g, beta, S0, o (fp32), S_T per slot, each 256-aligned
+    per = lambda n: (n + 255) // 256 * 256
+    slot = sum(per(2 * x) for x in (96 * 128 * 2, 96 * 128 * 2, 96 * 128 * 2, 96 * 4, 96 * 4, 128 * 128 * 4,
+                                    96 * 128 * 4, 128 * 128 * 4))
+    assert need == 2 * slot
+    args = (vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000), None, vp(0x100000), None)
+    ws = vp(0x9000000)
+    assert f(ctypes.byref(d), 0, *args, ws, need, None) == -1              # n_slices < 1
+    assert f(ctypes.byref(d), 4, *args, ws, need - 1, None) == -1          # workspace too small
+    assert f(ctypes.byref(d), 4, *args, None, need, None) == -1            # no workspace
+    assert f(ctypes.byref(d), 4, *args, vp(0x9000010), need, None) == -2   # workspace not 256-aligned
+    assert f(ctypes.byref(d), 4, vp(0x1000), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x5000), None, vp(0x2000),
+             None, ws, need, None) == -1                                   # o over an input
+    d = _desc(B=0)
+    assert f(ctypes.byref(d), 4, *args, None, 0, None) == 0                # empty batch: no-op
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -87,3 +87,115 @@ def test_segmented_rejects_uneven_split():
     x = make_prefill_inputs(w)
     with pytest.raises(gdn.GDNError):
         run(w, x, 3)
+
+
+# ---------------------------------------------------------------------------
+# Segments on different devices: maps, composition, per-run prefill
+# ---------------------------------------------------------------------------
+
+def _dev_inputs(w, x, a=0, b=None):
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    b = w.T if b is None else b
+    sl = lambda v_: None if v_ is None else v_[:, :, a:b]
+    return {k_: (None if v_ is None else dev(np.ascontiguousarray(sl(v_)) if k_ != "S0" else v_,
+                                             dt if k_ in ("q", "k", "v") else torch.float32))
+            for k_, v_ in x.items()}
+
+
+@pytest.mark.parametrize("update,gate", MODES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_segment_maps_match_oracle(update, gate, dtype):
+    w = workload(update, gate, dtype, 150)
+    x = make_prefill_inputs(w)
+    t = _dev_inputs(w, x)
+    H, Lam = gdn.segment_maps(t["q"], t["k"], t["v"], t["g"], t["beta"], update=update, gate=gate)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    rH, rL = oracle.segment_maps(update, gate, x["k"], x["v"], g=x["g"], beta=x["beta"])
+    assert rel_err(np64(H), rH) <= TOL[dtype] and rel_err(np64(Lam), rL) <= TOL[dtype]
+    # the map's action on a state of unit scale: S0 Lam + H
+    S0 = np.random.default_rng(5).standard_normal(rH.shape)
+    assert rel_err(S0 @ np64(Lam) + np64(H), S0 @ rL + rH) <= TOL[dtype]
+
+
+def test_strongly_decayed_transition_keeps_its_digits():
+    # 400 tokens at g ~ -0.022 decay the transition to entries of about 4e-6, below
+    # fp16's normal range unless the transition pass runs from a scaled identity
+    w = workload("delta", "scalar", "bf16", 400).with_(gate_dist=("uniform", -0.025, -0.020))
+    x = make_prefill_inputs(w)
+    t = _dev_inputs(w, x)
+    _, Lam = gdn.segment_maps(t["q"], t["k"], t["v"], t["g"], t["beta"], update="delta", gate="scalar")
+    torch.cuda.synchronize()
+    _, rL = oracle.segment_maps("delta", "scalar", x["k"], x["v"], g=x["g"], beta=x["beta"])
+    assert np.sqrt(np.mean(rL ** 2)) < 1e-5
+    assert rel_err(np64(Lam), rL) <= TOL["bf16"]
+
+
+def test_compose_matches_float64():
+    r = np.random.default_rng(41)
+    nseg, BH, d = 5, 3, 128
+    H = r.standard_normal((nseg, 1, BH, d, d)) * 0.1
+    L = np.eye(d) * 0.9 + r.standard_normal((nseg, 1, BH, d, d)) * 0.02
+    S0 = r.standard_normal((1, BH, d, d)) * 0.1
+    S_in, ST = gdn.compose_segments(dev(H), dev(L), dev(S0))
+    S = S0
+    for i in range(nseg):
+        assert rel_err(np64(S_in[i]), S) <= 1e-5
+        S = S @ L[i] + H[i]
+    assert rel_err(np64(ST), S) <= 1e-5
+    _, ST2 = gdn.compose_segments(dev(H), None, None, want_inputs=False)  # identity transitions, zero start
+    assert rel_err(np64(ST2), H.sum(0)) <= 1e-5
+
+
+@pytest.mark.parametrize("update,gate", [("delta", "scalar"), ("delta", "channel"), ("additive", "none"),
+                                         ("decay", "scalar")])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_runs_on_emulated_ranks_match_oracle(update, gate, dtype):
+    # three uneven runs (ragged chunks, one empty) as three devices would hold them
+    w = workload(update, gate, dtype, 300)
+    x = make_prefill_inputs(w)
+    cuts = [0, 70, 70, 229, 300]
+    maps = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        t = _dev_inputs(w, x, a, b)
+        maps.append(gdn.segment_maps(t["q"], t["k"], t["v"], t["g"], t["beta"], update=update, gate=gate))
+    H_all = torch.stack([m[0] for m in maps])
+    L_all = torch.stack([m[1] for m in maps])
+    S0 = dev(x["S0"])
+    S_in, ST = gdn.compose_segments(H_all, L_all, S0)
+    outs = []
+    for i, (a, b) in enumerate(zip(cuts[:-1], cuts[1:])):
+        t = _dev_inputs(w, x, a, b)
+        o, _ = gdn.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], S_in[i], update=update, gate=gate,
+                             return_state=False)
+        outs.append(np64(o))
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    ro, rS = oracle.gdn_forward(update, gate, x["q"], x["k"], x["v"], g=x["g"], beta=x["beta"], S0=x["S0"])
+    assert rel_err(np.concatenate(outs, axis=2), ro) <= TOL[dtype]
+    assert rel_err(np64(ST), rS) <= TOL[dtype]
+
+
+def test_seqpar_on_a_single_rank_group():
+    # the torch.distributed path end to end (one NCCL rank): equals gdn_chunk_fwd
+    import socket
+
+    import torch.distributed as dist
+
+    from gated_delta_rule_97_b200.seqpar import chunk_fwd_seqpar
+
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % port, rank=0, world_size=1)
+    try:
+        w = workload("delta", "scalar", "bf16", 256)
+        x = make_prefill_inputs(w)
+        t = _dev_inputs(w, x)
+        o, ST = chunk_fwd_seqpar(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], update="delta", gate="scalar")
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    ro, rS = oracle.gdn_forward("delta", "scalar", x["q"], x["k"], x["v"], g=x["g"], beta=x["beta"], S0=x["S0"])
+    assert rel_err(np64(o), ro) <= TOL["bf16"] and rel_err(np64(ST), rS) <= TOL["bf16"]

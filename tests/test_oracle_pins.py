@@ -341,6 +341,53 @@ def test_split_sequence_composes(oracle_mod):
     assert rel_err(np.concatenate([oa, ob], axis=1), o) < 1e-13 and rel_err(Sb, ST) < 1e-13
 
 
+SEG_MODES = [("additive", "none"), ("decay", "scalar"), ("decay", "channel"), ("delta", "none"),
+             ("delta", "scalar"), ("delta", "channel")]
+
+
+@pytest.mark.parametrize("update,gate", SEG_MODES)
+def test_segment_map_is_affine(oracle_mod, update, gate):
+    """The run's final state from any S0 is S0 Lam + H ("One chunk as an affine
+    recurrence"): the recurrence against the dense transition product."""
+    q, k, v, g, beta, S0 = rand_inputs(21, BH=2, T=30, dk=8, dv=6, gate=gate, delta=update == "delta", s0=True)
+    H, Lam = oracle.segment_maps(update, gate, k, v, g=g, beta=beta)
+    _, ST = oracle.gdn_forward(update, gate, q, k, v, g=g, beta=beta, S0=S0)
+    assert rel_err(S0 @ Lam + H, ST) < 1e-12
+    _, H0 = oracle.gdn_forward(update, gate, q, k, v, g=g, beta=beta)
+    assert rel_err(H, H0) < 1e-14
+
+
+def test_segment_map_special_cases(oracle_mod):
+    # additive write: the identity transition
+    q, k, v, _, _, _ = rand_inputs(22, BH=2, T=12, dk=8, dv=6)
+    assert np.array_equal(oracle.segment_maps("additive", "none", k, v)[1], np.broadcast_to(np.eye(8), (2, 8, 8)))
+    # delta write with beta = 0 under a scalar gate: exp(sum g) I, and H = 0
+    q, k, v, g, beta, _ = rand_inputs(23, BH=2, T=12, dk=8, dv=6, gate="scalar", delta=True)
+    H, Lam = oracle.segment_maps("delta", "scalar", k, v, g=g, beta=np.zeros_like(beta))
+    expect = np.exp(g.sum(-1))[:, None, None] * np.eye(8)
+    assert rel_err(Lam, expect) < 1e-14 and np.all(H == 0)
+    # beta = 1 on orthonormal keys, no gate: the projector onto their complement
+    kk = orthonormal_keys(8, 5, seed=24)[None]
+    H, Lam = oracle.segment_maps("delta", "none", kk, np.zeros((1, 5, 3)), beta=np.ones((1, 5)))
+    assert rel_err(Lam[0], np.eye(8) - kk[0].T @ kk[0]) < 1e-14
+
+
+def test_segment_maps_compose_along_the_sequence(oracle_mod):
+    """Three consecutive runs composed through their maps give the one-run
+    state; each run's incoming state is the composition of those before it."""
+    q, k, v, g, beta, S0 = rand_inputs(25, BH=2, T=36, dk=8, dv=6, gate="channel", delta=True, s0=True)
+    cuts = [0, 10, 23, 36]
+    S = S0
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        _, S_ref = oracle.gdn_forward("delta", "channel", q[:, :a], k[:, :a], v[:, :a], g=g[:, :a],
+                                      beta=beta[:, :a], S0=S0) if a else (None, S0)
+        assert rel_err(S, S_ref) < 1e-12
+        H, Lam = oracle.segment_maps("delta", "channel", k[:, a:b], v[:, a:b], g=g[:, a:b], beta=beta[:, a:b])
+        S = S @ Lam + H
+    _, ST = oracle.gdn_forward("delta", "channel", q, k, v, g=g, beta=beta, S0=S0)
+    assert rel_err(S, ST) < 1e-12
+
+
 # ---------------------------------------------------------------------------
 # Planted mistakes: each must break at least one pin
 # ---------------------------------------------------------------------------
