@@ -84,6 +84,10 @@ def load():
     lib.gdn_segmented_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_chunk_fwd_segmented.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.gdn_chunk_fwd_segmented.restype = ctypes.c_int
+    lib.gdn_noalloc_scratch_bytes.argtypes = []
+    lib.gdn_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.gdn_chunk_fwd_segmented_noalloc.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gdn_chunk_fwd_segmented_noalloc.restype = ctypes.c_int
     lib.gdn_host_workspace_bytes.argtypes = [dp, ctypes.c_int]
     lib.gdn_host_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_chunk_fwd_host.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
@@ -343,6 +347,45 @@ def chunk_fwd_segmented(q, k, v, g=None, beta=None, S0=None, *, update, gate, ns
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_chunk_fwd_segmented")
     return o, S_T
+
+
+def chunk_fwd_segmented_noalloc(q, k, v, g=None, beta=None, S0=None, *, update, gate, nseg, out_dtype=None,
+                                o=None, S_T=None, return_state=True, algo="auto", prologue=0, stream=None):
+    """gdn_chunk_fwd_segmented_noalloc: chunk_fwd_segmented with its scratch
+    in the library's fixed device array (noalloc_scratch_bytes()); nothing is
+    allocated when o (and S_T, or return_state=False) are given.  Returns (o, S_T)."""
+    import torch
+
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
+    if gate == "scalar":
+        _check(g, "g", (B, H, T), torch.float32)
+    elif gate == "channel":
+        _check(g, "g", (B, H, T, dk), torch.float32)
+    _check(beta, "beta", (B, H, T), torch.float32)
+    _check(S0, "S0", (B, H, dv, dk), torch.float32)
+    if out_dtype is None:
+        out_dtype = o.dtype if o is not None else torch.float32
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
+    _check(o, "o", (B, H, T, dv), out_dtype)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
+                  prologue=prologue)
+    rc = load().gdn_chunk_fwd_segmented_noalloc(ctypes.byref(d), int(nseg), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                                _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_chunk_fwd_segmented_noalloc")
+    return o, S_T
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(load().gdn_noalloc_scratch_bytes())
 
 
 def segmented_workspace_bytes(B, H, T, dk, dv, nseg) -> int:

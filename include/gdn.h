@@ -211,6 +211,24 @@ int gdn_chunk_fwd_segmented(const gdn_desc_t *desc, int nseg, const void *q, con
                             void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gdn_chunk_fwd_segmented_noalloc -- gdn_chunk_fwd_segmented with the
+ * workspace taken from a fixed device array of the library
+ * (GDN_NOALLOC_SCRATCH_BYTES per device, mapped on first use) instead of the
+ * caller, so the call allocates nothing and takes no workspace argument.  The
+ * pages have no counterpart: it is a calling convenience for callers that
+ * cannot allocate on the call path.  Requests whose workspace
+ * (gdn_segmented_workspace_bytes) exceeds the array return
+ * GDN_ERR_UNSUPPORTED; other arguments and results as gdn_chunk_fwd_segmented.
+ * Concurrent calls on one device share the array and must be ordered (one
+ * stream, or events).
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+size_t gdn_noalloc_scratch_bytes(void);
+int gdn_chunk_fwd_segmented_noalloc(const gdn_desc_t *desc, int nseg, const void *q, const void *k, const void *v,
+                                    const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                                    void *stream);
+
+/*
  * gdn_segment_maps -- the affine map of a run of tokens taken as one segment
  * ("One chunk as an affine recurrence", "Update the state"): for every (b,h),
  * the T tokens send an incoming state S_in to S_in Lambda + H, where
