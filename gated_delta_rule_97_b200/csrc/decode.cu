@@ -164,16 +164,144 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
     for (int r = 0; r < kRowsPerWarp; ++r) VecF<V>::store(Srow + (size_t)r * DK, s[r]);
 }
 
+// ---------------------------------------------------------------------------
+// T > 1 tokens per call.  The single-token layout above spreads a row over the
+// 32 lanes, so each row and token costs two 5-level butterflies: with several
+// tokens the shuffles, not the state stream, set the time.  Here lane l owns
+// columns [c0, c0 + E) of row l / 8 (E = dk / 8): the row sums take 3-level
+// butterflies that reduce the warp's four rows at once (9 shuffles per token
+// and warp instead of 45).  The state stays in registers across the tokens.
+template <typename TIn, int N>
+struct RowLoad;
+template <int N>
+struct RowLoad<__nv_bfloat16, N> {
+    __device__ static void load(const __nv_bfloat16 *p, float *x) {
+#pragma unroll
+        for (int i = 0; i < N / 8; ++i) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(p + 8 * i);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+                x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+            }
+        }
+    }
+};
+template <int N>
+struct RowLoad<float, N> {
+    __device__ static void load(const float *p, float *x) {
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i) {
+            const float4 f = *reinterpret_cast<const float4 *>(p + 4 * i);
+            x[4 * i] = f.x; x[4 * i + 1] = f.y; x[4 * i + 2] = f.z; x[4 * i + 3] = f.w;
+        }
+    }
+};
+
+__device__ __forceinline__ float row_sum8(float x) {  // over the 8 lanes of a row group
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    return x;
+}
+
+template <int DK, int UPD, int GATE, typename TIn, typename TOut, bool PRO>
+__global__ void __launch_bounds__(kThreads) decode_multi_kernel(DecodeArgs a) {
+    constexpr int E = DK / 8;
+    const long warp = ((long)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long row0 = warp * kRowsPerWarp;
+    if (row0 >= (long)a.BH * a.dv) return;
+    const long bh = row0 / a.dv;
+    const int i = (int)(row0 - bh * a.dv) + (lane >> 3);  // this lane's state row
+    const int c0 = (lane & 7) * E;
+    const int pro = PRO ? a.pro : 0;
+
+    float *Srow = a.S + ((size_t)bh * a.dv + i) * DK + c0;
+    float s[E];
+#pragma unroll
+    for (int e = 0; e < E; e += 4) VecF<4>::load(Srow + e, s + e);
+
+#pragma unroll 1
+    for (int t = 0; t < a.T; ++t) {
+        const long tok = bh * a.T + t;
+        float qq[E], kk[E];
+        RowLoad<TIn, E>::load(static_cast<const TIn *>(a.q) + tok * DK + c0, qq);
+        RowLoad<TIn, E>::load(static_cast<const TIn *>(a.k) + tok * DK + c0, kk);
+        const float vi = to_f32(static_cast<const TIn *>(a.v)[tok * a.dv + i]);
+        const float bt = (UPD == kDelta) ? pro_beta(a.beta[tok], pro) : 0.f;
+        if (pro) {
+            float sq = 0.f, sk = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                qq[e] = pro_feature(qq[e], pro);
+                kk[e] = pro_feature(kk[e], pro);
+                sq = fmaf(qq[e], qq[e], sq);
+                sk = fmaf(kk[e], kk[e], sk);
+            }
+            if (pro & kProL2) {  // unit q and k rows; a zero row stays zero
+                sq = row_sum8(sq);
+                sk = row_sum8(sk);
+                const float iq = sq > 0.f ? 1.f / sqrtf(sq) : 0.f, ik = sk > 0.f ? 1.f / sqrtf(sk) : 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    qq[e] *= iq;
+                    kk[e] *= ik;
+                }
+            }
+        }
+        float kq = 0.f, p = 0.f, rr = 0.f;
+        if (GATE == kGateChannel) {
+            float gg[E];
+            RowLoad<float, E>::load(a.g + tok * DK + c0, gg);
+#pragma unroll
+            for (int e = 0; e < E; ++e) s[e] *= __expf(pro_gate(gg[e], pro));
+        } else if (GATE == kGateScalar) {
+            const float al = __expf(pro_gate(a.g[tok], pro));
+#pragma unroll
+            for (int e = 0; e < E; ++e) s[e] *= al;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            kq = fmaf(kk[e], qq[e], kq);
+            p = fmaf(s[e], kk[e], p);
+            rr = fmaf(s[e], qq[e], rr);
+        }
+        kq += __shfl_xor_sync(0xffffffffu, kq, 1);
+        p += __shfl_xor_sync(0xffffffffu, p, 1);
+        rr += __shfl_xor_sync(0xffffffffu, rr, 1);
+        kq += __shfl_xor_sync(0xffffffffu, kq, 2);
+        p += __shfl_xor_sync(0xffffffffu, p, 2);
+        rr += __shfl_xor_sync(0xffffffffu, rr, 2);
+        kq += __shfl_xor_sync(0xffffffffu, kq, 4);
+        p += __shfl_xor_sync(0xffffffffu, p, 4);
+        rr += __shfl_xor_sync(0xffffffffu, rr, 4);
+        const float u = (UPD == kDelta) ? bt * (vi - p) : vi;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s[e] = fmaf(u, kk[e], s[e]);
+        if ((lane & 7) == 0) static_cast<TOut *>(a.o)[tok * a.dv + i] = from_f32<TOut>(fmaf(u, kq, rr));
+    }
+#pragma unroll
+    for (int e = 0; e < E; e += 4) VecF<4>::store(Srow + e, s + e);
+}
+
 template <int DK, int UPD, int GATE, typename TIn, typename TOut>
 int launch(const DecodeArgs &a, cudaStream_t stream) {
     const long rows = (long)a.BH * a.dv;
     const long warps = rows / kRowsPerWarp;
     const long blocks = (warps * 32 + kThreads - 1) / kThreads;
     if (blocks == 0) return 0;
-    if (a.pro)
+    if (a.T > 1) {
+        if (a.pro)
+            decode_multi_kernel<DK, UPD, GATE, TIn, TOut, true><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+        else
+            decode_multi_kernel<DK, UPD, GATE, TIn, TOut, false><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+    } else if (a.pro) {
         decode_kernel<DK, UPD, GATE, TIn, TOut, true><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
-    else
+    } else {
         decode_kernel<DK, UPD, GATE, TIn, TOut, false><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+    }
     return (int)cudaGetLastError();
 }
 
