@@ -425,6 +425,12 @@ def run_ours(args):
         if rank == 0:
             print(json.dumps({"only": "decode", "ms_per_step": ms_d}), flush=True)
         return
+    if args.only == "decode_multi":
+        wd = WORKLOADS["decode_gdn_bf16"]
+        ms_m = time_decode_multi(wd, 4, 25 if args.quick else 100, torch, gdn)
+        if rank == 0:
+            print(json.dumps({"only": "decode_multi", "tokens_per_call": 4, "ms_per_call": ms_m}), flush=True)
+        return
     w = WORKLOADS[args.workload]
     x = make_prefill_inputs(w)
     if args.only == "prefill":
@@ -583,7 +589,7 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=[k for k, w in WORKLOADS.items() if w.steps == 0])
     ap.add_argument("--quick", action="store_true", help="skip the extra prefill workloads; 100 decode steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_multi"], default="all",
                     help="profiling aid: run one part only (its line is not a benchmark result)")
     args = ap.parse_args()
     if args.warmup < 3:
