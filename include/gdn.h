@@ -101,7 +101,7 @@ typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TC = 2, GDN_ALGO_T
 
 typedef struct {
     int B, H;      /* batch and heads; B*H >= 0 */
-    int T;         /* tokens per sequence (gdn_chunk_fwd: T >= 0; decode: T == 1) */
+    int T;         /* tokens per sequence (gdn_chunk_fwd: T >= 0; decode: 0..GDN_DECODE_MAX_T) */
     int dk, dv;    /* key and value head dims, each 64 or 128 */
     int update;    /* gdn_update_t */
     int gate;      /* gdn_gate_t */
