@@ -2,8 +2,9 @@
 // (each segment's H and Lambda and its incoming state) lives in a fixed device
 // array of this library: a __device__ variable exists once per device context
 // that loads the library, and its address is looked up on the calling thread's
-// current device at every call.  The array is only mapped when this entry point
-// is first used (modules load lazily), so other callers pay nothing for it.
+// current device at every call.  This file holds no kernel, so with lazy module
+// loading (the CUDA default) the array is only mapped when this entry point is
+// first used and other callers pay nothing for it.
 // Calls that run at the same time on one device share the array: order them
 // (one stream, or events), or use gdn_chunk_fwd_segmented with a workspace each.
 #include <cuda_runtime.h>

@@ -151,7 +151,9 @@ int gdn_chunk_fwd(const gdn_desc_t *desc, const void *q, const void *k, const vo
  * host-resident use of the same prefill.)
  *
  *   workspace  device buffer of gdn_host_workspace_bytes(desc, n_slices)
- *              bytes, 256-byte aligned, owned by the caller
+ *              bytes, 256-byte aligned, owned by the caller, on the calling
+ *              thread's current device (where the two internal streams are
+ *              created; `stream` must belong to that device too)
  *
  * n_slices >= 1 (more slices than heads act as one head per slice).  On a
  * non-zero return some copies may already be in flight: synchronise the device
@@ -213,7 +215,8 @@ int gdn_chunk_fwd_segmented(const gdn_desc_t *desc, int nseg, const void *q, con
 /*
  * gdn_chunk_fwd_segmented_noalloc -- gdn_chunk_fwd_segmented with the
  * workspace taken from a fixed device array of the library
- * (GDN_NOALLOC_SCRATCH_BYTES per device, mapped on first use) instead of the
+ * (GDN_NOALLOC_SCRATCH_BYTES per device; with lazy module loading, the CUDA
+ * default, it is mapped on first use) instead of the
  * caller, so the call allocates nothing and takes no workspace argument.  The
  * pages have no counterpart: it is a calling convenience for callers that
  * cannot allocate on the call path.  Requests whose workspace
