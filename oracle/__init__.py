@@ -95,6 +95,15 @@ def _check(update, gate, q, k, v, g, beta):
         raise ValueError("g must be given iff gate != 'none'")
     if q.shape[:-1] != k.shape[:-1] or q.shape[-1] != k.shape[-1] or v.shape[:-1] != q.shape[:-1]:
         raise ValueError("shape mismatch")
+    # the gate is one value per token (scalar) or one per token and key channel;
+    # beta one per token: a tensor laid out along another axis is an error here,
+    # not a silently different recurrence
+    if g is not None:
+        want = q.shape[:-1] if gate == "scalar" else q.shape
+        if np.shape(g) != tuple(want):
+            raise ValueError("g has shape %s, expected %s" % (np.shape(g), tuple(want)))
+    if beta is not None and np.shape(beta) != tuple(q.shape[:-1]):
+        raise ValueError("beta has shape %s, expected %s" % (np.shape(beta), tuple(q.shape[:-1])))
 
 
 def gdn_forward(update, gate, q, k, v, g=None, beta=None, S0=None):

@@ -571,3 +571,71 @@ def test_prologue_l2_rows():
     q2, _, _, _ = oracle.prologue(oracle.PRO_QK_ELU1 | oracle.PRO_QK_L2, q=x)
     e = np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
     assert np.allclose(q2, e / np.linalg.norm(e, axis=-1, keepdims=True), atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Decode: consecutive single-token steps are the recurrence over the stacked
+# sequence ("Optional: Linear attention as an RNN": one state, one token at a
+# time).  decode_sequence is the reference of every decode GPU test, so its
+# stacking (per tensor, along the token axis) is pinned against explicit d x d
+# products over the same tokens, gathered by hand one step and head at a time.
+# ---------------------------------------------------------------------------
+
+def _decode_steps(seed, gate, update, B=2, H=2, n=9, dk=6, dv=5):
+    r = np.random.default_rng(seed)
+    steps = []
+    for _ in range(n):
+        k = r.standard_normal((B, H, 1, dk))
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+        s = {"q": r.standard_normal((B, H, 1, dk)), "k": k, "v": r.standard_normal((B, H, 1, dv)),
+             "beta": r.uniform(0.05, 1.0, (B, H, 1)) if update == "delta" else None, "g": None}
+        if gate == "scalar":
+            s["g"] = r.uniform(-0.4, 0.0, (B, H, 1))
+        elif gate == "channel":
+            s["g"] = r.uniform(-0.4, 0.0, (B, H, 1, dk))
+        steps.append(s)
+    S0 = 0.3 * r.standard_normal((B, H, dv, dk))
+    return steps, S0
+
+
+@pytest.mark.parametrize("update,gate", [("delta", "scalar"), ("delta", "channel"), ("delta", "none"),
+                                         ("decay", "scalar"), ("decay", "channel"), ("additive", "none")])
+def test_decode_sequence_equals_explicit_products(oracle_mod, update, gate):
+    steps, S0 = _decode_steps(61, gate, update)
+    o, S = oracle.decode_sequence(update, gate, S0, steps)
+    n = len(steps)
+    B, H = S0.shape[:2]
+    assert o.shape == (B, H, n, steps[0]["v"].shape[-1]) and S.shape == S0.shape
+    for b in range(B):
+        for h in range(H):
+            # this head's tokens, taken from each step's dict in order
+            q = np.stack([s["q"][b, h, 0] for s in steps])
+            k = np.stack([s["k"][b, h, 0] for s in steps])
+            v = np.stack([s["v"][b, h, 0] for s in steps])
+            g = None if gate == "none" else np.stack([np.asarray(s["g"][b, h, 0]) for s in steps])
+            beta = None if update != "delta" else np.array([s["beta"][b, h, 0] for s in steps])
+            ro, rS = brute_force_matrices(update, gate, q, k, v, g, beta, S0[b, h])
+            assert rel_err(o[b, h], ro) < TOL and rel_err(S[b, h], rS) < TOL
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_decode_sequence_chains_one_step_calls(oracle_mod, gate):
+    """n calls of one step each, the state handed on, equal one call of n steps."""
+    steps, S0 = _decode_steps(62, gate, "delta")
+    o, S = oracle.decode_sequence("delta", gate, S0, steps)
+    Sc = S0
+    for i, s in enumerate(steps):
+        oi, Sc = oracle.decode_sequence("delta", gate, Sc, [s])
+        assert rel_err(oi[..., 0, :], o[..., i, :]) < TOL
+    assert rel_err(Sc, S) < TOL
+
+
+def test_gate_and_beta_layouts_are_checked(oracle_mod):
+    """A gate or write strength laid out along the wrong axis is rejected."""
+    q, k, v, g, beta, _ = rand_inputs(63, BH=2, T=5, dk=4, dv=3, gate="channel", delta=True)
+    with pytest.raises(ValueError):
+        oracle.gdn_forward("delta", "channel", q, k, v, g=g[..., 0], beta=beta)
+    with pytest.raises(ValueError):
+        oracle.gdn_forward("delta", "scalar", q, k, v, g=g, beta=beta)
+    with pytest.raises(ValueError):
+        oracle.gdn_forward("delta", "channel", q, k, v, g=g, beta=beta[..., None])
