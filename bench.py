@@ -59,8 +59,14 @@ def measured_traffic(workload):
     return rec["dram_bytes_read"] + rec["dram_bytes_write"]
 
 
-def prefill_bytes(w, out_bytes=4):
+def prefill_bytes(w, out_bytes=None):
+    """Algorithmic bytes of one prefill launch: q, k, v, g, beta read once, o
+    written once, S0 read and S_T written once per head.  By default o is
+    counted in the input dtype (the survey's per-token bytes); ``out_bytes=4``
+    counts the fp32 o this benchmark actually writes."""
     in_b = 2 if w.dtype == "bf16" else 4
+    if out_bytes is None:
+        out_bytes = in_b
     per_tok = (2 * w.dk + w.dv) * in_b + w.dv * out_bytes
     if w.gate == "scalar":
         per_tok += 4
@@ -241,8 +247,10 @@ def time_product(w, nh, steps, warmup, torch, gdn):
     return e0.elapsed_time(e1) / steps
 
 
-def product_bytes(w, nh, out_bytes=4):
+def product_bytes(w, nh, out_bytes=None):
     in_b = 2 if w.dtype == "bf16" else 4
+    if out_bytes is None:
+        out_bytes = in_b
     per_tok = w.dk * in_b + nh * (w.dk + w.dv) * in_b + w.dv * out_bytes + 4 + 4 * nh
     state = w.dv * w.dk * 4 * ((1 if w.s0_std > 0 else 0) + 1)
     return w.n_heads * (w.T * per_tok + state)
@@ -395,6 +403,37 @@ def cpu_baseline(w, budget_s=15.0):
                       % (n_heads, w.n_heads, w.T, token_heads, dt)}
 
 
+def bench_config(w, world):
+    """The workload description both arms print (same keys, same values)."""
+    nbytes = prefill_bytes(w, out_bytes=4)
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "update": w.update,
+            "gate": w.gate, "chunk": w.chunk, "global_batch": w.B * world, "seq_len": w.T,
+            "parallelism": "replicas x%d (batch per GPU fixed)" % world,
+            "l2": "inputs and outputs (%.2f GB) larger than the 126 MB L2, no flush" % (nbytes / 1e9)}
+
+
+def roofline(w, ms, peaks, peak_kind):
+    """HBM roofline of one prefill launch.  ``frac`` counts the algorithmic bytes
+    with o in the input dtype (bf16 here); the kernel writes o in fp32, and
+    ``fp32_output`` gives the same figures with those bytes counted."""
+    nbytes = prefill_bytes(w)
+    nbytes32 = prefill_bytes(w, out_bytes=4)
+    flops = prefill_flops(w)
+    s = ms * 1e-3
+    achieved = nbytes / s / 1e9
+    t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    t_roof32 = max(nbytes32 / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(w.name), "peak_source": peak_kind,
+            "algorithmic_bytes_per_launch": nbytes, "bytes_note": "o counted in the input dtype (bf16)",
+            "flops_per_launch": flops, "achieved_tflops": flops / s / 1e12,
+            "tensor_frac": flops / s / 1e12 / peaks["bf16_tflops"],
+            "roofline_us": t_roof * 1e6, "frac_of_roofline_time": t_roof / s,
+            "fp32_output": {"bytes_per_launch": nbytes32, "achieved": nbytes32 / s / 1e9,
+                            "frac": nbytes32 / s / 1e9 / peaks["hbm_gbs"], "roofline_us": t_roof32 * 1e6,
+                            "note": "o counted as the fp32 tensor the kernel writes"}}
+
+
 def run_ours(args):
     import torch
 
@@ -443,24 +482,12 @@ def run_ours(args):
     clocks = clk.summary()
     tokens = w.B * w.T
     value = world * tokens / (ms * 1e-3)
-    nbytes = prefill_bytes(w)
-    flops = prefill_flops(w)
-    achieved_gbs = nbytes / (ms * 1e-3) / 1e9
-    t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
     result = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
               "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
               "vs_baseline": None, "dtype": "bf16 in / fp32 state, accumulation, output", "data": "synthetic",
-              "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
-                         "update": w.update, "gate": w.gate, "chunk": w.chunk, "global_batch": w.B * world,
-                         "seq_len": w.T, "parallelism": "replicas x%d (batch per GPU fixed)" % world,
-                         "l2": "inputs (%.2f GB) larger than the 126 MB L2" % (nbytes / 1e9)},
+              "config": bench_config(w, world),
               "token_heads_per_s": world * w.n_heads * w.T / (ms * 1e-3),
-              "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": measured_traffic(w.name),
-                           "peak_source": peak_kind, "algorithmic_bytes_per_launch": nbytes,
-                           "flops_per_launch": flops,
-                           "achieved_tflops": flops / (ms * 1e-3) / 1e12,
-                           "roofline_us": t_roof * 1e6, "frac_of_roofline_time": t_roof / (ms * 1e-3)},
+              "roofline": roofline(w, ms, peaks, peak_kind),
               "gpu_launches": args.steps, "clocks": clocks}
 
     ms_e2e, h2d, d2h = time_prefill_e2e(w, x, max(2, min(args.steps, 5)), args.warmup, torch, gdn)
@@ -499,11 +526,11 @@ def run_ours(args):
             mso = time_prefill(wo, xo, max(3, args.steps // 2), args.warmup, torch, gdn, dist)
             result["gpu_launches"] += max(3, args.steps // 2)
             del xo
-            nb, fl = prefill_bytes(wo), prefill_flops(wo)
-            tr = max(nb / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+            rf = roofline(wo, mso, peaks, peak_kind)
             others[name] = {"ms_per_step": mso, "tokens_per_s": wo.B * wo.T * world / (mso * 1e-3),
-                            "achieved_gbs": nb / (mso * 1e-3) / 1e9, "roofline_us": tr * 1e6,
-                            "frac_of_roofline_time": tr / (mso * 1e-3)}
+                            "achieved_gbs": rf["achieved"], "roofline_us": rf["roofline_us"],
+                            "frac_of_roofline_time": rf["frac_of_roofline_time"],
+                            "frac_fp32_output": rf["fp32_output"]["frac"]}
         # Gated DeltaProduct, 2 substeps per token, on the GDN workload's heads and
         # 4096 tokens (8192 virtual steps, the GDN workload's length)
         wp, nh = WORKLOADS["gdn_prefill_bf16"].with_(T=4096, name="gdp_prefill_bf16"), 2
@@ -561,7 +588,7 @@ def run_reference(args):
     xs = make_prefill_inputs(w, heads=heads)
     run = lambda: oracle.gdn_forward(w.update, w.gate, xs["q"], xs["k"], xs["v"], g=xs["g"], beta=xs["beta"],
                                      S0=xs["S0"])
-    for _ in range(min(args.warmup, 1)):
+    for _ in range(args.warmup):
         run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
@@ -573,11 +600,48 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "update": w.update,
-                   "gate": w.gate, "chunk": w.chunk},
+        "config": bench_config(w, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
         flush=True)
+
+
+def relaunch(n_procs):
+    """``--gpus N`` (N > 1) started as a single process: start N ranks of this
+    script on one node with torch.distributed.run (rendezvous on 127.0.0.1) and
+    return the launcher's exit status."""
+    import socket
+
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=%d" % n_procs,
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+def launch_check(args):
+    """The rank protocol alone, on CPU (gloo): every rank joins, takes the same
+    barrier and max-over-ranks steps as a timed run, and rank 0 prints the line's
+    rank-dependent keys.  No GPU work; a test of the launcher."""
+    import datetime
+
+    import torch.distributed as tdist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        tdist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        dist = tdist
+        dist.barrier()
+    ms = max_over_ranks(1.0 + rank, dist, "cpu")
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"launch_check": True, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": ms}), flush=True)
 
 
 def main():
@@ -591,10 +655,21 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_multi"], default="all",
                     help="profiling aid: run one part only (its line is not a benchmark result)")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="test aid: run only the rank protocol on CPU (gloo), no GPU work")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        sys.exit(relaunch(args.gpus))
+    if env_world is not None and int(env_world) != args.gpus:
+        ap.error("--gpus %d but WORLD_SIZE=%s" % (args.gpus, env_world))
+    if args.launch_check:
+        launch_check(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
