@@ -25,7 +25,7 @@ _LIB_PATH = os.path.join(_HERE, "libgdn.so")
 
 UPDATES = {"additive": 0, "decay": 1, "delta": 2}
 GATES = {"none": 0, "scalar": 1, "channel": 2}
-ALGOS = {"auto": 0, "simt": 1, "tc": 2, "tc_seq": 3}
+ALGOS = {"auto": 0, "simt": 1, "tc": 2}
 F32, BF16 = 0, 1
 
 DECODE_MAX_T = 16  # GDN_DECODE_MAX_T
@@ -128,11 +128,22 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, t):
+    """The stream to launch on: ``stream``, else the current stream of the
+    device that holds ``t``."""
     import torch
 
-    s = torch.cuda.current_stream() if stream is None else stream
+    s = torch.cuda.current_stream(t.device) if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _on_device(t):
+    """Makes the device that holds ``t`` current for the call: the library
+    launches on, and takes its status word and scratch from, the calling
+    thread's current device."""
+    import torch
+
+    return torch.cuda.device(t.device)
 
 
 def _dtype_code(dt):
@@ -197,8 +208,9 @@ def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=No
     _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
     d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
                   prologue=prologue)
-    rc = load().gdn_chunk_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
-                              _ptr(o), _ptr(S_T), _stream(stream))
+    with _on_device(q):
+        rc = load().gdn_chunk_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                  _ptr(o), _ptr(S_T), _stream(stream, q))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_chunk_fwd")
     return o, S_T
@@ -259,9 +271,10 @@ def chunk_fwd_host(q, k, v, g=None, beta=None, S0=None, *, update, gate, n_slice
                                 device=device if device is not None else torch.cuda.current_device())
     if not workspace.is_cuda or not workspace.is_contiguous() or workspace.numel() < need:
         raise ValueError("workspace needs %d contiguous CUDA bytes" % need)
-    rc = load().gdn_chunk_fwd_host(ctypes.byref(d), int(n_slices), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                   _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
-                                   _stream(stream))
+    with _on_device(workspace):
+        rc = load().gdn_chunk_fwd_host(ctypes.byref(d), int(n_slices), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                       _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                       _stream(stream, workspace))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_chunk_fwd_host")
     return o, S_T
@@ -300,8 +313,9 @@ def product_fwd(q, k, v, g=None, beta=None, S0=None, *, gate, out_dtype=None, o=
     _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
     d = make_desc(B, H, T, dk, dv, "delta", gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
                   prologue=prologue)
-    rc = load().gdn_product_fwd(ctypes.byref(d), ctypes.c_int(nh), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream))
+    with _on_device(q):
+        rc = load().gdn_product_fwd(ctypes.byref(d), ctypes.c_int(nh), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                    _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream, q))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_product_fwd")
     return o, S_T
@@ -341,9 +355,11 @@ def chunk_fwd_segmented(q, k, v, g=None, beta=None, S0=None, *, update, gate, ns
         workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
     if not workspace.is_cuda or not workspace.is_contiguous() or workspace.numel() * workspace.element_size() < need:
         raise ValueError("workspace needs %d contiguous CUDA bytes" % need)
-    rc = load().gdn_chunk_fwd_segmented(ctypes.byref(d), int(nseg), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                        _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
-                                        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+    with _on_device(q):
+        rc = load().gdn_chunk_fwd_segmented(ctypes.byref(d), int(nseg), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                            _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                                            ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                            _stream(stream, q))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_chunk_fwd_segmented")
     return o, S_T
@@ -377,8 +393,9 @@ def chunk_fwd_segmented_noalloc(q, k, v, g=None, beta=None, S0=None, *, update, 
     _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
     d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
                   prologue=prologue)
-    rc = load().gdn_chunk_fwd_segmented_noalloc(ctypes.byref(d), int(nseg), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                                _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream))
+    with _on_device(q):
+        rc = load().gdn_chunk_fwd_segmented_noalloc(ctypes.byref(d), int(nseg), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                                    _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream, q))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_chunk_fwd_segmented_noalloc")
     return o, S_T
@@ -417,8 +434,9 @@ def segment_maps(q, k, v, g=None, beta=None, *, update, gate, H=None, Lam=None, 
     _check(H, "H", (B, Hh, dv, dk), torch.float32)
     _check(Lam, "Lam", (B, Hh, dk, dk), torch.float32)
     d = make_desc(B, Hh, T, dk, dv, update, gate, _dtype_code(q.dtype), F32, algo, prologue=prologue)
-    rc = load().gdn_segment_maps(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(H),
-                                 _ptr(Lam), _stream(stream))
+    with _on_device(q):
+        rc = load().gdn_segment_maps(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(H),
+                                     _ptr(Lam), _stream(stream, q))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_segment_maps")
     return H, Lam
@@ -441,8 +459,9 @@ def compose_segments(H, Lam=None, S0=None, *, S_in=None, S_T=None, want_inputs=T
     if S_T is None:
         S_T = torch.empty((B, Hh, dv, dk), dtype=torch.float32, device=H.device)
     _check(S_T, "S_T", (B, Hh, dv, dk), torch.float32)
-    rc = load().gdn_compose_segments(B * Hh, nseg, dk, dv, _ptr(S0), _ptr(H), _ptr(Lam), _ptr(S_in), _ptr(S_T),
-                                     _stream(stream))
+    with _on_device(H):
+        rc = load().gdn_compose_segments(B * Hh, nseg, dk, dv, _ptr(S0), _ptr(H), _ptr(Lam), _ptr(S_in), _ptr(S_T),
+                                         _stream(stream, H))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_compose_segments")
     return S_in, S_T
@@ -476,8 +495,9 @@ def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, pr
         o = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
     _check(o, "o", (B, H, T, dv), out_dtype)
     d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), prologue=prologue)
-    rc = load().gdn_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
-                                _ptr(o), _stream(stream))
+    with _on_device(q):
+        rc = load().gdn_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                                    _ptr(o), _stream(stream, q))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_decode_step")
     return o

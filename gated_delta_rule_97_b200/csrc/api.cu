@@ -10,9 +10,8 @@
 __device__ int g_gdn_status = 0;
 __device__ int g_gdn_diag = 0;
 
-// tensor-core launchers (chunk_tc.cu, chunk_tc2.cu)
+// tensor-core launcher (chunk_tc2.cu)
 int gdn_tc_supported(const gdn_desc_t *d);
-int gdn_launch_chunk_tc(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
 int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
 
 namespace {
@@ -63,15 +62,12 @@ bool tc2_prologue_ok(const gdn_desc_t *d);
 
 // Kernel choice of gdn_chunk_fwd (and of the passes of the segmented prefill):
 // the requested kernel, or for AUTO the pipelined tensor-core kernel when it
-// serves the request and the SIMT kernel otherwise.  The input prologue runs in
-// the SIMT kernel and the pipelined tensor-core kernel, not in the sequential one.
+// serves the request and the SIMT kernel otherwise.  Both apply the input
+// prologue.
 int dispatch_chunk(const gdn_desc_t *d, gdn::ChunkArgs &a, cudaStream_t st) {
-    const bool tc_ok = gdn_tc_supported(d) != 0 && (d->prologue == 0 || d->algo != GDN_ALGO_TC_SEQ) &&
-                       tc2_prologue_ok(d);
-    if ((d->algo == GDN_ALGO_TC || d->algo == GDN_ALGO_TC_SEQ) && !tc_ok) return GDN_ERR_UNSUPPORTED;
-    if (a.mode != 0 && d->algo == GDN_ALGO_TC_SEQ) return GDN_ERR_UNSUPPORTED;
+    const bool tc_ok = gdn_tc_supported(d) != 0 && tc2_prologue_ok(d);
+    if (d->algo == GDN_ALGO_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
     if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));
-    if (d->algo == GDN_ALGO_TC_SEQ) return from_cuda(gdn_launch_chunk_tc(a, d, st));
     return from_cuda(gdn_launch_chunk_simt(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16, st));
 }
 
@@ -123,7 +119,7 @@ static int chunk_fwd_check(const gdn_desc_t *d, const void *q, const void *k, co
     int rc = validate_common(d);
     if (rc != GDN_OK) return rc;
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
-    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC_SEQ) return GDN_ERR_ARG;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC) return GDN_ERR_ARG;
     const long BH = (long)d->B * d->H;
     const size_t n_qk = (size_t)BH * d->T * d->dk, n_v = (size_t)BH * d->T * d->dv;
     const size_t n_S = (size_t)BH * d->dv * d->dk;
@@ -305,12 +301,12 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     if (nh > GDN_PRODUCT_MAX_NH) return GDN_ERR_UNSUPPORTED;
     if (nh == 1) return gdn_chunk_fwd(d, q, k, v, g, beta, S0, o, S_T, stream);
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
-    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC_SEQ) return GDN_ERR_ARG;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC) return GDN_ERR_ARG;
     // the pipelined tensor-core kernel takes whole tokens per chunk: nh a power of
     // two (it divides the chunk), scalar or no gate
     const bool pow2 = (nh & (nh - 1)) == 0;
     const bool tc_ok = gdn_tc_supported(d) != 0 && pow2 && d->gate != GDN_GATE_CHANNEL && tc2_prologue_ok(d);
-    if (d->algo == GDN_ALGO_TC_SEQ || (d->algo == GDN_ALGO_TC && !tc_ok)) return GDN_ERR_UNSUPPORTED;
+    if (d->algo == GDN_ALGO_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
     if ((long)d->T * nh > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
     const long BH = (long)d->B * d->H;
     const size_t Tr = (size_t)d->T, Tv = Tr * nh;
@@ -347,23 +343,38 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
 }
 
 extern "C" size_t gdn_segmented_workspace_bytes(const gdn_desc_t *d, int nseg) {
-    if (!d || nseg < 1) return 0;
-    const size_t segs = (size_t)d->B * d->H * nseg;
+    if (!d || nseg < 1 || d->B < 0 || d->H < 0 || d->dk < 0 || d->dv < 0) return 0;
+    // at most 2^30 segment-heads (larger requests are rejected), so the product
+    // below cannot wrap
+    const long bh = (long)d->B * d->H;
+    if (bh > (1L << 30) || bh * nseg > (1L << 30) || d->dk > 128 || d->dv > 128) return 0;
+    const size_t segs = (size_t)bh * nseg;
     return segs * ((size_t)2 * d->dv * d->dk + (size_t)d->dk * d->dk) * sizeof(float);
+}
+
+// The request rules of the segmented prefill that do not involve pointers (the
+// descriptor, the segment count and the total number of segment-heads), shared
+// with gdn_chunk_fwd_segmented_noalloc so that both reject a bad request with
+// the same code before looking at any scratch size.
+int gdn_segmented_request_check(const gdn_desc_t *d, int nseg) {
+    int rc = validate_common(d);
+    if (rc != GDN_OK) return rc;
+    if (nseg < 1) return GDN_ERR_ARG;
+    if (nseg == 1) return GDN_OK;
+    if (d->T % nseg != 0) return GDN_ERR_ARG;
+    if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC) return GDN_ERR_ARG;
+    if ((long)d->B * d->H * nseg > (1L << 30)) return GDN_ERR_ARG;
+    return GDN_OK;
 }
 
 extern "C" int gdn_chunk_fwd_segmented(const gdn_desc_t *d, int nseg, const void *q, const void *k, const void *v,
                                        const float *g, const float *beta, const float *S0, void *o, float *S_T,
                                        void *workspace, size_t workspace_bytes, void *stream) {
-    int rc = validate_common(d);
+    int rc = gdn_segmented_request_check(d, nseg);
     if (rc != GDN_OK) return rc;
-    if (nseg < 1) return GDN_ERR_ARG;
     if (nseg == 1) return gdn_chunk_fwd(d, q, k, v, g, beta, S0, o, S_T, stream);
-    if (d->T % nseg != 0) return GDN_ERR_ARG;
-    if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
-    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC_SEQ) return GDN_ERR_ARG;
     const long BH = (long)d->B * d->H;
-    if (BH * nseg > (1L << 30)) return GDN_ERR_ARG;
     const size_t need = gdn_segmented_workspace_bytes(d, nseg);
     if (BH > 0 && d->T > 0) {
         if (!workspace || workspace_bytes < need) return GDN_ERR_ARG;
@@ -372,9 +383,15 @@ extern "C" int gdn_chunk_fwd_segmented(const gdn_desc_t *d, int nseg, const void
     // the same argument rules as gdn_chunk_fwd, checked on the whole request
     rc = chunk_fwd_check(d, q, k, v, g, beta, S0, o, S_T);
     if (rc != GDN_OK) return rc;
-    const size_t n_o = (size_t)BH * d->T * d->dv * elem_size(d->out_dtype);
-    if (overlaps(workspace, need, o, n_o) || overlaps(workspace, need, S_T, (size_t)BH * d->dv * d->dk * 4) ||
-        overlaps(workspace, need, S0, (size_t)BH * d->dv * d->dk * 4))
+    // pass 1 writes the workspace and later passes re-read every input, so the
+    // workspace may overlap no input and no output
+    const size_t es = elem_size(d->dtype), n_tok = (size_t)BH * d->T;
+    const size_t n_o = n_tok * d->dv * elem_size(d->out_dtype), n_S = (size_t)BH * d->dv * d->dk * 4;
+    const size_t n_g = d->gate == GDN_GATE_CHANNEL ? n_tok * d->dk * 4 : n_tok * 4;
+    if (overlaps(workspace, need, o, n_o) || overlaps(workspace, need, S_T, n_S) ||
+        overlaps(workspace, need, S0, n_S) || overlaps(workspace, need, q, n_tok * d->dk * es) ||
+        overlaps(workspace, need, k, n_tok * d->dk * es) || overlaps(workspace, need, v, n_tok * d->dv * es) ||
+        overlaps(workspace, need, g, n_g) || overlaps(workspace, need, beta, n_tok * 4))
         return GDN_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (BH == 0) return GDN_OK;

@@ -13,13 +13,16 @@
 
 __device__ __align__(256) unsigned char g_gdn_scratch[GDN_NOALLOC_SCRATCH_BYTES];
 
+int gdn_segmented_request_check(const gdn_desc_t *d, int nseg);  // api.cu
+
 extern "C" size_t gdn_noalloc_scratch_bytes(void) { return GDN_NOALLOC_SCRATCH_BYTES; }
 
 extern "C" int gdn_chunk_fwd_segmented_noalloc(const gdn_desc_t *d, int nseg, const void *q, const void *k,
                                                const void *v, const float *g, const float *beta, const float *S0,
                                                void *o, float *S_T, void *stream) {
-    if (!d || nseg < 1 || d->B < 0 || d->H < 0 || d->T < 0) return GDN_ERR_ARG;
-    if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return GDN_ERR_ARG;
+    // a malformed request gets the workspace variant's code, whatever its size
+    const int rc = gdn_segmented_request_check(d, nseg);
+    if (rc != GDN_OK) return rc;
     // one segment, or nothing to split: no scratch is touched
     if (nseg == 1 || (long)d->B * d->H == 0 || d->T == 0)
         return gdn_chunk_fwd_segmented(d, nseg, q, k, v, g, beta, S0, o, S_T, nullptr, 0, stream);

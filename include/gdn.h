@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define GDN_VERSION 3
+#define GDN_VERSION 4
 
 /* Return codes. */
 #define GDN_OK 0
@@ -73,14 +73,13 @@ typedef enum { GDN_GATE_NONE = 0, GDN_GATE_SCALAR = 1, GDN_GATE_CHANNEL = 2 } gd
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
 
-/* Kernel choice for gdn_chunk_fwd.  AUTO picks a tensor-core kernel when one
+/* Kernel choice for gdn_chunk_fwd.  AUTO picks the tensor-core kernel when it
  * supports the request (bf16 inputs, dk = 128) and the fp32 SIMT kernel
  * otherwise.  TC is the warp-specialised tensor-core kernel (prep of the next
- * chunk overlapping the state update of the current one); TC_SEQ the
- * single-group tensor-core kernel that runs the phases of a chunk in sequence.
- * An explicit value forces that kernel (GDN_ERR_UNSUPPORTED if it cannot serve
- * the request). */
-typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TC = 2, GDN_ALGO_TC_SEQ = 3 } gdn_algo_t;
+ * chunk overlapping the state update of the current one).  An explicit value
+ * forces that kernel (GDN_ERR_UNSUPPORTED if it cannot serve the request); any
+ * other value is GDN_ERR_ARG. */
+typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TC = 2 } gdn_algo_t;
 
 /* Input prologue (bits of gdn_desc_t.prologue): maps the kernels apply to their
  * inputs as they load them, so that raw projections can be passed directly.
@@ -182,9 +181,8 @@ int gdn_chunk_fwd_host(const gdn_desc_t *desc, int n_slices, const void *q, cons
  * gdn_chunk_fwd.  For nh > 1, GDN_ALGO_AUTO takes the pipelined tensor-core
  * kernel when it serves the shape (bf16, dk = 128, dv in {64, 128}, scalar or no
  * gate, nh a power of two, so that a chunk holds whole tokens) and the fp32 SIMT
- * kernel otherwise; GDN_ALGO_TC demands the former, GDN_ALGO_SIMT the latter,
- * GDN_ALGO_TC_SEQ returns GDN_ERR_UNSUPPORTED.  The caller owns every buffer;
- * nothing is allocated.
+ * kernel otherwise; GDN_ALGO_TC demands the former, GDN_ALGO_SIMT the latter.
+ * The caller owns every buffer; nothing is allocated.
  */
 int gdn_product_fwd(const gdn_desc_t *desc, int nh, const void *q, const void *k, const void *v,
                     const float *g, const float *beta, const float *S0, void *o, float *S_T,
@@ -205,7 +203,12 @@ int gdn_product_fwd(const gdn_desc_t *desc, int nh, const void *q, const void *k
  *
  *   workspace  device buffer of at least gdn_segmented_workspace_bytes(desc,
  *              nseg) bytes, 16-byte aligned, owned by the caller; it must not
- *              overlap o, S0 or S_T.  Its contents on return are unspecified.
+ *              overlap any input (q, k, v, g, beta, S0) or output (o, S_T):
+ *              the first pass writes it and later passes re-read the inputs,
+ *              so an overlap returns GDN_ERR_ARG.  Its contents on return are
+ *              unspecified.  gdn_segmented_workspace_bytes returns 0 for a
+ *              request it cannot size (null desc, nseg < 1, more than 2^30
+ *              segment-heads).
  */
 size_t gdn_segmented_workspace_bytes(const gdn_desc_t *desc, int nseg);
 int gdn_chunk_fwd_segmented(const gdn_desc_t *desc, int nseg, const void *q, const void *k, const void *v,
@@ -219,8 +222,9 @@ int gdn_chunk_fwd_segmented(const gdn_desc_t *desc, int nseg, const void *q, con
  * default, it is mapped on first use) instead of the
  * caller, so the call allocates nothing and takes no workspace argument.  The
  * pages have no counterpart: it is a calling convenience for callers that
- * cannot allocate on the call path.  Requests whose workspace
- * (gdn_segmented_workspace_bytes) exceeds the array return
+ * cannot allocate on the call path.  A malformed request returns the code
+ * gdn_chunk_fwd_segmented returns for it (checked first); a well-formed one
+ * whose workspace (gdn_segmented_workspace_bytes) exceeds the array returns
  * GDN_ERR_UNSUPPORTED; other arguments and results as gdn_chunk_fwd_segmented.
  * Concurrent calls on one device share the array and must be ordered (one
  * stream, or events).

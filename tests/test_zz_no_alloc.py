@@ -39,6 +39,14 @@ def test_rejects_before_touching_the_device(lib):
     assert f(ctypes.byref(big), 4, *args) == -3                     # larger than the array
     empty = _desc(B=0)
     assert f(ctypes.byref(empty), 4, *args) == 0                    # nothing to do, no device work
+    # a malformed request is an argument error whatever its size, as in the
+    # workspace variant: T not a multiple of nseg, too many segment-heads
+    bad = _desc(B=64, H=16, T=4095)
+    assert f(ctypes.byref(bad), 4, *args) == -1
+    assert lib.gdn_chunk_fwd_segmented(ctypes.byref(bad), 4, *args[:-1], vp(0x7000000), 1 << 40, None) == -1
+    huge = _desc(B=1 << 15, H=1 << 15, T=64)                        # 2^30 heads x 2 segments
+    assert f(ctypes.byref(huge), 2, *args) == -1
+    assert lib.gdn_segmented_workspace_bytes(ctypes.byref(huge), 2) == 0
 
 
 @pytest.mark.gpu
@@ -62,13 +70,17 @@ def test_matches_workspace_variant_and_oracle_without_allocating():
     torch.cuda.synchronize()
     gdn.chunk_fwd_segmented_noalloc(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], update="delta",
                                     gate="scalar", nseg=5, o=o2, S_T=S2)  # warm: maps the array
-    torch.cuda.synchronize()
-    before = torch.cuda.memory_allocated()
     o2.zero_()
+    torch.cuda.synchronize()
+    # torch's allocator counter, and the device's free memory (which also sees a
+    # cudaMalloc / cudaMallocAsync inside the library)
+    before = torch.cuda.memory_allocated()
+    free_before = torch.cuda.mem_get_info()[0]
     gdn.chunk_fwd_segmented_noalloc(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], update="delta",
                                     gate="scalar", nseg=5, o=o2, S_T=S2)
     torch.cuda.synchronize()
     assert torch.cuda.memory_allocated() == before
+    assert torch.cuda.mem_get_info()[0] == free_before
     assert gdn.device_status() == 0
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
     ro, rS = oracle.gdn_forward("delta", "scalar", x["q"], x["k"], x["v"], g=x["g"], beta=x["beta"], S0=x["S0"])
