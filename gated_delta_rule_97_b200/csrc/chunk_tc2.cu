@@ -30,7 +30,11 @@
 // Hand-offs: bar_rdy (prep -> state, one phase per chunk), bar_fA (state MMAs
 // that read Q<, K<, V, T2 completed), bar_fB0/1 (state MMAs that read A', K>
 // of an even / odd chunk completed; A' and K> are double-buffered).  All waits
-// are bounded; intermediates are fp16 with a range flag (see chunk_tc.cu).
+// are bounded: on a timeout the CTA records GDN_ERR_TIMEOUT and the wait site.
+// Intermediates handed to the tensor cores (T2, Q<, K<, K>, V, A', -X, Z and
+// the state copy) are fp16 (11-bit significand; raw bf16 inputs are exact in
+// it); accumulators and the state master are fp32.  Every value converted to
+// fp16 is range-checked and an overflow is recorded as GDN_ERR_RANGE.
 #include <string.h>
 
 #include "../../include/gdn.h"
@@ -1348,6 +1352,10 @@ extern "C" int gdn_tc2_phase_times(unsigned long long *out, int clear) {
     return 0;
 }
 #endif
+
+int gdn_tc_supported(const gdn_desc_t *d) {
+    return d->dtype == GDN_BF16 && d->dk == 128 && (d->dv == 64 || d->dv == 128);
+}
 
 // Value-slice width: 128 keeps the per-chunk K-side work unduplicated; 64
 // doubles the CTA count when 128-wide slices would leave most SMs idle.

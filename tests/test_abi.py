@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_strerror_and_version(lib):
-    assert gdn.version() == 3  # segment maps and their composition joined the boundary
+    assert gdn.version() == 4  # the sequential tensor-core kernel choice left the boundary
     for code in (0, -1, -2, -3, -4, -5, -6, 123):
         assert isinstance(gdn.strerror(code), str) and gdn.strerror(code)
 
@@ -119,8 +119,9 @@ def test_product_rejects_bad_arguments(lib):
     assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -1      # only the delta rule has substeps
     d = _desc(algo="tc")
     assert lib.gdn_product_fwd(ctypes.byref(d), 3, *args) == -3      # tensor-core kernel: whole tokens per chunk
-    d = _desc(algo="tc_seq")
-    assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -3      # the sequential kernel has no remap
+    d = _desc()
+    d.algo = 3
+    assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -1      # no such kernel choice
     d = _desc(B=0)
     assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == 0       # empty batch: no-op
 
