@@ -14,7 +14,9 @@ Two implementations of the same definition:
 * ``prologue`` -- the optional input maps (feature map, L2 rows, sigmoid,
   -softplus) applied before the recurrence;
 * ``segment_maps`` -- the affine map (H, Lambda) of a run of tokens, Lambda as
-  the dense product of the per-token transition matrices.
+  the dense product of the per-token transition matrices;
+* ``gdn_backward_np`` -- the gradients of the recurrence (reverse mode through
+  the token loop, states recomputed from chunk-start checkpoints).
 
 Definition (column convention, S in R^{dv x dk}, stored [B,H,dv,dk]):
 ``S_t = S_{t-1} Diag(alpha_t)(I - beta_t k_t k_t^T) + beta_t v_t k_t^T``,
@@ -267,3 +269,91 @@ def decode_sequence(update, gate, S0, steps):
                               axis=-2 if name in ("q", "k", "v") or (name == "g" and gate == "channel") else -1)
 
     return gdn_forward(update, gate, cat("q"), cat("k"), cat("v"), cat("g"), cat("beta"), S0)
+
+
+def gdn_backward_np(update, gate, q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, checkpoint=64):
+    """Gradients of the recurrence (reverse mode through the token loop), float64.
+
+    For the scalar loss L = sum(dO * o) + sum(dS_T * S_T) of ``gdn_forward``
+    (dO [..., T, dv] and dS_T [..., dv, dk] are the upstream gradients; either
+    may be None = 0), returns (dq, dk, dv, dg, dbeta, dS0) shaped like q, k, v,
+    g, beta, S0 (dg / dbeta None when g / beta are None; dS0 always returned).
+
+    Each token's step is differentiated as written in ``gdn_forward_np``:
+    S' = S_{t-1} Diag(alpha_t); delta: r = v_t - S' k_t, u = beta_t r, else
+    u = v_t; S_t = S' + u k_t^T; o_t = S_t q_t.  Going back from t = T-1 with
+    dS = dL/dS_t: dq_t = S_t^T dO_t; dS += dO_t q_t^T; du = dS k_t;
+    dk_t = dS^T u; dS' = dS; delta: dbeta_t = du . r, dv_t = beta_t du,
+    dS' -= dv_t k_t^T, dk_t -= S'^T dv_t; else dv_t = du; the gate:
+    dg_t = sum(dS' * S') (over the key channel j alone for a per-channel gate,
+    since S'[:, j] = alpha_j S[:, j] and d alpha / d g = alpha); then
+    dL/dS_{t-1} = dS' Diag(alpha_t).  The states S' are recomputed a chunk of
+    ``checkpoint`` tokens at a time from the states saved at chunk starts
+    ("Update the state": autograd keeps the chunk-boundary states)."""
+    _check(update, gate, q, k, v, g, beta)
+    q, k, v, g, beta = _f64(q), _f64(k), _f64(v), _f64(g), _f64(beta)
+    lead = q.shape[:-2]
+    T, dk_ = q.shape[-2], q.shape[-1]
+    dv_ = v.shape[-1]
+    S = np.zeros(lead + (dv_, dk_)) if S0 is None else _f64(S0).copy()
+    dO = np.zeros(lead + (T, dv_)) if dO is None else _f64(dO)
+
+    def alpha(t):
+        if gate == "scalar":
+            return np.exp(g[..., t])[..., None, None]
+        if gate == "channel":
+            return np.exp(g[..., t, :])[..., None, :]
+        return None
+
+    def step(S, t):
+        """One token forward: returns (S', r or None, u, S_t)."""
+        a = alpha(t)
+        Sp = S * a if a is not None else S
+        kt = k[..., t, :]
+        if update == "delta":
+            r = v[..., t, :] - np.einsum("...ij,...j->...i", Sp, kt)
+            u = beta[..., t][..., None] * r
+        else:
+            r, u = None, v[..., t, :]
+        return Sp, r, u, Sp + u[..., :, None] * kt[..., None, :]
+
+    # forward: the state entering every chunk
+    starts = []
+    for t in range(T):
+        if t % checkpoint == 0:
+            starts.append(S.copy())
+        S = step(S, t)[3]
+    dS = np.zeros(lead + (dv_, dk_)) if dS_T is None else _f64(dS_T).copy()
+    dq, dk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dg = None if g is None else np.zeros_like(g)
+    db = None if beta is None else np.zeros_like(beta)
+    for c in range(len(starts) - 1, -1, -1):
+        t0, t1 = c * checkpoint, min(T, (c + 1) * checkpoint)
+        S = starts[c].copy()
+        saved = []
+        for t in range(t0, t1):
+            Sp, r, u, S = step(S, t)
+            saved.append((Sp, r, u, S))
+        for t in range(t1 - 1, t0 - 1, -1):
+            Sp, r, u, St = saved[t - t0]
+            qt, kt, dOt = q[..., t, :], k[..., t, :], dO[..., t, :]
+            dq[..., t, :] = np.einsum("...ij,...i->...j", St, dOt)
+            dS = dS + dOt[..., :, None] * qt[..., None, :]
+            du = np.einsum("...ij,...j->...i", dS, kt)
+            dk[..., t, :] = np.einsum("...ij,...i->...j", dS, u)
+            dSp = dS
+            if update == "delta":
+                db[..., t] = np.sum(du * r, axis=-1)
+                dvt = beta[..., t][..., None] * du
+                dvv[..., t, :] = dvt
+                dSp = dSp - dvt[..., :, None] * kt[..., None, :]
+                dk[..., t, :] -= np.einsum("...ij,...i->...j", Sp, dvt)
+            else:
+                dvv[..., t, :] = du
+            a = alpha(t)
+            if gate == "scalar":
+                dg[..., t] = np.sum(dSp * Sp, axis=(-2, -1))
+            elif gate == "channel":
+                dg[..., t, :] = np.sum(dSp * Sp, axis=-2)
+            dS = dSp * a if a is not None else dSp
+    return dq, dk, dvv, dg, db, dS

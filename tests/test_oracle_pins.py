@@ -639,3 +639,77 @@ def test_gate_and_beta_layouts_are_checked(oracle_mod):
         oracle.gdn_forward("delta", "scalar", q, k, v, g=g, beta=beta)
     with pytest.raises(ValueError):
         oracle.gdn_forward("delta", "channel", q, k, v, g=g, beta=beta[..., None])
+
+
+# ---------------------------------------------------------------------------
+# Backward: gdn_backward_np is pinned to central finite differences of the
+# forward definition (every input element of tiny cases, all six modes) and to
+# the closed-form gradients of causal linear attention.
+# ---------------------------------------------------------------------------
+
+BWD_MODES = [("additive", "none"), ("decay", "scalar"), ("decay", "channel"),
+             ("delta", "none"), ("delta", "scalar"), ("delta", "channel")]
+
+
+def _bwd_case(seed, update, gate, BH=2, T=7, dk=4, dv=3):
+    q, k, v, g, beta, S0 = rand_inputs(seed, BH=BH, T=T, dk=dk, dv=dv, gate=gate, delta=update == "delta",
+                                       s0=True, gmin=-0.6)
+    r = np.random.default_rng(seed + 1000)
+    dO = r.standard_normal((BH, T, dv))
+    dST = r.standard_normal((BH, dv, dk))
+    return q, k, v, g, beta, S0, dO, dST
+
+
+@pytest.mark.parametrize("update,gate", BWD_MODES)
+def test_backward_equals_finite_differences(oracle_mod, update, gate):
+    q, k, v, g, beta, S0, dO, dST = _bwd_case(71, update, gate)
+    got = oracle.gdn_backward_np(update, gate, q, k, v, g, beta, S0, dO, dST, checkpoint=3)
+    inputs = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "S0": S0}
+    names = ["q", "k", "v", "g", "beta", "S0"]
+
+    def loss(x):
+        o, ST = oracle.gdn_forward_np(update, gate, x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    h = 1e-6
+    for name, grad in zip(names, got):
+        if inputs[name] is None:
+            assert grad is None
+            continue
+        fd = np.zeros_like(inputs[name])
+        it = np.nditer(inputs[name], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = {n: (None if a is None else a.copy()) for n, a in inputs.items()}
+            xm = {n: (None if a is None else a.copy()) for n, a in inputs.items()}
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * h)
+        assert rel_err(grad, fd) < 1e-6, (name, rel_err(grad, fd))
+
+
+def test_backward_independent_of_checkpoint_spacing(oracle_mod):
+    q, k, v, g, beta, S0, dO, dST = _bwd_case(72, "delta", "channel", T=11)
+    ref = oracle.gdn_backward_np("delta", "channel", q, k, v, g, beta, S0, dO, dST, checkpoint=64)
+    for c in (1, 4, 5):
+        got = oracle.gdn_backward_np("delta", "channel", q, k, v, g, beta, S0, dO, dST, checkpoint=c)
+        for a, b in zip(got, ref):
+            assert np.array_equal(a, b)
+
+
+def test_backward_additive_closed_forms(oracle_mod):
+    """Causal linear attention o_t = sum_{s<=t} (q_t . k_s) v_s + S0 q_t and
+    S_T = S0 + V^T K ("Naive linear attention", causal): with M the causal
+    mask, dQ = (dO V^T (.) M) K + dO S0, dK = (dO V^T (.) M)^T Q + V dS_T,
+    dV = (Q K^T (.) M)^T dO + K dS_T^T, dS0 = dO^T Q + dS_T."""
+    q, k, v, _, _, S0, dO, dST = _bwd_case(73, "additive", "none", BH=2, T=29, dk=6, dv=5)
+    dq, dk, dv, dg, db, dS0 = oracle.gdn_backward_np("additive", "none", q, k, v, None, None, S0, dO, dST,
+                                                     checkpoint=8)
+    assert dg is None and db is None
+    M = np.tril(np.ones((29, 29)))
+    for h in range(2):
+        G = dO[h] @ v[h].T * M
+        assert rel_err(dq[h], G @ k[h] + dO[h] @ S0[h]) < TOL
+        assert rel_err(dk[h], G.T @ q[h] + v[h] @ dST[h]) < TOL
+        assert rel_err(dv[h], (q[h] @ k[h].T * M).T @ dO[h] + k[h] @ dST[h].T) < TOL
+        assert rel_err(dS0[h], dO[h].T @ q[h] + dST[h]) < TOL
