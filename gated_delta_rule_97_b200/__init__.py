@@ -18,7 +18,7 @@ import os
 __all__ = ["GDNError", "chunk_fwd", "decode_step", "device_status", "strerror", "version", "load",
            "lib_path", "Desc", "UPDATES", "GATES", "build", "device_diag", "product_fwd", "chunk_fwd_segmented",
            "segmented_workspace_bytes", "segment_maps", "compose_segments", "chunk_fwd_host",
-           "host_workspace_bytes"]
+           "host_workspace_bytes", "chunk_bwd", "bwd_workspace_bytes"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libgdn.so")
@@ -96,6 +96,10 @@ def load():
     lib.gdn_segment_maps.restype = ctypes.c_int
     lib.gdn_compose_segments.argtypes = [ctypes.c_int] * 4 + [vp] * 6
     lib.gdn_compose_segments.restype = ctypes.c_int
+    lib.gdn_bwd_workspace_bytes.argtypes = [dp]
+    lib.gdn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_chunk_bwd.argtypes = [dp] + [vp] * 15 + [ctypes.c_size_t, vp]
+    lib.gdn_chunk_bwd.restype = ctypes.c_int
     lib.gdn_strerror.argtypes = [ctypes.c_int]
     lib.gdn_strerror.restype = ctypes.c_char_p
     lib.gdn_device_status.argtypes = [ctypes.c_int]
@@ -501,3 +505,50 @@ def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, pr
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_decode_step")
     return o
+
+
+def bwd_workspace_bytes(B, H, T, dk, dv) -> int:
+    d = make_desc(B, H, T, dk, dv, "delta", "scalar", BF16, F32)
+    return int(load().gdn_bwd_workspace_bytes(ctypes.byref(d)))
+
+
+def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update, gate, workspace=None,
+              want_dS0=True, stream=None):
+    """gdn_chunk_bwd: gradients of chunk_fwd for upstream gradients dO [B,H,T,dv]
+    and dS_T [B,H,dv,dk] (fp32; None = 0).  Returns (dq, dk, dv, dg, dbeta, dS0),
+    fp32, dg / dbeta None when the mode has no gate / write strength, dS0 None
+    when ``want_dS0`` is false.  ``workspace``: a CUDA uint8 tensor of
+    bwd_workspace_bytes(...) bytes (allocated here when None)."""
+    import torch
+
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
+    if gate == "scalar":
+        _check(g, "g", (B, H, T), torch.float32)
+    elif gate == "channel":
+        _check(g, "g", (B, H, T, dk), torch.float32)
+    _check(beta, "beta", (B, H, T), torch.float32)
+    _check(S0, "S0", (B, H, dv, dk), torch.float32)
+    _check(dO, "dO", (B, H, T, dv), torch.float32)
+    _check(dS_T, "dS_T", (B, H, dv, dk), torch.float32)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    gq, gk, gv = torch.empty((B, H, T, dk), **f32), torch.empty((B, H, T, dk), **f32), torch.empty((B, H, T, dv), **f32)
+    gg = None if gate == "none" else torch.empty(tuple(g.shape), **f32)
+    gb = torch.empty((B, H, T), **f32) if update == "delta" else None
+    gS0 = torch.empty((B, H, dv, dk), **f32) if want_dS0 else None
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), F32)
+    need = int(load().gdn_bwd_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous() or workspace.numel() < need:
+        raise ValueError("workspace needs %d contiguous CUDA bytes" % need)
+    with _on_device(q):
+        rc = load().gdn_chunk_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                  _ptr(dO), _ptr(dS_T), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gg), _ptr(gb), _ptr(gS0),
+                                  _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream, q))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_chunk_bwd")
+    return gq, gk, gv, gg, gb, gS0

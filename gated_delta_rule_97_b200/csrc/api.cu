@@ -532,3 +532,62 @@ extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k
     return from_cuda(gdn_launch_decode(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16,
                                        static_cast<cudaStream_t>(stream)));
 }
+
+// ---------------------------------------------------------------------------
+// Backward (backward.cu)
+int gdn_launch_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta, const float *S0,
+                   const float *dO, const float *dST, float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                   float *dS0, float *ws, int BH, int T, int dk_, int dv_, int update, int gate, int in_bf16,
+                   cudaStream_t st);
+
+extern "C" size_t gdn_bwd_workspace_bytes(const gdn_desc_t *d) {
+    if (!d || validate_common(d) != GDN_OK) return 0;
+    const size_t nch = ((size_t)d->T + gdn::kChunk - 1) / gdn::kChunk;
+    return (size_t)d->B * d->H * nch * d->dv * d->dk * sizeof(float);
+}
+
+extern "C" int gdn_chunk_bwd(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *S0, const float *dO, const float *dS_T, float *dq,
+                             float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    int rc = validate_common(d);
+    if (rc != GDN_OK) return rc;
+    if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if (d->prologue != 0) return GDN_ERR_UNSUPPORTED;
+    const long BH = (long)d->B * d->H;
+    const size_t ntok = (size_t)BH * d->T;
+    const size_t es = elem_size(d->dtype);
+    const size_t n_qk = ntok * d->dk, n_v = ntok * d->dv, n_S = (size_t)BH * d->dv * d->dk;
+    const size_t n_g = d->gate == GDN_GATE_CHANNEL ? n_qk : ntok;
+    const bool has_tokens = ntok > 0;
+    if (has_tokens) {
+        if (!q || !k || !v || !dq || !dk || !dv) return GDN_ERR_ARG;
+        if ((d->update == GDN_DELTA) != (beta != nullptr) || (d->update == GDN_DELTA) != (dbeta != nullptr))
+            return GDN_ERR_ARG;
+        if ((d->gate != GDN_GATE_NONE) != (g != nullptr) || (d->gate != GDN_GATE_NONE) != (dg != nullptr))
+            return GDN_ERR_ARG;
+    }
+    const void *ptrs[] = {q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    const size_t need = gdn_bwd_workspace_bytes(d);
+    if (has_tokens && (!workspace || workspace_bytes < need)) return GDN_ERR_ARG;
+    // outputs (and the workspace) against every input and against each other
+    struct Span { const void *p; size_t n; };
+    const Span ins[] = {{q, n_qk * es}, {k, n_qk * es}, {v, n_v * es}, {g, n_g * 4}, {beta, ntok * 4},
+                        {S0, n_S * 4}, {dO, n_v * 4}, {dS_T, n_S * 4}};
+    const Span outs[] = {{dq, n_qk * 4}, {dk, n_qk * 4}, {dv, n_v * 4}, {dg, n_g * 4}, {dbeta, ntok * 4},
+                         {dS0, n_S * 4}, {workspace, has_tokens ? need : 0}};
+    for (const Span &o : outs) {
+        for (const Span &i : ins)
+            if (overlaps(o.p, o.n, i.p, i.n)) return GDN_ERR_ARG;
+        for (const Span &o2 : outs)
+            if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return GDN_ERR_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (BH == 0) return GDN_OK;
+    if (d->T == 0) return dS0 ? from_cuda(gdn_launch_copy_state(dS_T, dS0, (long)n_S, st)) : GDN_OK;
+    return from_cuda(gdn_launch_bwd(q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0,
+                                    static_cast<float *>(workspace), (int)BH, d->T, d->dk, d->dv, d->update, d->gate,
+                                    d->dtype == GDN_BF16, st));
+}

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define GDN_VERSION 4
+#define GDN_VERSION 5
 
 /* Return codes. */
 #define GDN_OK 0
@@ -295,6 +295,48 @@ int gdn_decode_step(const gdn_desc_t *desc, const void *q, const void *k, const 
 
 /* Static string naming a return code (never NULL). */
 const char *gdn_strerror(int code);
+
+/*
+ * gdn_chunk_bwd -- the gradients of gdn_chunk_fwd (training backward).  For the
+ * scalar loss L = sum(dO (.) o) + sum(dS_T (.) S_T) of gdn_chunk_fwd on the same
+ * desc and inputs, writes dq = dL/dq, dk, dv, dg (dL/d log alpha), dbeta and
+ * dS0.  Reverse mode through the recurrence of "Linear Attention, Visualized"
+ * ("Recurrent form" of DeltaNet, "Gated DeltaNet (GDN)", "Kimi Delta
+ * Attention (KDA)", "Mamba-2", "Gated Linear Attention (GLA)"; the additive
+ * and decay writes as in gdn_chunk_fwd): the state entering every chunk of 64
+ * tokens is kept ("Update the state": training keeps the chunk-boundary
+ * states) and each chunk is recomputed before its gradients are stepped back
+ * through it.  fp32 arithmetic.
+ *
+ *   desc        as for gdn_chunk_fwd (update, gate, dtype of q, k, v; dk, dv
+ *               in {64, 128}; chunk 0 or 64); out_dtype and algo are not read;
+ *               prologue must be 0 (GDN_ERR_UNSUPPORTED otherwise: the maps'
+ *               own gradients are not part of this call).
+ *   q, k, v, g, beta, S0   the forward inputs, laid out as in gdn_chunk_fwd
+ *               (S0 may be NULL = 0).
+ *   dO          [B,H,T,dv] float, the gradient of o (NULL = 0).
+ *   dS_T        [B,H,dv,dk] float, the gradient of S_T (NULL = 0).
+ *   dq, dk      [B,H,T,dk] float;  dv [B,H,T,dv] float (required when B*H*T > 0)
+ *   dg          [B,H,T] (scalar) or [B,H,T,dk] (channel) float; non-NULL iff
+ *               gate != NONE
+ *   dbeta       [B,H,T] float; non-NULL iff update == DELTA
+ *   dS0         [B,H,dv,dk] float, or NULL (not written)
+ *   workspace   device buffer of at least gdn_bwd_workspace_bytes(desc) bytes
+ *               (B*H*ceil(T/64)*dv*dk*4: the chunk-boundary states), 16-byte
+ *               aligned, owned by the caller; contents on return unspecified.
+ *
+ * Every pointer 16-byte aligned; no output may overlap another output, an
+ * input or the workspace (GDN_ERR_ARG).  dq, dk, dg and dbeta are sums over the
+ * value rows of the state, accumulated across slices of 32 rows with float
+ * atomics after being zeroed by the call, so they can differ from run to run
+ * in the last bits; dv and dS0 are written once.  T == 0 writes dS0 = dS_T (or
+ * zeros) and nothing else.  Asynchronous on `stream`; allocates nothing.
+ */
+size_t gdn_bwd_workspace_bytes(const gdn_desc_t *desc);
+int gdn_chunk_bwd(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
+                  const float *beta, const float *S0, const float *dO, const float *dS_T, float *dq, float *dk,
+                  float *dv, float *dg, float *dbeta, float *dS0, void *workspace, size_t workspace_bytes,
+                  void *stream);
 
 /*
  * gdn_device_status -- synchronises the current device, then returns the

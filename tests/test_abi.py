@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_strerror_and_version(lib):
-    assert gdn.version() == 4  # the sequential tensor-core kernel choice left the boundary
+    assert gdn.version() == 5  # the backward pass joined the boundary
     for code in (0, -1, -2, -3, -4, -5, -6, 123):
         assert isinstance(gdn.strerror(code), str) and gdn.strerror(code)
 
@@ -205,3 +205,32 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(gdn, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         gdn.load()
+
+
+def test_backward_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    f = lib.gdn_chunk_bwd
+    f.argtypes = [ctypes.c_void_p] * 16 + [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gdn_bwd_workspace_bytes.argtypes = [ctypes.c_void_p]
+    lib.gdn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    d = _desc(T=130)  # delta, scalar gate, B2 H3 dk=dv=128
+    need = lib.gdn_bwd_workspace_bytes(ctypes.byref(d))
+    assert need == 6 * 3 * 128 * 128 * 4  # six heads, three chunk-boundary states each
+    ins = [vp(0x100000), vp(0x200000), vp(0x300000), vp(0x400000), vp(0x500000), None, vp(0x600000), None]
+    outs = [vp(0x1000000), vp(0x1100000), vp(0x1200000), vp(0x1300000), vp(0x1400000), None]
+    ws = vp(0x2000000)
+    assert f(ctypes.byref(d), *ins, *outs, ws, need - 16, None) == -1          # workspace too small
+    assert f(ctypes.byref(d), *ins, *outs[:4], None, None, ws, need, None) == -1  # delta without dbeta
+    assert f(ctypes.byref(d), *ins, *outs[:3], None, outs[4], None, ws, need, None) == -1  # gate without dg
+    bad = list(outs)
+    bad[1] = vp(0x1100004)
+    assert f(ctypes.byref(d), *ins, *bad, ws, need, None) == -2                # misaligned
+    bad = list(outs)
+    bad[2] = vp(0x100010)
+    assert f(ctypes.byref(d), *ins, *bad, ws, need, None) == -1                # dv overlaps q
+    assert f(ctypes.byref(d), *ins, *outs, vp(0x1100000), need, None) == -1   # workspace overlaps dk
+    p = _desc(T=130)
+    p.prologue = 1
+    assert f(ctypes.byref(p), *ins, *outs, ws, need, None) == -3              # input maps not differentiated
+    e = _desc(B=0)
+    assert f(ctypes.byref(e), *ins, *outs, ws, 0, None) == 0                   # empty batch: no-op

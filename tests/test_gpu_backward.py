@@ -1,0 +1,105 @@
+"""GPU parity of the backward pass (gdn_chunk_bwd) against the float64 oracle
+``oracle.gdn_backward_np`` (itself pinned to finite differences of the forward
+definition): every mode, dk and dv in {64, 128}, fp32 and bf16 inputs, ragged
+lengths, with and without S0 and the two upstream gradients."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_97_b200 as gdn
+import oracle
+from gpu_util import dev, np64, rel_err
+from synth import round_to_bf16
+
+pytestmark = pytest.mark.gpu
+
+MODES = [("additive", "none"), ("decay", "scalar"), ("decay", "channel"),
+         ("delta", "none"), ("delta", "scalar"), ("delta", "channel")]
+# fp32 arithmetic against float64 on the same (rounded) inputs
+TOL = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    gdn.build()
+    gdn.device_status(clear=True)
+
+
+def inputs(seed, update, gate, B=1, H=2, T=130, dk=128, dv=128, bf16=False, s0=True, grads=(True, True)):
+    r = np.random.default_rng(seed)
+    q = r.standard_normal((B, H, T, dk))
+    k = r.standard_normal((B, H, T, dk))
+    if update == "additive":
+        q, k = np.where(q > 0, q + 1, np.exp(q)) / np.sqrt(dk), np.where(k > 0, k + 1, np.exp(k)) / np.sqrt(dk)
+    else:
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = r.standard_normal((B, H, T, dv))
+    if bf16:
+        q, k, v = (round_to_bf16(np.asarray(x, np.float32)).astype(np.float64) for x in (q, k, v))
+    else:
+        q, k, v = (np.asarray(x, np.float32).astype(np.float64) for x in (q, k, v))
+    g = None
+    if gate == "scalar":
+        g = -np.log1p(np.exp(r.standard_normal((B, H, T)) - 3.0))
+    elif gate == "channel":
+        g = -np.log1p(np.exp(r.standard_normal((B, H, T, dk)) - 4.0))
+    beta = 1.0 / (1.0 + np.exp(-r.standard_normal((B, H, T)))) if update == "delta" else None
+    S0 = 0.05 * r.standard_normal((B, H, dv, dk)) if s0 else None
+    dO = r.standard_normal((B, H, T, dv)) if grads[0] else None
+    dST = r.standard_normal((B, H, dv, dk)) if grads[1] else None
+    f32 = lambda x: None if x is None else np.asarray(x, np.float32).astype(np.float64)
+    return q, k, v, f32(g), f32(beta), f32(S0), f32(dO), f32(dST)
+
+
+def run(update, gate, x, bf16):
+    q, k, v, g, beta, S0, dO, dST = x
+    dt = torch.bfloat16 if bf16 else torch.float32
+    gdn.device_status(clear=True)
+    got = gdn.chunk_bwd(dev(q, dt), dev(k, dt), dev(v, dt), dev(g), dev(beta), dev(S0), dev(dO), dev(dST),
+                        update=update, gate=gate)
+    torch.cuda.synchronize()
+    assert gdn.device_status(clear=True) == 0
+    ref = oracle.gdn_backward_np(update, gate, q, k, v, g, beta, S0, dO, dST)
+    names = ["dq", "dk", "dv", "dg", "dbeta", "dS0"]
+    for name, a, b in zip(names, got, ref):
+        if b is None:
+            assert a is None, name
+            continue
+        err = rel_err(np64(a), b)
+        assert err <= TOL, (name, err)
+
+
+@pytest.mark.parametrize("update,gate", MODES)
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64)])
+def test_backward_modes(update, gate, dk, dv):
+    run(update, gate, inputs(3, update, gate, T=130, dk=dk, dv=dv), bf16=False)
+
+
+@pytest.mark.parametrize("update,gate", MODES)
+def test_backward_bf16_inputs(update, gate):
+    run(update, gate, inputs(4, update, gate, T=100, bf16=True), bf16=True)
+
+
+@pytest.mark.parametrize("T", [1, 7, 8, 63, 64, 65, 200])
+def test_backward_ragged_lengths(T):
+    run("delta", "scalar", inputs(5, "delta", "scalar", T=T), bf16=False)
+
+
+@pytest.mark.parametrize("s0,grads", [(False, (True, False)), (True, (False, True)), (False, (False, False))])
+def test_backward_optional_inputs(s0, grads):
+    run("delta", "channel", inputs(6, "delta", "channel", T=90, s0=s0, grads=grads), bf16=False)
+
+
+def test_backward_many_heads_and_value_slices():
+    run("delta", "scalar", inputs(7, "delta", "scalar", B=3, H=5, T=70, dv=128, bf16=True), bf16=True)
+
+
+def test_backward_empty_sequence_copies_state_gradient():
+    q = torch.zeros((1, 2, 0, 128), device="cuda")
+    dST = torch.randn((1, 2, 128, 128), device="cuda")
+    out = gdn.chunk_bwd(q, q, q, None, torch.zeros((1, 2, 0), device="cuda"), None, None, dST,
+                        update="delta", gate="none")
+    torch.cuda.synchronize()
+    assert torch.equal(out[5], dST) and out[0].numel() == 0
