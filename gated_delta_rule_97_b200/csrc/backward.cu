@@ -27,6 +27,9 @@
 //              dg_t = sum(dS' (.) S') (per key channel for a per-channel gate)
 //              dS <- dS' Diag(alpha_t)
 // Tokens past T are identity steps (q = k = v = dO = 0, beta = 0, alpha = 1).
+// The inputs of every sub-block are staged in shared memory (coalesced loads of
+// the next sub-block issued while the current one is processed), so the token
+// steps read shared memory only.
 #include <string.h>
 
 #include "../../include/gdn.h"
@@ -55,56 +58,97 @@ __device__ __forceinline__ float bwd_warp_sum(float x) {
     return x;
 }
 
-// One token's inputs as this thread sees them (its key channels and its warp's rows).
+// The inputs of one sub-block of kSub tokens, staged in shared memory as fp32:
+// key and query channels, alpha = exp(g) (per channel, or per token), this
+// CTA's kSlice value rows of v and dO, and beta.  Tokens past T read as the
+// identity step.  With kSub * kSlice == kBwdThreads, thread i stages value row
+// i % kSlice of token i / kSlice, and a contiguous run of DK / 32 channels.
+template <int DK, int GATE>
+struct StageLayout {
+    static constexpr int NA = (GATE == kGateChannel) ? kSub * DK : kSub;
+    static constexpr int K = 0, Q = kSub * DK, AL = 2 * kSub * DK, VV = AL + NA, DO = VV + kSub * kSlice,
+                         BT = DO + kSub * kSlice, FLOATS = BT + kSub;
+};
+
 template <int DK, int UPD, int GATE, typename TIn>
-struct BwdTok {
-    static constexpr int V = DK / 32;
-    float q[V], k[V], al[V], bt, v[kRows], dO[kRows];
-    __device__ void load(const BwdArgs &a, long bh, int t, int c0, int i0, bool need_q) {
-        if (t >= a.T) {
+struct StageRegs {
+    using SL = StageLayout<DK, GATE>;
+    static constexpr int EQ = kSub * DK / kBwdThreads;
+    float k[EQ], q[EQ], al[EQ], v, dO, bt;
+    __device__ void load(const BwdArgs &a, long bh, int tb, int rslice, int t_, bool need_q) {
+        const int T = a.T;
+        const int e0 = t_ * EQ, t = tb + e0 / DK, ch = e0 % DK;
 #pragma unroll
-            for (int e = 0; e < V; ++e) {
-                q[e] = 0.f;
-                k[e] = 0.f;
-                al[e] = 1.f;
-            }
-            bt = 0.f;
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-                v[r] = 0.f;
-                dO[r] = 0.f;
-            }
-            return;
-        }
-        const long tok = bh * a.T + t;
-        const TIn *kp = static_cast<const TIn *>(a.k) + tok * DK + c0;
-        const TIn *qp = static_cast<const TIn *>(a.q) + tok * DK + c0;
-#pragma unroll
-        for (int e = 0; e < V; ++e) {
-            k[e] = to_f32(kp[e]);
-            q[e] = need_q ? to_f32(qp[e]) : 0.f;
+        for (int e = 0; e < EQ; ++e) {
+            k[e] = 0.f;
+            q[e] = 0.f;
             al[e] = 1.f;
         }
-        if (GATE == kGateScalar) {
-            const float x = __expf(a.g[tok]);
+        if (t < T) {
+            const size_t off = ((size_t)bh * T + t) * DK + ch;
+            const TIn *kp = static_cast<const TIn *>(a.k) + off;
+            const TIn *qp = static_cast<const TIn *>(a.q) + off;
 #pragma unroll
-            for (int e = 0; e < V; ++e) al[e] = x;
-        } else if (GATE == kGateChannel) {
-#pragma unroll
-            for (int e = 0; e < V; ++e) al[e] = __expf(a.g[tok * DK + c0 + e]);
+            for (int e = 0; e < EQ; ++e) {
+                k[e] = to_f32(kp[e]);
+                if (need_q) q[e] = to_f32(qp[e]);
+                if (GATE == kGateChannel) al[e] = __expf(a.g[off + e]);
+            }
         }
-        bt = (UPD == kDelta) ? a.beta[tok] : 0.f;
-        const TIn *vp = static_cast<const TIn *>(a.v) + tok * a.DV + i0;
+        const int tv = tb + t_ / kSlice, row = rslice + t_ % kSlice;
+        v = 0.f;
+        dO = 0.f;
+        if (tv < T) {
+            const size_t ov = ((size_t)bh * T + tv) * a.DV + row;
+            v = to_f32(static_cast<const TIn *>(a.v)[ov]);
+            if (need_q && a.dO) dO = a.dO[ov];
+        }
+        bt = 0.f;
+        if (t_ < kSub && tb + t_ < T) {
+            const size_t ot = (size_t)bh * T + tb + t_;
+            if (UPD == kDelta) bt = a.beta[ot];
+            if (GATE == kGateScalar) al[0] = __expf(a.g[ot]);
+        }
+    }
+    __device__ void store(float *st, int t_) const {
+        const int e0 = t_ * EQ;
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-            v[r] = to_f32(vp[r]);
-            dO[r] = (need_q && a.dO) ? a.dO[tok * a.DV + i0 + r] : 0.f;
+        for (int e = 0; e < EQ; ++e) {
+            st[SL::K + e0 + e] = k[e];
+            st[SL::Q + e0 + e] = q[e];
+            if (GATE == kGateChannel) st[SL::AL + e0 + e] = al[e];
+        }
+        st[SL::VV + t_] = v;
+        st[SL::DO + t_] = dO;
+        if (t_ < kSub) {
+            st[SL::BT + t_] = bt;
+            if (GATE != kGateChannel) st[SL::AL + t_] = (GATE == kGateScalar) ? al[0] : 1.f;
         }
     }
 };
 
-// S <- S Diag(alpha); then the write (u = beta (v - S k) or v); returns u and
-// r = v - S k (delta) through the arrays.
+// One token's inputs as this thread reads them from a staged sub-block.
+template <int DK, int UPD, int GATE>
+struct BwdTok {
+    using SL = StageLayout<DK, GATE>;
+    static constexpr int V = DK / 32;
+    float q[V], k[V], al[V], bt, v[kRows], dO[kRows];
+    __device__ void read(const float *st, int tt, int c0, int lr, bool need_q) {
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            k[e] = st[SL::K + tt * DK + c0 + e];
+            q[e] = need_q ? st[SL::Q + tt * DK + c0 + e] : 0.f;
+            al[e] = (GATE == kGateChannel) ? st[SL::AL + tt * DK + c0 + e] : st[SL::AL + tt];
+        }
+        bt = st[SL::BT + tt];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+            v[r] = st[SL::VV + tt * kSlice + lr + r];
+            dO[r] = need_q ? st[SL::DO + tt * kSlice + lr + r] : 0.f;
+        }
+    }
+};
+
 template <int V, int UPD>
 __device__ __forceinline__ void fwd_write(float (&s)[kRows][V], const float *k, const float *v, float bt,
                                           float *u, float *rr) {
@@ -139,75 +183,110 @@ __device__ __forceinline__ void fwd_write(float (&s)[kRows][V], const float *k, 
         for (int e = 0; e < V; ++e) s[r][e] = fmaf(u[r], k[e], s[r][e]);
 }
 
+// The kernel walks a fixed sequence of sub-block visits: phase 1 visits the
+// sub-blocks of the sequence in order; phase 2 visits the chunks from the last,
+// each chunk's sub-blocks forward (recompute) and then backward.  Every visit's
+// inputs are staged in one of two shared-memory buffers; the next visit's are
+// loaded into registers while the current one is processed and stored into the
+// other buffer at its end.
+struct Visit {
+    int tb;     // first token of the sub-block
+    int phase;  // 1: forward of phase 1; 2: forward recompute of phase 2; 3: backward
+    int j;      // sub-block index inside its chunk
+    int c;      // chunk
+};
+
+__device__ __forceinline__ Visit visit_at(int n, int T, int nch) {
+    const int ns = (T + kSub - 1) / kSub;
+    Visit v;
+    if (n < ns) {
+        v.tb = n * kSub;
+        v.phase = 1;
+        v.j = n % (kChunkB / kSub);
+        v.c = n / (kChunkB / kSub);
+        return v;
+    }
+    n -= ns;
+    const int last = nch - 1;
+    const int nsub_last = (T - last * kChunkB + kSub - 1) / kSub;
+    int c, i, nsub;
+    if (n < 2 * nsub_last) {
+        c = last;
+        i = n;
+        nsub = nsub_last;
+    } else {
+        const int m = n - 2 * nsub_last;
+        nsub = kChunkB / kSub;
+        c = last - 1 - m / (2 * nsub);
+        i = m % (2 * nsub);
+    }
+    v.c = c;
+    v.phase = i < nsub ? 2 : 3;
+    v.j = i < nsub ? i : 2 * nsub - 1 - i;
+    v.tb = c * kChunkB + v.j * kSub;
+    return v;
+}
+
 template <int DK, int UPD, int GATE, typename TIn>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
     constexpr int V = DK / 32;
     constexpr int NW = kBwdThreads / 32;
-    using Tok = BwdTok<DK, UPD, GATE, TIn>;
+    using SL = StageLayout<DK, GATE>;
+    using Tok = BwdTok<DK, UPD, GATE>;
+    static_assert(kSub * kSlice == kBwdThreads, "one staged (token, value row) per thread");
     extern __shared__ float bsm[];
-    float *sub = bsm;                                        // [kSub][kSlice][DK] sub-block entry states
-    float *red = sub + kSub * kSlice * DK;                   // [2][NW][3][DK] per-warp partial sums
-    float *redb = red + 2 * NW * 3 * DK;                     // [2][NW] beta partials
+    float *sub = bsm;                          // [kSub][kSlice][DK] sub-block entry states
+    float *red = sub + kSub * kSlice * DK;     // [2][NW][3][DK] per-warp partial sums
+    float *redb = red + 2 * NW * 3 * DK;       // [2][NW] beta partials
+    float *stg = redb + 2 * NW;                // [2][SL::FLOATS] staged inputs
 
     const int t_ = threadIdx.x, warp = t_ >> 5, lane = t_ & 31;
     const int nsl = a.DV / kSlice;
     const long bh = blockIdx.x / nsl;
-    const int i0 = (blockIdx.x % nsl) * kSlice + warp * kRows;  // first value row of this warp
+    const int rslice = (blockIdx.x % nsl) * kSlice;
+    const int i0 = rslice + warp * kRows;  // first value row of this warp
     const int c0 = lane * V;
     const int T = a.T;
     const int lr = warp * kRows;  // row of this warp inside the slice
+    const int ns = (T + kSub - 1) / kSub;
+    const int last = a.nch - 1;
+    const int nvis = ns + 2 * ((T - last * kChunkB + kSub - 1) / kSub) + last * 2 * (kChunkB / kSub);
 
-    float s[kRows][V];
-    // ---------------------------------------------------------------- phase 1
+    float s[kRows][V], ds[kRows][V];
 #pragma unroll
     for (int r = 0; r < kRows; ++r)
 #pragma unroll
-        for (int e = 0; e < V; ++e) s[r][e] = a.S0 ? a.S0[((size_t)bh * a.DV + i0 + r) * DK + c0 + e] : 0.f;
-    for (int t = 0; t < T; ++t) {
-        if (t % kChunkB == 0) {
-            float *w = a.ws + (((size_t)bh * a.nch + t / kChunkB) * a.DV + i0) * DK + c0;
-#pragma unroll
-            for (int r = 0; r < kRows; ++r)
-#pragma unroll
-                for (int e = 0; e < V; ++e) w[r * DK + e] = s[r][e];
+        for (int e = 0; e < V; ++e) {
+            s[r][e] = a.S0 ? a.S0[((size_t)bh * a.DV + i0 + r) * DK + c0 + e] : 0.f;
+            ds[r][e] = a.dST ? a.dST[((size_t)bh * a.DV + i0 + r) * DK + c0 + e] : 0.f;
         }
-        Tok x;
-        x.load(a, bh, t, c0, i0, false);
-#pragma unroll
-        for (int r = 0; r < kRows; ++r)
-#pragma unroll
-            for (int e = 0; e < V; ++e) s[r][e] *= x.al[e];
-        float u[kRows], rr[kRows];
-        fwd_write<V, UPD>(s, x.k, x.v, x.bt, u, rr);
+    StageRegs<DK, UPD, GATE, TIn> R;
+    {
+        const Visit v0 = visit_at(0, T, a.nch);
+        R.load(a, bh, v0.tb, rslice, t_, v0.phase != 1);
+        R.store(stg, t_);
     }
-
-    // ---------------------------------------------------------------- phase 2
-    float ds[kRows][V];
-#pragma unroll
-    for (int r = 0; r < kRows; ++r)
-#pragma unroll
-        for (int e = 0; e < V; ++e) ds[r][e] = a.dST ? a.dST[((size_t)bh * a.DV + i0 + r) * DK + c0 + e] : 0.f;
+    __syncthreads();
     int par = 0;  // parity of the reduction buffer
-    for (int c = a.nch - 1; c >= 0; --c) {
-        const int t0 = c * kChunkB;
-        const int nsub = (min(T, t0 + kChunkB) - t0 + kSub - 1) / kSub;
-        {
-            const float *w = a.ws + (((size_t)bh * a.nch + c) * a.DV + i0) * DK + c0;
-#pragma unroll
-            for (int r = 0; r < kRows; ++r)
-#pragma unroll
-                for (int e = 0; e < V; ++e) s[r][e] = w[r * DK + e];
+    for (int n = 0; n < nvis; ++n) {
+        const Visit vi = visit_at(n, T, a.nch);
+        const float *st = stg + (n & 1) * SL::FLOATS;
+        if (n + 1 < nvis) {
+            const Visit vn = visit_at(n + 1, T, a.nch);
+            R.load(a, bh, vn.tb, rslice, t_, vn.phase != 1);
         }
-        // the state entering each sub-block (own entries only)
-        for (int j = 0; j < nsub; ++j) {
-            float *sp = sub + ((size_t)j * kSlice + lr) * DK + c0;
+        if (vi.phase == 1) {
+            // forward; the state entering every chunk goes to the workspace
+            if (vi.j == 0) {
+                float *w = a.ws + (((size_t)bh * a.nch + vi.c) * a.DV + i0) * DK + c0;
 #pragma unroll
-            for (int r = 0; r < kRows; ++r)
+                for (int r = 0; r < kRows; ++r)
 #pragma unroll
-                for (int e = 0; e < V; ++e) sp[r * DK + e] = s[r][e];
+                    for (int e = 0; e < V; ++e) w[r * DK + e] = s[r][e];
+            }
             for (int tt = 0; tt < kSub; ++tt) {
                 Tok x;
-                x.load(a, bh, t0 + j * kSub + tt, c0, i0, false);
+                x.read(st, tt, c0, lr, false);
 #pragma unroll
                 for (int r = 0; r < kRows; ++r)
 #pragma unroll
@@ -215,12 +294,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
                 float u[kRows], rr[kRows];
                 fwd_write<V, UPD>(s, x.k, x.v, x.bt, u, rr);
             }
-        }
-        for (int j = nsub - 1; j >= 0; --j) {
-            // the sub-block's decayed states S'_t in registers
+        } else if (vi.phase == 2) {
+            // recompute forward from the chunk's stored state, keeping each sub-block's entry state
+            if (vi.j == 0) {
+                const float *w = a.ws + (((size_t)bh * a.nch + vi.c) * a.DV + i0) * DK + c0;
+#pragma unroll
+                for (int r = 0; r < kRows; ++r)
+#pragma unroll
+                    for (int e = 0; e < V; ++e) s[r][e] = w[r * DK + e];
+            }
+            float *sp = sub + ((size_t)vi.j * kSlice + lr) * DK + c0;
+#pragma unroll
+            for (int r = 0; r < kRows; ++r)
+#pragma unroll
+                for (int e = 0; e < V; ++e) sp[r * DK + e] = s[r][e];
+            for (int tt = 0; tt < kSub; ++tt) {
+                Tok x;
+                x.read(st, tt, c0, lr, false);
+#pragma unroll
+                for (int r = 0; r < kRows; ++r)
+#pragma unroll
+                    for (int e = 0; e < V; ++e) s[r][e] *= x.al[e];
+                float u[kRows], rr[kRows];
+                fwd_write<V, UPD>(s, x.k, x.v, x.bt, u, rr);
+            }
+        } else {
+            // the sub-block's decayed states S'_t in registers, then back through it
             float Sp[kSub][kRows][V];
             {
-                const float *sp = sub + ((size_t)j * kSlice + lr) * DK + c0;
+                const float *sp = sub + ((size_t)vi.j * kSlice + lr) * DK + c0;
 #pragma unroll
                 for (int r = 0; r < kRows; ++r)
 #pragma unroll
@@ -229,7 +331,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
 #pragma unroll
             for (int tt = 0; tt < kSub; ++tt) {
                 Tok x;
-                x.load(a, bh, t0 + j * kSub + tt, c0, i0, false);
+                x.read(st, tt, c0, lr, false);
 #pragma unroll
                 for (int r = 0; r < kRows; ++r)
 #pragma unroll
@@ -242,21 +344,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
             }
 #pragma unroll
             for (int tt = kSub - 1; tt >= 0; --tt) {
-                const int t = t0 + j * kSub + tt;
+                const int t = vi.tb + tt;
                 Tok x;
-                x.load(a, bh, t, c0, i0, true);
-                float st[kRows][V], u[kRows], rr[kRows];
+                x.read(st, tt, c0, lr, true);
+                float stt[kRows][V], u[kRows], rr[kRows];
 #pragma unroll
                 for (int r = 0; r < kRows; ++r)
 #pragma unroll
-                    for (int e = 0; e < V; ++e) st[r][e] = Sp[tt][r][e];
-                fwd_write<V, UPD>(st, x.k, x.v, x.bt, u, rr);  // st = S_t
+                    for (int e = 0; e < V; ++e) stt[r][e] = Sp[tt][r][e];
+                fwd_write<V, UPD>(stt, x.k, x.v, x.bt, u, rr);  // stt = S_t
                 float dqp[V], dkp[V], dgp[V];
 #pragma unroll
                 for (int e = 0; e < V; ++e) {
                     float acc = 0.f;
 #pragma unroll
-                    for (int r = 0; r < kRows; ++r) acc = fmaf(st[r][e], x.dO[r], acc);
+                    for (int r = 0; r < kRows; ++r) acc = fmaf(stt[r][e], x.dO[r], acc);
                     dqp[e] = acc;
                 }
                 // dS += dO q^T;  du = dS k
@@ -303,14 +405,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
                     }
                     dgp[e] = acc;
                 }
-                if (t < T) {
-                    if (lane == 0) {
-                        float *dvp = a.dv + ((size_t)bh * T + t) * a.DV + i0;
+                if (t < T && lane == 0) {
+                    float *dvp = a.dv + ((size_t)bh * T + t) * a.DV + i0;
 #pragma unroll
-                        for (int r = 0; r < kRows; ++r) dvp[r] = dvt[r];
-                    }
+                    for (int r = 0; r < kRows; ++r) dvp[r] = dvt[r];
                 }
-                // per-warp partials, then the CTA's sums over its 32 rows
+                // per-warp partials, then the CTA's sums over its kSlice rows
                 float *rp = red + ((size_t)par * NW + warp) * 3 * DK;
 #pragma unroll
                 for (int e = 0; e < V; ++e) {
@@ -349,6 +449,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
                 par ^= 1;
             }
         }
+        // the next visit's inputs into the other buffer (its last readers passed the
+        // barrier that ended the previous visit)
+        if (n + 1 < nvis) R.store(stg + ((n + 1) & 1) * SL::FLOATS, t_);
+        __syncthreads();
     }
     if (a.dS0) {
 #pragma unroll
@@ -361,7 +465,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
 template <int DK, int UPD, int GATE, typename TIn>
 int launch_bwd(const BwdArgs &a, cudaStream_t st) {
     constexpr int NW = kBwdThreads / 32;
-    const size_t smem = ((size_t)kSub * kSlice * DK + 2 * NW * 3 * DK + 2 * NW) * sizeof(float);
+    const size_t smem =
+        ((size_t)kSub * kSlice * DK + 2 * NW * 3 * DK + 2 * NW + 2 * StageLayout<DK, GATE>::FLOATS) * sizeof(float);
     auto kern = bwd_kernel<DK, UPD, GATE, TIn>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
