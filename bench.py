@@ -366,6 +366,44 @@ def time_decode_multi(w, T, n_calls, torch, gdn, warmup=3):
     return e0.elapsed_time(e1) / n_calls
 
 
+def time_backward(w, steps, torch, gdn, warmup=1):
+    """Device time of gdn_chunk_bwd (gradients of the prefill) on workload ``w``
+    with random upstream gradients of o and S_T; returns ms per call."""
+    x = make_prefill_inputs(w)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q, k, v = to_dev(x["q"], dt, torch), to_dev(x["k"], dt, torch), to_dev(x["v"], dt, torch)
+    g, beta, S0 = (to_dev(x[n], torch.float32, torch) for n in ("g", "beta", "S0"))
+    del x
+    gen = torch.Generator(device="cuda").manual_seed(w.seed)
+    dO = torch.randn((w.B, w.H, w.T, w.dv), device="cuda", generator=gen)
+    dST = torch.randn((w.B, w.H, w.dv, w.dk), device="cuda", generator=gen)
+    ws = torch.empty(gdn.bwd_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv), dtype=torch.uint8, device="cuda")
+
+    def step():
+        gdn.chunk_bwd(q, k, v, g, beta, S0, dO, dST, update=w.update, gate=w.gate, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(torch.cuda.current_stream())
+    for _ in range(steps):
+        step()
+    e1.record(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    if gdn.device_status() != 0:
+        raise RuntimeError("device status after the backward pass")
+    return e0.elapsed_time(e1) / steps
+
+
+def backward_flops(w):
+    """fp32 arithmetic of gdn_chunk_bwd per launch: four forward token steps per
+    token (the forward pass, the chunk recompute, the sub-block recompute and the
+    S_t of the backward step; 4 dv dk each) and the backward step (dq, dO q^T, du,
+    dk, dS', the gate term, the decay: 15 dv dk)."""
+    return w.n_heads * w.T * (4 * 4 + 15) * w.dv * w.dk
+
+
 def max_over_ranks(value, dist, device):
     """Max of a per-rank float over all ranks (timing only; not on the data path)."""
     if dist is None:
@@ -562,6 +600,17 @@ def run_ours(args):
                                    "achieved_gbs": nb / (msn * 1e-3) / 1e9,
                                    "frac_of_roofline_time": nb / (peaks["hbm_gbs"] * 1e9) / (msn * 1e-3)}
         result["prefill_workloads"] = others
+        # training backward (gdn_chunk_bwd) on the GDN workload
+        nb_steps = 2
+        msb = max_over_ranks(time_backward(w, nb_steps, torch, gdn), dist, "cuda")
+        result["gpu_launches"] += nb_steps * 5  # four output zeroings and the kernel per call
+        fl = backward_flops(w)
+        fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # FP32 lanes x FMA x max SM clock
+        result["backward"] = {"workload": w.name, "ms_per_call": msb,
+                              "tokens_per_s": w.B * w.T * world / (msb * 1e-3),
+                              "flops_per_call": fl, "achieved_tflops": fl / (msb * 1e-3) / 1e12,
+                              "bound": "alu", "fp32_peak_tflops": fp32_peak,
+                              "frac": fl / (msb * 1e-3) / 1e12 / fp32_peak}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w)
