@@ -509,6 +509,15 @@ def run_ours(args):
             print(json.dumps({"only": "decode_multi", "tokens_per_call": 4, "ms_per_call": ms_m}), flush=True)
         return
     w = WORKLOADS[args.workload]
+    if args.only in ("prefill", "backward"):
+        # profiling aids: the workload's distributions on an optionally smaller shape
+        w = w.with_(B=args.batch or w.B, H=args.heads or w.H, T=args.seq_len or w.T)
+    if args.only == "backward":
+        ms = time_backward(w, args.steps, torch, gdn, warmup=args.warmup)
+        if rank == 0:
+            print(json.dumps({"only": "backward", "workload": w.name, "B": w.B, "H": w.H, "T": w.T,
+                              "ms_per_call": ms}), flush=True)
+        return
     x = make_prefill_inputs(w)
     if args.only == "prefill":
         ms = time_prefill(w, x, args.steps, args.warmup, torch, gdn, dist)
@@ -702,7 +711,10 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=[k for k, w in WORKLOADS.items() if w.steps == 0])
     ap.add_argument("--quick", action="store_true", help="skip the extra prefill workloads; 100 decode steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_multi"], default="all",
+    ap.add_argument("--batch", type=int, default=0, help="with --only prefill/backward: override B")
+    ap.add_argument("--heads", type=int, default=0, help="with --only prefill/backward: override H")
+    ap.add_argument("--seq-len", type=int, default=0, help="with --only prefill/backward: override T")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_multi", "backward"], default="all",
                     help="profiling aid: run one part only (its line is not a benchmark result)")
     ap.add_argument("--launch-check", action="store_true",
                     help="test aid: run only the rank protocol on CPU (gloo), no GPU work")
