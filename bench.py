@@ -578,9 +578,9 @@ def run_ours(args):
                             "achieved_gbs": rf["achieved"], "roofline_us": rf["roofline_us"],
                             "frac_of_roofline_time": rf["frac_of_roofline_time"],
                             "frac_fp32_output": rf["fp32_output"]["frac"]}
-        # Gated DeltaProduct, 2 substeps per token, on the GDN workload's heads and
-        # 4096 tokens (8192 virtual steps, the GDN workload's length)
-        wp, nh = WORKLOADS["gdn_prefill_bf16"].with_(T=4096, name="gdp_prefill_bf16"), 2
+        # Gated DeltaProduct with the pages' 3 substeps per token, on the GDN workload's
+        # heads and 2731 tokens (8193 virtual steps, about the GDN workload's length)
+        wp, nh = WORKLOADS["gdn_prefill_bf16"].with_(T=2731, name="gdp_prefill_bf16"), 3
         msp = max_over_ranks(time_product(wp, nh, max(3, args.steps // 2), args.warmup, torch, gdn), dist, "cuda")
         nb = product_bytes(wp, nh)
         fl = prefill_flops(wp.with_(T=wp.T * nh))

@@ -302,10 +302,9 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     if (nh == 1) return gdn_chunk_fwd(d, q, k, v, g, beta, S0, o, S_T, stream);
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
     if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC) return GDN_ERR_ARG;
-    // the pipelined tensor-core kernel takes whole tokens per chunk: nh a power of
-    // two (it divides the chunk), scalar or no gate
-    const bool pow2 = (nh & (nh - 1)) == 0;
-    const bool tc_ok = gdn_tc_supported(d) != 0 && pow2 && d->gate != GDN_GATE_CHANNEL && tc2_prologue_ok(d);
+    // the pipelined tensor-core kernel takes 64 / nh whole tokens per chunk (the
+    // remaining rows are identity steps), scalar or no gate
+    const bool tc_ok = gdn_tc_supported(d) != 0 && d->gate != GDN_GATE_CHANNEL && tc2_prologue_ok(d);
     if (d->algo == GDN_ALGO_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
     if ((long)d->T * nh > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
     const long BH = (long)d->B * d->H;

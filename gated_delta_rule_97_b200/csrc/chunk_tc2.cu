@@ -82,7 +82,9 @@ struct Params {
     int *status;
     int *diag;
     int BH, T, dv, nslices;
-    int lnh;  // log2 of the substeps per token (Gated DeltaProduct), else 0
+    int nh, cv, tpc;  // Gated DeltaProduct: substeps per token, virtual steps and tokens per chunk
+    // and the rows of a chunk that are a token's first / last substep (bit l = row l)
+    unsigned long long firstmask, lastmask;
     int pro;   // GDN_PRO_* input maps
     int mode;  // kMode* bits (internal passes of the segmented prefill)
 };
@@ -158,12 +160,15 @@ __device__ __forceinline__ int v16_slot(int buf) {
     return (UPD != kDelta && GATE != kGateChannel && buf) ? L::KT : L::V16;
 }
 
-// PROD: Gated DeltaProduct with 2^lnh substeps per token ("GDP as GDN over a
+// PROD: Gated DeltaProduct with nh substeps per token ("GDP as GDN over a
 // virtual sequence"): T counts virtual steps; k, v, beta are per virtual step,
-// while q, g and o are per token.  A chunk covers 64 >> lnh whole tokens: their q
-// rows arrive compact and are moved to each token's last substep (zeros
-// elsewhere), the gate sits on each token's first substep, and only each
-// token's last substep is written out.
+// while q, g and o are per token.  A chunk covers tpc = 64 / nh whole tokens,
+// i.e. cv = tpc * nh virtual steps; when nh does not divide 64 its last 64 - cv
+// rows are identity steps (k, beta and g zero, so T2 has zero columns there
+// and they neither read nor change the state).  The tokens' q rows arrive
+// compact and are moved to each token's last substep (zeros elsewhere), the
+// gate sits on each token's first substep, and only each token's last substep
+// is written out.
 //
 // EXT: the input prologue and the segmented prefill's pass modes are compiled
 // in only for calls that use them; the plain path (EXT = false) sees both as
@@ -202,7 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     const int bh = blockIdx.x / p.nslices;
     const int v0 = (blockIdx.x % p.nslices) * DVS;
     const int T = p.T, dv = p.dv;
-    const int nchunks = (T + C - 1) / C;
+    // virtual steps and tokens per chunk, substeps per token (compile-time C, C, 1
+    // unless PROD)
+    const int CV = PROD ? p.cv : C, TPC = PROD ? p.tpc : C, NH = PROD ? p.nh : 1;
+    const int nchunks = (T + CV - 1) / CV;
 
     if (t == 0) {
         mbar_init(&ms.bar_tma, 1);
@@ -255,15 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         float gpre0 = 0.f, gpre1 = 0.f, bpre = 0.f;
         // raw gates (warp 4, two tokens a lane) and betas (warps 4-5) of chunk r into registers
         auto load_gate_beta = [&](int r) {
-            const int t0 = r * C;
+            const int t0 = r * CV;
             if (GATE == kGateScalar && warp == 4) {
                 const int l0 = 2 * lane;
                 if (PROD) {
-                    // the token's gate on its first substep, 1 (g = 0) on the others
-                    const int m0 = t0 + l0, m1 = m0 + 1, msk = (1 << p.lnh) - 1;
-                    const size_t gb = (size_t)bh * (T >> p.lnh);
-                    gpre0 = (m0 < T && (m0 & msk) == 0) ? pro_gate(p.g[gb + (m0 >> p.lnh)], pro) : 0.f;
-                    gpre1 = (m1 < T && (m1 & msk) == 0) ? pro_gate(p.g[gb + (m1 >> p.lnh)], pro) : 0.f;
+                    // the token's gate on its first substep, 1 (g = 0) on the others and
+                    // on the identity rows past cv
+                    const size_t gb = (size_t)bh * (T / NH) + (size_t)r * TPC;
+                    const int l1 = l0 + 1;
+                    const unsigned long long fm = p.firstmask;
+                    // the token of a first-substep row is the number of first substeps before it
+                    gpre0 = (t0 + l0 < T && ((fm >> l0) & 1)) ? pro_gate(p.g[gb + __popcll(fm & ((1ull << l0) - 1))], pro)
+                                                             : 0.f;
+                    gpre1 = (t0 + l1 < T && ((fm >> l1) & 1)) ? pro_gate(p.g[gb + __popcll(fm & ((1ull << l1) - 1))], pro)
+                                                             : 0.f;
                 } else {
                     gpre0 = (t0 + l0 < T) ? pro_gate(p.g[(size_t)bh * T + t0 + l0], pro) : 0.f;
                     gpre1 = (t0 + l0 + 1 < T) ? pro_gate(p.g[(size_t)bh * T + t0 + l0 + 1], pro) : 0.f;
@@ -271,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             }
             if (DELTA && t >= 128 && t < 128 + C) {
                 const int l = t - 128;
-                bpre = (t0 + l < T) ? pro_beta(p.beta[(size_t)bh * T + t0 + l], pro) : 0.f;
+                bpre = (t0 + l < T && l < CV) ? pro_beta(p.beta[(size_t)bh * T + t0 + l], pro) : 0.f;
             }
         };
         // scalar gate prefix of chunk r and its factors b = e^G, gamma = e^{G_C-G},
@@ -303,16 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         // q, k (+ the channel gate tile) on bar_tma; v on bar_tv when split, else also on bar_tma
         auto issue_tma_v = [&](int r, uint64_t *bar) {
             for (int j = 0; j < NB; ++j)
-                tma_load_3d(sm + L::RAW_V + j * 8192, &p.v_map, v0 + j * 64, r * C, bh, bar);
+                tma_load_3d(sm + L::RAW_V + j * 8192, &p.v_map, v0 + j * 64, r * CV, bh, bar);
         };
         auto issue_tma = [&](int r) {
-            const int t0 = r * C;
-            const uint32_t qbytes = PROD ? 2u * (64u >> p.lnh) * 128u : 16384u;
+            const int t0 = r * CV;
+            const uint32_t qbytes = PROD ? 2u * (uint32_t)TPC * 128u : 16384u;
             const uint32_t bytes =
                 qbytes + 16384 + ((kSplitV || zeroV) ? 0 : DVS * 128) + (GATE == kGateChannel ? 32768 : 0);
             mbar_arrive_expect_tx(&ms.bar_tma, bytes);
             for (int h = 0; h < 2; ++h) {
-                tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, PROD ? (t0 >> p.lnh) : t0, bh,
+                tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, PROD ? r * TPC : t0, bh,
                             &ms.bar_tma);
                 tma_load_3d(sm + L::RAW_QK + h * 16384 + 8192, &p.k_map, h * 64, t0, bh, &ms.bar_tma);
             }
@@ -345,15 +358,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             TC2_MARK(0, 0);
             if (!mbar_wait(&ms.bar_tma, ph)) note_timeout(ms, 1, r);
             if (PROD) {
-                // compact q rows j -> row (j + 1) * nh - 1, the rest zero (both key halves)
-                const int lnh = p.lnh, msk = (1 << lnh) - 1;
+                // compact q rows j -> row (j + 1) * nh - 1, the rest zero (both key halves);
+                // the k rows past cv (the next chunk's first steps, loaded by the 64-row box)
+                // become the zero keys of identity steps
                 uint4 qv[4];
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
                     const int i = t + 256 * s4, h = i >> 9, d = (i & 511) >> 3, c = i & 7;
                     qv[s4] = make_uint4(0, 0, 0, 0);
-                    if ((d & msk) == msk) {
-                        const int j = d >> lnh;
+                    if ((p.lastmask >> d) & 1) {
+                        const int j = __popcll(p.lastmask & ((1ull << d) - 1));  // the row's token
                         qv[s4] = *reinterpret_cast<const uint4 *>(sm + L::RAW_QK + h * 16384 + j * 128 +
                                                                    ((c ^ (j & 7)) << 4));
                     }
@@ -363,6 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 for (int s4 = 0; s4 < 4; ++s4) {
                     const int i = t + 256 * s4, h = i >> 9, d = (i & 511) >> 3, c = i & 7;
                     *reinterpret_cast<uint4 *>(sm + L::RAW_QK + h * 16384 + d * 128 + ((c ^ (d & 7)) << 4)) = qv[s4];
+                    if (d >= CV)
+                        *reinterpret_cast<uint4 *>(sm + L::RAW_QK + h * 16384 + 8192 + d * 128 + ((c ^ (d & 7)) << 4)) =
+                            make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
                 named_bar(kPrepBar, 256);
@@ -372,9 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 // halves of a row are adjacent lanes.  Rows past T and, for the
                 // product, q rows that are not a token's last substep stay zero.
                 const int ten = t >> 7, row = (t >> 1) & 63, hk = t & 1;
-                const int m = r * C + row;
-                bool valid = m < T;
-                if (PROD && ten == 0) valid = valid && ((row & ((1 << p.lnh) - 1)) == (1 << p.lnh) - 1);
+                const int m = r * CV + row;
+                bool valid = m < T && row < CV;
+                if (PROD && ten == 0) valid = valid && ((p.lastmask >> row) & 1);
                 unsigned char *base = sm + L::RAW_QK + hk * 16384 + ten * 8192 + row * 128;
                 float f[64];
                 float ss = 0.f;
@@ -1056,7 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         for (int r = 0; r < nchunks; ++r) {
             if (ms.s_abort) break;
             const uint32_t ph = r & 1;
-            const int t0 = r * C;
+            const int t0 = r * CV;
             const int buf = r & 1;
             if (GATE != kGateChannel && r > 0) {
                 if (!mbar_wait(&ms.bar_rdy, ph)) note_timeout(ms, 6, r);
@@ -1196,15 +1213,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 named_bar(kStateBar, 128);
                 if (has_row && PROD) {
                     // each token's last substep, compacted to one row per token
-                    const int msk = (1 << p.lnh) - 1;
+                    const unsigned long long lm = p.lastmask;
+                    int row = 0;
 #pragma unroll
                     for (int l = 0; l < 64; ++l) {
-                        if ((l & msk) != msk) continue;
-                        const int row = l >> p.lnh;
+                        if (!((lm >> l) & 1)) continue;
                         if (OUT_BF16)
                             reinterpret_cast<__nv_bfloat16 *>(ost)[row * DVS + vrow] = __float2bfloat16_rn(ov[l]);
                         else
                             ost[row * DVS + vrow] = ov[l];
+                        ++row;
                     }
                 } else if (has_row) {
                     if (OUT_BF16) {
@@ -1219,7 +1237,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 fence_proxy_async_smem();
                 named_bar(kStateBar, 128);
                 if (ts == 0) {
-                    tma_store_3d(&p.o_map, ost, v0, PROD ? (t0 >> p.lnh) : t0, bh);
+                    tma_store_3d(&p.o_map, ost, v0, PROD ? r * TPC : t0, bh);
                     bulk_commit();
                 }
             }
@@ -1370,12 +1388,12 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     Params prm;
     memset(&prm, 0, sizeof(prm));
     const uint64_t BH = (uint64_t)a.BH, T = (uint64_t)a.T;
-    // Gated DeltaProduct: T counts virtual steps; q and o have T / nh token rows
-    int lnh = 0;
-    while ((1 << lnh) < a.nh) ++lnh;
-    if ((1 << lnh) != a.nh || lnh > 6 || d->gate == GDN_GATE_CHANNEL && lnh > 0) return (int)cudaErrorInvalidValue;
-    const uint64_t Tr = T >> lnh;
-    const uint32_t rows = 64u >> lnh;
+    // Gated DeltaProduct: T counts virtual steps; q and o have T / nh token rows, a
+    // chunk holds rows = 64 / nh whole tokens
+    const int nh = a.nh;
+    if (nh < 1 || nh > 64 || (d->gate == GDN_GATE_CHANNEL && nh > 1)) return (int)cudaErrorInvalidValue;
+    const uint64_t Tr = T / nh;
+    const uint32_t rows = 64u / nh;
     if (!make_map_3d(&prm.q_map, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, Tr, BH, 64, rows, 1, true) ||
         !make_map_3d(&prm.k_map, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, T, BH, 64, 64, 1, true))
         return (int)cudaErrorInvalidValue;
@@ -1402,12 +1420,18 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     prm.T = a.T;
     prm.dv = a.dv;
     prm.nslices = a.dv / dvs;
-    prm.lnh = lnh;
+    prm.nh = nh;
+    prm.tpc = (int)rows;
+    prm.cv = (int)rows * nh;
+    for (int l = 0; l < prm.cv; ++l) {
+        if (l % nh == 0) prm.firstmask |= 1ull << l;
+        if (l % nh == nh - 1) prm.lastmask |= 1ull << l;
+    }
     prm.pro = a.pro;
     prm.mode = a.mode;
     const long grid = (long)a.BH * prm.nslices;
     if (grid == 0) return 0;
-    if (lnh > 0) {
+    if (nh > 1) {
         if (dvs == 64)
             return d->gate == GDN_GATE_SCALAR ? launch_prod<64, kGateScalar>(prm, (int)grid, ob, stream)
                                               : launch_prod<64, kGateNone>(prm, (int)grid, ob, stream);

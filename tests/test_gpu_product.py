@@ -77,18 +77,19 @@ def test_product_empty_sequence_copies_state():
     assert o.shape == (2, 2, 0, 64) and torch.equal(ST, S0)
 
 
-def test_product_rejects_tensor_core_choice_without_whole_tokens():
-    w = workload("scalar", "bf16", T=8, d=128)
-    x = make_product_inputs(w, 3)
+def test_product_rejects_tensor_core_choice_with_channel_gate():
+    w = workload("channel", "bf16", T=8, d=128)
+    x = make_product_inputs(w, 2)
     with pytest.raises(gdn.GDNError):
-        run(w, x, 3, algo="tc")
+        run(w, x, 2, algo="tc")
 
 
 @pytest.mark.parametrize("gate", ["none", "scalar"])
-@pytest.mark.parametrize("nh", [2, 4, 8, 16])
+@pytest.mark.parametrize("nh", [2, 3, 4, 5, 7, 8, 16])
 @pytest.mark.parametrize("dv,T", [(128, 37), (128, 200), (64, 100)])
 def test_product_tensor_core_matches_oracle(gate, nh, dv, T):
-    # a chunk holds 64 / nh whole tokens; T ragged in tokens
+    # a chunk holds 64 / nh whole tokens (with nh = 3, 5, 7 its last rows are identity
+    # steps and tokens never straddle a chunk); T ragged in tokens
     w = workload(gate, "bf16", T=T, d=128).with_(dv=dv)
     x = make_product_inputs(w, nh)
     o, ST = run(w, x, nh, algo="tc")
@@ -97,9 +98,10 @@ def test_product_tensor_core_matches_oracle(gate, nh, dv, T):
     assert eo <= TOL["bf16"] and es <= TOL["bf16"], (eo, es)
 
 
-def test_product_tensor_core_matches_simt():
+@pytest.mark.parametrize("nh", [3, 4])
+def test_product_tensor_core_matches_simt(nh):
     w = workload("scalar", "bf16", T=300, d=128, B=1, H=4)
-    x = make_product_inputs(w, 4)
-    o_tc, S_tc = run(w, x, 4, algo="tc")
-    o_s, S_s = run(w, x, 4, algo="simt")
+    x = make_product_inputs(w, nh)
+    o_tc, S_tc = run(w, x, nh, algo="tc")
+    o_s, S_s = run(w, x, nh, algo="simt")
     assert rel_err(np64(o_tc), np64(o_s)) <= TOL["bf16"] and rel_err(np64(S_tc), np64(S_s)) <= TOL["bf16"]
