@@ -303,8 +303,8 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
     if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_TC) return GDN_ERR_ARG;
     // the pipelined tensor-core kernel takes 64 / nh whole tokens per chunk (the
-    // remaining rows are identity steps), scalar or no gate
-    const bool tc_ok = gdn_tc_supported(d) != 0 && d->gate != GDN_GATE_CHANNEL && tc2_prologue_ok(d);
+    // remaining rows are identity steps)
+    const bool tc_ok = gdn_tc_supported(d) != 0 && tc2_prologue_ok(d);
     if (d->algo == GDN_ALGO_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
     if ((long)d->T * nh > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
     const long BH = (long)d->B * d->H;

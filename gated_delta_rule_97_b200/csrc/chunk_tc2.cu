@@ -321,8 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         auto issue_tma = [&](int r) {
             const int t0 = r * CV;
             const uint32_t qbytes = PROD ? 2u * (uint32_t)TPC * 128u : 16384u;
+            const uint32_t gbytes = PROD ? 512u * (uint32_t)TPC : 32768u;  // the channel gate tile
             const uint32_t bytes =
-                qbytes + 16384 + ((kSplitV || zeroV) ? 0 : DVS * 128) + (GATE == kGateChannel ? 32768 : 0);
+                qbytes + 16384 + ((kSplitV || zeroV) ? 0 : DVS * 128) + (GATE == kGateChannel ? gbytes : 0);
             mbar_arrive_expect_tx(&ms.bar_tma, bytes);
             for (int h = 0; h < 2; ++h) {
                 tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, PROD ? r * TPC : t0, bh,
@@ -331,7 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             }
             if (!kSplitV && !zeroV) issue_tma_v(r, &ms.bar_tma);
             if (GATE == kGateChannel)
-                for (int j = 0; j < 4; ++j) tma_load_3d(sm + L::GCH + j * 8192, &p.g_map, j * 32, t0, bh, &ms.bar_tma);
+                for (int j = 0; j < 4; ++j)
+                    tma_load_3d(sm + L::GCH + j * 8192, &p.g_map, j * 32, PROD ? r * TPC : t0, bh, &ms.bar_tma);
         };
         auto issue_tma_split_v = [&](int r) {
             mbar_arrive_expect_tx(&ms.bar_tv, DVS * 128);
@@ -372,7 +374,29 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                                                                    ((c ^ (j & 7)) << 4));
                     }
                 }
+                // the per-channel gate: each token's row (compact, as loaded) moves to the
+                // token's first substep, every other row is g = 0 (four 32-channel sub-tiles)
+                uint4 gw[GATE == kGateChannel ? 8 : 1];
+                if (GATE == kGateChannel) {
+#pragma unroll
+                    for (int s8 = 0; s8 < 8; ++s8) {
+                        const int i = t + 256 * s8, st = i >> 9, d = (i & 511) >> 3, c = i & 7;
+                        gw[s8] = make_uint4(0, 0, 0, 0);
+                        if ((p.firstmask >> d) & 1) {
+                            const int j = __popcll(p.firstmask & ((1ull << d) - 1));  // the row's token
+                            gw[s8] = *reinterpret_cast<const uint4 *>(sm + L::GCH + st * 8192 + j * 128 +
+                                                                       ((c ^ (j & 7)) << 4));
+                        }
+                    }
+                }
                 named_bar(kPrepBar, 256);
+                if (GATE == kGateChannel) {
+#pragma unroll
+                    for (int s8 = 0; s8 < 8; ++s8) {
+                        const int i = t + 256 * s8, st = i >> 9, d = (i & 511) >> 3, c = i & 7;
+                        *reinterpret_cast<uint4 *>(sm + L::GCH + st * 8192 + d * 128 + ((c ^ (d & 7)) << 4)) = gw[s8];
+                    }
+                }
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
                     const int i = t + 256 * s4, h = i >> 9, d = (i & 511) >> 3, c = i & 7;
@@ -464,7 +488,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 #pragma unroll
                 for (int l = 0; l < 32; ++l) {
                     gv[l] = gt[gch_idx(32 * hf + l, c)];
-                    if (r * C + 32 * hf + l < T) gv[l] = pro_gate(gv[l], pro);  // padding stays g = 0
+                    // padding (and, for the product, every row but a token's first substep) stays g = 0
+                    const bool real = PROD ? ((p.firstmask >> (32 * hf + l)) & 1) != 0 : true;
+                    if (r * CV + 32 * hf + l < T && real) gv[l] = pro_gate(gv[l], pro);
                 }
 #pragma unroll
                 for (int l = 1; l < 32; ++l) gv[l] += gv[l - 1];
@@ -1391,7 +1417,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     // Gated DeltaProduct: T counts virtual steps; q and o have T / nh token rows, a
     // chunk holds rows = 64 / nh whole tokens
     const int nh = a.nh;
-    if (nh < 1 || nh > 64 || (d->gate == GDN_GATE_CHANNEL && nh > 1)) return (int)cudaErrorInvalidValue;
+    if (nh < 1 || nh > 64) return (int)cudaErrorInvalidValue;
     const uint64_t Tr = T / nh;
     const uint32_t rows = 64u / nh;
     if (!make_map_3d(&prm.q_map, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, Tr, BH, 64, rows, 1, true) ||
@@ -1401,7 +1427,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
         !make_map_3d(&prm.v_map, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.dv, T, BH, 64, 64, 1, true))
         return (int)cudaErrorInvalidValue;
     if (d->gate == GDN_GATE_CHANNEL &&
-        !make_map_3d(&prm.g_map, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, T, BH, 32, 64, 1, true))
+        !make_map_3d(&prm.g_map, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, Tr, BH, 32, rows, 1, true))
         return (int)cudaErrorInvalidValue;
     const int dvs = tc2_slice(d);
     const bool ob = d->out_dtype == GDN_BF16;
@@ -1432,6 +1458,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     const long grid = (long)a.BH * prm.nslices;
     if (grid == 0) return 0;
     if (nh > 1) {
+        if (d->gate == GDN_GATE_CHANNEL) return launch_prod<64, kGateChannel>(prm, (int)grid, ob, stream);
         if (dvs == 64)
             return d->gate == GDN_GATE_SCALAR ? launch_prod<64, kGateScalar>(prm, (int)grid, ob, stream)
                                               : launch_prod<64, kGateNone>(prm, (int)grid, ob, stream);

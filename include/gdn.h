@@ -179,9 +179,10 @@ int gdn_chunk_fwd_host(const gdn_desc_t *desc, int n_slices, const void *q, cons
  *
  * desc->update must be GDN_DELTA and desc->T counts real tokens.  nh == 1 is
  * gdn_chunk_fwd.  For nh > 1, GDN_ALGO_AUTO takes the pipelined tensor-core
- * kernel when it serves the shape (bf16, dk = 128, dv in {64, 128}, scalar or no
- * gate, nh a power of two, so that a chunk holds whole tokens) and the fp32 SIMT
- * kernel otherwise; GDN_ALGO_TC demands the former, GDN_ALGO_SIMT the latter.
+ * kernel when it serves the shape (bf16, dk = 128, dv in {64, 128}, any gate; a
+ * chunk holds floor(64 / nh) whole tokens and identity steps fill its remaining
+ * rows) and the fp32 SIMT kernel otherwise; GDN_ALGO_TC demands the former,
+ * GDN_ALGO_SIMT the latter.
  * The caller owns every buffer; nothing is allocated.
  */
 int gdn_product_fwd(const gdn_desc_t *desc, int nh, const void *q, const void *k, const void *v,

@@ -117,8 +117,8 @@ def test_product_rejects_bad_arguments(lib):
     assert lib.gdn_product_fwd(ctypes.byref(d), 17, *args) == -3     # nh > GDN_PRODUCT_MAX_NH
     d = _desc(update="additive", gate="none")
     assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -1      # only the delta rule has substeps
-    d = _desc(algo="tc", gate="channel")
-    assert lib.gdn_product_fwd(ctypes.byref(d), 3, *args) == -3      # tensor-core kernel: scalar or no gate
+    d = _desc(algo="tc", dtype=gdn.F32)
+    assert lib.gdn_product_fwd(ctypes.byref(d), 3, *args) == -3      # tensor-core kernel: bf16 inputs only
     d = _desc()
     d.algo = 3
     assert lib.gdn_product_fwd(ctypes.byref(d), 2, *args) == -1      # no such kernel choice

@@ -77,11 +77,17 @@ def test_product_empty_sequence_copies_state():
     assert o.shape == (2, 2, 0, 64) and torch.equal(ST, S0)
 
 
-def test_product_rejects_tensor_core_choice_with_channel_gate():
-    w = workload("channel", "bf16", T=8, d=128)
-    x = make_product_inputs(w, 2)
-    with pytest.raises(gdn.GDNError):
-        run(w, x, 2, algo="tc")
+@pytest.mark.parametrize("nh", [2, 3, 5, 16])
+@pytest.mark.parametrize("dv,T", [(128, 37), (64, 100)])
+def test_product_tensor_core_channel_gate(nh, dv, T):
+    # per-channel (KDA) gate: each token's gate row sits on its first substep and
+    # the other rows of the chunk carry g = 0
+    w = workload("channel", "bf16", T=T, d=128).with_(dv=dv)
+    x = make_product_inputs(w, nh)
+    o, ST = run(w, x, nh, algo="tc")
+    ro, rS = oracle.gdp_forward("channel", x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
+    eo, es = rel_err(np64(o), ro), rel_err(np64(ST), rS)
+    assert eo <= TOL["bf16"] and es <= TOL["bf16"], (eo, es)
 
 
 @pytest.mark.parametrize("gate", ["none", "scalar"])
