@@ -528,6 +528,7 @@ extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.o = o;
     a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
     a.pro = d->prologue;
+    a.status = status_ptr();
     return from_cuda(gdn_launch_decode(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16,
                                        static_cast<cudaStream_t>(stream)));
 }

@@ -70,6 +70,7 @@ struct DecodeArgs {
     void *o;                 // [BH,T,dv]
     int BH, T, dk, dv;
     int pro;                 // GDN_PRO_* input maps
+    int *status;             // device status word
 };
 
 // Input prologue maps (GDN_PRO_* bits, mirrored here for device code).
