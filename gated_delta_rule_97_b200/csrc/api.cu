@@ -13,6 +13,9 @@ __device__ int g_gdn_diag = 0;
 // tensor-core launcher (chunk_tc2.cu)
 int gdn_tc_supported(const gdn_desc_t *d);
 int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
+// linear-attention launcher (chunk_la.cu)
+int gdn_la_supported(const gdn_desc_t *d, int mode);
+int gdn_launch_chunk_la(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream);
 
 namespace {
 
@@ -61,10 +64,12 @@ int from_cuda(int e) { return e == 0 ? GDN_OK : GDN_ERR_CUDA; }
 bool tc2_prologue_ok(const gdn_desc_t *d);
 
 // Kernel choice of gdn_chunk_fwd (and of the passes of the segmented prefill):
-// the requested kernel, or for AUTO the pipelined tensor-core kernel when it
-// serves the request and the SIMT kernel otherwise.  Both apply the input
-// prologue.
+// the requested kernel, or for AUTO the linear-attention kernel for a plain
+// additive request it serves, else the pipelined tensor-core kernel when it
+// serves the request and the SIMT kernel otherwise.  The latter two apply the
+// input prologue.
 int dispatch_chunk(const gdn_desc_t *d, gdn::ChunkArgs &a, cudaStream_t st) {
+    if (d->algo == GDN_ALGO_AUTO && gdn_la_supported(d, a.mode)) return from_cuda(gdn_launch_chunk_la(a, d, st));
     const bool tc_ok = gdn_tc_supported(d) != 0 && tc2_prologue_ok(d);
     if (d->algo == GDN_ALGO_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
     if (d->algo == GDN_ALGO_TC || (d->algo == GDN_ALGO_AUTO && tc_ok)) return from_cuda(gdn_launch_chunk_tc2(a, d, st));

@@ -215,6 +215,17 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
         : "memory");
 }
 
+// D (fp32, TMEM) (+)= A (fp32 read as tf32, TMEM) x B (tf32, shared memory).
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+
 // Each thread of the warp writes 32 consecutive 32-bit columns of its lane.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
     asm volatile(
@@ -237,6 +248,20 @@ __device__ __forceinline__ void tmem_st32f(uint32_t taddr, const float *v) {
 // Barrier over `count` threads (a multiple of 32) with hardware barrier `id` (1..15).
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// The same barrier, returning whether `pred` held on every participating thread.
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, a;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "barrier.red.and.pred a, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, a;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 
 // ---------------------------------------------------------------- descriptors
@@ -262,6 +287,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_bf16, int 
            | ((uint32_t)a_neg << 13)                   // negate A
            | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16)
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::tf32 with fp32 accumulation, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Byte offset of element (row, col) inside a 128-byte-swizzled tile whose rows

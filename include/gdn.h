@@ -73,10 +73,13 @@ typedef enum { GDN_GATE_NONE = 0, GDN_GATE_SCALAR = 1, GDN_GATE_CHANNEL = 2 } gd
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
 
-/* Kernel choice for gdn_chunk_fwd.  AUTO picks the tensor-core kernel when it
- * supports the request (bf16 inputs, dk = 128) and the fp32 SIMT kernel
- * otherwise.  TC is the warp-specialised tensor-core kernel (prep of the next
- * chunk overlapping the state update of the current one).  An explicit value
+/* Kernel choice for gdn_chunk_fwd.  AUTO picks, for the additive update without
+ * gate and without input prologue (bf16, dk = 128, dv in {64, 128}), the
+ * linear-attention tensor-core kernel (state kept fp32 in tensor memory); else
+ * the tensor-core kernel below when it supports the request (bf16 inputs,
+ * dk = 128) and the fp32 SIMT kernel otherwise.  TC is the warp-specialised
+ * tensor-core kernel for every mode (prep of the next chunk overlapping the
+ * state update of the current one).  An explicit value
  * forces that kernel (GDN_ERR_UNSUPPORTED if it cannot serve the request); any
  * other value is GDN_ERR_ARG. */
 typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TC = 2 } gdn_algo_t;
