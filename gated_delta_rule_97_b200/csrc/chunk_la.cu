@@ -121,10 +121,12 @@ __global__ void __launch_bounds__(kLAThreads, 1) chunk_la_kernel(const __grid_co
     tc_fence_after();
     const uint32_t tmem = bs.tmem_base;
 
-    // a wait that runs out stops every role (each then finds its next wait cut short too)
+    // a wait that runs out stops every role (each then finds its next wait cut
+    // short too); the waits on the chunk-to-chunk chain poll without suspending
     auto wait = [&](uint64_t *bar, uint32_t par) -> bool {
+        if (mbar_test_wait(bar, par)) return true;
         if (*reinterpret_cast<volatile int *>(&bs.abort_flag)) return false;
-        if (mbar_wait(bar, par)) return true;
+        if (mbar_wait_spin(bar, par)) return true;
         if (atomicExch(&bs.abort_flag, 1) == 0) record_status(p.status, kStatusTimeout);
         return false;
     };
