@@ -574,7 +574,9 @@ def run_ours(args):
             result["gpu_launches"] += max(3, args.steps // 2)
             del xo
             rf = roofline(wo, mso, peaks, peak_kind)
-            others[name] = {"ms_per_step": mso, "tokens_per_s": wo.B * wo.T * world / (mso * 1e-3),
+            others[name] = {"kernel": "chunk_la (additive, 128-token chunks)" if wo.update == "additive"
+                            else "chunk_tc2 (pipelined, 64-token chunks)",
+                            "ms_per_step": mso, "tokens_per_s": wo.B * wo.T * world / (mso * 1e-3),
                             "achieved_gbs": rf["achieved"], "roofline_us": rf["roofline_us"],
                             "frac_of_roofline_time": rf["frac_of_roofline_time"],
                             "frac_fp32_output": rf["fp32_output"]["frac"]}
