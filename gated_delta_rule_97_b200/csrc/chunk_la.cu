@@ -89,7 +89,9 @@ __global__ void __launch_bounds__(kLAThreads, 1) chunk_la_kernel(const __grid_co
     using L = LASmem;
     constexpr int DVS = kDVS;
     extern __shared__ unsigned char dsm_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned by an offset on the shared pointer (a cast through an integer
+    // would turn every access into a generic one)
+    unsigned char *sm = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
     __shared__ LABars bs;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int bh = blockIdx.x / p.nslices, v0 = (blockIdx.x % p.nslices) * DVS;
