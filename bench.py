@@ -366,6 +366,66 @@ def time_decode_multi(w, T, n_calls, torch, gdn, warmup=3):
     return e0.elapsed_time(e1) / n_calls
 
 
+# The prefill -> decode serving loop: a prompt of SERVE_PROMPT tokens per
+# sequence is prefilled (gdn_chunk_fwd writes S_T into the decode state
+# buffer), then SERVE_DECODE tokens are generated one at a time in place
+# (gdn_decode_step), the forward(x, state) -> (o, state) hand-off of the pages.
+SERVE_B, SERVE_H, SERVE_PROMPT, SERVE_DECODE = 32, 32, 1024, 128
+
+
+def serving_workloads():
+    wp = WORKLOADS["gdn_prefill_bf16"].with_(B=SERVE_B, H=SERVE_H, T=SERVE_PROMPT, name="serve_prompt")
+    wd = WORKLOADS["decode_gdn_bf16"].with_(B=SERVE_B, H=SERVE_H, name="serve_decode")
+    return wp, wd
+
+
+def time_serving_loop(reps, torch, gdn, warmup=1):
+    """Device time of one serving loop (prefill of the prompt into the state,
+    then SERVE_DECODE single-token steps on it); returns (ms per loop, ms of
+    the prefill, ms per decode step)."""
+    wp, wd = serving_workloads()
+    x = make_prefill_inputs(wp)
+    dt = torch.bfloat16
+    q, k, v = (to_dev(x[n], dt, torch) for n in ("q", "k", "v"))
+    g, beta, S0 = (to_dev(x[n], torch.float32, torch) for n in ("g", "beta", "S0"))
+    del x
+    steps = []
+    for _, blk in iter_decode_blocks(wd, SERVE_DECODE):
+        steps += [{n: to_dev(a, dt if n in ("q", "k", "v") else torch.float32, torch) for n, a in st.items()}
+                  for st in blk]
+    S = torch.empty((wp.B, wp.H, wp.dv, wp.dk), dtype=torch.float32, device="cuda")
+    o_pf = torch.empty((wp.B, wp.H, wp.T, wp.dv), dtype=torch.float32, device="cuda")
+    o_dec = torch.empty((wd.B, wd.H, 1, wd.dv), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+
+    def loop(timed):
+        if timed:
+            ev[0].record(stream)
+        gdn.chunk_fwd(q, k, v, g, beta, S0, update=wp.update, gate=wp.gate, o=o_pf, S_T=S)
+        if timed:
+            ev[1].record(stream)
+        for st in steps:
+            gdn.decode_step(st["q"], st["k"], st["v"], st["g"], st["beta"], S, update=wd.update, gate=wd.gate,
+                            o=o_dec)
+        if timed:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        loop(False)
+    torch.cuda.synchronize()
+    tot, pf = [], []
+    for _ in range(reps):
+        loop(True)
+        torch.cuda.synchronize()
+        tot.append(ev[0].elapsed_time(ev[2]))
+        pf.append(ev[0].elapsed_time(ev[1]))
+    if gdn.device_status() != 0:
+        raise RuntimeError("device status after the serving loop")
+    ms, ms_pf = sorted(tot)[len(tot) // 2], sorted(pf)[len(pf) // 2]
+    return ms, ms_pf, (ms - ms_pf) / SERVE_DECODE
+
+
 def time_backward(w, steps, torch, gdn, warmup=1):
     """Device time of gdn_chunk_bwd (gradients of the prefill) on workload ``w``
     with random upstream gradients of o and S_T; returns ms per call."""
@@ -502,6 +562,12 @@ def run_ours(args):
         if rank == 0:
             print(json.dumps({"only": "decode", "ms_per_step": ms_d}), flush=True)
         return
+    if args.only == "serving":
+        ms_sv, ms_pf, ms_dec = time_serving_loop(3, torch, gdn)
+        if rank == 0:
+            print(json.dumps({"only": "serving", "ms_per_loop": ms_sv, "ms_prefill": ms_pf,
+                              "ms_per_decode_step": ms_dec}), flush=True)
+        return
     if args.only == "decode_multi":
         wd = WORKLOADS["decode_gdn_bf16"]
         ms_m = time_decode_multi(wd, 4, 25 if args.quick else 100, torch, gdn)
@@ -611,6 +677,16 @@ def run_ours(args):
                                    "achieved_gbs": nb / (msn * 1e-3) / 1e9,
                                    "frac_of_roofline_time": nb / (peaks["hbm_gbs"] * 1e9) / (msn * 1e-3)}
         result["prefill_workloads"] = others
+        # the prefill -> decode serving loop (second workload)
+        ms_sv, ms_pf, ms_dec = time_serving_loop(3, torch, gdn)
+        ms_sv = max_over_ranks(ms_sv, dist, "cuda")
+        result["gpu_launches"] += 3 * (1 + SERVE_DECODE)
+        result["serving_loop"] = {
+            "B": SERVE_B, "H": SERVE_H, "prompt_tokens": SERVE_PROMPT, "decode_tokens": SERVE_DECODE,
+            "ms_per_loop": ms_sv, "ms_prefill": ms_pf, "ms_per_decode_step": ms_dec,
+            "tokens_per_s": SERVE_B * (SERVE_PROMPT + SERVE_DECODE) * world / (ms_sv * 1e-3),
+            "decode_tokens_per_s": SERVE_B * world / (ms_dec * 1e-3),
+            "note": "gdn_chunk_fwd writes S_T into the decode state, then gdn_decode_step runs in place"}
         # training backward (gdn_chunk_bwd) on the GDN workload
         nb_steps = 2
         msb = max_over_ranks(time_backward(w, nb_steps, torch, gdn), dist, "cuda")
@@ -716,7 +792,7 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="with --only prefill/backward: override B")
     ap.add_argument("--heads", type=int, default=0, help="with --only prefill/backward: override H")
     ap.add_argument("--seq-len", type=int, default=0, help="with --only prefill/backward: override T")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_multi", "backward"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_multi", "backward", "serving"], default="all",
                     help="profiling aid: run one part only (its line is not a benchmark result)")
     ap.add_argument("--launch-check", action="store_true",
                     help="test aid: run only the rank protocol on CPU (gloo), no GPU work")
