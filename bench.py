@@ -426,9 +426,12 @@ def time_serving_loop(reps, torch, gdn, warmup=1):
     return ms, ms_pf, (ms - ms_pf) / SERVE_DECODE
 
 
-def time_backward(w, steps, torch, gdn, warmup=1):
+def time_backward(w, steps, torch, gdn, warmup=1, saved=False):
     """Device time of gdn_chunk_bwd (gradients of the prefill) on workload ``w``
-    with random upstream gradients of o and S_T; returns ms per call."""
+    with random upstream gradients of o and S_T; returns ms per call.  With
+    ``saved``: a training step's forward gdn_chunk_fwd_states and then
+    gdn_chunk_bwd_states from its chunk states; returns (ms of the forward, ms
+    of the backward) per step."""
     x = make_prefill_inputs(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     q, k, v = to_dev(x["q"], dt, torch), to_dev(x["k"], dt, torch), to_dev(x["v"], dt, torch)
@@ -438,6 +441,26 @@ def time_backward(w, steps, torch, gdn, warmup=1):
     dO = torch.randn((w.B, w.H, w.T, w.dv), device="cuda", generator=gen)
     dST = torch.randn((w.B, w.H, w.dv, w.dk), device="cuda", generator=gen)
     ws = torch.empty(gdn.bwd_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv), dtype=torch.uint8, device="cuda")
+    if saved:
+        states = ws.view(torch.float32).view(w.B, w.H, (w.T + 63) // 64, w.dv, w.dk)
+        o = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device="cuda")
+        ST = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device="cuda")
+        stream = torch.cuda.current_stream()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        fw, bw = [], []
+        for it in range(warmup + steps):
+            ev[0].record(stream)
+            gdn.chunk_fwd(q, k, v, g, beta, S0, update=w.update, gate=w.gate, o=o, S_T=ST, states=states)
+            ev[1].record(stream)
+            gdn.chunk_bwd(q, k, v, g, beta, None, dO, dST, update=w.update, gate=w.gate, states=states)
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            if it >= warmup:
+                fw.append(ev[0].elapsed_time(ev[1]))
+                bw.append(ev[1].elapsed_time(ev[2]))
+        if gdn.device_status() != 0:
+            raise RuntimeError("device status after the saved-state training step")
+        return sum(fw) / len(fw), sum(bw) / len(bw)
 
     def step():
         gdn.chunk_bwd(q, k, v, g, beta, S0, dO, dST, update=w.update, gate=w.gate, workspace=ws)
@@ -580,9 +603,11 @@ def run_ours(args):
         w = w.with_(B=args.batch or w.B, H=args.heads or w.H, T=args.seq_len or w.T)
     if args.only == "backward":
         ms = time_backward(w, args.steps, torch, gdn, warmup=args.warmup)
+        msf_s, msb_s = time_backward(w, args.steps, torch, gdn, warmup=1, saved=True)
         if rank == 0:
             print(json.dumps({"only": "backward", "workload": w.name, "B": w.B, "H": w.H, "T": w.T,
-                              "ms_per_call": ms}), flush=True)
+                              "ms_per_call": ms, "saved_states": {"ms_forward": msf_s, "ms_backward": msb_s}}),
+                  flush=True)
         return
     x = make_prefill_inputs(w)
     if args.only == "prefill":
@@ -698,6 +723,14 @@ def run_ours(args):
                               "flops_per_call": fl, "achieved_tflops": fl / (msb * 1e-3) / 1e12,
                               "bound": "alu", "fp32_peak_tflops": fp32_peak,
                               "frac": fl / (msb * 1e-3) / 1e12 / fp32_peak}
+        # the same gradients from the chunk states a training forward saved
+        msf_s, msb_s = time_backward(w, nb_steps, torch, gdn, saved=True)
+        msf_s, msb_s = max_over_ranks(msf_s, dist, "cuda"), max_over_ranks(msb_s, dist, "cuda")
+        result["gpu_launches"] += (nb_steps + 1) * 6
+        result["backward"]["from_saved_states"] = {
+            "ms_forward_with_states": msf_s, "ms_backward": msb_s,
+            "note": "gdn_chunk_fwd_states (tensor-core forward writing the chunk-entry states), then "
+                    "gdn_chunk_bwd_states (no forward pass of its own)"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w)

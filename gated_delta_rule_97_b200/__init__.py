@@ -30,6 +30,7 @@ F32, BF16 = 0, 1
 
 DECODE_MAX_T = 16  # GDN_DECODE_MAX_T
 PRODUCT_MAX_NH = 16  # GDN_PRODUCT_MAX_NH
+CHUNK = 64  # chunk length of the saved states (gdn_chunk_fwd_states)
 GDN_OK = 0
 ERRORS = {-1: "GDN_ERR_ARG", -2: "GDN_ERR_ALIGN", -3: "GDN_ERR_UNSUPPORTED", -4: "GDN_ERR_CUDA",
           -5: "GDN_ERR_TIMEOUT", -6: "GDN_ERR_RANGE"}
@@ -100,6 +101,10 @@ def load():
     lib.gdn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_chunk_bwd.argtypes = [dp] + [vp] * 15 + [ctypes.c_size_t, vp]
     lib.gdn_chunk_bwd.restype = ctypes.c_int
+    lib.gdn_chunk_fwd_states.argtypes = [dp] + [vp] * 10
+    lib.gdn_chunk_fwd_states.restype = ctypes.c_int
+    lib.gdn_chunk_bwd_states.argtypes = [dp] + [vp] * 15
+    lib.gdn_chunk_bwd_states.restype = ctypes.c_int
     lib.gdn_strerror.argtypes = [ctypes.c_int]
     lib.gdn_strerror.restype = ctypes.c_char_p
     lib.gdn_device_status.argtypes = [ctypes.c_int]
@@ -182,8 +187,11 @@ def _check(t, name, shape, dtype=None):
 
 
 def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=None, o=None, S_T=None,
-              return_state=True, algo="auto", prologue=0, stream=None):
+              return_state=True, algo="auto", prologue=0, states=None, stream=None):
     """Prefill over T tokens (gdn_chunk_fwd).  Returns (o, S_T).
+
+    ``states``: a CUDA float32 tensor [B,H,ceil(T/64),dv,dk] that receives the
+    state entering every chunk (gdn_chunk_fwd_states, for chunk_bwd(states=...)).
 
     q, k [B,H,T,dk]; v [B,H,T,dv] (bf16 or fp32, same dtype); g [B,H,T] or
     [B,H,T,dk] fp32 (log of the gate) or None; beta [B,H,T] fp32 (delta);
@@ -212,6 +220,14 @@ def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=No
     _check(S_T, "S_T", (B, H, dv, dk), torch.float32)
     d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), _dtype_code(out_dtype), algo,
                   prologue=prologue)
+    if states is not None:
+        _check(states, "states", (B, H, (T + CHUNK - 1) // CHUNK, dv, dk), torch.float32)
+        with _on_device(q):
+            rc = load().gdn_chunk_fwd_states(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                             _ptr(S0), _ptr(o), _ptr(S_T), _ptr(states), _stream(stream, q))
+        if rc != GDN_OK:
+            raise GDNError(rc, "gdn_chunk_fwd_states")
+        return o, S_T
     with _on_device(q):
         rc = load().gdn_chunk_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
                                   _ptr(o), _ptr(S_T), _stream(stream, q))
@@ -513,12 +529,14 @@ def bwd_workspace_bytes(B, H, T, dk, dv) -> int:
 
 
 def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update, gate, workspace=None,
-              want_dS0=True, stream=None):
+              want_dS0=True, states=None, stream=None):
     """gdn_chunk_bwd: gradients of chunk_fwd for upstream gradients dO [B,H,T,dv]
     and dS_T [B,H,dv,dk] (fp32; None = 0).  Returns (dq, dk, dv, dg, dbeta, dS0),
     fp32, dg / dbeta None when the mode has no gate / write strength, dS0 None
     when ``want_dS0`` is false.  ``workspace``: a CUDA uint8 tensor of
-    bwd_workspace_bytes(...) bytes (allocated here when None)."""
+    bwd_workspace_bytes(...) bytes (allocated here when None).  With ``states``
+    (written by chunk_fwd(states=...)) the call is gdn_chunk_bwd_states: S0 and
+    the workspace are not used."""
     import torch
 
     B, H, T, dk = q.shape
@@ -540,6 +558,15 @@ def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update
     gb = torch.empty((B, H, T), **f32) if update == "delta" else None
     gS0 = torch.empty((B, H, dv, dk), **f32) if want_dS0 else None
     d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), F32)
+    if states is not None:
+        _check(states, "states", (B, H, (T + CHUNK - 1) // CHUNK, dv, dk), torch.float32)
+        with _on_device(q):
+            rc = load().gdn_chunk_bwd_states(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                             _ptr(states), _ptr(dO), _ptr(dS_T), _ptr(gq), _ptr(gk), _ptr(gv),
+                                             _ptr(gg), _ptr(gb), _ptr(gS0), _stream(stream, q))
+        if rc != GDN_OK:
+            raise GDNError(rc, "gdn_chunk_bwd_states")
+        return gq, gk, gv, gg, gb, gS0
     need = int(load().gdn_bwd_workspace_bytes(ctypes.byref(d)))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)

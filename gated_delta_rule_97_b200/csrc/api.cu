@@ -160,7 +160,7 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     if (BH == 0) return GDN_OK;
     if (d->T == 0) return from_cuda(gdn_launch_copy_state(S0, S_T, (long)n_S, st));
 
-    gdn::ChunkArgs a;
+    gdn::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
     a.status = status_ptr();
     a.diag = diag_ptr();
@@ -334,7 +334,7 @@ extern "C" int gdn_product_fwd(const gdn_desc_t *d, int nh, const void *q, const
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (BH == 0) return GDN_OK;
     if (d->T == 0) return from_cuda(gdn_launch_copy_state(S0, S_T, (long)n_S, st));
-    gdn::ChunkArgs a;
+    gdn::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
     a.status = status_ptr();
     a.diag = diag_ptr();
@@ -411,7 +411,7 @@ extern "C" int gdn_chunk_fwd_segmented(const gdn_desc_t *d, int nseg, const void
     sd.B = (int)BH;
     sd.H = nseg;
     sd.T = d->T / nseg;
-    gdn::ChunkArgs a;
+    gdn::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o;
     a.status = status_ptr();
     a.diag = diag_ptr();
@@ -468,7 +468,7 @@ extern "C" int gdn_segment_maps(const gdn_desc_t *d, const void *q, const void *
     if (d->T == 0) {
         if ((rc = from_cuda(gdn_launch_copy_state(nullptr, H, (long)BH * d->dv * d->dk, st))) != GDN_OK) return rc;
     } else {
-        gdn::ChunkArgs a;
+        gdn::ChunkArgs a{};
         a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = nullptr;
         a.status = status_ptr();
         a.diag = diag_ptr();
@@ -543,7 +543,7 @@ extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k
 int gdn_launch_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta, const float *S0,
                    const float *dO, const float *dST, float *dq, float *dk, float *dv, float *dg, float *dbeta,
                    float *dS0, float *ws, int BH, int T, int dk_, int dv_, int update, int gate, int in_bf16,
-                   cudaStream_t st);
+                   int skip_fwd, cudaStream_t st);
 
 extern "C" size_t gdn_bwd_workspace_bytes(const gdn_desc_t *d) {
     if (!d || validate_common(d) != GDN_OK) return 0;
@@ -551,10 +551,15 @@ extern "C" size_t gdn_bwd_workspace_bytes(const gdn_desc_t *d) {
     return (size_t)d->B * d->H * nch * d->dv * d->dk * sizeof(float);
 }
 
-extern "C" int gdn_chunk_bwd(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
-                             const float *beta, const float *S0, const float *dO, const float *dS_T, float *dq,
-                             float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
-                             size_t workspace_bytes, void *stream) {
+namespace {
+
+// gdn_chunk_bwd and gdn_chunk_bwd_states: `saved` holds the chunk-entry states
+// written by gdn_chunk_fwd_states (read only, the forward pass is skipped), or
+// is null and `workspace` receives them from the backward's own forward pass.
+int chunk_bwd_impl(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const float *S0, const float *saved, const float *dO, const float *dS_T,
+                   float *dq, float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
+                   size_t workspace_bytes, void *stream) {
     int rc = validate_common(d);
     if (rc != GDN_OK) return rc;
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
@@ -572,17 +577,18 @@ extern "C" int gdn_chunk_bwd(const gdn_desc_t *d, const void *q, const void *k, 
         if ((d->gate != GDN_GATE_NONE) != (g != nullptr) || (d->gate != GDN_GATE_NONE) != (dg != nullptr))
             return GDN_ERR_ARG;
     }
-    const void *ptrs[] = {q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace};
+    const void *ptrs[] = {q, k, v, g, beta, S0, saved, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     const size_t need = gdn_bwd_workspace_bytes(d);
-    if (has_tokens && (!workspace || workspace_bytes < need)) return GDN_ERR_ARG;
+    if (has_tokens && !saved && (!workspace || workspace_bytes < need)) return GDN_ERR_ARG;
+    if (has_tokens && saved && workspace) return GDN_ERR_ARG;
     // outputs (and the workspace) against every input and against each other
     struct Span { const void *p; size_t n; };
     const Span ins[] = {{q, n_qk * es}, {k, n_qk * es}, {v, n_v * es}, {g, n_g * 4}, {beta, ntok * 4},
-                        {S0, n_S * 4}, {dO, n_v * 4}, {dS_T, n_S * 4}};
+                        {S0, n_S * 4}, {saved, has_tokens ? need : 0}, {dO, n_v * 4}, {dS_T, n_S * 4}};
     const Span outs[] = {{dq, n_qk * 4}, {dk, n_qk * 4}, {dv, n_v * 4}, {dg, n_g * 4}, {dbeta, ntok * 4},
-                         {dS0, n_S * 4}, {workspace, has_tokens ? need : 0}};
+                         {dS0, n_S * 4}, {workspace, has_tokens && !saved ? need : 0}};
     for (const Span &o : outs) {
         for (const Span &i : ins)
             if (overlaps(o.p, o.n, i.p, i.n)) return GDN_ERR_ARG;
@@ -592,7 +598,59 @@ extern "C" int gdn_chunk_bwd(const gdn_desc_t *d, const void *q, const void *k, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (BH == 0) return GDN_OK;
     if (d->T == 0) return dS0 ? from_cuda(gdn_launch_copy_state(dS_T, dS0, (long)n_S, st)) : GDN_OK;
-    return from_cuda(gdn_launch_bwd(q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0,
-                                    static_cast<float *>(workspace), (int)BH, d->T, d->dk, d->dv, d->update, d->gate,
-                                    d->dtype == GDN_BF16, st));
+    float *ws = saved ? const_cast<float *>(saved) : static_cast<float *>(workspace);
+    return from_cuda(gdn_launch_bwd(q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, ws, (int)BH, d->T,
+                                    d->dk, d->dv, d->update, d->gate, d->dtype == GDN_BF16, saved != nullptr, st));
+}
+
+}  // namespace
+
+extern "C" int gdn_chunk_bwd(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *S0, const float *dO, const float *dS_T, float *dq,
+                             float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    return chunk_bwd_impl(d, q, k, v, g, beta, S0, nullptr, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace,
+                          workspace_bytes, stream);
+}
+
+extern "C" int gdn_chunk_bwd_states(const gdn_desc_t *d, const void *q, const void *k, const void *v,
+                                    const float *g, const float *beta, const float *states, const float *dO,
+                                    const float *dS_T, float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                                    float *dS0, void *stream) {
+    if (d && (long)d->B * d->H * d->T > 0 && !states) return GDN_ERR_ARG;
+    return chunk_bwd_impl(d, q, k, v, g, beta, nullptr, states, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, nullptr, 0,
+                          stream);
+}
+
+extern "C" int gdn_chunk_fwd_states(const gdn_desc_t *d, const void *q, const void *k, const void *v,
+                                    const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                                    float *states, void *stream) {
+    const int rc = chunk_fwd_check(d, q, k, v, g, beta, S0, o, S_T);
+    if (rc != GDN_OK) return rc;
+    if (d->prologue != 0 || d->algo == GDN_ALGO_SIMT || !gdn_tc_supported(d)) return GDN_ERR_UNSUPPORTED;
+    const long BH = (long)d->B * d->H;
+    const size_t n_S = (size_t)BH * d->dv * d->dk;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (BH == 0) return GDN_OK;
+    if (d->T == 0) return from_cuda(gdn_launch_copy_state(S0, S_T, (long)n_S, st));
+    if (!states) return GDN_ERR_ARG;
+    if (!aligned16(states)) return GDN_ERR_ALIGN;
+    const size_t ns = gdn_bwd_workspace_bytes(d);
+    const size_t es = elem_size(d->dtype), eo = elem_size(d->out_dtype);
+    const size_t ntok = (size_t)BH * d->T;
+    const size_t n_qk = ntok * d->dk, n_v = ntok * d->dv;
+    const size_t n_g = d->gate == GDN_GATE_CHANNEL ? n_qk : ntok;
+    if (overlaps(states, ns, q, n_qk * es) || overlaps(states, ns, k, n_qk * es) || overlaps(states, ns, v, n_v * es) ||
+        overlaps(states, ns, g, n_g * 4) || overlaps(states, ns, beta, ntok * 4) || overlaps(states, ns, S0, n_S * 4) ||
+        overlaps(states, ns, o, n_v * eo) || overlaps(states, ns, S_T, n_S * 4))
+        return GDN_ERR_ARG;
+    gdn::ChunkArgs a{};
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
+    a.status = status_ptr();
+    a.diag = diag_ptr();
+    a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
+    a.nh = 1;
+    a.mode = gdn::kModeSaveStates;
+    a.states = states;
+    return from_cuda(gdn_launch_chunk_tc2(a, d, st));
 }

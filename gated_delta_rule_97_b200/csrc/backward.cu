@@ -12,7 +12,8 @@
 // consecutive rows, lane l holds key channels [l V, l V + V), V = dk / 32.
 //
 //   phase 1: the forward recurrence from S0, storing the state entering every
-//            chunk of kChunkB = 64 tokens into the workspace;
+//            chunk of kChunkB = 64 tokens into the workspace (skipped when the
+//            tensor-core forward saved those states already);
 //   phase 2: the chunks in reverse.  A chunk is recomputed forward from its
 //            stored state, keeping the state entering each sub-block of kSub =
 //            8 tokens in shared memory (each thread keeps only its own
@@ -50,6 +51,7 @@ struct BwdArgs {
     float *dq, *dk, *dv, *dg, *dbeta, *dS0;
     float *ws;  // [BH][nchunks][dv][DK]: the state entering every chunk
     int BH, T, DV, nch;  // DV: value dimension
+    int skip_fwd;        // ws already holds the states (a forward wrote them): no phase 1
 };
 
 __device__ __forceinline__ float bwd_warp_sum(float x) {
@@ -251,6 +253,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
     const int ns = (T + kSub - 1) / kSub;
     const int last = a.nch - 1;
     const int nvis = ns + 2 * ((T - last * kChunkB + kSub - 1) / kSub) + last * 2 * (kChunkB / kSub);
+    const int n0 = a.skip_fwd ? ns : 0;  // first visit
 
     float s[kRows][V], ds[kRows][V];
 #pragma unroll
@@ -262,15 +265,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
         }
     StageRegs<DK, UPD, GATE, TIn> R;
     {
-        const Visit v0 = visit_at(0, T, a.nch);
+        const Visit v0 = visit_at(n0, T, a.nch);
         R.load(a, bh, v0.tb, rslice, t_, v0.phase != 1);
         R.store(stg, t_);
     }
     __syncthreads();
     int par = 0;  // parity of the reduction buffer
-    for (int n = 0; n < nvis; ++n) {
+    for (int n = n0; n < nvis; ++n) {
         const Visit vi = visit_at(n, T, a.nch);
-        const float *st = stg + (n & 1) * SL::FLOATS;
+        const float *st = stg + ((n - n0) & 1) * SL::FLOATS;
         if (n + 1 < nvis) {
             const Visit vn = visit_at(n + 1, T, a.nch);
             R.load(a, bh, vn.tb, rslice, t_, vn.phase != 1);
@@ -451,7 +454,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
         }
         // the next visit's inputs into the other buffer (its last readers passed the
         // barrier that ended the previous visit)
-        if (n + 1 < nvis) R.store(stg + ((n + 1) & 1) * SL::FLOATS, t_);
+        if (n + 1 < nvis) R.store(stg + ((n + 1 - n0) & 1) * SL::FLOATS, t_);
         __syncthreads();
     }
     if (a.dS0) {
@@ -494,7 +497,7 @@ int launch_bwd_modes(const BwdArgs &a, int update, int gate, cudaStream_t st) {
 int gdn_launch_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta, const float *S0,
                    const float *dO, const float *dST, float *dq, float *dk, float *dv, float *dg, float *dbeta,
                    float *dS0, float *ws, int BH, int T, int dk_, int dv_, int update, int gate, int in_bf16,
-                   cudaStream_t st) {
+                   int skip_fwd, cudaStream_t st) {
     using namespace gdn;
     const size_t ntok = (size_t)BH * T;
     cudaError_t e = cudaMemsetAsync(dq, 0, ntok * dk_ * sizeof(float), st);
@@ -508,6 +511,7 @@ int gdn_launch_bwd(const void *q, const void *k, const void *v, const float *g, 
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta; a.dS0 = dS0; a.ws = ws;
     a.BH = BH; a.T = T; a.DV = dv_;
     a.nch = (T + kChunkB - 1) / kChunkB;
+    a.skip_fwd = skip_fwd;
     if (dk_ == 128)
         return in_bf16 ? launch_bwd_modes<128, __nv_bfloat16>(a, update, gate, st)
                        : launch_bwd_modes<128, float>(a, update, gate, st);

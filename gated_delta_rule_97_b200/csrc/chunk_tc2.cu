@@ -86,7 +86,8 @@ struct Params {
     // and the rows of a chunk that are a token's first / last substep (bit l = row l)
     unsigned long long firstmask, lastmask;
     int pro;   // GDN_PRO_* input maps
-    int mode;  // kMode* bits (internal passes of the segmented prefill)
+    int mode;  // kMode* bits (internal passes of the segmented prefill, saved states)
+    float *states;  // kModeSaveStates: the chunk-entry states [BH][nchunks][dv][dk]
 };
 
 template <int DVS, int GATE>
@@ -1062,6 +1063,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 }
                 sv[j] = x.x; sv[j + 1] = x.y; sv[j + 2] = x.z; sv[j + 3] = x.w;
             }
+            if ((mode & kModeSaveStates) && has_row && nchunks > 0) {  // the state entering chunk 0
+                float *st = p.states + ((size_t)bh * nchunks * dv + v0 + vrow) * DK + h * 64;
+#pragma unroll
+                for (int j = 0; j < 64; j += 4)
+                    __stcs(reinterpret_cast<float4 *>(st + j), make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]));
+            }
             __syncwarp();
             tmem_st32f(lane_addr + TSM + h * 64, sv);
             tmem_st32f(lane_addr + TSM + h * 64 + 32, sv + 32);
@@ -1294,6 +1301,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     w[c] = pack_h2(sv[2 * c], sv[2 * c + 1]);
                 }
                 tmem_st32(lane_addr + TS16 + h * 32, w);
+                if ((mode & kModeSaveStates) && has_row && more) {  // the state entering chunk r + 1
+                    float *st = p.states + (((size_t)bh * nchunks + r + 1) * dv + v0 + vrow) * DK + h * 64;
+#pragma unroll
+                    for (int j = 0; j < 64; j += 4)
+                        __stcs(reinterpret_cast<float4 *>(st + j), make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]));
+                }
                 if (GATE != kGateNone && more) {
 #pragma unroll
                     for (int i = 0; i < 64; ++i)
@@ -1455,6 +1468,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     }
     prm.pro = a.pro;
     prm.mode = a.mode;
+    prm.states = a.states;
     const long grid = (long)a.BH * prm.nslices;
     if (grid == 0) return 0;
     if (nh > 1) {

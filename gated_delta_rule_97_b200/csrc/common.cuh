@@ -50,12 +50,17 @@ struct ChunkArgs {
     int nh;
     int pro;   // GDN_PRO_* input maps
     int mode;  // kMode* bits (internal passes of the segmented prefill), 0 = plain
+    float *states;  // kModeSaveStates: the chunk-entry states, else null
 };
 
 // Internal pass modes: values taken as zero (v not read), no output written,
 // initial state the identity (dv == dk); with all three the pass yields the
 // transition of the sequence (S_T = S0 Lambda with S0 = I).
 constexpr int kModeZeroV = 1, kModeNoOut = 2, kModeS0Eye = 4;
+// Forward for training: the state entering every chunk (before that chunk's
+// decay) is also written to ChunkArgs::states [BH][nchunks][dv][dk], for the
+// backward pass to start from.
+constexpr int kModeSaveStates = 8;
 // The tensor-core kernel runs kModeS0Eye from kEyeScale * I and stores S_T /
 // kEyeScale (exact, a power of two): a transition that decays far below 1 then
 // stays in fp16's normal range in the state's fp16 operand copy, while entries

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define GDN_VERSION 5
+#define GDN_VERSION 6
 
 /* Return codes. */
 #define GDN_OK 0
@@ -341,6 +341,32 @@ int gdn_chunk_bwd(const gdn_desc_t *desc, const void *q, const void *k, const vo
                   const float *beta, const float *S0, const float *dO, const float *dS_T, float *dq, float *dk,
                   float *dv, float *dg, float *dbeta, float *dS0, void *workspace, size_t workspace_bytes,
                   void *stream);
+
+/*
+ * gdn_chunk_fwd_states -- gdn_chunk_fwd for training: the same o and S_T, and
+ * in `states` the state entering every chunk of 64 tokens (before that chunk's
+ * first decay; chunk 0's is S0), the chunk-boundary states that training keeps
+ * ("Linear Attention, Visualized", "Update the state").  Runs the pipelined
+ * tensor-core kernel, so the request must be one it serves: bf16 inputs,
+ * dk = 128, dv in {64, 128}, prologue 0, algo AUTO or TC (GDN_ERR_UNSUPPORTED
+ * otherwise).  The states carry that kernel's rounding (fp16 operands, fp32
+ * accumulation).
+ *
+ *   states   [B,H,ceil(T/64),dv,dk] float, gdn_bwd_workspace_bytes(desc) bytes,
+ *            16-byte aligned, owned by the caller; overlaps no other argument
+ *            (GDN_ERR_ARG).  Not written when T == 0.
+ *   others   as for gdn_chunk_fwd.
+ *
+ * gdn_chunk_bwd_states -- gdn_chunk_bwd from those saved states: the backward's
+ * own forward pass over the sequence is skipped (each chunk is still recomputed
+ * from its saved state).  Arguments as for gdn_chunk_bwd, with `states` (read
+ * only; required when B*H*T > 0) in place of S0 and the workspace.
+ */
+int gdn_chunk_fwd_states(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, const float *S0, void *o, float *S_T, float *states, void *stream);
+int gdn_chunk_bwd_states(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, const float *states, const float *dO, const float *dS_T, float *dq,
+                         float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *stream);
 
 /*
  * gdn_device_status -- synchronises the current device, then returns the

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_strerror_and_version(lib):
-    assert gdn.version() == 5  # the backward pass joined the boundary
+    assert gdn.version() == 6  # saved chunk states for the backward joined the boundary
     for code in (0, -1, -2, -3, -4, -5, -6, 123):
         assert isinstance(gdn.strerror(code), str) and gdn.strerror(code)
 
@@ -234,3 +234,28 @@ def test_backward_rejects_bad_arguments(lib):
     assert f(ctypes.byref(p), *ins, *outs, ws, need, None) == -3              # input maps not differentiated
     e = _desc(B=0)
     assert f(ctypes.byref(e), *ins, *outs, ws, 0, None) == 0                   # empty batch: no-op
+
+
+def test_saved_state_entry_points_reject_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    lib.gdn_chunk_fwd_states.argtypes = [ctypes.c_void_p] + [ctypes.c_void_p] * 10
+    lib.gdn_chunk_bwd_states.argtypes = [ctypes.c_void_p] + [ctypes.c_void_p] * 15
+    fw = lambda d, states: lib.gdn_chunk_fwd_states(ctypes.byref(d), vp(0x10000), vp(0x20000), vp(0x30000),
+                                                     vp(0x40000), vp(0x50000), None, vp(0x9000000), None,
+                                                     states, None)
+    d = _desc()
+    assert fw(d, None) == -1                                  # no states buffer
+    assert fw(d, vp(0x7000008)) == -2                         # misaligned
+    assert fw(d, vp(0x10000)) == -1                           # overlaps q
+    assert fw(_desc(dtype=gdn.F32), vp(0x70000000)) == -3     # the tensor-core forward takes bf16 only
+    d = _desc()
+    d.prologue = 1
+    assert fw(d, vp(0x70000000)) == -3                        # no input prologue with saved states
+    bw = lambda d, states: lib.gdn_chunk_bwd_states(ctypes.byref(d), vp(0x10000), vp(0x20000), vp(0x30000),
+                                                     vp(0x40000), vp(0x50000), states, None, None,
+                                                     vp(0x1000000), vp(0x2000000), vp(0x3000000),
+                                                     vp(0x4000000), vp(0x5000000), None, None)
+    assert bw(_desc(), None) == -1                            # states required
+    d = _desc()
+    d.prologue = 1
+    assert bw(d, vp(0x70000000)) == -3

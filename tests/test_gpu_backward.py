@@ -103,3 +103,71 @@ def test_backward_empty_sequence_copies_state_gradient():
                         update="delta", gate="none")
     torch.cuda.synchronize()
     assert torch.equal(out[5], dST) and out[0].numel() == 0
+
+
+# ----------------------------------------------------------------------------
+# Saved chunk states: gdn_chunk_fwd_states writes the state entering every chunk
+# of 64 tokens (the tensor-core forward, fp16 operands), gdn_chunk_bwd_states
+# starts from them.  Their rounding bounds these cases, so the bound is the
+# bf16 one of the forward parity tests.
+TOL_STATES = 2e-2
+
+
+def _dev_inputs(x):
+    q, k, v, g, beta, S0, dO, dST = x
+    dt = torch.bfloat16
+    return dev(q, dt), dev(k, dt), dev(v, dt), dev(g), dev(beta), dev(S0), dev(dO), dev(dST)
+
+
+@pytest.mark.parametrize("update,gate", MODES)
+@pytest.mark.parametrize("dv,T", [(128, 150), (64, 64), (128, 1)])
+def test_forward_states_are_the_chunk_boundary_states(update, gate, dv, T):
+    x = inputs(17, update, gate, T=T, dv=dv, bf16=True)
+    q, k, v, g, beta, S0 = _dev_inputs(x)[:6]
+    nch = (T + 63) // 64
+    states = torch.empty((1, 2, nch, dv, 128), dtype=torch.float32, device="cuda")
+    gdn.device_status(clear=True)
+    o1, S1 = gdn.chunk_fwd(q, k, v, g, beta, S0, update=update, gate=gate, states=states)
+    o2, S2 = gdn.chunk_fwd(q, k, v, g, beta, S0, update=update, gate=gate, algo="tc")
+    torch.cuda.synchronize()
+    assert gdn.device_status(clear=True) == 0
+    # the same forward as the plain tensor-core call
+    assert rel_err(np64(o1), np64(o2)) <= 1e-6 and rel_err(np64(S1), np64(S2)) <= 1e-6
+    qn, kn, vn, gn, bn, S0n = x[:6]
+    for c in range(nch):
+        if c == 0:
+            ref = S0n
+        else:
+            t = 64 * c
+            sl = lambda a: None if a is None else np.ascontiguousarray(a[:, :, :t])
+            _, ref = oracle.gdn_forward(update, gate, sl(qn), sl(kn), sl(vn), g=sl(gn), beta=sl(bn), S0=S0n)
+        assert rel_err(np64(states[:, :, c]), ref) <= TOL_STATES, c
+
+
+@pytest.mark.parametrize("update,gate", MODES)
+@pytest.mark.parametrize("dv,T", [(128, 150), (64, 200)])
+def test_backward_from_saved_states(update, gate, dv, T):
+    x = inputs(23, update, gate, T=T, dv=dv, bf16=True)
+    q, k, v, g, beta, S0, dO, dST = _dev_inputs(x)
+    states = torch.empty((1, 2, (T + 63) // 64, dv, 128), dtype=torch.float32, device="cuda")
+    gdn.device_status(clear=True)
+    gdn.chunk_fwd(q, k, v, g, beta, S0, update=update, gate=gate, states=states)
+    got = gdn.chunk_bwd(q, k, v, g, beta, None, dO, dST, update=update, gate=gate, states=states)
+    plain = gdn.chunk_bwd(q, k, v, g, beta, S0, dO, dST, update=update, gate=gate)
+    torch.cuda.synchronize()
+    assert gdn.device_status(clear=True) == 0
+    ref = oracle.gdn_backward_np(update, gate, *x)
+    for name, a, b, c in zip(["dq", "dk", "dv", "dg", "dbeta", "dS0"], got, ref, plain):
+        if b is None:
+            assert a is None, name
+            continue
+        assert rel_err(np64(a), b) <= TOL_STATES, (name, rel_err(np64(a), b))
+        assert rel_err(np64(a), np64(c)) <= TOL_STATES, name
+
+
+def test_saved_states_reject_requests_the_tensor_core_forward_cannot_serve():
+    x = inputs(29, "delta", "scalar", T=70, dv=128)
+    q, k, v, g, beta, S0 = (dev(a) for a in x[:6])  # fp32 inputs
+    states = torch.empty((1, 2, 2, 128, 128), dtype=torch.float32, device="cuda")
+    with pytest.raises(gdn.GDNError):
+        gdn.chunk_fwd(q, k, v, g, beta, S0, update="delta", gate="scalar", states=states)
