@@ -42,7 +42,7 @@ def test_la_matches_oracle(T, dv):
 
 
 def test_la_wide_value_slice():
-    """More heads than SMs: each CTA takes all 128 value rows (M = 128 MMAs)."""
+    """More heads than SMs: 320 CTAs of 64 value rows, in several waves."""
     w = workload(130, B=2, H=80)
     check(w, make_prefill_inputs(w))
 
@@ -107,3 +107,15 @@ def test_la_state_chains_across_calls():
     torch.cuda.synchronize()
     assert rel_err(np64(torch.cat([oa, ob], dim=2)), np64(o)) <= 1e-5
     assert rel_err(np64(Sb), np64(S)) <= 1e-5
+
+
+def test_la_state_in_place():
+    """S_T may be S0 itself: each CTA reads its rows of S0 before it writes them."""
+    w = workload(200, B=2, H=3)
+    x = make_prefill_inputs(w)
+    t = {k_: dev(x[k_], torch.bfloat16) for k_ in ("q", "k", "v")}
+    o1, S1 = gdn.chunk_fwd(t["q"], t["k"], t["v"], None, None, dev(x["S0"]), update="additive", gate="none")
+    S = dev(x["S0"])
+    o2, S2 = gdn.chunk_fwd(t["q"], t["k"], t["v"], None, None, S, update="additive", gate="none", S_T=S)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2) and S2.data_ptr() == S.data_ptr()

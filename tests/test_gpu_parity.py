@@ -163,6 +163,45 @@ def test_decode_multi_token_all_modes(update, gate, T):
     assert rel_err(np64(o), ro) <= TOL["bf16"] and rel_err(np64(S), rS) <= TOL["bf16"]
 
 
+def _decode_multi_case(update, gate, dtype, T, dk, dv, B, H, seed=3, gfix=None):
+    w = small_workload(update, gate, dtype, T=1, dk=dk, dv=dv, B=B, H=H, seed=seed).with_(steps=T, q_map="none")
+    steps = make_decode_inputs(w, T)
+    if gfix is not None:  # a fixed log-gate per token
+        for s_ in steps:
+            s_["g"] = np.full_like(s_["g"], gfix)
+    x = _stack_steps(steps)
+    S0 = np.random.default_rng(seed).standard_normal((B, H, dv, dk)).astype(np.float32) * 0.05
+    S = dev(S0)
+    io = torch.bfloat16 if dtype == "bf16" else torch.float32
+    d = {k_: (None if v_ is None else dev(v_, io if k_ in ("q", "k", "v") else torch.float32)) for k_, v_ in x.items()}
+    o = gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], S, update=update, gate=gate)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    ro, rS = oracle.decode_sequence(update, gate, S0, steps)
+    eo, es = rel_err(np64(o), ro), rel_err(np64(S), rS)
+    assert eo <= TOL[dtype] and es <= TOL[dtype], (eo, es)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 64), (64, 128)])
+@pytest.mark.parametrize("update,gate", [("delta", "scalar"), ("delta", "channel"), ("additive", "none")])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_multi_token_head_dims(dk, dv, update, gate, dtype):
+    # the persistent kernel's other layouts: dk = 64 (two column blocks per lane), 4 tasks per head at dv = 64
+    _decode_multi_case(update, gate, dtype, T=3, dk=dk, dv=dv, B=3, H=7)
+
+
+def test_decode_multi_token_deep_scalar_decay():
+    # g = -30 per token: the carried decay factor falls below 2^-64 after three tokens and is folded
+    # into the rows (fp32 inputs, fp32 bound)
+    _decode_multi_case("delta", "scalar", "f32", T=9, dk=128, dv=128, B=2, H=3, gfix=-30.0)
+
+
+def test_decode_multi_token_many_tasks_per_warp():
+    # more 16-row tasks (4096) than warps of the persistent grid: every warp walks several tasks and
+    # its two state slots cycle through their mbarrier phases
+    _decode_multi_case("delta", "scalar", "bf16", T=4, dk=128, dv=128, B=16, H=32, seed=9)
+
+
 def test_decode_multi_token_equals_single_steps():
     w = small_workload("delta", "channel", "f32", T=1, dk=128, dv=128, B=2, H=3).with_(steps=8, q_map="none")
     steps = make_decode_inputs(w, 8)
