@@ -54,6 +54,23 @@ struct BwdArgs {
     int skip_fwd;        // ws already holds the states (a forward wrote them): no phase 1
 };
 
+// Warp sums of four per-lane partials x[0..3] (one per row of the warp), every
+// sum returned to every lane: a transposing butterfly (6 shuffles, after which
+// lane l holds the sum of row (l >> 3) & 3), then one broadcast per row.
+__device__ __forceinline__ void warp_sum_rows(float (&x)[kRows]) {
+    static_assert(kRows == 4, "four rows per warp");
+    const int lane = threadIdx.x & 31;
+    const bool b4 = lane & 16, b3 = lane & 8;
+    const float a0 = (b4 ? x[2] : x[0]) + __shfl_xor_sync(0xffffffffu, b4 ? x[0] : x[2], 16);
+    const float a1 = (b4 ? x[3] : x[1]) + __shfl_xor_sync(0xffffffffu, b4 ? x[1] : x[3], 16);
+    float b = (b3 ? a1 : a0) + __shfl_xor_sync(0xffffffffu, b3 ? a0 : a1, 8);
+    b += __shfl_xor_sync(0xffffffffu, b, 4);
+    b += __shfl_xor_sync(0xffffffffu, b, 2);
+    b += __shfl_xor_sync(0xffffffffu, b, 1);
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) x[r] = __shfl_sync(0xffffffffu, b, ((r >> 1) << 4) | ((r & 1) << 3));
+}
+
 __device__ __forceinline__ float bwd_warp_sum(float x) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
@@ -163,10 +180,7 @@ __device__ __forceinline__ void fwd_write(float (&s)[kRows][V], const float *k, 
             for (int e = 0; e < V; ++e) x = fmaf(s[r][e], k[e], x);
             p[r] = x;
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) p[r] += __shfl_xor_sync(0xffffffffu, p[r], off);
+        warp_sum_rows(p);
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
             rr[r] = v[r] - p[r];
@@ -376,10 +390,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs a) {
                     }
                     du[r] = acc;
                 }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-                    for (int r = 0; r < kRows; ++r) du[r] += __shfl_xor_sync(0xffffffffu, du[r], off);
+                warp_sum_rows(du);
                 float dvt[kRows], dbp = 0.f;
 #pragma unroll
                 for (int r = 0; r < kRows; ++r) {
