@@ -101,6 +101,8 @@ def load():
     lib.gdn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_chunk_bwd.argtypes = [dp] + [vp] * 15 + [ctypes.c_size_t, vp]
     lib.gdn_chunk_bwd.restype = ctypes.c_int
+    lib.gdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.gdn_set_wait_limit_ns.restype = ctypes.c_int
     lib.gdn_chunk_fwd_states.argtypes = [dp] + [vp] * 10
     lib.gdn_chunk_fwd_states.restype = ctypes.c_int
     lib.gdn_chunk_bwd_states.argtypes = [dp] + [vp] * 15
@@ -131,6 +133,12 @@ def device_status(clear: bool = True) -> int:
 def device_diag() -> int:
     """Where the first recorded kernel timeout happened (0 if none)."""
     return int(load().gdn_device_diag())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Bound of the kernels' hand-off waits in ns (0 = the default, 1 s): a test
+    hook for the timeout path (gdn_set_wait_limit_ns)."""
+    load().gdn_set_wait_limit_ns(ctypes.c_ulonglong(int(ns)))
 
 
 def _ptr(t):

@@ -81,6 +81,16 @@ bool tc2_prologue_ok(const gdn_desc_t *) { return true; }
 
 }  // namespace
 
+// Bound of the kernels' hand-off waits in ns (0 = the default, 1 s); a test
+// hook (gdn_set_wait_limit_ns), read by the launchers.
+static unsigned long long g_wait_limit_ns = 0;
+unsigned long long gdn_wait_limit_ns() { return g_wait_limit_ns; }
+
+extern "C" int gdn_set_wait_limit_ns(unsigned long long ns) {
+    g_wait_limit_ns = ns;
+    return GDN_OK;
+}
+
 extern "C" int gdn_version(void) { return GDN_VERSION; }
 
 extern "C" const char *gdn_strerror(int code) {
@@ -534,6 +544,7 @@ extern "C" int gdn_decode_step(const gdn_desc_t *d, const void *q, const void *k
     a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
     a.pro = d->prologue;
     a.status = status_ptr();
+    a.wait_ns = g_wait_limit_ns;
     return from_cuda(gdn_launch_decode(a, d->update, d->gate, d->dtype == GDN_BF16, d->out_dtype == GDN_BF16,
                                        static_cast<cudaStream_t>(stream)));
 }

@@ -53,6 +53,7 @@ struct LAParams {
     float *ST;
     int *status;
     int BH, T, dv, nslices;
+    unsigned long long wait_ns;  // bound of the hand-off waits (gdn_set_wait_limit_ns)
 };
 
 // Stage: Q then K, each [2 key halves][128 rows][64] bf16 (16 KB per half),
@@ -125,10 +126,11 @@ __global__ void __launch_bounds__(kLAThreads, 1) chunk_la_kernel(const __grid_co
 
     // a wait that runs out stops every role (each then finds its next wait cut
     // short too); the waits on the chunk-to-chunk chain poll without suspending
+    const uint64_t wlim = p.wait_ns ? p.wait_ns : 1000000000ull;
     auto wait = [&](uint64_t *bar, uint32_t par) -> bool {
         if (mbar_test_wait(bar, par)) return true;
         if (*reinterpret_cast<volatile int *>(&bs.abort_flag)) return false;
-        if (mbar_wait_spin(bar, par)) return true;
+        if (wlim >= 1000ull && mbar_wait_spin(bar, par, wlim)) return true;  // under 1 us: no waiting
         if (atomicExch(&bs.abort_flag, 1) == 0) record_status(p.status, kStatusTimeout);
         return false;
     };
@@ -379,6 +381,8 @@ int launch_la(const LAParams &prm, int grid, cudaStream_t stream) {
 }  // namespace
 }  // namespace gdn
 
+unsigned long long gdn_wait_limit_ns();  // api.cu
+
 // The request this kernel serves: additive update without gate, bf16 inputs,
 // dk = 128, dv in {64, 128}, no input prologue, a plain forward (no internal
 // pass mode).
@@ -402,6 +406,7 @@ int gdn_launch_chunk_la(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream
     prm.S0 = a.S0;
     prm.ST = a.ST;
     prm.status = a.status;
+    prm.wait_ns = gdn_wait_limit_ns();
     prm.BH = a.BH;
     prm.T = a.T;
     prm.dv = a.dv;

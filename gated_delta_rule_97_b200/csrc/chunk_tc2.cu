@@ -88,6 +88,7 @@ struct Params {
     int pro;   // GDN_PRO_* input maps
     int mode;  // kMode* bits (internal passes of the segmented prefill, saved states)
     float *states;  // kModeSaveStates: the chunk-entry states [BH][nchunks][dv][dk]
+    unsigned long long wait_ns;  // bound of the hand-off waits (gdn_set_wait_limit_ns)
 };
 
 template <int DVS, int GATE>
@@ -117,9 +118,10 @@ struct Misc {
     float beta[2][64];  // by chunk parity: the solve of chunk r overlaps the gate pass of r+1
     float GC[128];
     int abort_flag, range_flag, slow_chunk, abort_site;
-    int p_abort, s_abort, pad0, pad1;
+    int p_abort, s_abort, n_tma, n_tv;  // n_tma / n_tv: phases armed on bar_tma / bar_tv
     uint32_t tmem_base, pad2[3];
     uint64_t bar_tma, bar_p1, bar_x, bar_rdy, bar_fA, bar_fB0, bar_fB1, bar_tv;
+    uint64_t bar_drain;  // after a timeout: every MMA issued has completed
 };
 
 static_assert(sizeof(Misc) <= 3072, "the Misc block has 3 KB of shared memory");
@@ -180,6 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     constexpr bool DELTA = (UPD == kDelta);
     const int pro = EXT ? p.pro : 0;
     const int mode = EXT ? p.mode : 0;
+    // the hand-off waits, bounded (1 s unless a test shortens it)
+    const uint64_t wlim = p.wait_ns ? p.wait_ns : 1000000000ull;
+    auto mwait = [wlim](uint64_t *bar, uint32_t par) { return mbar_wait_bounded(bar, par, wlim); };
     // P = [Q;K]K^T of a chunk is issued by the state group's MMA thread right after
     // rdy when the prep group is the longer side (delta rule, scalar / no gate), else
     // by the prep group itself (it then has slack; the channel gate's P also needs
@@ -216,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     if (t == 0) {
         mbar_init(&ms.bar_tma, 1);
         mbar_init(&ms.bar_tv, 1);
+        mbar_init(&ms.bar_drain, 2);  // the two MMA-issuing threads
         mbar_init(&ms.bar_p1, 1);
         mbar_init(&ms.bar_x, 1);
         mbar_init(&ms.bar_rdy, 1);
@@ -227,6 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         ms.range_flag = 0;
         ms.p_abort = 0;
         ms.s_abort = 0;
+        ms.n_tma = 0;
+        ms.n_tv = 0;
         tma_prefetch_desc(&p.q_map);
         tma_prefetch_desc(&p.k_map);
         if (!(mode & kModeZeroV)) tma_prefetch_desc(&p.v_map);
@@ -326,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             const uint32_t bytes =
                 qbytes + 16384 + ((kSplitV || zeroV) ? 0 : DVS * 128) + (GATE == kGateChannel ? gbytes : 0);
             mbar_arrive_expect_tx(&ms.bar_tma, bytes);
+            ++ms.n_tma;
             for (int h = 0; h < 2; ++h) {
                 tma_load_3d(sm + L::RAW_QK + h * 16384, &p.q_map, h * 64, PROD ? r * TPC : t0, bh,
                             &ms.bar_tma);
@@ -338,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         };
         auto issue_tma_split_v = [&](int r) {
             mbar_arrive_expect_tx(&ms.bar_tv, DVS * 128);
+            ++ms.n_tv;
             issue_tma_v(r, &ms.bar_tv);
         };
         if (t == 0 && nchunks > 0) {
@@ -359,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             const int buf = r & 1;
             const float *bet = ms.beta[buf];
             TC2_MARK(0, 0);
-            if (!mbar_wait(&ms.bar_tma, ph)) note_timeout(ms, 1, r);
+            if (!mwait(&ms.bar_tma, ph)) note_timeout(ms, 1, r);
             if (PROD) {
                 // compact q rows j -> row (j + 1) * nh - 1, the rest zero (both key halves);
                 // the k rows past cv (the next chunk's first steps, loaded by the 64-row box)
@@ -525,23 +535,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             // A'[buf] and K>[buf] were last read by the state's chunk r-2
             if (r >= 2) {
                 uint64_t *fb = buf ? &ms.bar_fB1 : &ms.bar_fB0;
-                if (!mbar_wait(fb, ((r - 2) >> 1) & 1)) note_timeout(ms, 10, r);
+                if (!mwait(fb, ((r - 2) >> 1) & 1)) note_timeout(ms, 10, r);
             }
             // the history operands were last read by the state's chunk r-1: Q<, K<, V by
             // its first MMA group (bar_x; fA without the delta rule), T2 also by the
             // correction MMA (fA), the single V tile of the channel modes by its last MMAs
             auto wait_first_mmas = [&]() {
                 if (DELTA && r >= 1) {
-                    if (!mbar_wait(&ms.bar_x, (r - 1) & 1)) note_timeout(ms, 12, r);
+                    if (!mwait(&ms.bar_x, (r - 1) & 1)) note_timeout(ms, 12, r);
                 }
             };
             auto wait_history = [&]() {
                 if (r >= 1) {
                     if (DELTA || GATE != kGateChannel) {
-                        if (!mbar_wait(&ms.bar_fA, (r - 1) & 1)) note_timeout(ms, 9, r);
+                        if (!mwait(&ms.bar_fA, (r - 1) & 1)) note_timeout(ms, 9, r);
                     } else {
                         uint64_t *fb = ((r - 1) & 1) ? &ms.bar_fB1 : &ms.bar_fB0;
-                        if (!mbar_wait(fb, ((r - 1) >> 1) & 1)) note_timeout(ms, 10, r);
+                        if (!mwait(fb, ((r - 1) >> 1) & 1)) note_timeout(ms, 10, r);
                     }
                 }
             };
@@ -691,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 mma_commit(&ms.bar_p1);
             }
             TC2_MARK(0, 4);
-            if (!mbar_wait(&ms.bar_p1, ph)) note_timeout(ms, 2, r);
+            if (!mwait(&ms.bar_p1, ph)) note_timeout(ms, 2, r);
             TC2_MARK(0, 5);
             tc_fence_after();
 
@@ -900,7 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                     if (kSplitV && !zeroV) {
                         // V -> fp16 (its slot was released with bar_x(r-1), waited in the
                         // window), then the next chunk's v load
-                        if (!mbar_wait(&ms.bar_tv, ph)) note_timeout(ms, 13, r);
+                        if (!mwait(&ms.bar_tv, ph)) note_timeout(ms, 13, r);
                         constexpr int NV = 512 * NB, ITV = NV / 128;
                         const int wt = t - 128;
                         uint4 raw[ITV];
@@ -1030,7 +1040,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         // P = [Q;K] K^T of chunk r from the raw bf16 tiles, issued by this group's MMA
         // thread (the prep group's threads then never stall on the tensor pipe's queue)
         auto issue_p1 = [&](int r) {
-            if (!mbar_wait(&ms.bar_tma, r & 1)) note_timeout(ms, 11, r);
+            if (!mwait(&ms.bar_tma, r & 1)) note_timeout(ms, 11, r);
             tc_fence_after();
             const uint32_t qk = smem_u32(sm + L::RAW_QK);
             constexpr uint32_t id = idesc_f16(128, 64, 1, 0, 0);
@@ -1084,7 +1094,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
         // the first chunk's decay is applied here; later ones ride on the fp16
         // write-back at the end of the previous chunk
         if (nchunks > 0) {
-            if (!mbar_wait(&ms.bar_rdy, 0)) note_timeout(ms, 6, 0);
+            if (!mwait(&ms.bar_rdy, 0)) note_timeout(ms, 6, 0);
             tc_fence_after();
             if (GATE != kGateNone) {
 #pragma unroll
@@ -1109,7 +1119,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             const int t0 = r * CV;
             const int buf = r & 1;
             if (GATE != kGateChannel && r > 0) {
-                if (!mbar_wait(&ms.bar_rdy, ph)) note_timeout(ms, 6, r);
+                if (!mwait(&ms.bar_rdy, ph)) note_timeout(ms, 6, r);
                 tc_fence_after();
             }
             TC2_MARK(256, 17);
@@ -1161,7 +1171,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             if (DELTA) {
                 // history correction Z^T = U^T - (S K<^T) T2^T: X^T = S K<^T leaves TMEM as
                 // -X^T in fp16 (the A operand of the product with T2)
-                if (!mbar_wait(&ms.bar_x, ph)) note_timeout(ms, 3, r);
+                if (!mwait(&ms.bar_x, ph)) note_timeout(ms, 3, r);
                 tc_fence_after();
                 {
                     float x[64];
@@ -1191,7 +1201,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 }
             }
             if (DELTA) {
-                if (!mbar_wait(&ms.bar_fA, ph)) note_timeout(ms, 7, r);
+                if (!mwait(&ms.bar_fA, ph)) note_timeout(ms, 7, r);
             }
             TC2_MARK(256, 19);
             tc_fence_after();
@@ -1230,7 +1240,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
                 mma_commit(fb);
             }
             TC2_MARK(256, 21);
-            if (!mbar_wait(fb, (r >> 1) & 1)) note_timeout(ms, 8, r);
+            if (!mwait(fb, (r >> 1) & 1)) note_timeout(ms, 8, r);
             TC2_MARK(256, 22);
             tc_fence_after();
             if (!(mode & kModeNoOut)) {
@@ -1282,7 +1292,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
             // scalar gate's was published with rdy(r) (the prep group runs a chunk's
             // gate pass one chunk early), so S16 and the decay need not wait
             if (GATE == kGateChannel && more) {
-                if (!mbar_wait(&ms.bar_rdy, (r + 1) & 1)) note_timeout(ms, 6, r + 1);
+                if (!mwait(&ms.bar_rdy, (r + 1) & 1)) note_timeout(ms, 6, r + 1);
                 tc_fence_after();
             }
             TC2_MARK(256, 25);
@@ -1344,6 +1354,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 
     if (!(rmax <= 65504.f)) ms.range_flag = 1;
     __syncthreads();
+    if (ms.abort_flag) {
+        // a wait ran out: let every MMA and TMA load this CTA issued land before
+        // its TMEM and shared memory are released (each wait bounded at 1 s)
+        if (t == 0 || t == 256) mma_commit(&ms.bar_drain);  // the two MMA-issuing threads
+        if (t == 0) {
+            mbar_wait(&ms.bar_drain, 0);
+            if (ms.n_tma > 0) mbar_wait(&ms.bar_tma, (ms.n_tma - 1) & 1);
+            if (ms.n_tv > 0) mbar_wait(&ms.bar_tv, (ms.n_tv - 1) & 1);
+        }
+        __syncthreads();
+    }
     if (t == 0) {
         if (ms.abort_flag) {
             record_status(p.status, kStatusTimeout);
@@ -1410,6 +1431,8 @@ extern "C" int gdn_tc2_phase_times(unsigned long long *out, int clear) {
 }
 #endif
 
+unsigned long long gdn_wait_limit_ns();  // api.cu
+
 int gdn_tc_supported(const gdn_desc_t *d) {
     return d->dtype == GDN_BF16 && d->dk == 128 && (d->dv == 64 || d->dv == 128);
 }
@@ -1469,6 +1492,7 @@ int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStrea
     prm.pro = a.pro;
     prm.mode = a.mode;
     prm.states = a.states;
+    prm.wait_ns = gdn_wait_limit_ns();
     const long grid = (long)a.BH * prm.nslices;
     if (grid == 0) return 0;
     if (nh > 1) {

@@ -76,6 +76,7 @@ struct DecodeArgs {
     int BH, T, dk, dv;
     int pro;                 // GDN_PRO_* input maps
     int *status;             // device status word
+    unsigned long long wait_ns;  // bound of the bulk-copy waits (0 = 1 s)
 };
 
 // Input prologue maps (GDN_PRO_* bits, mirrored here for device code).

@@ -275,6 +275,7 @@ __global__ void __launch_bounds__(kMWarps * 32, 3) decode_multi_kernel(DecodeArg
     const long nwarps = (long)gridDim.x * kMWarps;
     const long w0 = (long)blockIdx.x * kMWarps + wib;
     const int bpr = a.dv / kMRows;  // tasks per head
+    const uint64_t wlim = a.wait_ns ? a.wait_ns : 1000000000ull;
 
     auto issue = [&](long task, int sl) {
         if (lane == 0) {
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(kMWarps * 32, 3) decode_multi_kernel(DecodeArg
     int it = 0;
     for (long task = w0; task < ntasks; task += nwarps, ++it) {
         const int sl = it % kMSlots;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar[sl], (it / kMSlots) & 1));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar[sl], (it / kMSlots) & 1, wlim));
         if (!ok) {
             // give up: record it, let the copies still in flight land (bounded), leave
             record_status(a.status, kStatusTimeout);

@@ -104,6 +104,14 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, u
     }
 }
 
+// A wait with a caller-chosen bound.  A bound under 1 us means no waiting at
+// all: the phase must already be complete (the setting with which a test forces
+// the expiry path; a suspending try_wait would outlast any such bound).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    if (limit_ns < 1000ull) return mbar_test_wait(bar, parity);
+    return mbar_wait(bar, parity, limit_ns);
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -387,6 +387,20 @@ int gdn_device_status(int clear);
  */
 int gdn_device_diag(void);
 
+/*
+ * gdn_set_wait_limit_ns -- the bound, in ns, of the waits by which a kernel's
+ * warps hand work to one another (the mbarrier phases of TMA loads, MMAs and
+ * producer / consumer steps of the tensor-core prefill, linear-attention and
+ * multi-token decode kernels); 0 restores the default of 1 s.  A wait that
+ * runs out records GDN_ERR_TIMEOUT in the status word (the tensor-core prefill
+ * also its site in the diagnostic word); the kernel then lets every copy and
+ * MMA it issued land
+ * (each of those waits bounded at 1 s whatever this setting) and returns,
+ * with o and S_T unspecified.  For tests of that path: a process-wide setting
+ * read when a call launches, not thread-safe.  Returns GDN_OK.
+ */
+int gdn_set_wait_limit_ns(unsigned long long ns);
+
 /* GDN_VERSION of the built library. */
 int gdn_version(void);
 

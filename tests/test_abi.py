@@ -259,3 +259,9 @@ def test_saved_state_entry_points_reject_bad_arguments(lib):
     d = _desc()
     d.prologue = 1
     assert bw(d, vp(0x70000000)) == -3
+
+
+def test_wait_limit_hook(lib):
+    lib.gdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    assert lib.gdn_set_wait_limit_ns(5) == 0
+    assert lib.gdn_set_wait_limit_ns(0) == 0  # back to the default bound
