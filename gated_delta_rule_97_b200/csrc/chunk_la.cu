@@ -85,7 +85,8 @@ __device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-template <bool OB>
+// TW: a test's short wait bound (gdn_set_wait_limit_ns), compiled in only for it.
+template <bool OB, bool TW>
 __global__ void __launch_bounds__(kLAThreads, 1) chunk_la_kernel(const __grid_constant__ LAParams p) {
     using L = LASmem;
     constexpr int DVS = kDVS;
@@ -126,11 +127,10 @@ __global__ void __launch_bounds__(kLAThreads, 1) chunk_la_kernel(const __grid_co
 
     // a wait that runs out stops every role (each then finds its next wait cut
     // short too); the waits on the chunk-to-chunk chain poll without suspending
-    const uint64_t wlim = p.wait_ns ? p.wait_ns : 1000000000ull;
     auto wait = [&](uint64_t *bar, uint32_t par) -> bool {
         if (mbar_test_wait(bar, par)) return true;
         if (*reinterpret_cast<volatile int *>(&bs.abort_flag)) return false;
-        if (wlim >= 1000ull && mbar_wait_spin(bar, par, wlim)) return true;  // under 1 us: no waiting
+        if (TW ? mbar_wait_bounded(bar, par, p.wait_ns) : mbar_wait_spin(bar, par)) return true;
         if (atomicExch(&bs.abort_flag, 1) == 0) record_status(p.status, kStatusTimeout);
         return false;
     };
@@ -367,9 +367,9 @@ __global__ void __launch_bounds__(kLAThreads, 1) chunk_la_kernel(const __grid_co
     }
 }
 
-template <bool OB>
+template <bool OB, bool TW>
 int launch_la(const LAParams &prm, int grid, cudaStream_t stream) {
-    auto kern = chunk_la_kernel<OB>;
+    auto kern = chunk_la_kernel<OB, TW>;
     constexpr int smem = LASmem::DYN;
     static_assert(smem <= 232448, "shared memory of one CTA");
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -413,5 +413,6 @@ int gdn_launch_chunk_la(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream
     prm.nslices = a.dv / kDVS;
     const long grid = (long)a.BH * prm.nslices;
     if (grid == 0) return 0;
-    return ob ? launch_la<true>(prm, (int)grid, stream) : launch_la<false>(prm, (int)grid, stream);
+    if (prm.wait_ns) return ob ? launch_la<true, true>(prm, (int)grid, stream) : launch_la<false, true>(prm, (int)grid, stream);
+    return ob ? launch_la<true, false>(prm, (int)grid, stream) : launch_la<false, false>(prm, (int)grid, stream);
 }

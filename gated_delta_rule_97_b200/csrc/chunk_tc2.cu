@@ -182,9 +182,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
     constexpr bool DELTA = (UPD == kDelta);
     const int pro = EXT ? p.pro : 0;
     const int mode = EXT ? p.mode : 0;
-    // the hand-off waits, bounded (1 s unless a test shortens it)
-    const uint64_t wlim = p.wait_ns ? p.wait_ns : 1000000000ull;
-    auto mwait = [wlim](uint64_t *bar, uint32_t par) { return mbar_wait_bounded(bar, par, wlim); };
+    // the hand-off waits, bounded at 1 s; a test's shorter bound is compiled
+    // into the EXT instantiation only, so the plain kernel's waits are unchanged
+    auto mwait = [&p](uint64_t *bar, uint32_t par) {
+        if (EXT && p.wait_ns) return mbar_wait_bounded(bar, par, p.wait_ns);
+        return mbar_wait(bar, par);
+    };
     // P = [Q;K]K^T of a chunk is issued by the state group's MMA thread right after
     // rdy when the prep group is the longer side (delta rule, scalar / no gate), else
     // by the prep group itself (it then has slack; the channel gate's P also needs
@@ -1382,7 +1385,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc2_kernel(const __grid_con
 template <int DVS, int UPD, int GATE, bool OB, bool PROD = false>
 int launch_one(const Params &prm, int grid, cudaStream_t stream) {
     using L = Smem<DVS, GATE>;
-    auto kern = (prm.pro != 0 || prm.mode != 0) ? chunk_tc2_kernel<DVS, UPD, GATE, OB, PROD, true>
+    auto kern = (prm.pro != 0 || prm.mode != 0 || prm.wait_ns != 0) ? chunk_tc2_kernel<DVS, UPD, GATE, OB, PROD, true>
                                                 : chunk_tc2_kernel<DVS, UPD, GATE, OB, PROD, false>;
     static_assert(L::DYN <= 232448, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN);
