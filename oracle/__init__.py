@@ -357,3 +357,40 @@ def gdn_backward_np(update, gate, q, k, v, g=None, beta=None, S0=None, dO=None, 
                 dg[..., t, :] = np.sum(dSp * Sp, axis=-2)
             dS = dSp * a if a is not None else dSp
     return dq, dk, dvv, dg, db, dS
+
+
+def gdn_backward_prologue_np(update, gate, flags, q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None):
+    """Gradients of the recurrence with the input prologue ``flags`` (the maps
+    of ``prologue``) in front of it, with respect to the raw inputs, float64.
+
+    The maps are applied, ``gdn_backward_np`` runs on the mapped inputs, and the
+    chain rule takes each gradient back through its map:
+      unit rows y = e / |e| (|e| > 0):  de = (dy - y (y . dy)) / |e|; zero row: 0
+      elu(x) + 1:                       dx = de where x > 0, de e^x elsewhere
+      beta = sigmoid(b):                db = dbeta sigmoid(b) (1 - sigmoid(b))
+      g = -softplus(x):                 dx = -dg sigmoid(x)
+    Returns (dq, dk, dv, dg, dbeta, dS0) shaped like the raw inputs."""
+    qm, km, bm, gm = prologue(flags, q=q, k=k, beta=beta, g=g)
+    dqm, dkm, dv, dgm, dbm, dS0 = gdn_backward_np(update, gate, qm, km, v, gm, bm, S0, dO, dS_T)
+
+    def back_feat(x, dy):
+        x = _f64(x)
+        e = np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0))) if flags & PRO_QK_ELU1 else x
+        de = dy
+        if flags & PRO_QK_L2:
+            n = np.sqrt(np.sum(e * e, axis=-1, keepdims=True))
+            safe = np.where(n > 0, n, 1.0)
+            y = e / safe
+            de = np.where(n > 0, (dy - y * np.sum(y * dy, axis=-1, keepdims=True)) / safe, 0.0)
+        if flags & PRO_QK_ELU1:
+            de = np.where(x > 0, de, de * np.exp(np.minimum(x, 0.0)))
+        return de
+
+    dq, dk = back_feat(q, dqm), back_feat(k, dkm)
+    dbeta, dg = dbm, dgm
+    if dbm is not None and flags & PRO_BETA_SIGMOID:
+        sb = 1.0 / (1.0 + np.exp(-_f64(beta)))
+        dbeta = dbm * sb * (1.0 - sb)
+    if dgm is not None and flags & PRO_G_NEG_SOFTPLUS:
+        dg = -dgm / (1.0 + np.exp(-_f64(g)))
+    return dq, dk, dv, dg, dbeta, dS0

@@ -713,3 +713,56 @@ def test_backward_additive_closed_forms(oracle_mod):
         assert rel_err(dk[h], G.T @ q[h] + v[h] @ dST[h]) < TOL
         assert rel_err(dv[h], (q[h] @ k[h].T * M).T @ dO[h] + k[h] @ dST[h].T) < TOL
         assert rel_err(dS0[h], dO[h].T @ q[h] + dST[h]) < TOL
+
+
+
+@pytest.mark.parametrize("update,gate,flags", [
+    ("delta", "scalar", oracle.PRO_QK_L2 | oracle.PRO_BETA_SIGMOID | oracle.PRO_G_NEG_SOFTPLUS),
+    ("delta", "channel", oracle.PRO_QK_ELU1 | oracle.PRO_QK_L2 | oracle.PRO_G_NEG_SOFTPLUS),
+    ("delta", "none", oracle.PRO_QK_ELU1 | oracle.PRO_BETA_SIGMOID),
+    ("additive", "none", oracle.PRO_QK_ELU1),
+    ("decay", "scalar", oracle.PRO_QK_L2 | oracle.PRO_G_NEG_SOFTPLUS),
+])
+def test_prologue_backward_equals_finite_differences(oracle_mod, update, gate, flags):
+    """The gradients with respect to the raw inputs match central differences
+    of the loss through the maps and the recurrence (raw gate and beta drawn as
+    logits, some raw q / k entries negative so both branches of elu are hit)."""
+    q, k, v, g, beta, S0, dO, dST = _bwd_case(91, update, gate)
+    r = np.random.default_rng(92)
+    q = q + 0.3 * r.standard_normal(q.shape)
+    k = k + 0.3 * r.standard_normal(k.shape)
+    if beta is not None:
+        beta = r.standard_normal(beta.shape)
+    if g is not None:
+        g = r.standard_normal(g.shape) - 2.0
+    got = oracle.gdn_backward_prologue_np(update, gate, flags, q, k, v, g, beta, S0, dO, dST)
+    inputs = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "S0": S0}
+
+    def loss(x):
+        qm, km, bm, gm = oracle.prologue(flags, q=x["q"], k=x["k"], beta=x["beta"], g=x["g"])
+        o, ST = oracle.gdn_forward_np(update, gate, qm, km, x["v"], gm, bm, x["S0"])
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    h = 1e-6
+    for name, grad in zip(["q", "k", "v", "g", "beta", "S0"], got):
+        if inputs[name] is None:
+            assert grad is None
+            continue
+        fd = np.zeros_like(inputs[name])
+        it = np.nditer(inputs[name], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = {n: (None if a is None else a.copy()) for n, a in inputs.items()}
+            xm = {n: (None if a is None else a.copy()) for n, a in inputs.items()}
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * h)
+        assert rel_err(grad, fd) < 1e-6, (name, rel_err(grad, fd))
+
+
+def test_prologue_backward_without_maps_is_the_plain_backward(oracle_mod):
+    q, k, v, g, beta, S0, dO, dST = _bwd_case(93, "delta", "channel")
+    a = oracle.gdn_backward_prologue_np("delta", "channel", 0, q, k, v, g, beta, S0, dO, dST)
+    b = oracle.gdn_backward_np("delta", "channel", q, k, v, g, beta, S0, dO, dST)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
