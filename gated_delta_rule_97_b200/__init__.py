@@ -531,20 +531,22 @@ def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, pr
     return o
 
 
-def bwd_workspace_bytes(B, H, T, dk, dv) -> int:
-    d = make_desc(B, H, T, dk, dv, "delta", "scalar", BF16, F32)
+def bwd_workspace_bytes(B, H, T, dk, dv, update="delta", gate="scalar", prologue=0) -> int:
+    d = make_desc(B, H, T, dk, dv, update, gate, BF16, F32, prologue=prologue)
     return int(load().gdn_bwd_workspace_bytes(ctypes.byref(d)))
 
 
 def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update, gate, workspace=None,
-              want_dS0=True, states=None, stream=None):
+              want_dS0=True, states=None, prologue=0, stream=None):
     """gdn_chunk_bwd: gradients of chunk_fwd for upstream gradients dO [B,H,T,dv]
     and dS_T [B,H,dv,dk] (fp32; None = 0).  Returns (dq, dk, dv, dg, dbeta, dS0),
     fp32, dg / dbeta None when the mode has no gate / write strength, dS0 None
     when ``want_dS0`` is false.  ``workspace``: a CUDA uint8 tensor of
     bwd_workspace_bytes(...) bytes (allocated here when None).  With ``states``
     (written by chunk_fwd(states=...)) the call is gdn_chunk_bwd_states: S0 and
-    the workspace are not used."""
+    the workspace are not used.  ``prologue``: the GDN_PRO_* maps the forward
+    applied to the raw q, k, beta, g; the gradients are then with respect to
+    those raw inputs."""
     import torch
 
     B, H, T, dk = q.shape
@@ -565,7 +567,7 @@ def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update
     gg = None if gate == "none" else torch.empty(tuple(g.shape), **f32)
     gb = torch.empty((B, H, T), **f32) if update == "delta" else None
     gS0 = torch.empty((B, H, dv, dk), **f32) if want_dS0 else None
-    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), F32)
+    d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), F32, prologue=prologue)
     if states is not None:
         _check(states, "states", (B, H, (T + CHUNK - 1) // CHUNK, dv, dk), torch.float32)
         with _on_device(q):

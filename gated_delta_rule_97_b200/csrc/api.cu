@@ -555,11 +555,44 @@ int gdn_launch_bwd(const void *q, const void *k, const void *v, const float *g, 
                    const float *dO, const float *dST, float *dq, float *dk, float *dv, float *dg, float *dbeta,
                    float *dS0, float *ws, int BH, int T, int dk_, int dv_, int update, int gate, int in_bf16,
                    int skip_fwd, cudaStream_t st);
+// input prologue of the backward (prologue_bwd.cu)
+int gdn_launch_prologue_map(const void *q, const void *k, const void *v, const float *g, const float *beta, float *qm,
+                            float *km, float *vf, float *gm, float *bm, long rows, int dk, int dv, int gate,
+                            int in_bf16, int pro, cudaStream_t st);
+int gdn_launch_prologue_grad(const void *q, const void *k, const float *g, const float *beta, float *dq, float *dk,
+                             float *dg, float *dbeta, long rows, int dk_, int gate, int in_bf16, int pro,
+                             cudaStream_t st);
+
+// Workspace of gdn_chunk_bwd: the chunk-entry states, then (with an input
+// prologue) the mapped inputs in fp32: q, k, v, beta, g, each on a 256-byte
+// boundary.
+struct BwdLayout {
+    size_t states, qm, km, vf, bm, gm, bytes;
+};
+
+static size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+static BwdLayout bwd_layout(const gdn_desc_t *d) {
+    BwdLayout L{};
+    const size_t BH = (size_t)d->B * d->H, ntok = BH * d->T;
+    const size_t nch = ((size_t)d->T + gdn::kChunk - 1) / gdn::kChunk;
+    L.states = 0;
+    size_t off = BH * nch * d->dv * d->dk * sizeof(float);
+    if (d->prologue != 0) {
+        off = round256(off);
+        L.qm = off; off = round256(off + ntok * d->dk * 4);
+        L.km = off; off = round256(off + ntok * d->dk * 4);
+        L.vf = off; off = round256(off + ntok * d->dv * 4);
+        L.bm = off; off = round256(off + (d->update == GDN_DELTA ? ntok * 4 : 0));
+        L.gm = off; off += d->gate == GDN_GATE_NONE ? 0 : ntok * (d->gate == GDN_GATE_CHANNEL ? d->dk : 1) * 4;
+    }
+    L.bytes = off;
+    return L;
+}
 
 extern "C" size_t gdn_bwd_workspace_bytes(const gdn_desc_t *d) {
     if (!d || validate_common(d) != GDN_OK) return 0;
-    const size_t nch = ((size_t)d->T + gdn::kChunk - 1) / gdn::kChunk;
-    return (size_t)d->B * d->H * nch * d->dv * d->dk * sizeof(float);
+    return bwd_layout(d).bytes;
 }
 
 namespace {
@@ -574,7 +607,7 @@ int chunk_bwd_impl(const gdn_desc_t *d, const void *q, const void *k, const void
     int rc = validate_common(d);
     if (rc != GDN_OK) return rc;
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
-    if (d->prologue != 0) return GDN_ERR_UNSUPPORTED;
+    if (d->prologue != 0 && saved) return GDN_ERR_UNSUPPORTED;  // the saved states carry no maps
     const long BH = (long)d->B * d->H;
     const size_t ntok = (size_t)BH * d->T;
     const size_t es = elem_size(d->dtype);
@@ -610,8 +643,27 @@ int chunk_bwd_impl(const gdn_desc_t *d, const void *q, const void *k, const void
     if (BH == 0) return GDN_OK;
     if (d->T == 0) return dS0 ? from_cuda(gdn_launch_copy_state(dS_T, dS0, (long)n_S, st)) : GDN_OK;
     float *ws = saved ? const_cast<float *>(saved) : static_cast<float *>(workspace);
-    return from_cuda(gdn_launch_bwd(q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, ws, (int)BH, d->T,
-                                    d->dk, d->dv, d->update, d->gate, d->dtype == GDN_BF16, saved != nullptr, st));
+    const int in_bf16 = d->dtype == GDN_BF16;
+    if (d->prologue == 0)
+        return from_cuda(gdn_launch_bwd(q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, ws, (int)BH,
+                                        d->T, d->dk, d->dv, d->update, d->gate, in_bf16, saved != nullptr, st));
+    // input prologue: map the inputs (fp32, into the workspace), run the
+    // recurrence's backward on them, then take dq, dk, dbeta, dg back through the maps
+    const BwdLayout L = bwd_layout(d);
+    char *w = static_cast<char *>(workspace);
+    float *qm = reinterpret_cast<float *>(w + L.qm), *km = reinterpret_cast<float *>(w + L.km);
+    float *vf = reinterpret_cast<float *>(w + L.vf);
+    float *bm = d->update == GDN_DELTA ? reinterpret_cast<float *>(w + L.bm) : nullptr;
+    float *gm = d->gate != GDN_GATE_NONE ? reinterpret_cast<float *>(w + L.gm) : nullptr;
+    int e = gdn_launch_prologue_map(q, k, v, g, beta, qm, km, vf, gm, bm, (long)ntok, d->dk, d->dv, d->gate, in_bf16,
+                                    d->prologue, st);
+    if (e == 0)
+        e = gdn_launch_bwd(qm, km, vf, gm, bm, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, ws, (int)BH, d->T, d->dk,
+                           d->dv, d->update, d->gate, 0, 0, st);
+    if (e == 0)
+        e = gdn_launch_prologue_grad(q, k, g, beta, dq, dk, dg, dbeta, (long)ntok, d->dk, d->gate, in_bf16,
+                                     d->prologue, st);
+    return from_cuda(e);
 }
 
 }  // namespace

@@ -313,9 +313,11 @@ const char *gdn_strerror(int code);
  * through it.  fp32 arithmetic.
  *
  *   desc        as for gdn_chunk_fwd (update, gate, dtype of q, k, v; dk, dv
- *               in {64, 128}; chunk 0 or 64); out_dtype and algo are not read;
- *               prologue must be 0 (GDN_ERR_UNSUPPORTED otherwise: the maps'
- *               own gradients are not part of this call).
+ *               in {64, 128}; chunk 0 or 64); out_dtype and algo are not read.
+ *               With prologue bits the inputs are the raw q, k, beta, g the
+ *               forward mapped, and dq, dk, dbeta, dg are the gradients with
+ *               respect to them (the chain rule through each map follows the
+ *               recurrence's backward).
  *   q, k, v, g, beta, S0   the forward inputs, laid out as in gdn_chunk_fwd
  *               (S0 may be NULL = 0).
  *   dO          [B,H,T,dv] float, the gradient of o (NULL = 0).
@@ -326,8 +328,9 @@ const char *gdn_strerror(int code);
  *   dbeta       [B,H,T] float; non-NULL iff update == DELTA
  *   dS0         [B,H,dv,dk] float, or NULL (not written)
  *   workspace   device buffer of at least gdn_bwd_workspace_bytes(desc) bytes
- *               (B*H*ceil(T/64)*dv*dk*4: the chunk-boundary states), 16-byte
- *               aligned, owned by the caller; contents on return unspecified.
+ *               (B*H*ceil(T/64)*dv*dk*4: the chunk-boundary states; with prologue
+ *               bits also the mapped q, k, v, beta, g in fp32), 16-byte aligned,
+ *               owned by the caller; contents on return unspecified.
  *
  * Every pointer 16-byte aligned; no output may overlap another output, an
  * input or the workspace (GDN_ERR_ARG).  dq, dk, dg and dbeta are sums over the
@@ -360,7 +363,7 @@ int gdn_chunk_bwd(const gdn_desc_t *desc, const void *q, const void *k, const vo
  * gdn_chunk_bwd_states -- gdn_chunk_bwd from those saved states: the backward's
  * own forward pass over the sequence is skipped (each chunk is still recomputed
  * from its saved state).  Arguments as for gdn_chunk_bwd, with `states` (read
- * only; required when B*H*T > 0) in place of S0 and the workspace.
+ * only; required when B*H*T > 0) in place of S0 and the workspace; prologue 0.
  */
 int gdn_chunk_fwd_states(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
                          const float *beta, const float *S0, void *o, float *S_T, float *states, void *stream);

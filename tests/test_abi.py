@@ -230,8 +230,12 @@ def test_backward_rejects_bad_arguments(lib):
     assert f(ctypes.byref(d), *ins, *bad, ws, need, None) == -1                # dv overlaps q
     assert f(ctypes.byref(d), *ins, *outs, vp(0x1100000), need, None) == -1   # workspace overlaps dk
     p = _desc(T=130)
-    p.prologue = 1
-    assert f(ctypes.byref(p), *ins, *outs, ws, need, None) == -3              # input maps not differentiated
+    p.prologue = 1 | 2 | 4 | 8
+    need_p = lib.gdn_bwd_workspace_bytes(ctypes.byref(p))
+    ntok = 6 * 130
+    extra = sum((x + 255) // 256 * 256 for x in (ntok * 128 * 4, ntok * 128 * 4, ntok * 128 * 4, ntok * 4)) + ntok * 4
+    assert need_p == (need + 255) // 256 * 256 + extra  # + the mapped q, k, v, beta, g in fp32
+    assert f(ctypes.byref(p), *ins, *outs, ws, need, None) == -1              # room for the mapped inputs too
     e = _desc(B=0)
     assert f(ctypes.byref(e), *ins, *outs, ws, 0, None) == 0                   # empty batch: no-op
 

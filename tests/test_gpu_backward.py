@@ -171,3 +171,56 @@ def test_saved_states_reject_requests_the_tensor_core_forward_cannot_serve():
     states = torch.empty((1, 2, 2, 128, 128), dtype=torch.float32, device="cuda")
     with pytest.raises(gdn.GDNError):
         gdn.chunk_fwd(q, k, v, g, beta, S0, update="delta", gate="scalar", states=states)
+
+
+# ----------------------------------------------------------------------------
+# Input prologue: the gradients with respect to the raw q, k, beta, g that the
+# forward's maps took (oracle.gdn_backward_prologue_np, pinned by central
+# differences through maps and recurrence).
+PRO_CASES = [("delta", "scalar", oracle.PRO_QK_L2 | oracle.PRO_BETA_SIGMOID | oracle.PRO_G_NEG_SOFTPLUS),
+             ("delta", "channel", oracle.PRO_QK_ELU1 | oracle.PRO_QK_L2 | oracle.PRO_G_NEG_SOFTPLUS),
+             ("delta", "none", oracle.PRO_QK_ELU1 | oracle.PRO_QK_L2 | oracle.PRO_BETA_SIGMOID),
+             ("additive", "none", oracle.PRO_QK_ELU1),
+             ("decay", "scalar", oracle.PRO_QK_L2 | oracle.PRO_G_NEG_SOFTPLUS)]
+
+
+def raw_inputs(seed, update, gate, T=130, dk=128, dv=128, bf16=False):
+    r = np.random.default_rng(seed)
+    q = r.standard_normal((1, 2, T, dk)) / (np.sqrt(dk) if update == "additive" else 1.0)
+    k = r.standard_normal((1, 2, T, dk)) / (np.sqrt(dk) if update == "additive" else 1.0)
+    v = r.standard_normal((1, 2, T, dv))
+    rnd = (lambda x: round_to_bf16(np.asarray(x, np.float32)).astype(np.float64)) if bf16 else \
+        (lambda x: np.asarray(x, np.float32).astype(np.float64))
+    q, k, v = rnd(q), rnd(k), rnd(v)
+    f32 = lambda x: None if x is None else np.asarray(x, np.float32).astype(np.float64)
+    g = None
+    if gate == "scalar":
+        g = f32(r.standard_normal((1, 2, T)) - 3.0)
+    elif gate == "channel":
+        g = f32(r.standard_normal((1, 2, T, dk)) - 4.0)
+    beta = f32(r.standard_normal((1, 2, T))) if update == "delta" else None
+    S0 = f32(0.05 * r.standard_normal((1, 2, dv, dk)))
+    dO = f32(r.standard_normal((1, 2, T, dv)))
+    dST = f32(r.standard_normal((1, 2, dv, dk)))
+    return q, k, v, g, beta, S0, dO, dST
+
+
+@pytest.mark.parametrize("update,gate,flags", PRO_CASES)
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_backward_with_input_prologue(update, gate, flags, dk, dv, bf16):
+    x = raw_inputs(41, update, gate, dk=dk, dv=dv, bf16=bf16)
+    q, k, v, g, beta, S0, dO, dST = x
+    dt = torch.bfloat16 if bf16 else torch.float32
+    gdn.device_status(clear=True)
+    got = gdn.chunk_bwd(dev(q, dt), dev(k, dt), dev(v, dt), dev(g), dev(beta), dev(S0), dev(dO), dev(dST),
+                        update=update, gate=gate, prologue=flags)
+    torch.cuda.synchronize()
+    assert gdn.device_status(clear=True) == 0
+    ref = oracle.gdn_backward_prologue_np(update, gate, flags, *x)
+    for name, a, b in zip(["dq", "dk", "dv", "dg", "dbeta", "dS0"], got, ref):
+        if b is None:
+            assert a is None, name
+            continue
+        err = rel_err(np64(a), b)
+        assert err <= TOL, (name, err)
