@@ -373,17 +373,18 @@ def time_decode_multi(w, T, n_calls, torch, gdn, warmup=3):
 SERVE_B, SERVE_H, SERVE_PROMPT, SERVE_DECODE = 32, 32, 1024, 128
 
 
-def serving_workloads():
-    wp = WORKLOADS["gdn_prefill_bf16"].with_(B=SERVE_B, H=SERVE_H, T=SERVE_PROMPT, name="serve_prompt")
-    wd = WORKLOADS["decode_gdn_bf16"].with_(B=SERVE_B, H=SERVE_H, name="serve_decode")
+def serving_workloads(B=SERVE_B):
+    wp = WORKLOADS["gdn_prefill_bf16"].with_(B=B, H=SERVE_H, T=SERVE_PROMPT, name="serve_prompt")
+    wd = WORKLOADS["decode_gdn_bf16"].with_(B=B, H=SERVE_H, name="serve_decode")
     return wp, wd
 
 
-def time_serving_loop(reps, torch, gdn, warmup=1):
+def time_serving_loop(reps, torch, gdn, warmup=1, B=SERVE_B, graph=False):
     """Device time of one serving loop (prefill of the prompt into the state,
     then SERVE_DECODE single-token steps on it); returns (ms per loop, ms of
-    the prefill, ms per decode step)."""
-    wp, wd = serving_workloads()
+    the prefill, ms per decode step).  With ``graph`` the decode steps are
+    captured once in a CUDA graph and replayed (the prefill runs eagerly)."""
+    wp, wd = serving_workloads(B)
     x = make_prefill_inputs(wp)
     dt = torch.bfloat16
     q, k, v = (to_dev(x[n], dt, torch) for n in ("q", "k", "v"))
@@ -399,15 +400,32 @@ def time_serving_loop(reps, torch, gdn, warmup=1):
     stream = torch.cuda.current_stream()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
 
+    def decode_all():
+        for st in steps:
+            gdn.decode_step(st["q"], st["k"], st["v"], st["g"], st["beta"], S, update=wd.update, gate=wd.gate,
+                            o=o_dec)
+
+    cg = None
+    if graph:
+        decode_all()  # warm (first-use attribute setup happens outside the capture)
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg, stream=side):
+            decode_all()
+        torch.cuda.synchronize()
+
     def loop(timed):
         if timed:
             ev[0].record(stream)
         gdn.chunk_fwd(q, k, v, g, beta, S0, update=wp.update, gate=wp.gate, o=o_pf, S_T=S)
         if timed:
             ev[1].record(stream)
-        for st in steps:
-            gdn.decode_step(st["q"], st["k"], st["v"], st["g"], st["beta"], S, update=wd.update, gate=wd.gate,
-                            o=o_dec)
+        if cg is not None:
+            cg.replay()
+        else:
+            decode_all()
         if timed:
             ev[2].record(stream)
 
@@ -586,10 +604,14 @@ def run_ours(args):
             print(json.dumps({"only": "decode", "ms_per_step": ms_d}), flush=True)
         return
     if args.only == "serving":
-        ms_sv, ms_pf, ms_dec = time_serving_loop(3, torch, gdn)
+        out = {"only": "serving"}
+        for B in (SERVE_B, 1):
+            for graph in (False, True):
+                ms_sv, ms_pf, ms_dec = time_serving_loop(3, torch, gdn, B=B, graph=graph)
+                out["B%d_%s" % (B, "graph" if graph else "eager")] = {
+                    "ms_per_loop": ms_sv, "ms_prefill": ms_pf, "ms_per_decode_step": ms_dec}
         if rank == 0:
-            print(json.dumps({"only": "serving", "ms_per_loop": ms_sv, "ms_prefill": ms_pf,
-                              "ms_per_decode_step": ms_dec}), flush=True)
+            print(json.dumps(out), flush=True)
         return
     if args.only == "decode_multi":
         wd = WORKLOADS["decode_gdn_bf16"]
@@ -702,16 +724,21 @@ def run_ours(args):
                                    "achieved_gbs": nb / (msn * 1e-3) / 1e9,
                                    "frac_of_roofline_time": nb / (peaks["hbm_gbs"] * 1e9) / (msn * 1e-3)}
         result["prefill_workloads"] = others
-        # the prefill -> decode serving loop (second workload)
-        ms_sv, ms_pf, ms_dec = time_serving_loop(3, torch, gdn)
-        ms_sv = max_over_ranks(ms_sv, dist, "cuda")
-        result["gpu_launches"] += 3 * (1 + SERVE_DECODE)
-        result["serving_loop"] = {
-            "B": SERVE_B, "H": SERVE_H, "prompt_tokens": SERVE_PROMPT, "decode_tokens": SERVE_DECODE,
-            "ms_per_loop": ms_sv, "ms_prefill": ms_pf, "ms_per_decode_step": ms_dec,
-            "tokens_per_s": SERVE_B * (SERVE_PROMPT + SERVE_DECODE) * world / (ms_sv * 1e-3),
-            "decode_tokens_per_s": SERVE_B * world / (ms_dec * 1e-3),
-            "note": "gdn_chunk_fwd writes S_T into the decode state, then gdn_decode_step runs in place"}
+        # the prefill -> decode serving loop (second workload), eager and with the
+        # decode steps replayed from one CUDA graph, at 32 and at 1 sequence
+        sv = {"H": SERVE_H, "prompt_tokens": SERVE_PROMPT, "decode_tokens": SERVE_DECODE,
+              "note": "gdn_chunk_fwd writes S_T into the decode state, then gdn_decode_step runs in place; "
+                      "graph: the decode steps captured once in a CUDA graph and replayed"}
+        for B in (SERVE_B, 1):
+            for graph in (False, True):
+                ms_sv, ms_pf, ms_dec = time_serving_loop(3, torch, gdn, B=B, graph=graph)
+                ms_sv = max_over_ranks(ms_sv, dist, "cuda")
+                result["gpu_launches"] += 3 * (1 + SERVE_DECODE)
+                sv["B%d_%s" % (B, "graph" if graph else "eager")] = {
+                    "ms_per_loop": ms_sv, "ms_prefill": ms_pf, "ms_per_decode_step": ms_dec,
+                    "tokens_per_s": B * (SERVE_PROMPT + SERVE_DECODE) * world / (ms_sv * 1e-3),
+                    "decode_tokens_per_s": B * world / (ms_dec * 1e-3)}
+        result["serving_loop"] = sv
         # training backward (gdn_chunk_bwd) on the GDN workload
         nb_steps = 2
         msb = max_over_ranks(time_backward(w, nb_steps, torch, gdn), dist, "cuda")
