@@ -444,12 +444,13 @@ def time_serving_loop(reps, torch, gdn, warmup=1, B=SERVE_B, graph=False):
     return ms, ms_pf, (ms - ms_pf) / SERVE_DECODE
 
 
-def time_backward(w, steps, torch, gdn, warmup=1, saved=False):
+def time_backward(w, steps, torch, gdn, warmup=1, saved=False, tc=False):
     """Device time of gdn_chunk_bwd (gradients of the prefill) on workload ``w``
     with random upstream gradients of o and S_T; returns ms per call.  With
     ``saved``: a training step's forward gdn_chunk_fwd_states and then
-    gdn_chunk_bwd_states from its chunk states; returns (ms of the forward, ms
-    of the backward) per step."""
+    gdn_chunk_bwd_states (``tc``: gdn_chunk_bwd_tc, the chunkwise tensor-core
+    backward) from its chunk states; returns (ms of the forward, ms of the
+    backward) per step."""
     x = make_prefill_inputs(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     q, k, v = to_dev(x["q"], dt, torch), to_dev(x["k"], dt, torch), to_dev(x["v"], dt, torch)
@@ -465,12 +466,20 @@ def time_backward(w, steps, torch, gdn, warmup=1, saved=False):
         ST = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device="cuda")
         stream = torch.cuda.current_stream()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        wtc = None
+        if tc:
+            wtc = torch.empty(gdn.bwd_tc_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.update, w.gate),
+                              dtype=torch.uint8, device="cuda")
         fw, bw = [], []
         for it in range(warmup + steps):
             ev[0].record(stream)
             gdn.chunk_fwd(q, k, v, g, beta, S0, update=w.update, gate=w.gate, o=o, S_T=ST, states=states)
             ev[1].record(stream)
-            gdn.chunk_bwd(q, k, v, g, beta, None, dO, dST, update=w.update, gate=w.gate, states=states)
+            if tc:
+                gdn.chunk_bwd(q, k, v, g, beta, None, dO, dST, update=w.update, gate=w.gate, states=states,
+                              algo="tc", workspace=wtc)
+            else:
+                gdn.chunk_bwd(q, k, v, g, beta, None, dO, dST, update=w.update, gate=w.gate, states=states)
             ev[2].record(stream)
             torch.cuda.synchronize()
             if it >= warmup:
@@ -626,9 +635,11 @@ def run_ours(args):
     if args.only == "backward":
         ms = time_backward(w, args.steps, torch, gdn, warmup=args.warmup)
         msf_s, msb_s = time_backward(w, args.steps, torch, gdn, warmup=1, saved=True)
+        msf_t, msb_t = time_backward(w, args.steps, torch, gdn, warmup=1, saved=True, tc=True)
         if rank == 0:
             print(json.dumps({"only": "backward", "workload": w.name, "B": w.B, "H": w.H, "T": w.T,
-                              "ms_per_call": ms, "saved_states": {"ms_forward": msf_s, "ms_backward": msb_s}}),
+                              "ms_per_call": ms, "saved_states": {"ms_forward": msf_s, "ms_backward": msb_s},
+                              "tensor_core": {"ms_forward": msf_t, "ms_backward": msb_t}}),
                   flush=True)
         return
     x = make_prefill_inputs(w)

@@ -107,6 +107,10 @@ def load():
     lib.gdn_chunk_fwd_states.restype = ctypes.c_int
     lib.gdn_chunk_bwd_states.argtypes = [dp] + [vp] * 15
     lib.gdn_chunk_bwd_states.restype = ctypes.c_int
+    lib.gdn_bwd_tc_workspace_bytes.argtypes = [dp]
+    lib.gdn_bwd_tc_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_chunk_bwd_tc.argtypes = [dp] + [vp] * 15 + [ctypes.c_size_t, vp]
+    lib.gdn_chunk_bwd_tc.restype = ctypes.c_int
     lib.gdn_strerror.argtypes = [ctypes.c_int]
     lib.gdn_strerror.restype = ctypes.c_char_p
     lib.gdn_device_status.argtypes = [ctypes.c_int]
@@ -536,8 +540,14 @@ def bwd_workspace_bytes(B, H, T, dk, dv, update="delta", gate="scalar", prologue
     return int(load().gdn_bwd_workspace_bytes(ctypes.byref(d)))
 
 
+def bwd_tc_workspace_bytes(B, H, T, dk, dv, update="delta", gate="scalar") -> int:
+    """Workspace of gdn_chunk_bwd_tc (0 for a request it does not serve)."""
+    d = make_desc(B, H, T, dk, dv, update, gate, BF16, F32)
+    return int(load().gdn_bwd_tc_workspace_bytes(ctypes.byref(d)))
+
+
 def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update, gate, workspace=None,
-              want_dS0=True, states=None, prologue=0, stream=None):
+              want_dS0=True, states=None, prologue=0, algo="token", stream=None):
     """gdn_chunk_bwd: gradients of chunk_fwd for upstream gradients dO [B,H,T,dv]
     and dS_T [B,H,dv,dk] (fp32; None = 0).  Returns (dq, dk, dv, dg, dbeta, dS0),
     fp32, dg / dbeta None when the mode has no gate / write strength, dS0 None
@@ -546,7 +556,9 @@ def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update
     (written by chunk_fwd(states=...)) the call is gdn_chunk_bwd_states: S0 and
     the workspace are not used.  ``prologue``: the GDN_PRO_* maps the forward
     applied to the raw q, k, beta, g; the gradients are then with respect to
-    those raw inputs."""
+    those raw inputs.  ``algo="tc"`` (with ``states``) is gdn_chunk_bwd_tc, the
+    chunkwise tensor-core backward; ``workspace`` is then one of
+    bwd_tc_workspace_bytes(...) bytes."""
     import torch
 
     B, H, T, dk = q.shape
@@ -568,6 +580,25 @@ def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update
     gb = torch.empty((B, H, T), **f32) if update == "delta" else None
     gS0 = torch.empty((B, H, dv, dk), **f32) if want_dS0 else None
     d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), F32, prologue=prologue)
+    if algo == "tc":
+        if states is None:
+            raise ValueError("algo='tc' runs from saved states (chunk_fwd(states=...))")
+        _check(states, "states", (B, H, (T + CHUNK - 1) // CHUNK, dv, dk), torch.float32)
+        need = int(load().gdn_bwd_tc_workspace_bytes(ctypes.byref(d)))
+        if workspace is None:
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        if not workspace.is_cuda or not workspace.is_contiguous() or workspace.numel() < need:
+            raise ValueError("workspace needs %d contiguous CUDA bytes" % need)
+        with _on_device(q):
+            rc = load().gdn_chunk_bwd_tc(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(states), _ptr(dO), _ptr(dS_T), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gg),
+                                         _ptr(gb), _ptr(gS0), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                         _stream(stream, q))
+        if rc != GDN_OK:
+            raise GDNError(rc, "gdn_chunk_bwd_tc")
+        return gq, gk, gv, gg, gb, gS0
+    if algo != "token":
+        raise ValueError("algo is 'token' or 'tc'")
     if states is not None:
         _check(states, "states", (B, H, (T + CHUNK - 1) // CHUNK, dv, dk), torch.float32)
         with _on_device(q):

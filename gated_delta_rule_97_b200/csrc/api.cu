@@ -597,17 +597,13 @@ extern "C" size_t gdn_bwd_workspace_bytes(const gdn_desc_t *d) {
 
 namespace {
 
-// gdn_chunk_bwd and gdn_chunk_bwd_states: `saved` holds the chunk-entry states
-// written by gdn_chunk_fwd_states (read only, the forward pass is skipped), or
-// is null and `workspace` receives them from the backward's own forward pass.
-int chunk_bwd_impl(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
-                   const float *beta, const float *S0, const float *saved, const float *dO, const float *dS_T,
-                   float *dq, float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
-                   size_t workspace_bytes, void *stream) {
-    int rc = validate_common(d);
-    if (rc != GDN_OK) return rc;
-    if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
-    if (d->prologue != 0 && saved) return GDN_ERR_UNSUPPORTED;  // the saved states carry no maps
+// Argument rules shared by the backward entry points: pointers, alignment, the
+// workspace (`need` bytes, required unless `ws_optional`) and overlaps of every
+// output (and the workspace) with every input and with each other.
+int bwd_check(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g, const float *beta,
+              const float *S0, const float *saved, size_t saved_bytes, const float *dO, const float *dS_T,
+              float *dq, float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
+              size_t workspace_bytes, size_t need) {
     const long BH = (long)d->B * d->H;
     const size_t ntok = (size_t)BH * d->T;
     const size_t es = elem_size(d->dtype);
@@ -624,21 +620,40 @@ int chunk_bwd_impl(const gdn_desc_t *d, const void *q, const void *k, const void
     const void *ptrs[] = {q, k, v, g, beta, S0, saved, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
-    const size_t need = gdn_bwd_workspace_bytes(d);
-    if (has_tokens && !saved && (!workspace || workspace_bytes < need)) return GDN_ERR_ARG;
-    if (has_tokens && saved && workspace) return GDN_ERR_ARG;
-    // outputs (and the workspace) against every input and against each other
+    if (has_tokens && need && (!workspace || workspace_bytes < need)) return GDN_ERR_ARG;
+    if (has_tokens && !need && workspace) return GDN_ERR_ARG;
     struct Span { const void *p; size_t n; };
     const Span ins[] = {{q, n_qk * es}, {k, n_qk * es}, {v, n_v * es}, {g, n_g * 4}, {beta, ntok * 4},
-                        {S0, n_S * 4}, {saved, has_tokens ? need : 0}, {dO, n_v * 4}, {dS_T, n_S * 4}};
+                        {S0, n_S * 4}, {saved, has_tokens ? saved_bytes : 0}, {dO, n_v * 4}, {dS_T, n_S * 4}};
     const Span outs[] = {{dq, n_qk * 4}, {dk, n_qk * 4}, {dv, n_v * 4}, {dg, n_g * 4}, {dbeta, ntok * 4},
-                         {dS0, n_S * 4}, {workspace, has_tokens && !saved ? need : 0}};
+                         {dS0, n_S * 4}, {workspace, has_tokens ? need : 0}};
     for (const Span &o : outs) {
         for (const Span &i : ins)
             if (overlaps(o.p, o.n, i.p, i.n)) return GDN_ERR_ARG;
         for (const Span &o2 : outs)
             if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return GDN_ERR_ARG;
     }
+    return GDN_OK;
+}
+
+// gdn_chunk_bwd and gdn_chunk_bwd_states: `saved` holds the chunk-entry states
+// written by gdn_chunk_fwd_states (read only, the forward pass is skipped), or
+// is null and `workspace` receives them from the backward's own forward pass.
+int chunk_bwd_impl(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const float *S0, const float *saved, const float *dO, const float *dS_T,
+                   float *dq, float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+    int rc = validate_common(d);
+    if (rc != GDN_OK) return rc;
+    if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if (d->prologue != 0 && saved) return GDN_ERR_UNSUPPORTED;  // the saved states carry no maps
+    const long BH = (long)d->B * d->H;
+    const size_t ntok = (size_t)BH * d->T;
+    const size_t n_S = (size_t)BH * d->dv * d->dk;
+    const size_t need = gdn_bwd_workspace_bytes(d);
+    rc = bwd_check(d, q, k, v, g, beta, S0, saved, need, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace,
+                   workspace_bytes, saved ? 0 : need);
+    if (rc != GDN_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (BH == 0) return GDN_OK;
     if (d->T == 0) return dS0 ? from_cuda(gdn_launch_copy_state(dS_T, dS0, (long)n_S, st)) : GDN_OK;
@@ -683,6 +698,46 @@ extern "C" int gdn_chunk_bwd_states(const gdn_desc_t *d, const void *q, const vo
     if (d && (long)d->B * d->H * d->T > 0 && !states) return GDN_ERR_ARG;
     return chunk_bwd_impl(d, q, k, v, g, beta, nullptr, states, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, nullptr, 0,
                           stream);
+}
+
+size_t gdn_bwd_tc_layout(long BH, int nch, int dk, int dv, int delta, size_t *off);  // backward_tc.cu
+int gdn_launch_bwd_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                      const float *states, const float *dO, const float *dST, float *dq, float *dk, float *dv,
+                      float *dg, float *dbeta, float *dS0, void *ws, int BH, int T, int dv_, int update, int gate,
+                      int in_bf16, cudaStream_t st);
+
+static bool bwd_tc_supported(const gdn_desc_t *d) {
+    return d->prologue == 0 && d->gate != GDN_GATE_CHANNEL && d->dk == 128 && (d->dv == 64 || d->dv == 128) &&
+           (d->chunk == 0 || d->chunk == gdn::kChunk);
+}
+
+extern "C" size_t gdn_bwd_tc_workspace_bytes(const gdn_desc_t *d) {
+    if (!d || validate_common(d) != GDN_OK || !bwd_tc_supported(d)) return 0;
+    const long BH = (long)d->B * d->H;
+    const int nch = (d->T + gdn::kChunk - 1) / gdn::kChunk;
+    return gdn_bwd_tc_layout(BH, nch, d->dk, d->dv, d->update == GDN_DELTA, nullptr);
+}
+
+extern "C" int gdn_chunk_bwd_tc(const gdn_desc_t *d, const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *states, const float *dO, const float *dS_T,
+                                float *dq, float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    int rc = validate_common(d);
+    if (rc != GDN_OK) return rc;
+    if (!bwd_tc_supported(d)) return GDN_ERR_UNSUPPORTED;
+    const long BH = (long)d->B * d->H;
+    const size_t ntok = (size_t)BH * d->T, n_S = (size_t)BH * d->dv * d->dk;
+    const int nch = (d->T + gdn::kChunk - 1) / gdn::kChunk;
+    if (ntok > 0 && !states) return GDN_ERR_ARG;
+    const size_t need = gdn_bwd_tc_workspace_bytes(d);
+    rc = bwd_check(d, q, k, v, g, beta, nullptr, states, (size_t)BH * nch * d->dv * d->dk * 4, dO, dS_T, dq, dk,
+                   dv, dg, dbeta, dS0, workspace, workspace_bytes, need);
+    if (rc != GDN_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (BH == 0) return GDN_OK;
+    if (d->T == 0) return dS0 ? from_cuda(gdn_launch_copy_state(dS_T, dS0, (long)n_S, st)) : GDN_OK;
+    return from_cuda(gdn_launch_bwd_tc(q, k, v, g, beta, states, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace,
+                                       (int)BH, d->T, d->dv, d->update, d->gate, d->dtype == GDN_BF16, st));
 }
 
 extern "C" int gdn_chunk_fwd_states(const gdn_desc_t *d, const void *q, const void *k, const void *v,

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define GDN_VERSION 6
+#define GDN_VERSION 7
 
 /* Return codes. */
 #define GDN_OK 0
@@ -370,6 +370,38 @@ int gdn_chunk_fwd_states(const gdn_desc_t *desc, const void *q, const void *k, c
 int gdn_chunk_bwd_states(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
                          const float *beta, const float *states, const float *dO, const float *dS_T, float *dq,
                          float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *stream);
+
+/*
+ * gdn_chunk_bwd_tc -- the same gradients as gdn_chunk_bwd_states, computed at
+ * chunk granularity on tensor cores: reverse mode through the chunkwise form
+ * ("Linear Attention, Visualized": "The triangular correction system",
+ * "Optional: Use UT...", "Correct the incoming state", "Update the state"),
+ * not through the token loop.  Three passes: every chunk's T = (I + L)^-1, W,
+ * A and Q~ = diag(b) q - A W (all chunks in parallel); the gradient of the state
+ * entering each chunk, dS_r = b_C dS_{r+1} - (dS_{r+1} K>^T) W + dO^T Q~ (the one
+ * sequential pass, chunks last to first); every chunk-local gradient (all
+ * chunks in parallel).  Products on tf32 tensor cores with fp32 accumulation,
+ * so the results carry tf32 rounding (10-bit significand) on top of the saved
+ * states'.  dq, dk, dv, dg, dbeta are written once per token (deterministic).
+ *
+ *   desc        update any, gate NONE or SCALAR, dk = 128, dv in {64, 128},
+ *               dtype bf16 or f32, prologue 0, chunk 0 or 64
+ *               (GDN_ERR_UNSUPPORTED otherwise).
+ *   states      [B,H,ceil(T/64),dv,dk] float, the chunk-entry states
+ *               (gdn_chunk_fwd_states); required when B*H*T > 0.
+ *   workspace   device buffer of at least gdn_bwd_tc_workspace_bytes(desc)
+ *               bytes, 16-byte aligned, owned by the caller; contents on
+ *               return unspecified.  Per chunk and head: T, A, P (.) Gamma
+ *               (64 x 64), W, K>, Q~ (64 x dk), the state gradient (dv x dk)
+ *               and b_C, in fp32 (T, P (.) Gamma, W, K> only for the delta rule).
+ *   others      as for gdn_chunk_bwd_states.
+ * gdn_bwd_tc_workspace_bytes returns 0 for a request the call does not serve.
+ */
+size_t gdn_bwd_tc_workspace_bytes(const gdn_desc_t *desc);
+int gdn_chunk_bwd_tc(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
+                     const float *beta, const float *states, const float *dO, const float *dS_T, float *dq,
+                     float *dk, float *dv, float *dg, float *dbeta, float *dS0, void *workspace,
+                     size_t workspace_bytes, void *stream);
 
 /*
  * gdn_device_status -- synchronises the current device, then returns the

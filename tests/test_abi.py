@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_strerror_and_version(lib):
-    assert gdn.version() == 6  # saved chunk states for the backward joined the boundary
+    assert gdn.version() == 7  # the chunkwise tensor-core backward joined the boundary
     for code in (0, -1, -2, -3, -4, -5, -6, 123):
         assert isinstance(gdn.strerror(code), str) and gdn.strerror(code)
 
@@ -263,6 +263,42 @@ def test_saved_state_entry_points_reject_bad_arguments(lib):
     d = _desc()
     d.prologue = 1
     assert bw(d, vp(0x70000000)) == -3
+
+
+def test_tensor_core_backward_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    lib.gdn_bwd_tc_workspace_bytes.argtypes = [ctypes.c_void_p]
+    lib.gdn_bwd_tc_workspace_bytes.restype = ctypes.c_size_t
+    f = lib.gdn_chunk_bwd_tc
+    f.argtypes = [ctypes.c_void_p] * 16 + [ctypes.c_size_t, ctypes.c_void_p]
+    d = _desc(T=130)  # delta, scalar gate, B2 H3 dk=dv=128: 18 chunk-heads
+    n = 6 * 3
+    cc, cd, ss = n * 64 * 64 * 4, n * 64 * 128 * 4, n * 128 * 128 * 4
+    # T, A, P (.) Gamma; W, K>, Q~; the state gradients; b_C (on 256-byte boundaries)
+    assert lib.gdn_bwd_tc_workspace_bytes(ctypes.byref(d)) == 3 * cc + 3 * cd + ss + 256
+    a = _desc(T=130, update="additive", gate="none")
+    assert lib.gdn_bwd_tc_workspace_bytes(ctypes.byref(a)) == cc + cd + ss + 256  # A, Q~ only
+    need = lib.gdn_bwd_tc_workspace_bytes(ctypes.byref(d))
+    ins = [vp(0x100000), vp(0x200000), vp(0x300000), vp(0x400000), vp(0x500000), vp(0x600000), None, None]
+    outs = [vp(0x1000000), vp(0x1100000), vp(0x1200000), vp(0x1300000), vp(0x1400000), None]
+    ws = vp(0x20000000)
+    assert f(ctypes.byref(d), *ins, *outs, ws, need - 16, None) == -1          # workspace too small
+    assert f(ctypes.byref(d), *ins, *outs, None, need, None) == -1             # no workspace
+    no_states = list(ins)
+    no_states[5] = None
+    assert f(ctypes.byref(d), *no_states, *outs, ws, need, None) == -1         # states required
+    bad = list(outs)
+    bad[0] = vp(0x1000008)
+    assert f(ctypes.byref(d), *ins, *bad, ws, need, None) == -2                # misaligned
+    assert f(ctypes.byref(d), *ins, *outs, vp(0x1100000), need, None) == -1   # workspace overlaps dk
+    for unsupported in (_desc(T=130, gate="channel"), _desc(T=130, dk=64, dv=64)):
+        assert lib.gdn_bwd_tc_workspace_bytes(ctypes.byref(unsupported)) == 0
+        assert f(ctypes.byref(unsupported), *ins, *outs, ws, need, None) == -3
+    p = _desc(T=130)
+    p.prologue = 1
+    assert f(ctypes.byref(p), *ins, *outs, ws, need, None) == -3              # no input prologue
+    e = _desc(B=0)
+    assert f(ctypes.byref(e), *ins, *outs, ws, 0, None) == 0                   # empty batch: no-op
 
 
 def test_wait_limit_hook(lib):
