@@ -506,6 +506,18 @@ def time_backward(w, steps, torch, gdn, warmup=1, saved=False, tc=False):
     return e0.elapsed_time(e1) / steps
 
 
+def backward_tc_flops(w):
+    """Dense MACs x 2 of gdn_chunk_bwd_tc per launch, per chunk of C = 64 tokens
+    and head (d = dk = dv): prep (q k^T, k k^T, W = T Mk, A W: 4 C^2 d; the solve
+    C^3 / 3), chain (dS Kc^T, X W, dO^T Q~: 3 C d^2), local (W S^T, k dSn^T,
+    Z dSn, dO S, dZ S: 5 C d^2; T Mv, A^T dO, dO Z^T, dZ v^T, T^T dZ: 5 C^2 d;
+    dW k^T, T^T dW, E k, E^T k, F^T q, F k: 6 C^2 d; dT T^T, T^T Y: 2 C^3)."""
+    C, d = 64, w.dk
+    nch = (w.T + C - 1) // C
+    macs = 4 * C * C * d + C ** 3 / 3 + 3 * C * d * d + 5 * C * d * d + 11 * C * C * d + 2 * C ** 3
+    return 2 * macs * nch * w.n_heads
+
+
 def backward_flops(w):
     """fp32 arithmetic of gdn_chunk_bwd per launch: four forward token steps per
     token (the forward pass, the chunk recompute, the sub-block recompute and the
@@ -769,6 +781,20 @@ def run_ours(args):
             "ms_forward_with_states": msf_s, "ms_backward": msb_s,
             "note": "gdn_chunk_fwd_states (tensor-core forward writing the chunk-entry states), then "
                     "gdn_chunk_bwd_states (no forward pass of its own)"}
+        # the chunkwise tensor-core backward from the same saved states
+        msf_t, msb_t = time_backward(w, nb_steps, torch, gdn, saved=True, tc=True)
+        msf_t, msb_t = max_over_ranks(msf_t, dist, "cuda"), max_over_ranks(msb_t, dist, "cuda")
+        result["gpu_launches"] += (nb_steps + 1) * 4  # the forward kernel, then prep, chain, local
+        fl_tc = backward_tc_flops(w)
+        tf32_peak = peaks["bf16_tflops"] / 2.0
+        result["backward"]["tensor_core"] = {
+            "ms_forward_with_states": msf_t, "ms_backward": msb_t,
+            "tokens_per_s": w.B * w.T * world / (msb_t * 1e-3),
+            "flops_per_call": fl_tc, "achieved_tflops": fl_tc / (msb_t * 1e-3) / 1e12,
+            "bound": "tensor", "tf32_peak_tflops": tf32_peak,
+            "frac": fl_tc / (msb_t * 1e-3) / 1e12 / tf32_peak,
+            "note": "gdn_chunk_bwd_tc: prep, state-gradient chain and local kernels on tf32 warp MMAs; "
+                    "peak = measured bf16 dense x 1/2 (the nominal tf32 : bf16 ratio)"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w)

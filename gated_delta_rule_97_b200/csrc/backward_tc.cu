@@ -21,7 +21,8 @@
 //
 // Three kernels:
 //   prep  (one CTA per chunk and head, all in parallel): T by blocked forward
-//         substitution, A, P (.) Gamma, W, Q~ = Qb - A W, Kc, b_C -> workspace;
+//         substitution, A, P (.) Gamma, W, Q~ = Qb - A W, Kc, b_C -> workspace
+//         (W, Q~, Kc rounded to tf32 there, the chain's operands as stored);
 //   chain (one CTA per head, chunks last to first): the only sequential part,
 //         dS_r from dS_{r+1} with three products per chunk, storing dS_{r+1}
 //         for every chunk; each warp owns 16 value rows of dS in mma
@@ -33,7 +34,8 @@
 //         value rows go through in slices of 32, the sums over value rows
 //         (dKc, dQb, dW, dA, dT) stay in registers across the slices.
 // Every product is a warp-level tf32 tensor-core MMA (m16n8k8, fp32
-// accumulation) on fp32 tiles in shared memory.  dq, dk, dv, dg, dbeta are
+// accumulation) on fp32 tiles in shared memory; an operand tile is rounded to
+// tf32 (nearest) once, where it is written, so the MMA loops convert nothing.  dq, dk, dv, dg, dbeta are
 // written once per token (no atomics): a chunk's CTA owns its tokens.
 #include <stddef.h>
 
@@ -71,33 +73,45 @@ struct TcBwdArgs {
 // B(k,n) = B[k SBK + n SBN] (pointers at the block's first row / column), B
 // optionally scaled by sck[k].  Fragments (g = lane / 4, t = lane % 4):
 // acc[j] = {(g, 8j+2t), (g, 8j+2t+1), (g+8, 8j+2t), (g+8, 8j+2t+1)}.
-template <int NT, int SAM, int SAK, int SBK, int SBN, bool SCK = false>
+// PERM: the k slots t and t + 4 of each 8-wide step take k = k0 + 2t and
+// k0 + 2t + 1 (a permutation of the summation, the same for A and B): with
+// row strides of 4 (mod 32) words, B rows k0 + 2t then fall on distinct banks,
+// and so do the rows of a transposed A.
+// CVT false: both operands are stored rounded to tf32 already (no conversion).
+template <int NT, int SAM, int SAK, int SBK, int SBN, bool SCK = false, bool PERM = false, bool CVT = true>
 __device__ __forceinline__ void wmma(float (&acc)[NT][4], const float *A, const float *B, int k_begin, int k_end,
                                      const float *sck = nullptr) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int ka = PERM ? 2 * t : t, kb = PERM ? 2 * t + 1 : t + 4;
+    auto op = [](float x) { return CVT ? f2tf32(x) : __float_as_uint(x); };
     for (int k0 = k_begin; k0 < k_end; k0 += 8) {
         uint32_t a[4];
-        a[0] = f2tf32(A[g * SAM + (k0 + t) * SAK]);
-        a[1] = f2tf32(A[(g + 8) * SAM + (k0 + t) * SAK]);
-        a[2] = f2tf32(A[g * SAM + (k0 + t + 4) * SAK]);
-        a[3] = f2tf32(A[(g + 8) * SAM + (k0 + t + 4) * SAK]);
+        a[0] = op(A[g * SAM + (k0 + ka) * SAK]);
+        a[1] = op(A[(g + 8) * SAM + (k0 + ka) * SAK]);
+        a[2] = op(A[g * SAM + (k0 + kb) * SAK]);
+        a[3] = op(A[(g + 8) * SAM + (k0 + kb) * SAK]);
         float s0 = 1.f, s1 = 1.f;
         if (SCK) {
-            s0 = sck[k0 + t];
-            s1 = sck[k0 + t + 4];
+            s0 = sck[k0 + ka];
+            s1 = sck[k0 + kb];
         }
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-            float b0 = B[(k0 + t) * SBK + (8 * j + g) * SBN], b1 = B[(k0 + t + 4) * SBK + (8 * j + g) * SBN];
+            float b0 = B[(k0 + ka) * SBK + (8 * j + g) * SBN], b1 = B[(k0 + kb) * SBK + (8 * j + g) * SBN];
             if (SCK) {
                 b0 *= s0;
                 b1 *= s1;
             }
-            const uint32_t b[2] = {f2tf32(b0), f2tf32(b1)};
+            const uint32_t b[2] = {(SCK || CVT) ? f2tf32(b0) : __float_as_uint(b0),
+                                   (SCK || CVT) ? f2tf32(b1) : __float_as_uint(b1)};
             mma_tf32_16x8x8(acc[j], a, b);
         }
     }
 }
+
+// x rounded to tf32 (nearest, ties away), kept as an fp32 value: an MMA operand
+// stored this way needs no conversion when it is read.
+__device__ __forceinline__ float tf32r(float x) { return __uint_as_float(f2tf32(x)); }
 
 template <int NT>
 __device__ __forceinline__ void zero(float (&a)[NT][4]) {
@@ -105,28 +119,33 @@ __device__ __forceinline__ void zero(float (&a)[NT][4]) {
     for (int j = 0; j < NT; ++j) a[j][0] = a[j][1] = a[j][2] = a[j][3] = 0.f;
 }
 
-// Accumulator block -> shared tile (row stride LD), times `s`.
-template <int NT, int LD>
+// Accumulator block -> shared tile (row stride LD), times `s`; RND: rounded to
+// tf32 (a later MMA operand).
+template <int NT, int LD, bool RND = false>
 __device__ __forceinline__ void store_frag(float *dst, const float (&a)[NT][4], float s = 1.f) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    auto f = [&](float x) { return RND ? tf32r(s * x) : s * x; };
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
-        *reinterpret_cast<float2 *>(dst + g * LD + 8 * j + 2 * t) = make_float2(s * a[j][0], s * a[j][1]);
-        *reinterpret_cast<float2 *>(dst + (g + 8) * LD + 8 * j + 2 * t) = make_float2(s * a[j][2], s * a[j][3]);
+        *reinterpret_cast<float2 *>(dst + g * LD + 8 * j + 2 * t) = make_float2(f(a[j][0]), f(a[j][1]));
+        *reinterpret_cast<float2 *>(dst + (g + 8) * LD + 8 * j + 2 * t) = make_float2(f(a[j][2]), f(a[j][3]));
     }
 }
 
-// Accumulator block -> global rows (row stride ld floats), rows >= nrow skipped.
-template <int NT>
+// Accumulator block -> global rows (row stride ld floats), rows >= nrow skipped;
+// RND: rounded to tf32.
+template <int NT, bool RND = false>
 __device__ __forceinline__ void store_frag_global(float *dst, size_t ld, const float (&a)[NT][4], int row0, int nrow) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    auto f = [](float x) { return RND ? tf32r(x) : x; };
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
         if (row0 + g < nrow)
-            *reinterpret_cast<float2 *>(dst + (size_t)(row0 + g) * ld + 8 * j + 2 * t) = make_float2(a[j][0], a[j][1]);
+            *reinterpret_cast<float2 *>(dst + (size_t)(row0 + g) * ld + 8 * j + 2 * t) =
+                make_float2(f(a[j][0]), f(a[j][1]));
         if (row0 + g + 8 < nrow)
             *reinterpret_cast<float2 *>(dst + (size_t)(row0 + g + 8) * ld + 8 * j + 2 * t) =
-                make_float2(a[j][2], a[j][3]);
+                make_float2(f(a[j][2]), f(a[j][3]));
     }
 }
 
@@ -148,32 +167,46 @@ __device__ __forceinline__ void load_f32(float *dst, const float *src, size_t sw
 template <typename TIn, int W, int LD, int NTH>
 __device__ __forceinline__ void load_in(float *dst, const void *src, size_t sw, int nvalid) {
     if constexpr (sizeof(TIn) == 4) {
-        load_f32<W, LD, NTH>(dst, static_cast<const float *>(src), sw, nvalid);
-    } else {
-        constexpr int V = W / 8;
-        const __nv_bfloat16 *s = static_cast<const __nv_bfloat16 *>(src);
+        // fp32 inputs rounded to tf32 as staged (MMA operands); bf16 values are tf32 already
+        const float *s = static_cast<const float *>(src);
+        constexpr int V = W / 4;
         for (int i = threadIdx.x; i < C * V; i += NTH) {
-            const int r = i / V, c = (i % V) * 8;
-            float f[8];
-            if (r < nvalid) {
-                tcu::unpack_bf16x8(__ldg(reinterpret_cast<const uint4 *>(s + (size_t)r * sw + c)), f);
-            } else {
+            const int r = i / V, c = (i % V) * 4;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < nvalid) x = __ldg(reinterpret_cast<const float4 *>(s + (size_t)r * sw + c));
+            *reinterpret_cast<float4 *>(dst + r * LD + c) = make_float4(tf32r(x.x), tf32r(x.y), tf32r(x.z), tf32r(x.w));
+        }
+    } else {
+        constexpr int V = W / 8, N = (C * V + NTH - 1) / NTH;
+        const __nv_bfloat16 *s = static_cast<const __nv_bfloat16 *>(src);
+        uint4 u[N];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = 0.f;
-            }
+        for (int n = 0; n < N; ++n) {  // every load in flight before the first store
+            const int i = threadIdx.x + n * NTH, r = i / V, c = (i % V) * 8;
+            u[n] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < C * V && r < nvalid) u[n] = __ldg(reinterpret_cast<const uint4 *>(s + (size_t)r * sw + c));
+        }
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+            const int i = threadIdx.x + n * NTH, r = i / V, c = (i % V) * 8;
+            if (i >= C * V) break;
+            float f[8];
+            tcu::unpack_bf16x8(u[n], f);
             *reinterpret_cast<float4 *>(dst + r * LD + c) = make_float4(f[0], f[1], f[2], f[3]);
             *reinterpret_cast<float4 *>(dst + r * LD + c + 4) = make_float4(f[4], f[5], f[6], f[7]);
         }
     }
 }
 
-// Shared tile (row stride LD) -> dense global [rows][W].
-template <int W, int LD>
+// Shared tile (row stride LD) -> dense global [rows][W]; RND: rounded to tf32.
+template <int W, int LD, bool RND = false>
 __device__ __forceinline__ void store_tile(float *dst, const float *src, int rows = C) {
     constexpr int V = W / 4;
     for (int i = threadIdx.x; i < rows * V; i += kThreads) {
         const int r = i / V, c = (i % V) * 4;
-        *reinterpret_cast<float4 *>(dst + (size_t)r * W + c) = *reinterpret_cast<const float4 *>(src + r * LD + c);
+        float4 x = *reinterpret_cast<const float4 *>(src + r * LD + c);
+        if (RND) x = make_float4(tf32r(x.x), tf32r(x.y), tf32r(x.z), tf32r(x.w));
+        *reinterpret_cast<float4 *>(dst + (size_t)r * W + c) = x;
     }
 }
 
@@ -188,12 +221,18 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// [64][W] fp32 rows of global memory into a shared tile, asynchronously; rows
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
+__device__ __forceinline__ void l2_prefetch(const void *p, uint32_t bytes) {
+    if (p && bytes) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// [ROWS][W] fp32 rows of global memory into a shared tile, asynchronously; rows
 // >= nvalid (or a null source) are zero-filled.
-template <int W, int LD, int NTH>
+template <int W, int LD, int NTH, int ROWS = C>
 __device__ __forceinline__ void cp_tile(float *dst, const float *src, size_t sw, int nvalid, const void *dummy) {
     constexpr int V = W / 4;
-    for (int i = threadIdx.x; i < C * V; i += NTH) {
+#pragma unroll 4
+    for (int i = threadIdx.x; i < ROWS * V; i += NTH) {
         const int r = i / V, c = (i % V) * 4;
         const bool ok = src && r < nvalid;
         cp_async16(dst + r * LD + c, ok ? static_cast<const void *>(src + (size_t)r * sw + c) : dummy, ok);
@@ -261,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_prep_kernel(TcBwdArgs p) {
         float aq[4][4], ap[4][4];
         zero(aq);
         zero(ap);
-        wmma<4, LK, 1, 1, LK>(aq, qs + 16 * mt * LK, ks + nb * LK, 0, DKB);
-        if (DELTA) wmma<4, LK, 1, 1, LK>(ap, ks + 16 * mt * LK, ks + nb * LK, 0, DKB);
+        wmma<4, LK, 1, 1, LK, false, false, false>(aq, qs + 16 * mt * LK, ks + nb * LK, 0, DKB);
+        if (DELTA) wmma<4, LK, 1, 1, LK, false, false, false>(ap, ks + 16 * mt * LK, ks + nb * LK, 0, DKB);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -317,7 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_prep_kernel(TcBwdArgs p) {
         const int mt = warp & 3, nb = (warp >> 2) * 64;
         float acc[8][4];
         zero(acc);
-        wmma<8, LC, 1, LK, 1, true>(acc, Ts + 16 * mt * LC, ks + nb, 0, 16 * (mt + 1), bsc);
+        wmma<8, LC, 1, LK, 1, true, true>(acc, Ts + 16 * mt * LC, ks + nb, 0, 16 * (mt + 1), bsc);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[j][e] = tf32r(acc[j][e]);
         store_frag<8, LK>(Ws + 16 * mt * LK + nb, acc);
         __syncthreads();
     }
@@ -326,25 +369,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_prep_kernel(TcBwdArgs p) {
         const int mt = warp & 3, nb = (warp >> 2) * 64;
         float acc[8][4];
         zero(acc);
-        if (DELTA) wmma<8, LC, 1, LK, 1>(acc, As + 16 * mt * LC, Ws + nb, 0, 16 * (mt + 1));
+        if (DELTA) wmma<8, LC, 1, LK, 1, false, true>(acc, As + 16 * mt * LC, Ws + nb, 0, 16 * (mt + 1));
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int l = 16 * mt + g + 8 * (e >> 1), i = nb + 8 * j + 2 * t + (e & 1);
-                qs[l * LK + i] = bs[l] * qs[l * LK + i] - acc[j][e];
+                qs[l * LK + i] = tf32r(bs[l] * qs[l * LK + i] - acc[j][e]);
             }
         if (DELTA)
             for (int i = tid; i < C * DKB; i += kThreads) {
                 const int l = i / DKB, c = i % DKB;
-                ks[l * LK + c] *= es[l];
+                ks[l * LK + c] = tf32r(ks[l * LK + c] * es[l]);
             }
     }
     __syncthreads();
     store_tile<DKB, LK>(p.Qtm + cidx * C * DKB, qs);
-    store_tile<C, LC>(p.Am + cidx * C * C, As);
+    store_tile<C, LC, true>(p.Am + cidx * C * C, As);
     if (DELTA) {
-        store_tile<C, LC>(p.Tm + cidx * C * C, Ts);
+        store_tile<C, LC, true>(p.Tm + cidx * C * C, Ts);
         store_tile<C, LC>(p.PGm + cidx * C * C, PGs);
         store_tile<DKB, LK>(p.Wm + cidx * C * DKB, Ws);
         store_tile<DKB, LK>(p.Kcm + cidx * C * DKB, ks);
@@ -406,7 +449,7 @@ __global__ void __launch_bounds__(DV * 2, 1) bwdtc_chain_kernel(TcBwdArgs p) {
     float bc = p.bC[(size_t)bh * R + R - 1];
     for (int r = R - 1; r >= 0; --r) {
         const size_t cidx = (size_t)bh * R + r;
-        store_frag_global<16>(p.dSn + (cidx * DV + v0) * DKB, DKB, acc, 0, 16);
+        store_frag_global<16, true>(p.dSn + (cidx * DV + v0) * DKB, DKB, acc, 0, 16);  // a local-kernel operand
         const float bc_next = r > 0 ? p.bC[cidx - 1] : 1.f;
         float X[8][4];  // X = dS Kc^T: rows v0 + g (+8), tokens 8n + 2t (+1)
         cp_async_wait<2>();
@@ -419,7 +462,7 @@ __global__ void __launch_bounds__(DV * 2, 1) bwdtc_chain_kernel(TcBwdArgs p) {
 #pragma unroll
                 for (int n = 0; n < 8; ++n) {
                     const float2 kk = *reinterpret_cast<const float2 *>(Kcs + (8 * n + g) * LKC + 8 * j + 2 * t);
-                    const uint32_t b[2] = {f2tf32(kk.x), f2tf32(kk.y)};
+                    const uint32_t b[2] = {__float_as_uint(kk.x), __float_as_uint(kk.y)};  // stored as tf32
                     mma_tf32_16x8x8(X[n], a, b);
                 }
             }
@@ -443,7 +486,7 @@ __global__ void __launch_bounds__(DV * 2, 1) bwdtc_chain_kernel(TcBwdArgs p) {
                 const float *w0 = Wss + (8 * n + 2 * t) * LK + g;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const uint32_t b[2] = {f2tf32(w0[8 * j]), f2tf32(w0[LK + 8 * j])};
+                    const uint32_t b[2] = {__float_as_uint(w0[8 * j]), __float_as_uint(w0[LK + 8 * j])};
                     mma_tf32_16x8x8(acc[j], a, b);
                 }
             }
@@ -465,7 +508,7 @@ __global__ void __launch_bounds__(DV * 2, 1) bwdtc_chain_kernel(TcBwdArgs p) {
             const float *q0 = Qts + l0 * LK + g;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const uint32_t b[2] = {f2tf32(q0[8 * j]), f2tf32(q0[LK + 8 * j])};
+                const uint32_t b[2] = {__float_as_uint(q0[8 * j]), __float_as_uint(q0[LK + 8 * j])};
                 mma_tf32_16x8x8(acc[j], a, b);
             }
         }
@@ -520,12 +563,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
     const size_t cidx = (size_t)bh * p.nch + r;
     const float *Sr = p.states + cidx * DV * DKB, *dSr = p.dSn + cidx * DV * DKB;
 
-    load_in<TIn, DKB, LK, kThreads>(ks, static_cast<const char *>(p.k) + tok0 * DKB * sizeof(TIn), DKB, nv);
-    load_f32<C, LC, kThreads>(As, p.Am + cidx * C * C, C, C);
-    if (DELTA) {
-        load_f32<DKB, LK, kThreads>(Ws, p.Wm + cidx * C * DKB, DKB, C);
-        load_f32<C, LC, kThreads>(Ts, p.Tm + cidx * C * C, C, C);
+    const void *dummy = p.Am;
+    if (tid == 0) {  // everything read after the first tiles, into L2 now
+        l2_prefetch(Sr, DV * DKB * 4);
+        l2_prefetch(dSr, DV * DKB * 4);
+        l2_prefetch(static_cast<const char *>(p.v) + tok0 * DV * sizeof(TIn), nv * DV * sizeof(TIn));
+        if (p.dO) l2_prefetch(p.dO + tok0 * DV, nv * DV * 4);
+        l2_prefetch(static_cast<const char *>(p.q) + tok0 * DKB * sizeof(TIn), nv * DKB * sizeof(TIn));
+        if (DELTA) l2_prefetch(p.PGm + cidx * C * C, C * C * 4);
     }
+    cp_tile<C, LC, kThreads>(As, p.Am + cidx * C * C, C, C, dummy);
+    if (DELTA) {
+        cp_tile<DKB, LK, kThreads>(Ws, p.Wm + cidx * C * DKB, DKB, C, dummy);
+        cp_tile<C, LC, kThreads>(Ts, p.Tm + cidx * C * C, C, C, dummy);
+    }
+    cp_async_commit();
+    load_in<TIn, DKB, LK, kThreads>(ks, static_cast<const char *>(p.k) + tok0 * DKB * sizeof(TIn), DKB, nv);
     if (tid < C) betas[tid] = (DELTA && tid < nv) ? p.beta[tok0 + tid] : 0.f;
     for (int i = tid; i < 7 * C; i += kThreads) dbp[i] = 0.f;  // dbp, dgp, cpp
     if (warp == 0) gate_prefix<GATED>(p.g, tok0, nv, Gs, bs, es);
@@ -540,16 +593,26 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
     for (int s = 0; s < NSL; ++s) {
         const int vb = s * VJ;
         __syncthreads();
+        cp_tile<DKB, LK, kThreads, VJ>(Sj, Sr + (size_t)vb * DKB, DKB, VJ, dummy);
+        cp_tile<DKB, LK, kThreads, VJ>(dSj, dSr + (size_t)vb * DKB, DKB, VJ, dummy);
+        cp_tile<VJ, LJ, kThreads>(dOj, p.dO ? p.dO + tok0 * DV + vb : nullptr, DV, nv, dummy);
+        cp_async_commit();
+        load_in<TIn, VJ, LJ, kThreads>(vj, static_cast<const char *>(p.v) + (tok0 * DV + vb) * sizeof(TIn), DV, nv);
+        cp_async_wait<0>();
+        // the thread's own copies are visible to it: sum of dSn (.) S over them,
+        // and S and dO rounded to tf32 in place (MMA operands; dSn is stored so)
         for (int i = tid; i < VJ * (DKB / 4); i += kThreads) {
             const int rr = i / (DKB / 4), c = (i % (DKB / 4)) * 4;
-            const float4 a = __ldg(reinterpret_cast<const float4 *>(Sr + (size_t)(vb + rr) * DKB + c));
-            const float4 b = __ldg(reinterpret_cast<const float4 *>(dSr + (size_t)(vb + rr) * DKB + c));
-            *reinterpret_cast<float4 *>(Sj + rr * LK + c) = a;
-            *reinterpret_cast<float4 *>(dSj + rr * LK + c) = b;
+            float4 a = *reinterpret_cast<const float4 *>(Sj + rr * LK + c);
+            const float4 b = *reinterpret_cast<const float4 *>(dSj + rr * LK + c);
             sds += a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+            *reinterpret_cast<float4 *>(Sj + rr * LK + c) = make_float4(tf32r(a.x), tf32r(a.y), tf32r(a.z), tf32r(a.w));
         }
-        load_in<TIn, VJ, LJ, kThreads>(vj, static_cast<const char *>(p.v) + (tok0 * DV + vb) * sizeof(TIn), DV, nv);
-        load_f32<VJ, LJ, kThreads>(dOj, p.dO ? p.dO + tok0 * DV + vb : nullptr, DV, nv);
+        for (int i = tid; i < C * (VJ / 4); i += kThreads) {
+            const int rr = i / (VJ / 4), c = (i % (VJ / 4)) * 4;
+            const float4 a = *reinterpret_cast<const float4 *>(dOj + rr * LJ + c);
+            *reinterpret_cast<float4 *>(dOj + rr * LJ + c) = make_float4(tf32r(a.x), tf32r(a.y), tf32r(a.z), tf32r(a.w));
+        }
         __syncthreads();
         // Z and dZ for this slice: warp (mt, nh) owns rows 16 mt, columns 16 nh
         {
@@ -559,14 +622,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
             if (DELTA) {
                 float au[2][4];
                 zero(au);
-                wmma<2, LC, 1, LJ, 1, true>(au, Ts + 16 * mt * LC, vj + 16 * nh, 0, 16 * (mt + 1), betas);
-                wmma<2, LK, 1, 1, LK>(az, Ws + 16 * mt * LK, Sj + 16 * nh * LK, 0, DKB);
+                wmma<2, LC, 1, LJ, 1, true, false, false>(au, Ts + 16 * mt * LC, vj + 16 * nh, 0, 16 * (mt + 1),
+                                                          betas);
+                wmma<2, LK, 1, 1, LK, false, false, false>(az, Ws + 16 * mt * LK, Sj + 16 * nh * LK, 0, DKB);
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) az[j][e] = au[j][e] - az[j][e];
             }
-            wmma<2, LK, 1, 1, LK>(adz, ks + 16 * mt * LK, dSj + 16 * nh * LK, 0, DKB);
+            wmma<2, LK, 1, 1, LK, false, false, false>(adz, ks + 16 * mt * LK, dSj + 16 * nh * LK, 0, DKB);
             if (GATED) {
                 const float e0 = es[16 * mt + g], e1 = es[16 * mt + g + 8];
 #pragma unroll
@@ -577,23 +641,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
                     adz[j][3] *= e1;
                 }
             }
-            wmma<2, 1, LC, LJ, 1>(adz, As + 16 * mt, dOj + 16 * nh, 16 * mt, C);
-            if (DELTA) store_frag<2, LJ>(Zj + 16 * mt * LJ + 16 * nh, az);
-            store_frag<2, LJ>(dZj + 16 * mt * LJ + 16 * nh, adz);
+            wmma<2, 1, LC, LJ, 1, false, true, false>(adz, As + 16 * mt, dOj + 16 * nh, 16 * mt, C);
+            if (DELTA) store_frag<2, LJ, true>(Zj + 16 * mt * LJ + 16 * nh, az);
+            store_frag<2, LJ, true>(dZj + 16 * mt * LJ + 16 * nh, adz);
             if (!DELTA) store_frag_global<2>(p.dv + tok0 * DV + vb + 16 * nh, DV, adz, 16 * mt, nv);
         }
         __syncthreads();
         const float *Zs = DELTA ? Zj : vj;
-        wmma<8, LJ, 1, LK, 1>(dKc, Zs + 16 * mt * LJ, dSj + 64 * nh, 0, VJ);
-        wmma<8, LJ, 1, LK, 1>(dQb, dOj + 16 * mt * LJ, Sj + 64 * nh, 0, VJ);
-        wmma<4, LJ, 1, 1, LJ>(dA, dOj + 16 * mt * LJ, Zs + 32 * nh * LJ, 0, VJ);
+        wmma<8, LJ, 1, LK, 1, false, true, false>(dKc, Zs + 16 * mt * LJ, dSj + 64 * nh, 0, VJ);
+        wmma<8, LJ, 1, LK, 1, false, true, false>(dQb, dOj + 16 * mt * LJ, Sj + 64 * nh, 0, VJ);
+        wmma<4, LJ, 1, 1, LJ, false, false, false>(dA, dOj + 16 * mt * LJ, Zs + 32 * nh * LJ, 0, VJ);
         if (DELTA) {
-            wmma<8, LJ, 1, LK, 1>(dWa, dZj + 16 * mt * LJ, Sj + 64 * nh, 0, VJ);
-            wmma<4, LJ, 1, 1, LJ>(dTv, dZj + 16 * mt * LJ, vj + 32 * nh * LJ, 0, VJ);
+            wmma<8, LJ, 1, LK, 1, false, true, false>(dWa, dZj + 16 * mt * LJ, Sj + 64 * nh, 0, VJ);
+            wmma<4, LJ, 1, 1, LJ, false, false, false>(dTv, dZj + 16 * mt * LJ, vj + 32 * nh * LJ, 0, VJ);
             // dv = diag(beta) T^T dZ;  dbeta += rows of (T^T dZ) (.) v
             float ad[2][4];
             zero(ad);
-            wmma<2, 1, LC, LJ, 1>(ad, Ts + 16 * mt, dZj + 16 * nh, 16 * mt, C);
+            wmma<2, 1, LC, LJ, 1, false, true, false>(ad, Ts + 16 * mt, dZj + 16 * nh, 16 * mt, C);
             float rb0 = 0.f, rb1 = 0.f;
             const int l0 = 16 * mt + g;
 #pragma unroll
@@ -624,10 +688,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
     __syncthreads();
 
     float *dAs = sm + S::dAs, *qs = sm + S::qs, *PGs = sm + S::PGs;
-    if (DELTA) store_frag<8, LK>(Ws + 16 * mt * LK + 64 * nh, dWa, -1.f);  // dW
+    if (DELTA) store_frag<8, LK, true>(Ws + 16 * mt * LK + 64 * nh, dWa, -1.f);  // dW
     store_frag<4, LC>(dAs + 16 * mt * LC + 32 * nh, dA);
+    if (DELTA) cp_tile<C, LC, kThreads>(PGs, p.PGm + cidx * C * C, C, C, dummy);
+    cp_async_commit();
     load_in<TIn, DKB, LK, kThreads>(qs, static_cast<const char *>(p.q) + tok0 * DKB * sizeof(TIn), DKB, nv);
-    if (DELTA) load_f32<C, LC, kThreads>(PGs, p.PGm + cidx * C * C, C, C);
+    cp_async_wait<0>();
     __syncthreads();
 
     if (DELTA) {
@@ -635,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
         {
             float a2[4][4];
             zero(a2);
-            wmma<4, LK, 1, 1, LK>(a2, Ws + 16 * mt * LK, ks + 32 * nh * LK, 0, DKB);
+            wmma<4, LK, 1, 1, LK, false, false, false>(a2, Ws + 16 * mt * LK, ks + 32 * nh * LK, 0, DKB);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -643,20 +709,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
                     const int m = 32 * nh + 8 * j + 2 * t + (e & 1);
                     dTv[j][e] = betas[m] * (dTv[j][e] + bs[m] * a2[j][e]);
                 }
-            store_frag<4, LC>(X0 + 16 * mt * LC + 32 * nh, dTv);
+            store_frag<4, LC, true>(X0 + 16 * mt * LC + 32 * nh, dTv);
         }
         __syncthreads();
         {  // Y = dT T^T
             float y[4][4];
             zero(y);
-            wmma<4, LC, 1, 1, LC>(y, X0 + 16 * mt * LC, Ts + 32 * nh * LC, 0, C);
-            store_frag<4, LC>(X1 + 16 * mt * LC + 32 * nh, y);
+            wmma<4, LC, 1, 1, LC, false, false, false>(y, X0 + 16 * mt * LC, Ts + 32 * nh * LC, 0, C);
+            store_frag<4, LC, true>(X1 + 16 * mt * LC + 32 * nh, y);
         }
         __syncthreads();
         {  // dL = strict-lower(-T^T Y)
             float dl[4][4];
             zero(dl);
-            wmma<4, 1, LC, LC, 1>(dl, Ts + 16 * mt, X1 + 32 * nh, 16 * mt, C);
+            wmma<4, 1, LC, LC, 1, false, true, false>(dl, Ts + 16 * mt, X1 + 32 * nh, 16 * mt, C);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -680,12 +746,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
             const float gam = m <= l ? (GATED ? expf(Gl - Gs[m]) : 1.f) : 0.f;
             const float da = dAs[l * LC + m];
             float h = m < l ? da * As[l * LC + m] : 0.f;
-            dAs[l * LC + m] = da * gam;
+            dAs[l * LC + m] = tf32r(da * gam);
             if (DELTA) {
                 const float dl = X0[l * LC + m], pg = PGs[l * LC + m];
                 h += dl * bl * pg;
                 rowB += dl * pg;
-                X0[l * LC + m] = dl * bl * gam;
+                X0[l * LC + m] = tf32r(dl * bl * gam);
             }
             X1[l * LC + m] = h;
             rowH += h;
@@ -713,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
         if (DELTA) {
             float kb[8][4];
             zero(kb);
-            wmma<8, 1, LC, LK, 1>(kb, Ts + 16 * mt, Ws + nb, 16 * mt, C);  // T^T dW
+            wmma<8, 1, LC, LK, 1, false, true, false>(kb, Ts + 16 * mt, Ws + nb, 16 * mt, C);  // T^T dW
 #pragma unroll
             for (int j = 0; j < 8; ++j)
 #pragma unroll
@@ -736,11 +802,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
                 dqacc[j][e] = bs[l] * dQb[j][e];
             }
         if (DELTA) {
-            wmma<8, LC, 1, LK, 1>(dkacc, X0 + 16 * mt * LC, ks + nb, 0, 16 * (mt + 1));  // E k
-            wmma<8, 1, LC, LK, 1>(dkacc, X0 + 16 * mt, ks + nb, 16 * mt, C);             // E^T k
+            wmma<8, LC, 1, LK, 1, false, true, false>(dkacc, X0 + 16 * mt * LC, ks + nb, 0, 16 * (mt + 1));  // E k
+            wmma<8, 1, LC, LK, 1, false, true, false>(dkacc, X0 + 16 * mt, ks + nb, 16 * mt, C);  // E^T k
         }
-        wmma<8, 1, LC, LK, 1>(dkacc, dAs + 16 * mt, qs + nb, 16 * mt, C);             // F^T q
-        wmma<8, LC, 1, LK, 1>(dqacc, dAs + 16 * mt * LC, ks + nb, 0, 16 * (mt + 1));  // F k
+        wmma<8, 1, LC, LK, 1, false, true, false>(dkacc, dAs + 16 * mt, qs + nb, 16 * mt, C);  // F^T q
+        wmma<8, LC, 1, LK, 1, false, true, false>(dqacc, dAs + 16 * mt * LC, ks + nb, 0, 16 * (mt + 1));  // F k
         store_frag_global<8>(p.dk + tok0 * DKB + nb, DKB, dkacc, 16 * mt, nv);
         store_frag_global<8>(p.dq + tok0 * DKB + nb, DKB, dqacc, 16 * mt, nv);
 #pragma unroll

@@ -94,11 +94,14 @@ def test_tc_backward_many_heads():
 
 def test_tc_backward_deep_decay():
     """About -2 nats per token: e^G of a chunk falls below the fp32 range; the
-    gradient must stay finite and match."""
+    gradient must stay finite and match.  Bound: the tensor-core one (2e-2) of
+    the forward parity tests; this stress case measures 1.2e-2 on dk (every
+    product's operands rounded to tf32; rounding q and k alone gives 2.5e-3 in a
+    float64 model of the chunk algebra)."""
     x = list(inputs(35, "delta", "scalar", T=200))
     r = np.random.default_rng(35)
     x[3] = np.asarray(-2.0 + 0.3 * r.standard_normal(x[3].shape), np.float32).astype(np.float64)
-    got = run_tc("delta", "scalar", tuple(x), bf16=False)
+    got = run_tc("delta", "scalar", tuple(x), bf16=False, tol=TOL_STATES)
     assert all(a is None or torch.isfinite(a).all() for a in got)
 
 
