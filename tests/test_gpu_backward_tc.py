@@ -154,3 +154,39 @@ def test_tc_backward_rejects_unsupported_requests():
     states = torch.zeros((1, 2, 2, 64, 64), device="cuda")
     with pytest.raises(gdn.GDNError):
         gdn.chunk_bwd(q, k, v, g, beta, None, None, None, update="delta", gate="scalar", states=states, algo="tc")
+
+
+def test_tc_backward_full_size_sampled_heads():
+    """The GDN workload (8 x 16 x 8192) at full size, in the launch configuration
+    the benchmark times: gdn_chunk_fwd_states, then gdn_chunk_bwd_tc over all 128
+    heads.  Sampled heads are compared whole against the oracle's gradients."""
+    from synth import WORKLOADS, make_prefill_inputs
+
+    w = WORKLOADS["gdn_prefill_bf16"]
+    x = make_prefill_inputs(w)
+    t = [dev(x["q"], torch.bfloat16), dev(x["k"], torch.bfloat16), dev(x["v"], torch.bfloat16), dev(x["g"]),
+         dev(x["beta"])]
+    S0 = dev(x["S0"])
+    del x
+    gen = torch.Generator(device="cuda").manual_seed(41)
+    dO = torch.randn((w.B, w.H, w.T, w.dv), device="cuda", generator=gen)
+    dST = torch.randn((w.B, w.H, w.dv, w.dk), device="cuda", generator=gen)
+    states = torch.empty((w.B, w.H, (w.T + 63) // 64, w.dv, w.dk), device="cuda")
+    gdn.device_status(clear=True)
+    gdn.chunk_fwd(*t, S0, update=w.update, gate=w.gate, states=states)
+    got = gdn.chunk_bwd(*t, None, dO, dST, update=w.update, gate=w.gate, states=states, algo="tc")
+    torch.cuda.synchronize()
+    assert gdn.device_status(clear=True) == 0
+    assert all(a is None or torch.isfinite(a).all() for a in got)
+    heads = [(0, 0), (7, 15), (3, 9)]
+    xs = make_prefill_inputs(w, heads=heads)
+    for i, (b, h) in enumerate(heads):
+        one = lambda a: None if a is None else np.asarray(a[i:i + 1], np.float64)
+        ref = oracle.gdn_backward_np(w.update, w.gate, one(xs["q"]), one(xs["k"]), one(xs["v"]), one(xs["g"]),
+                                     one(xs["beta"]), one(xs["S0"]), np64(dO[b, h])[None, None],
+                                     np64(dST[b, h])[None, None])
+        for name, a, r in zip(NAMES, got, ref):
+            if r is None:
+                continue
+            err = rel_err(np64(a[b, h]), r[0, 0])
+            assert err <= TOL_STATES, ((b, h), name, err)
