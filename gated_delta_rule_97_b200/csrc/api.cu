@@ -706,9 +706,10 @@ int gdn_launch_bwd_tc(const void *q, const void *k, const void *v, const float *
                       float *dg, float *dbeta, float *dS0, void *ws, int BH, int T, int dv_, int update, int gate,
                       int in_bf16, cudaStream_t st);
 
+// The per-chunk kernels put the heads on the grid's y dimension (at most 65535).
 static bool bwd_tc_supported(const gdn_desc_t *d) {
     return d->prologue == 0 && d->gate != GDN_GATE_CHANNEL && d->dk == 128 && (d->dv == 64 || d->dv == 128) &&
-           (d->chunk == 0 || d->chunk == gdn::kChunk);
+           (d->chunk == 0 || d->chunk == gdn::kChunk) && (long)d->B * d->H <= 65535;
 }
 
 extern "C" size_t gdn_bwd_tc_workspace_bytes(const gdn_desc_t *d) {

@@ -385,7 +385,7 @@ int gdn_chunk_bwd_states(const gdn_desc_t *desc, const void *q, const void *k, c
  * states'.  dq, dk, dv, dg, dbeta are written once per token (deterministic).
  *
  *   desc        update any, gate NONE or SCALAR, dk = 128, dv in {64, 128},
- *               dtype bf16 or f32, prologue 0, chunk 0 or 64
+ *               dtype bf16 or f32, prologue 0, chunk 0 or 64, B*H <= 65535
  *               (GDN_ERR_UNSUPPORTED otherwise).
  *   states      [B,H,ceil(T/64),dv,dk] float, the chunk-entry states
  *               (gdn_chunk_fwd_states); required when B*H*T > 0.

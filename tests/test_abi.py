@@ -291,7 +291,7 @@ def test_tensor_core_backward_rejects_bad_arguments(lib):
     bad[0] = vp(0x1000008)
     assert f(ctypes.byref(d), *ins, *bad, ws, need, None) == -2                # misaligned
     assert f(ctypes.byref(d), *ins, *outs, vp(0x1100000), need, None) == -1   # workspace overlaps dk
-    for unsupported in (_desc(T=130, gate="channel"), _desc(T=130, dk=64, dv=64)):
+    for unsupported in (_desc(T=130, gate="channel"), _desc(T=130, dk=64, dv=64), _desc(B=65536, H=1, T=130)):
         assert lib.gdn_bwd_tc_workspace_bytes(ctypes.byref(unsupported)) == 0
         assert f(ctypes.byref(unsupported), *ins, *outs, ws, need, None) == -3
     p = _desc(T=130)
