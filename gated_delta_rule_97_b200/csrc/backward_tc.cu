@@ -539,6 +539,7 @@ struct LocalSmem {
     // dbp[2][64] beta gradient by column half, dgp[3][64] gate gradient (element
     // pass, then the two column halves), cpp[2][64] the K> gate term, redw[8]
     // per-warp sums of dSn (.) S
+    static_assert(VJ * LK <= C * LC, "an S slice must fit the X0 / X1 tiles");
     static constexpr int X0 = Rend, X1 = X0 + C * LC, Gs = X1 + C * LC, bs = Gs + C, es = bs + C, betas = es + C,
                          dbp = betas + C, dgp = dbp + 2 * C, cpp = dgp + 3 * C, redw = cpp + 2 * C,
                          floats = redw + 8;
@@ -551,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
     extern __shared__ float4 smem4[];
     float *sm = reinterpret_cast<float *>(smem4);
     float *ks = sm + S::ks, *Ws = sm + S::Ws, *Ts = sm + S::Ts, *As = sm + S::As;
-    float *Sj = sm + S::Sj, *dSj = sm + S::dSj, *vj = sm + S::vj, *dOj = sm + S::dOj, *Zj = sm + S::Zj,
+    float *Sj0 = sm + S::Sj, *dSj0 = sm + S::dSj, *vj = sm + S::vj, *dOj = sm + S::dOj, *Zj = sm + S::Zj,
           *dZj = sm + S::dZj;
     float *X0 = sm + S::X0, *X1 = sm + S::X1, *Gs = sm + S::Gs, *bs = sm + S::bs, *es = sm + S::es,
           *betas = sm + S::betas, *dbp = sm + S::dbp, *dgp = sm + S::dgp, *cpp = sm + S::cpp, *redw = sm + S::redw;
@@ -590,15 +591,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_local_kernel(TcBwdArgs p) {
     zero(dA);
     zero(dTv);
     float sds = 0.f;  // sum of dSn (.) S over the thread's loads
+    // S and dSn rows go through two buffers: slice s in (Sj0, dSj0) for even s and in
+    // (X0, X1), free until the element pass, for odd s; slice s + 1 is copied while
+    // slice s is processed
+    cp_tile<DKB, LK, kThreads, VJ>(Sj0, Sr, DKB, VJ, dummy);
+    cp_tile<DKB, LK, kThreads, VJ>(dSj0, dSr, DKB, VJ, dummy);
+    cp_async_commit();
     for (int s = 0; s < NSL; ++s) {
         const int vb = s * VJ;
+        float *Sj = (s & 1) ? X0 : Sj0, *dSj = (s & 1) ? X1 : dSj0;
         __syncthreads();
-        cp_tile<DKB, LK, kThreads, VJ>(Sj, Sr + (size_t)vb * DKB, DKB, VJ, dummy);
-        cp_tile<DKB, LK, kThreads, VJ>(dSj, dSr + (size_t)vb * DKB, DKB, VJ, dummy);
         cp_tile<VJ, LJ, kThreads>(dOj, p.dO ? p.dO + tok0 * DV + vb : nullptr, DV, nv, dummy);
         cp_async_commit();
+        if (s + 1 < NSL) {
+            cp_tile<DKB, LK, kThreads, VJ>((s & 1) ? Sj0 : X0, Sr + (size_t)(vb + VJ) * DKB, DKB, VJ, dummy);
+            cp_tile<DKB, LK, kThreads, VJ>((s & 1) ? dSj0 : X1, dSr + (size_t)(vb + VJ) * DKB, DKB, VJ, dummy);
+        }
+        cp_async_commit();
         load_in<TIn, VJ, LJ, kThreads>(vj, static_cast<const char *>(p.v) + (tok0 * DV + vb) * sizeof(TIn), DV, nv);
-        cp_async_wait<0>();
+        cp_async_wait<1>();  // all but the next slice's copies
         // the thread's own copies are visible to it: sum of dSn (.) S over them,
         // and S and dO rounded to tf32 in place (MMA operands; dSn is stored so)
         for (int i = tid; i < VJ * (DKB / 4); i += kThreads) {
