@@ -99,3 +99,103 @@ def chunk_forward_heads(update, gate, q, k, v, g=None, beta=None, S0=None, C=64,
                                    None if bf is None else bf[i], None if sf is None else sf[i], C,
                                    emulate_bf16)
     return O.reshape(lead + (T, dv)), S.reshape(lead + (dv, dk))
+
+
+def chunk_backward(update, gate, q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, C=64):
+    """Reverse mode through the chunk algebra above, float64, one head, the
+    scalar or no gate: the passes the tensor-core backward runs.  Returns (dq,
+    dk, dv, dg, dbeta, dS0) (dg / dbeta None without gate / delta rule).
+
+    Per chunk, with S the state entering it and dSn the gradient of the state
+    leaving it (Qb = diag(b) q, Kb = diag(b) k, Kc = diag(b_C / b) k, PG =
+    strict-lower(k k^T) Gamma, Mv = diag(beta) v, Mk = diag(beta) Kb):
+      dZ = A^T dO + Kc dSn^T;   dKc = Z dSn;   dA = dO Z^T;   dQb = dO S
+      delta: dW = -dZ S;  dT = dZ Mv^T + dW Mk^T;  dL = strict-lower(-T^T dT T^T)
+             dv = diag(beta) T^T dZ;  dKb = diag(beta) T^T dW
+      else:  dv = dZ
+      dS_r = b_C dSn + dO^T Qb - dZ^T W = b_C dSn - (dSn Kc^T) W + dO^T (Qb - A W)
+    then dq, dk, dbeta through Qb, Kb, Kc, L = diag(beta) PG and A = lower(q k^T)
+    Gamma, and the gate through every exponential: dG_l from b_l, b_C / b_l,
+    Gamma and b_C S, with dg_s = sum_{l >= s} dG_l."""
+    assert gate in ("none", "scalar")
+    T, dk = q.shape
+    dv_ = v.shape[1]
+    delta, gated = update == "delta", gate == "scalar"
+    n = max(1, -(-T // C))
+    pad = lambda a, w: np.concatenate([a, np.zeros((n * C - T,) + a.shape[1:])]) if a is not None else np.zeros(w)
+    qq, kk, vv = pad(q, None), pad(k, None), pad(v, None)
+    gg = pad(g, None) if gated else np.zeros(n * C)
+    bb = pad(beta, None) if delta else np.zeros(n * C)
+    do = pad(dO, None) if dO is not None else np.zeros((n * C, dv_))
+    S = np.zeros((dv_, dk)) if S0 is None else np.array(S0, np.float64)
+    # forward over the chunks: the states entering them and the chunk tiles
+    states, tiles = [], []
+    for r in range(n):
+        sl = slice(r * C, r * C + C)
+        qc, kc, vc, bc = qq[sl], kk[sl], vv[sl], bb[sl]
+        G = np.cumsum(gg[sl])
+        b, ec, bC = np.exp(G), np.exp(G[-1] - G), np.exp(G[-1])
+        Gam = np.tril(np.exp(G[:, None] - G[None, :]))
+        A = np.tril(qc @ kc.T) * Gam
+        tl = dict(G=G, b=b, ec=ec, bC=bC, Gam=Gam, A=A)
+        if delta:
+            tl["PG"] = np.tril(kc @ kc.T, -1) * Gam
+            tl["T"] = np.linalg.inv(np.eye(C) + bc[:, None] * tl["PG"])
+            tl["W"] = tl["T"] @ ((bc * b)[:, None] * kc)
+            Z = tl["T"] @ (bc[:, None] * vc) - tl["W"] @ S.T
+        else:
+            Z = vc
+        tl["Qt"] = b[:, None] * qc - (A @ tl["W"] if delta else 0.0)
+        tl["Kc"] = ec[:, None] * kc
+        states.append(S)
+        tiles.append(tl)
+        S = bC * S + Z.T @ tl["Kc"]
+    # the state-gradient chain, chunks last to first
+    dS = np.zeros((dv_, dk)) if dS_T is None else np.array(dS_T, np.float64)
+    dSn = [None] * n
+    for r in range(n - 1, -1, -1):
+        tl, doc = tiles[r], do[r * C:(r + 1) * C]
+        dSn[r] = dS
+        nxt = tl["bC"] * dS + doc.T @ tl["Qt"]
+        if delta:
+            nxt = nxt - (dS @ tl["Kc"].T) @ tl["W"]
+        dS = nxt
+    out_q, out_k, out_v = np.zeros((n * C, dk)), np.zeros((n * C, dk)), np.zeros((n * C, dv_))
+    out_g, out_b = np.zeros(n * C), np.zeros(n * C)
+    # every chunk's local gradients
+    for r in range(n):
+        tl, sl = tiles[r], slice(r * C, r * C + C)
+        qc, kc, vc, bc, doc = qq[sl], kk[sl], vv[sl], bb[sl], do[sl]
+        Sr, dSr = states[r], dSn[r]
+        b, ec, bC, Gam, A = tl["b"], tl["ec"], tl["bC"], tl["Gam"], tl["A"]
+        Z = (tl["T"] @ (bc[:, None] * vc) - tl["W"] @ Sr.T) if delta else vc
+        dZ = ec[:, None] * (kc @ dSr.T) + A.T @ doc
+        dKc, dQb, dA = Z @ dSr, doc @ Sr, doc @ Z.T
+        dG, db = np.zeros(C), np.zeros(C)
+        H = np.tril(dA * A, -1)
+        dkk = ec[:, None] * dKc
+        if delta:
+            Tm, PG = tl["T"], tl["PG"]
+            dW = -dZ @ Sr
+            tdz, kb = Tm.T @ dZ, Tm.T @ dW
+            dvv = bc[:, None] * tdz
+            dT = bc[None, :] * (dZ @ vc.T + b[None, :] * (dW @ kc.T))
+            dL = np.tril(-Tm.T @ dT @ Tm.T, -1)
+            E = dL * bc[:, None] * Gam
+            s = np.sum(kb * kc, axis=1)
+            db += np.sum(tdz * vc, axis=1) + b * s + np.sum(dL * PG, axis=1)
+            dG += b * bc * s
+            H = H + dL * bc[:, None] * PG
+            dkk = dkk + (b * bc)[:, None] * kb + E @ kc + E.T @ kc
+        else:
+            dvv = dZ
+        F = np.tril(dA) * Gam
+        dkk = dkk + F.T @ qc
+        dqq = b[:, None] * dQb + F @ kc
+        cp = ec * np.sum(kc * dKc, axis=1)
+        dG += b * np.sum(qc * dQb, axis=1) - cp + H.sum(1) - H.sum(0)
+        dG[-1] += bC * np.sum(dSr * Sr) + cp.sum()
+        out_q[sl], out_k[sl], out_v[sl] = dqq, dkk, dvv
+        out_g[sl] = np.cumsum(dG[::-1])[::-1]
+        out_b[sl] = db
+    return (out_q[:T], out_k[:T], out_v[:T], out_g[:T] if gated else None, out_b[:T] if delta else None, dS)

@@ -63,3 +63,32 @@ def test_bf16_operands_would_exceed_tolerance(oracle_mod):
     oc, _ = chunk_forward_heads("delta", "scalar", x["q"], x["k"], x["v"], g=x["g"], beta=x["beta"],
                                 S0=x["S0"], C=64, emulate_bf16="bf16")
     assert rel_err(oc, o) > 2e-2
+
+
+# ----------------------------------------------------------------------------
+# The chunkwise backward (the passes of the tensor-core backward) equals the
+# oracle's reverse mode through the token loop, for every chunk size.
+BWD_CASES = [("additive", "none"), ("decay", "scalar"), ("delta", "none"), ("delta", "scalar")]
+
+
+@pytest.mark.parametrize("update,gate", BWD_CASES)
+@pytest.mark.parametrize("C,T", [(64, 150), (16, 40), (64, 1), (4, 64)])
+@pytest.mark.parametrize("s0,grads", [(True, (True, True)), (False, (True, False)), (True, (False, True))])
+def test_chunk_backward_model_matches_oracle(update, gate, C, T, s0, grads):
+    from chunk_model import chunk_backward
+
+    q, k, v, g, beta, S0 = rand_inputs(43, BH=2, T=T, dk=16, dv=12, gate=gate,
+                                       delta=(update == "delta"), s0=s0, gmin=-0.5)
+    r = np.random.default_rng(44)
+    dO = r.standard_normal((2, T, 12)) if grads[0] else None
+    dST = r.standard_normal((2, 12, 16)) if grads[1] else None
+    ref = oracle.gdn_backward_np(update, gate, q, k, v, g, beta, S0, dO, dST)
+    for h in range(2):
+        one = lambda a: None if a is None else a[h]
+        got = chunk_backward(update, gate, one(q), one(k), one(v), one(g), one(beta), one(S0), one(dO), one(dST),
+                             C=C)
+        for name, a, b in zip(["dq", "dk", "dv", "dg", "dbeta", "dS0"], got, ref):
+            if b is None:
+                assert a is None, name
+                continue
+            assert rel_err(a, b[h]) < 1e-10, (name, rel_err(a, b[h]))
