@@ -265,27 +265,30 @@ __device__ __forceinline__ void gate_prefix(const float *g, long tok0, int nv, f
 }
 
 // ------------------------------------------------------------------ prep
+// Four large tiles, reused: q then W; k; P (.) Gamma then A; T.  L = diag(beta)
+// P (.) Gamma is taken from P (.) Gamma when read.  107 KB: two CTAs per SM.
 struct PrepSmem {
-    static constexpr int qs = 0, ks = qs + C * LK, Ws = ks + C * LK, Ls = Ws + C * LK, As = Ls + C * LC,
-                         PGs = As + C * LC, Ts = PGs + C * LC, Rs = Ts + C * LC, Gs = Rs + 16 * 52, bs = Gs + C,
-                         es = bs + C, betas = es + C, bsc = betas + C, floats = bsc + C;
+    static constexpr int qs = 0, ks = qs + C * LK, PGs = ks + C * LK, Ts = PGs + C * LC, Rs = Ts + C * LC,
+                         Gs = Rs + 16 * 52, bs = Gs + C, es = bs + C, betas = es + C, bsc = betas + C,
+                         floats = bsc + C;
 };
 
 template <bool DELTA, bool GATED, typename TIn>
-__global__ void __launch_bounds__(kThreads, 1) bwdtc_prep_kernel(TcBwdArgs p) {
+__global__ void __launch_bounds__(kThreads, 2) bwdtc_prep_kernel(TcBwdArgs p) {
     extern __shared__ float4 smem4[];
     float *sm = reinterpret_cast<float *>(smem4);
     using S = PrepSmem;
-    float *qs = sm + S::qs, *ks = sm + S::ks, *Ws = sm + S::Ws, *Ls = sm + S::Ls, *As = sm + S::As,
-          *PGs = sm + S::PGs, *Ts = sm + S::Ts, *Rs = sm + S::Rs, *Gs = sm + S::Gs, *bs = sm + S::bs,
-          *es = sm + S::es, *betas = sm + S::betas, *bsc = sm + S::bsc;
+    float *qs = sm + S::qs, *ks = sm + S::ks, *PGs = sm + S::PGs, *Ts = sm + S::Ts, *Rs = sm + S::Rs,
+          *Gs = sm + S::Gs, *bs = sm + S::bs, *es = sm + S::es, *betas = sm + S::betas, *bsc = sm + S::bsc;
+    float *Ws = qs, *As = PGs;  // W over q once A is formed; A over P (.) Gamma after the solve
     const int r = blockIdx.x, bh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
     const long tok0 = (long)bh * p.T + (long)r * C;
     const int nv = min(C, p.T - r * C);
     const size_t cidx = (size_t)bh * p.nch + r;
+    const TIn *qg = static_cast<const TIn *>(p.q) + tok0 * DKB;
 
-    load_in<TIn, DKB, LK, kThreads>(qs, static_cast<const char *>(p.q) + tok0 * DKB * sizeof(TIn), DKB, nv);
+    load_in<TIn, DKB, LK, kThreads>(qs, qg, DKB, nv);
     load_in<TIn, DKB, LK, kThreads>(ks, static_cast<const char *>(p.k) + tok0 * DKB * sizeof(TIn), DKB, nv);
     if (tid < C) betas[tid] = (DELTA && tid < nv) ? p.beta[tok0 + tid] : 0.f;
     if (DELTA)
@@ -293,43 +296,37 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_prep_kernel(TcBwdArgs p) {
     if (warp == 0) gate_prefix<GATED>(p.g, tok0, nv, Gs, bs, es);
     __syncthreads();
     if (tid < C) bsc[tid] = betas[tid] * bs[tid];
-
-    // A = q k^T (.) Gamma (lower incl.), P (.) Gamma and L = diag(beta) P (.) Gamma (strict lower)
-    {
-        const int mt = warp & 3, nb = (warp >> 2) * 32;
-        float aq[4][4], ap[4][4];
-        zero(aq);
-        zero(ap);
-        wmma<4, LK, 1, 1, LK, false, false, false>(aq, qs + 16 * mt * LK, ks + nb * LK, 0, DKB);
-        if (DELTA) wmma<4, LK, 1, 1, LK, false, false, false>(ap, ks + 16 * mt * LK, ks + nb * LK, 0, DKB);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int l = 16 * mt + g + 8 * (e >> 1), m = nb + 8 * j + 2 * t + (e & 1);
-                const float gam = m <= l ? (GATED ? expf(Gs[l] - Gs[m]) : 1.f) : 0.f;
-                As[l * LC + m] = aq[j][e] * gam;
-                if (DELTA) {
-                    const float pg = m < l ? ap[j][e] * gam : 0.f;
-                    PGs[l * LC + m] = pg;
-                    Ls[l * LC + m] = betas[l] * pg;
-                }
-            }
-    }
-    __syncthreads();
+    const int mt = warp & 3, nb32 = (warp >> 2) * 32, nb64 = (warp >> 2) * 64;
+    auto gamma = [&](int l, int m) { return m <= l ? (GATED ? expf(Gs[l] - Gs[m]) : 1.f) : 0.f; };
 
     if (DELTA) {
-        // T = (I + L)^-1: the four 16 x 16 diagonal blocks by forward substitution
-        // (lane c of warp I solves column c of block I), then block rows 1..3:
-        // T_IJ = -T_II sum_K L_IK T_KJ
+        // P (.) Gamma, strict lower
+        {
+            float ap[4][4];
+            zero(ap);
+            wmma<4, LK, 1, 1, LK, false, false, false>(ap, ks + 16 * mt * LK, ks + nb32 * LK, 0, DKB);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int l = 16 * mt + g + 8 * (e >> 1), m = nb32 + 8 * j + 2 * t + (e & 1);
+                    PGs[l * LC + m] = m < l ? ap[j][e] * gamma(l, m) : 0.f;
+                }
+        }
+        __syncthreads();
+        store_tile<C, LC>(p.PGm + cidx * C * C, PGs);
+        // T = (I + L)^-1, L = diag(beta) P (.) Gamma: the four 16 x 16 diagonal blocks
+        // by forward substitution (lane c of warp I solves column c of block I), then
+        // block rows 1..3: T_IJ = -T_II sum_K L_IK T_KJ
         if (warp < 4 && lane < 16) {
             const int o = 16 * warp, c = lane;
             float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 float s = (i == c) ? 1.f : 0.f;
+                const float bi = betas[o + i];
 #pragma unroll
-                for (int m = 0; m < i; ++m) s -= Ls[(o + i) * LC + o + m] * x[m];
+                for (int m = 0; m < i; ++m) s -= bi * PGs[(o + i) * LC + o + m] * x[m];
                 x[i] = s;
                 Ts[(o + i) * LC + o + c] = s;
             }
@@ -340,7 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_prep_kernel(TcBwdArgs p) {
             if (warp < nt) {
                 float acc[1][4];
                 zero(acc);
-                wmma<1, LC, 1, LC, 1>(acc, Ls + 16 * I * LC, Ts + 8 * warp, 8 * warp, 16 * I);
+                wmma<1, LC, 1, LC, 1>(acc, PGs + 16 * I * LC, Ts + 8 * warp, 8 * warp, 16 * I);
+                const float b0 = betas[16 * I + g], b1 = betas[16 * I + g + 8];
+                acc[0][0] *= b0;
+                acc[0][1] *= b0;
+                acc[0][2] *= b1;
+                acc[0][3] *= b1;
                 store_frag<1, 52>(Rs + 8 * warp, acc);
             }
             __syncthreads();
@@ -352,45 +354,69 @@ __global__ void __launch_bounds__(kThreads, 1) bwdtc_prep_kernel(TcBwdArgs p) {
             }
             __syncthreads();
         }
-        // W = T diag(beta b) k
-        const int mt = warp & 3, nb = (warp >> 2) * 64;
+    }
+    // A = q k^T (.) Gamma, lower incl. (over P (.) Gamma)
+    {
+        float aq[4][4];
+        zero(aq);
+        wmma<4, LK, 1, 1, LK, false, false, false>(aq, qs + 16 * mt * LK, ks + nb32 * LK, 0, DKB);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int l = 16 * mt + g + 8 * (e >> 1), m = nb32 + 8 * j + 2 * t + (e & 1);
+                As[l * LC + m] = aq[j][e] * gamma(l, m);
+            }
+    }
+    __syncthreads();
+    store_tile<C, LC, true>(p.Am + cidx * C * C, As);
+    if (DELTA) {
+        // W = T diag(beta b) k, rounded, over q (no warp reads q any more)
         float acc[8][4];
         zero(acc);
-        wmma<8, LC, 1, LK, 1, true, true>(acc, Ts + 16 * mt * LC, ks + nb, 0, 16 * (mt + 1), bsc);
+        wmma<8, LC, 1, LK, 1, true, true>(acc, Ts + 16 * mt * LC, ks + nb64, 0, 16 * (mt + 1), bsc);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[j][e] = tf32r(acc[j][e]);
-        store_frag<8, LK>(Ws + 16 * mt * LK + nb, acc);
+        store_frag<8, LK>(Ws + 16 * mt * LK + nb64, acc);
         __syncthreads();
+        store_tile<C, LC, true>(p.Tm + cidx * C * C, Ts);
+        store_tile<DKB, LK>(p.Wm + cidx * C * DKB, Ws);
     }
-    // Q~ = diag(b) q - A W (in place over q), Kc = diag(e^{G_C - G}) k (over k)
+    // Q~ = diag(b) q - A W, rounded (q read back from global memory when W holds its tile)
     {
-        const int mt = warp & 3, nb = (warp >> 2) * 64;
         float acc[8][4];
         zero(acc);
-        if (DELTA) wmma<8, LC, 1, LK, 1, false, true>(acc, As + 16 * mt * LC, Ws + nb, 0, 16 * (mt + 1));
+        if (DELTA) wmma<8, LC, 1, LK, 1, false, true>(acc, As + 16 * mt * LC, Ws + nb64, 0, 16 * (mt + 1));
+        float *dst = p.Qtm + cidx * C * DKB;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int l = 16 * mt + g + 8 * (e >> 1), i = nb + 8 * j + 2 * t + (e & 1);
-                qs[l * LK + i] = tf32r(bs[l] * qs[l * LK + i] - acc[j][e]);
-            }
-        if (DELTA)
-            for (int i = tid; i < C * DKB; i += kThreads) {
-                const int l = i / DKB, c = i % DKB;
-                ks[l * LK + c] = tf32r(ks[l * LK + c] * es[l]);
+            for (int h = 0; h < 2; ++h) {
+                const int l = 16 * mt + g + 8 * h, i = nb64 + 8 * j + 2 * t;
+                float q0 = 0.f, q1 = 0.f;
+                if (!DELTA) {
+                    q0 = qs[l * LK + i];
+                    q1 = qs[l * LK + i + 1];
+                } else if (l < nv) {
+                    q0 = to_f32(qg[(size_t)l * DKB + i]);
+                    q1 = to_f32(qg[(size_t)l * DKB + i + 1]);
+                }
+                *reinterpret_cast<float2 *>(dst + l * DKB + i) =
+                    make_float2(tf32r(bs[l] * q0 - acc[j][2 * h]), tf32r(bs[l] * q1 - acc[j][2 * h + 1]));
             }
     }
-    __syncthreads();
-    store_tile<DKB, LK>(p.Qtm + cidx * C * DKB, qs);
-    store_tile<C, LC, true>(p.Am + cidx * C * C, As);
+    // K> = diag(e^{G_C - G}) k, rounded
     if (DELTA) {
-        store_tile<C, LC, true>(p.Tm + cidx * C * C, Ts);
-        store_tile<C, LC>(p.PGm + cidx * C * C, PGs);
-        store_tile<DKB, LK>(p.Wm + cidx * C * DKB, Ws);
-        store_tile<DKB, LK>(p.Kcm + cidx * C * DKB, ks);
+        float *dst = p.Kcm + cidx * C * DKB;
+        for (int i = tid; i < C * (DKB / 4); i += kThreads) {
+            const int l = i / (DKB / 4), c = (i % (DKB / 4)) * 4;
+            const float4 x = *reinterpret_cast<const float4 *>(ks + l * LK + c);
+            const float e = es[l];
+            *reinterpret_cast<float4 *>(dst + l * DKB + c) =
+                make_float4(tf32r(x.x * e), tf32r(x.y * e), tf32r(x.z * e), tf32r(x.w * e));
+        }
     }
     if (tid == 0) p.bC[cidx] = GATED ? expf(Gs[C - 1]) : 1.f;
 }
