@@ -62,7 +62,7 @@ def measured_traffic(workload):
 def prefill_bytes(w, out_bytes=None):
     """Algorithmic bytes of one prefill launch: q, k, v, g, beta read once, o
     written once, S0 read and S_T written once per head.  By default o is
-    counted in the input dtype (the survey's per-token bytes); ``out_bytes=4``
+    counted in the input dtype (o as the pages' layer returns it); ``out_bytes=4``
     counts the fp32 o this benchmark actually writes."""
     in_b = 2 if w.dtype == "bf16" else 4
     if out_bytes is None:
