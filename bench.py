@@ -445,6 +445,7 @@ def time_serving_loop(reps, torch, gdn, warmup=1, B=SERVE_B, graph=False):
 
 
 def time_backward(w, steps, torch, gdn, warmup=1, saved=False, tc=False):
+    # tc without saved: gdn_chunk_bwd with GDN_ALGO_TC (forward states + chunkwise backward in one call)
     """Device time of gdn_chunk_bwd (gradients of the prefill) on workload ``w``
     with random upstream gradients of o and S_T; returns ms per call.  With
     ``saved``: a training step's forward gdn_chunk_fwd_states and then
@@ -489,8 +490,13 @@ def time_backward(w, steps, torch, gdn, warmup=1, saved=False, tc=False):
             raise RuntimeError("device status after the saved-state training step")
         return sum(fw) / len(fw), sum(bw) / len(bw)
 
+    if tc:
+        ws = torch.empty(gdn.bwd_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.update, w.gate, algo="tc"),
+                         dtype=torch.uint8, device="cuda")
+
     def step():
-        gdn.chunk_bwd(q, k, v, g, beta, S0, dO, dST, update=w.update, gate=w.gate, workspace=ws)
+        gdn.chunk_bwd(q, k, v, g, beta, S0, dO, dST, update=w.update, gate=w.gate, workspace=ws,
+                      algo="tc" if tc else "token")
 
     for _ in range(warmup):
         step()
@@ -648,10 +654,11 @@ def run_ours(args):
         ms = time_backward(w, args.steps, torch, gdn, warmup=args.warmup)
         msf_s, msb_s = time_backward(w, args.steps, torch, gdn, warmup=1, saved=True)
         msf_t, msb_t = time_backward(w, args.steps, torch, gdn, warmup=1, saved=True, tc=True)
+        ms_one = time_backward(w, args.steps, torch, gdn, warmup=1, tc=True)
         if rank == 0:
             print(json.dumps({"only": "backward", "workload": w.name, "B": w.B, "H": w.H, "T": w.T,
                               "ms_per_call": ms, "saved_states": {"ms_forward": msf_s, "ms_backward": msb_s},
-                              "tensor_core": {"ms_forward": msf_t, "ms_backward": msb_t}}),
+                              "tensor_core": {"ms_forward": msf_t, "ms_backward": msb_t, "ms_one_call": ms_one}}),
                   flush=True)
         return
     x = make_prefill_inputs(w)
@@ -795,6 +802,10 @@ def run_ours(args):
             "frac": fl_tc / (msb_t * 1e-3) / 1e12 / tf32_peak,
             "note": "gdn_chunk_bwd_tc: prep, state-gradient chain and local kernels on tf32 warp MMAs; "
                     "peak = measured bf16 dense x 1/2 (the nominal tf32 : bf16 ratio)"}
+        # gdn_chunk_bwd with GDN_ALGO_TC: the states from its own tensor-core forward, one call
+        ms_one = max_over_ranks(time_backward(w, nb_steps, torch, gdn, tc=True), dist, "cuda")
+        result["gpu_launches"] += (nb_steps + 1) * 4
+        result["backward"]["tensor_core"]["ms_one_call"] = ms_one
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w)

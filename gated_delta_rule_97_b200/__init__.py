@@ -535,8 +535,8 @@ def decode_step(q, k, v, g, beta, S, *, update, gate, out_dtype=None, o=None, pr
     return o
 
 
-def bwd_workspace_bytes(B, H, T, dk, dv, update="delta", gate="scalar", prologue=0) -> int:
-    d = make_desc(B, H, T, dk, dv, update, gate, BF16, F32, prologue=prologue)
+def bwd_workspace_bytes(B, H, T, dk, dv, update="delta", gate="scalar", prologue=0, algo="auto") -> int:
+    d = make_desc(B, H, T, dk, dv, update, gate, BF16, F32, algo, prologue=prologue)
     return int(load().gdn_bwd_workspace_bytes(ctypes.byref(d)))
 
 
@@ -556,9 +556,11 @@ def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update
     (written by chunk_fwd(states=...)) the call is gdn_chunk_bwd_states: S0 and
     the workspace are not used.  ``prologue``: the GDN_PRO_* maps the forward
     applied to the raw q, k, beta, g; the gradients are then with respect to
-    those raw inputs.  ``algo="tc"`` (with ``states``) is gdn_chunk_bwd_tc, the
-    chunkwise tensor-core backward; ``workspace`` is then one of
-    bwd_tc_workspace_bytes(...) bytes."""
+    those raw inputs.  ``algo="tc"``: the chunkwise tensor-core backward, from
+    ``states`` (gdn_chunk_bwd_tc; ``workspace`` of bwd_tc_workspace_bytes(...)
+    bytes) or, without them, gdn_chunk_bwd with GDN_ALGO_TC (the tensor-core
+    forward writes the states into the workspace first; bwd_workspace_bytes(...,
+    algo="tc") bytes)."""
     import torch
 
     B, H, T, dk = q.shape
@@ -580,9 +582,22 @@ def chunk_bwd(q, k, v, g=None, beta=None, S0=None, dO=None, dS_T=None, *, update
     gb = torch.empty((B, H, T), **f32) if update == "delta" else None
     gS0 = torch.empty((B, H, dv, dk), **f32) if want_dS0 else None
     d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), F32, prologue=prologue)
+    if algo == "tc" and states is None:
+        d = make_desc(B, H, T, dk, dv, update, gate, _dtype_code(q.dtype), F32, "tc", prologue=prologue)
+        need = int(load().gdn_bwd_workspace_bytes(ctypes.byref(d)))
+        if workspace is None:
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        if not workspace.is_cuda or not workspace.is_contiguous() or workspace.numel() < need:
+            raise ValueError("workspace needs %d contiguous CUDA bytes" % need)
+        with _on_device(q):
+            rc = load().gdn_chunk_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                      _ptr(dO), _ptr(dS_T), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gg), _ptr(gb),
+                                      _ptr(gS0), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                      _stream(stream, q))
+        if rc != GDN_OK:
+            raise GDNError(rc, "gdn_chunk_bwd")
+        return gq, gk, gv, gg, gb, gS0
     if algo == "tc":
-        if states is None:
-            raise ValueError("algo='tc' runs from saved states (chunk_fwd(states=...))")
         _check(states, "states", (B, H, (T + CHUNK - 1) // CHUNK, dv, dk), torch.float32)
         need = int(load().gdn_bwd_tc_workspace_bytes(ctypes.byref(d)))
         if workspace is None:

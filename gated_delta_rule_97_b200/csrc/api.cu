@@ -563,9 +563,22 @@ int gdn_launch_prologue_grad(const void *q, const void *k, const float *g, const
                              float *dg, float *dbeta, long rows, int dk_, int gate, int in_bf16, int pro,
                              cudaStream_t st);
 
+size_t gdn_bwd_tc_layout(long BH, int nch, int dk, int dv, int delta, size_t *off);  // backward_tc.cu
+int gdn_launch_bwd_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                      const float *states, const float *dO, const float *dST, float *dq, float *dk, float *dv,
+                      float *dg, float *dbeta, float *dS0, void *ws, int BH, int T, int dv_, int update, int gate,
+                      int in_bf16, cudaStream_t st);
+
+// The per-chunk kernels put the heads on the grid's y dimension (at most 65535).
+static bool bwd_tc_supported(const gdn_desc_t *d) {
+    return d->prologue == 0 && d->gate != GDN_GATE_CHANNEL && d->dk == 128 && (d->dv == 64 || d->dv == 128) &&
+           (d->chunk == 0 || d->chunk == gdn::kChunk) && (long)d->B * d->H <= 65535;
+}
+
 // Workspace of gdn_chunk_bwd: the chunk-entry states, then (with an input
 // prologue) the mapped inputs in fp32: q, k, v, beta, g, each on a 256-byte
-// boundary.
+// boundary.  With GDN_ALGO_TC: the states, then the tensor-core backward's
+// workspace.
 struct BwdLayout {
     size_t states, qm, km, vf, bm, gm, bytes;
 };
@@ -590,8 +603,24 @@ static BwdLayout bwd_layout(const gdn_desc_t *d) {
     return L;
 }
 
+// gdn_chunk_bwd on the tensor-core path: the tensor-core forward writes the
+// chunk states (bf16 inputs, dk = 128), then the chunkwise backward.
+static bool bwd_algo_tc(const gdn_desc_t *d) { return d->algo == GDN_ALGO_TC; }
+static bool bwd_algo_tc_served(const gdn_desc_t *d) { return bwd_tc_supported(d) && gdn_tc_supported(d); }
+
+static size_t bwd_states_bytes(const gdn_desc_t *d) {
+    const size_t nch = ((size_t)d->T + gdn::kChunk - 1) / gdn::kChunk;
+    return (size_t)d->B * d->H * nch * d->dv * d->dk * sizeof(float);
+}
+
 extern "C" size_t gdn_bwd_workspace_bytes(const gdn_desc_t *d) {
     if (!d || validate_common(d) != GDN_OK) return 0;
+    if (bwd_algo_tc(d)) {
+        if (!bwd_algo_tc_served(d)) return 0;
+        const int nch = (d->T + gdn::kChunk - 1) / gdn::kChunk;
+        return round256(bwd_states_bytes(d)) +
+               gdn_bwd_tc_layout((long)d->B * d->H, nch, d->dk, d->dv, d->update == GDN_DELTA, nullptr);
+    }
     return bwd_layout(d).bytes;
 }
 
@@ -647,18 +676,37 @@ int chunk_bwd_impl(const gdn_desc_t *d, const void *q, const void *k, const void
     if (rc != GDN_OK) return rc;
     if (d->chunk != 0 && d->chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
     if (d->prologue != 0 && saved) return GDN_ERR_UNSUPPORTED;  // the saved states carry no maps
+    const bool tc = !saved && bwd_algo_tc(d);
+    if (tc && !bwd_algo_tc_served(d)) return GDN_ERR_UNSUPPORTED;
     const long BH = (long)d->B * d->H;
     const size_t ntok = (size_t)BH * d->T;
     const size_t n_S = (size_t)BH * d->dv * d->dk;
-    const size_t need = gdn_bwd_workspace_bytes(d);
-    rc = bwd_check(d, q, k, v, g, beta, S0, saved, need, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace,
-                   workspace_bytes, saved ? 0 : need);
+    const size_t need = saved ? 0 : gdn_bwd_workspace_bytes(d);
+    rc = bwd_check(d, q, k, v, g, beta, S0, saved, bwd_states_bytes(d), dO, dS_T, dq, dk, dv, dg, dbeta, dS0,
+                   workspace, workspace_bytes, need);
     if (rc != GDN_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (BH == 0) return GDN_OK;
     if (d->T == 0) return dS0 ? from_cuda(gdn_launch_copy_state(dS_T, dS0, (long)n_S, st)) : GDN_OK;
     float *ws = saved ? const_cast<float *>(saved) : static_cast<float *>(workspace);
     const int in_bf16 = d->dtype == GDN_BF16;
+    if (tc) {
+        // the tensor-core forward writes the chunk-entry states (no o, no S_T), then
+        // the chunkwise backward runs from them
+        gdn::ChunkArgs a{};
+        a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = nullptr; a.ST = nullptr;
+        a.status = status_ptr();
+        a.diag = diag_ptr();
+        a.BH = (int)BH; a.T = d->T; a.dk = d->dk; a.dv = d->dv;
+        a.nh = 1;
+        a.mode = gdn::kModeSaveStates | gdn::kModeNoOut;
+        a.states = ws;
+        const int e = gdn_launch_chunk_tc2(a, d, st);
+        if (e != 0) return from_cuda(e);
+        return from_cuda(gdn_launch_bwd_tc(q, k, v, g, beta, ws, dO, dS_T, dq, dk, dv, dg, dbeta, dS0,
+                                           static_cast<char *>(workspace) + round256(bwd_states_bytes(d)), (int)BH,
+                                           d->T, d->dv, d->update, d->gate, in_bf16, st));
+    }
     if (d->prologue == 0)
         return from_cuda(gdn_launch_bwd(q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, ws, (int)BH,
                                         d->T, d->dk, d->dv, d->update, d->gate, in_bf16, saved != nullptr, st));
@@ -698,18 +746,6 @@ extern "C" int gdn_chunk_bwd_states(const gdn_desc_t *d, const void *q, const vo
     if (d && (long)d->B * d->H * d->T > 0 && !states) return GDN_ERR_ARG;
     return chunk_bwd_impl(d, q, k, v, g, beta, nullptr, states, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, nullptr, 0,
                           stream);
-}
-
-size_t gdn_bwd_tc_layout(long BH, int nch, int dk, int dv, int delta, size_t *off);  // backward_tc.cu
-int gdn_launch_bwd_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
-                      const float *states, const float *dO, const float *dST, float *dq, float *dk, float *dv,
-                      float *dg, float *dbeta, float *dS0, void *ws, int BH, int T, int dv_, int update, int gate,
-                      int in_bf16, cudaStream_t st);
-
-// The per-chunk kernels put the heads on the grid's y dimension (at most 65535).
-static bool bwd_tc_supported(const gdn_desc_t *d) {
-    return d->prologue == 0 && d->gate != GDN_GATE_CHANNEL && d->dk == 128 && (d->dv == 64 || d->dv == 128) &&
-           (d->chunk == 0 || d->chunk == gdn::kChunk) && (long)d->B * d->H <= 65535;
 }
 
 extern "C" size_t gdn_bwd_tc_workspace_bytes(const gdn_desc_t *d) {
@@ -754,7 +790,7 @@ extern "C" int gdn_chunk_fwd_states(const gdn_desc_t *d, const void *q, const vo
     if (d->T == 0) return from_cuda(gdn_launch_copy_state(S0, S_T, (long)n_S, st));
     if (!states) return GDN_ERR_ARG;
     if (!aligned16(states)) return GDN_ERR_ALIGN;
-    const size_t ns = gdn_bwd_workspace_bytes(d);
+    const size_t ns = bwd_states_bytes(d);
     const size_t es = elem_size(d->dtype), eo = elem_size(d->out_dtype);
     const size_t ntok = (size_t)BH * d->T;
     const size_t n_qk = ntok * d->dk, n_v = ntok * d->dv;

@@ -313,7 +313,13 @@ const char *gdn_strerror(int code);
  * through it.  fp32 arithmetic.
  *
  *   desc        as for gdn_chunk_fwd (update, gate, dtype of q, k, v; dk, dv
- *               in {64, 128}; chunk 0 or 64); out_dtype and algo are not read.
+ *               in {64, 128}; chunk 0 or 64); out_dtype is not read.  algo
+ *               GDN_ALGO_TC: the tensor-core path -- the tensor-core forward
+ *               writes the chunk-entry states into the workspace, then the
+ *               chunkwise backward of gdn_chunk_bwd_tc runs from them (its
+ *               requests only, GDN_ERR_UNSUPPORTED otherwise; results at the
+ *               rounding of those two kernels).  Any other algo: the fp32 token
+ *               backward described here.
  *               With prologue bits the inputs are the raw q, k, beta, g the
  *               forward mapped, and dq, dk, dbeta, dg are the gradients with
  *               respect to them (the chain rule through each map follows the
@@ -329,8 +335,10 @@ const char *gdn_strerror(int code);
  *   dS0         [B,H,dv,dk] float, or NULL (not written)
  *   workspace   device buffer of at least gdn_bwd_workspace_bytes(desc) bytes
  *               (B*H*ceil(T/64)*dv*dk*4: the chunk-boundary states; with prologue
- *               bits also the mapped q, k, v, beta, g in fp32), 16-byte aligned,
- *               owned by the caller; contents on return unspecified.
+ *               bits also the mapped q, k, v, beta, g in fp32; with GDN_ALGO_TC
+ *               also gdn_bwd_tc_workspace_bytes(desc)), 16-byte aligned, owned by
+ *               the caller; contents on return unspecified.  0 for a GDN_ALGO_TC
+ *               request the tensor-core path does not serve.
  *
  * Every pointer 16-byte aligned; no output may overlap another output, an
  * input or the workspace (GDN_ERR_ARG).  dq, dk, dg and dbeta are sums over the
@@ -363,7 +371,9 @@ int gdn_chunk_bwd(const gdn_desc_t *desc, const void *q, const void *k, const vo
  * gdn_chunk_bwd_states -- gdn_chunk_bwd from those saved states: the backward's
  * own forward pass over the sequence is skipped (each chunk is still recomputed
  * from its saved state).  Arguments as for gdn_chunk_bwd, with `states` (read
- * only; required when B*H*T > 0) in place of S0 and the workspace; prologue 0.
+ * only; required when B*H*T > 0) in place of S0 and the workspace; prologue 0;
+ * always the fp32 token backward (algo is not read: gdn_chunk_bwd_tc is the
+ * tensor-core form from saved states).
  */
 int gdn_chunk_fwd_states(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
                          const float *beta, const float *S0, void *o, float *S_T, float *states, void *stream);

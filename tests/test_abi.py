@@ -299,6 +299,19 @@ def test_tensor_core_backward_rejects_bad_arguments(lib):
     assert f(ctypes.byref(p), *ins, *outs, ws, need, None) == -3              # no input prologue
     e = _desc(B=0)
     assert f(ctypes.byref(e), *ins, *outs, ws, 0, None) == 0                   # empty batch: no-op
+    # gdn_chunk_bwd with GDN_ALGO_TC: the forward's states, then the same workspace
+    lib.gdn_bwd_workspace_bytes.argtypes = [ctypes.c_void_p]
+    lib.gdn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    b = lib.gdn_chunk_bwd
+    b.argtypes = [ctypes.c_void_p] * 16 + [ctypes.c_size_t, ctypes.c_void_p]
+    t = _desc(T=130, algo="tc")
+    need_t = lib.gdn_bwd_workspace_bytes(ctypes.byref(t))
+    assert need_t == ss + need  # 18 chunk states of 64 KB (256-byte multiple), then the tensor-core workspace
+    bins = [vp(0x100000), vp(0x200000), vp(0x300000), vp(0x400000), vp(0x500000), None, None, None]
+    assert b(ctypes.byref(t), *bins, *outs, ws, need_t - 16, None) == -1       # workspace too small
+    for unsupported in (_desc(T=130, gate="channel", algo="tc"), _desc(T=130, dtype=gdn.F32, algo="tc")):
+        assert lib.gdn_bwd_workspace_bytes(ctypes.byref(unsupported)) == 0
+        assert b(ctypes.byref(unsupported), *bins, *outs, ws, need_t, None) == -3
 
 
 def test_wait_limit_hook(lib):

@@ -190,3 +190,29 @@ def test_tc_backward_full_size_sampled_heads():
                 continue
             err = rel_err(np64(a[b, h]), r[0, 0])
             assert err <= TOL_STATES, ((b, h), name, err)
+
+
+@pytest.mark.parametrize("update,gate", MODES)
+@pytest.mark.parametrize("dv,T", [(128, 150), (64, 200)])
+def test_one_call_tensor_core_backward(update, gate, dv, T):
+    """gdn_chunk_bwd with GDN_ALGO_TC (no saved states): the tensor-core forward
+    writes the states into the workspace (without o), then the chunkwise
+    backward.  Equals the two-call training path bit for bit, and the oracle at
+    the tensor-core bound."""
+    x = inputs(47, update, gate, T=T, dv=dv, bf16=True)
+    q, k, v, g, beta, S0, dO, dST = x
+    t = [dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), dev(g), dev(beta)]
+    gdn.device_status(clear=True)
+    one = gdn.chunk_bwd(*t, dev(S0), dev(dO), dev(dST), update=update, gate=gate, algo="tc")
+    states = torch.empty((1, 2, (T + 63) // 64, dv, 128), dtype=torch.float32, device="cuda")
+    gdn.chunk_fwd(*t, dev(S0), update=update, gate=gate, states=states)
+    two = gdn.chunk_bwd(*t, None, dev(dO), dev(dST), update=update, gate=gate, states=states, algo="tc")
+    torch.cuda.synchronize()
+    assert gdn.device_status(clear=True) == 0
+    ref = oracle.gdn_backward_np(update, gate, *x)
+    for name, a, b, r in zip(NAMES, one, two, ref):
+        if r is None:
+            assert a is None, name
+            continue
+        assert torch.equal(a, b), name
+        assert rel_err(np64(a), r) <= TOL_STATES, (name, rel_err(np64(a), r))
