@@ -31,12 +31,14 @@
 //         operand fragments coincide);
 //   local (one CTA per chunk and head, all in parallel): every chunk-local
 //         gradient from the saved S_r, the stored dSn and the prep's tiles;
-//         value rows go through in slices of 32, the sums over value rows
-//         (dKc, dQb, dW, dA, dT) stay in registers across the slices.
+//         value rows go through in slices of 32 (the next slice's S and dSn
+//         copied while one is processed), the sums over value rows (dKc, dQb,
+//         dW, dA, dT) stay in registers across the slices.
 // Every product is a warp-level tf32 tensor-core MMA (m16n8k8, fp32
 // accumulation) on fp32 tiles in shared memory; an operand tile is rounded to
-// tf32 (nearest) once, where it is written, so the MMA loops convert nothing.  dq, dk, dv, dg, dbeta are
-// written once per token (no atomics): a chunk's CTA owns its tokens.
+// tf32 (nearest) once, where it is written, so the MMA loops of the chain and
+// local kernels convert nothing.  dq, dk, dv, dg, dbeta are written once per
+// token and the CTA reductions run in a fixed order: no atomics, deterministic.
 #include <stddef.h>
 
 #include "../../include/gdn.h"
