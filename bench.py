@@ -445,13 +445,13 @@ def time_serving_loop(reps, torch, gdn, warmup=1, B=SERVE_B, graph=False):
 
 
 def time_backward(w, steps, torch, gdn, warmup=1, saved=False, tc=False):
-    # tc without saved: gdn_chunk_bwd with GDN_ALGO_TC (forward states + chunkwise backward in one call)
     """Device time of gdn_chunk_bwd (gradients of the prefill) on workload ``w``
-    with random upstream gradients of o and S_T; returns ms per call.  With
-    ``saved``: a training step's forward gdn_chunk_fwd_states and then
-    gdn_chunk_bwd_states (``tc``: gdn_chunk_bwd_tc, the chunkwise tensor-core
-    backward) from its chunk states; returns (ms of the forward, ms of the
-    backward) per step."""
+    with random upstream gradients of o and S_T; returns ms per call (``tc``:
+    with GDN_ALGO_TC, the tensor-core forward's states and the chunkwise
+    backward in one call).  With ``saved``: a training step's forward
+    gdn_chunk_fwd_states and then gdn_chunk_bwd_states (``tc``:
+    gdn_chunk_bwd_tc, the chunkwise tensor-core backward) from its chunk
+    states; returns (ms of the forward, ms of the backward) per step."""
     x = make_prefill_inputs(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     q, k, v = to_dev(x["q"], dt, torch), to_dev(x["k"], dt, torch), to_dev(x["v"], dt, torch)
@@ -460,7 +460,9 @@ def time_backward(w, steps, torch, gdn, warmup=1, saved=False, tc=False):
     gen = torch.Generator(device="cuda").manual_seed(w.seed)
     dO = torch.randn((w.B, w.H, w.T, w.dv), device="cuda", generator=gen)
     dST = torch.randn((w.B, w.H, w.dv, w.dk), device="cuda", generator=gen)
-    ws = torch.empty(gdn.bwd_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv), dtype=torch.uint8, device="cuda")
+    algo = "tc" if tc and not saved else "auto"
+    ws = torch.empty(gdn.bwd_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.update, w.gate, algo=algo),
+                     dtype=torch.uint8, device="cuda")
     if saved:
         states = ws.view(torch.float32).view(w.B, w.H, (w.T + 63) // 64, w.dv, w.dk)
         o = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device="cuda")
@@ -489,10 +491,6 @@ def time_backward(w, steps, torch, gdn, warmup=1, saved=False, tc=False):
         if gdn.device_status() != 0:
             raise RuntimeError("device status after the saved-state training step")
         return sum(fw) / len(fw), sum(bw) / len(bw)
-
-    if tc:
-        ws = torch.empty(gdn.bwd_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.update, w.gate, algo="tc"),
-                         dtype=torch.uint8, device="cuda")
 
     def step():
         gdn.chunk_bwd(q, k, v, g, beta, S0, dO, dST, update=w.update, gate=w.gate, workspace=ws,
