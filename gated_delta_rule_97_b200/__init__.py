@@ -107,6 +107,8 @@ def load():
     lib.gdn_chunk_fwd_states.restype = ctypes.c_int
     lib.gdn_chunk_bwd_states.argtypes = [dp] + [vp] * 15
     lib.gdn_chunk_bwd_states.restype = ctypes.c_int
+    lib.gdn_chunk_fwd_checked.argtypes = [dp] + [vp] * 9
+    lib.gdn_chunk_fwd_checked.restype = ctypes.c_int
     lib.gdn_bwd_tc_workspace_bytes.argtypes = [dp]
     lib.gdn_bwd_tc_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_chunk_bwd_tc.argtypes = [dp] + [vp] * 15 + [ctypes.c_size_t, vp]
@@ -199,11 +201,14 @@ def _check(t, name, shape, dtype=None):
 
 
 def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=None, o=None, S_T=None,
-              return_state=True, algo="auto", prologue=0, states=None, stream=None):
+              return_state=True, algo="auto", prologue=0, states=None, checked=False, stream=None):
     """Prefill over T tokens (gdn_chunk_fwd).  Returns (o, S_T).
 
     ``states``: a CUDA float32 tensor [B,H,ceil(T/64),dv,dk] that receives the
     state entering every chunk (gdn_chunk_fwd_states, for chunk_bwd(states=...)).
+    ``checked``: gdn_chunk_fwd_checked (synchronous; an fp16 operand overflow
+    of a tensor-core kernel runs the request again on the fp32 kernel); returns
+    (o, S_T, reran) then.
 
     q, k [B,H,T,dk]; v [B,H,T,dv] (bf16 or fp32, same dtype); g [B,H,T] or
     [B,H,T,dk] fp32 (log of the gate) or None; beta [B,H,T] fp32 (delta);
@@ -240,6 +245,13 @@ def chunk_fwd(q, k, v, g=None, beta=None, S0=None, *, update, gate, out_dtype=No
         if rc != GDN_OK:
             raise GDNError(rc, "gdn_chunk_fwd_states")
         return o, S_T
+    if checked:
+        with _on_device(q):
+            rc = load().gdn_chunk_fwd_checked(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                              _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream, q))
+        if rc not in (GDN_OK, 1):
+            raise GDNError(rc, "gdn_chunk_fwd_checked")
+        return o, S_T, rc == 1
     with _on_device(q):
         rc = load().gdn_chunk_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
                                   _ptr(o), _ptr(S_T), _stream(stream, q))

@@ -181,6 +181,41 @@ extern "C" int gdn_chunk_fwd(const gdn_desc_t *d, const void *q, const void *k, 
     return dispatch_chunk(d, a, st);
 }
 
+// gdn_chunk_fwd, then the device status word: an fp16 operand overflow of the
+// tensor-core kernel (GDN_ERR_RANGE) runs the request again on the fp32 SIMT
+// kernel.  Synchronous.
+extern "C" int gdn_chunk_fwd_checked(const gdn_desc_t *d, const void *q, const void *k, const void *v,
+                                     const float *g, const float *beta, const float *S0, void *o, float *S_T,
+                                     void *stream) {
+    int rc = chunk_fwd_check(d, q, k, v, g, beta, S0, o, S_T);
+    if (rc != GDN_OK) return rc;
+    const size_t n_S = (size_t)d->B * d->H * d->dv * d->dk;
+    if (overlaps(S0, n_S * 4, S_T, n_S * 4)) return GDN_ERR_ARG;  // the second run reads S0
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int status = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&status, g_gdn_status, sizeof(int)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (status != 0) return status;  // an earlier error the caller has not cleared
+    rc = gdn_chunk_fwd(d, q, k, v, g, beta, S0, o, S_T, stream);
+    if (rc != GDN_OK) return rc;
+    if (cudaStreamSynchronize(st) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&status, g_gdn_status, sizeof(int)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (status == 0) return GDN_OK;
+    if (status != GDN_ERR_RANGE) return status;
+    const int z = 0;
+    if (cudaMemcpyToSymbol(g_gdn_status, &z, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+    gdn_desc_t d2 = *d;
+    d2.algo = GDN_ALGO_SIMT;
+    rc = gdn_chunk_fwd(&d2, q, k, v, g, beta, S0, o, S_T, stream);
+    if (rc != GDN_OK) return rc;
+    if (cudaStreamSynchronize(st) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&status, g_gdn_status, sizeof(int)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return status != 0 ? status : 1;
+}
+
 namespace {
 
 // Byte layout of one slot of the host pipeline's device workspace: the inputs

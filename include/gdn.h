@@ -301,6 +301,29 @@ int gdn_decode_step(const gdn_desc_t *desc, const void *q, const void *k, const 
 const char *gdn_strerror(int code);
 
 /*
+ * gdn_chunk_fwd_checked -- gdn_chunk_fwd with recovery from an fp16 overflow.
+ * The tensor-core kernels hand fp16 operands to the tensor cores, and a value
+ * beyond fp16's range there is reported as GDN_ERR_RANGE in the device status
+ * word, with unspecified results.  This call synchronises `stream`, reads the
+ * word, and after a GDN_ERR_RANGE clears it and runs the request again on the
+ * fp32 SIMT kernel (fp32 range, fp32 arithmetic; "Linear Attention,
+ * Visualized": the same recurrence).
+ *
+ *   arguments   as for gdn_chunk_fwd; S_T may not overlap S0 (GDN_ERR_ARG):
+ *               the second run reads S0.
+ *   returns     GDN_OK, 1 when the fp32 kernel ran again (the results are
+ *               its), a negative code otherwise.  If the status word already
+ *               holds an error on entry, that code is returned and nothing
+ *               runs (clear it with gdn_device_status(1) first).
+ *
+ * Blocks the host until `stream` is idle.  The status word is shared by the
+ * library's kernels on the device: a range error of another call running at
+ * the same time also triggers the second run.
+ */
+int gdn_chunk_fwd_checked(const gdn_desc_t *desc, const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *S0, void *o, float *S_T, void *stream);
+
+/*
  * gdn_chunk_bwd -- the gradients of gdn_chunk_fwd (training backward).  For the
  * scalar loss L = sum(dO (.) o) + sum(dS_T (.) S_T) of gdn_chunk_fwd on the same
  * desc and inputs, writes dq = dL/dq, dk, dv, dg (dL/d log alpha), dbeta and

@@ -314,6 +314,19 @@ def test_tensor_core_backward_rejects_bad_arguments(lib):
         assert b(ctypes.byref(unsupported), *bins, *outs, ws, need_t, None) == -3
 
 
+def test_checked_prefill_rejects_bad_arguments(lib):
+    f = lib.gdn_chunk_fwd_checked
+    f.argtypes = [ctypes.c_void_p] * 10
+    vp = ctypes.c_void_p
+    d = _desc()
+    args = [vp(0x10000), vp(0x20000), vp(0x30000), vp(0x40000), vp(0x50000)]
+    assert f(ctypes.byref(d), *args, vp(0x7000000), vp(0x9000000), vp(0x7000000), None) == -1  # S_T is S0
+    assert f(None, *args, None, vp(0x9000000), None, None) == -1                               # no desc
+    bad = _desc()
+    bad.update = 7
+    assert f(ctypes.byref(bad), *args, None, vp(0x9000000), None, None) == -1
+
+
 def test_wait_limit_hook(lib):
     lib.gdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     assert lib.gdn_set_wait_limit_ns(5) == 0

@@ -6,7 +6,7 @@ import torch
 import gated_delta_rule_97_b200 as gdn
 import oracle
 from gpu_util import TOL, dev, io_dtype, np64, rel_err, run_prefill
-from synth import WORKLOADS, make_prefill_inputs
+from synth import WORKLOADS, make_prefill_inputs, round_to_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -119,6 +119,37 @@ def test_tc_range_overflow_is_reported():
                   update="additive", gate="none", algo="tc")
     assert gdn.device_status(clear=True) == -6
     assert gdn.device_status() == 0
+
+
+def test_checked_prefill_recovers_from_range_overflow():
+    """gdn_chunk_fwd_checked on values far beyond fp16 range: the tensor-core
+    kernel reports GDN_ERR_RANGE, the call runs the request again on the fp32
+    kernel and returns its results, at fp32 parity with the oracle."""
+    w = workload("delta", "scalar", T=130, B=1, H=2)
+    x = make_prefill_inputs(w)
+    x["v"] = round_to_bf16((x["v"] * 1e6).astype(np.float32))  # the bf16 values both sides read
+    dt = io_dtype(w)
+    t = [dev(x["q"], dt), dev(x["k"], dt), dev(x["v"], dt), dev(x["g"]), dev(x["beta"]), dev(x["S0"])]
+    gdn.device_status(clear=True)
+    o, S, reran = gdn.chunk_fwd(*t, update="delta", gate="scalar", checked=True)
+    assert reran and gdn.device_status() == 0
+    ro, rS = oracle.gdn_forward("delta", "scalar", x["q"], x["k"], x["v"], g=x["g"], beta=x["beta"], S0=x["S0"])
+    assert rel_err(np64(o), ro) <= TOL["f32"] and rel_err(np64(S), rS) <= TOL["f32"]
+    o2, S2 = run_prefill(w, x, algo="simt")
+    assert torch.equal(o, o2) and torch.equal(S, S2)
+
+
+def test_checked_prefill_without_overflow_is_the_plain_call():
+    w = workload("delta", "scalar", T=200, B=1, H=2)
+    x = make_prefill_inputs(w)
+    dt = io_dtype(w)
+    t = [dev(x["q"], dt), dev(x["k"], dt), dev(x["v"], dt), dev(x["g"]), dev(x["beta"]), dev(x["S0"])]
+    gdn.device_status(clear=True)
+    o, S, reran = gdn.chunk_fwd(*t, update="delta", gate="scalar", checked=True)
+    o2, S2 = gdn.chunk_fwd(*t, update="delta", gate="scalar")
+    torch.cuda.synchronize()
+    assert not reran and gdn.device_status() == 0
+    assert torch.equal(o, o2) and torch.equal(S, S2)
 
 
 @pytest.mark.parametrize("update,gate", MODES)
