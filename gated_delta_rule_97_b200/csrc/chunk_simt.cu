@@ -317,7 +317,7 @@ int gdn_launch_chunk_simt(const gdn::ChunkArgs &a, int update, int gate, int in_
 int gdn_launch_copy_state(const float *S0, float *ST, long n, cudaStream_t stream) {
     if (n <= 0 || ST == nullptr || ST == S0) return 0;
     long blocks = (n + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > gdn::gdn_sm_count() * 16L) blocks = gdn::gdn_sm_count() * 16L;
     gdn::copy_state_kernel<<<(unsigned)blocks, 256, 0, stream>>>(S0, ST, n);
     return (int)cudaGetLastError();
 }

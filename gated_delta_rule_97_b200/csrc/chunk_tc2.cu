@@ -1445,7 +1445,7 @@ int gdn_tc_supported(const gdn_desc_t *d) {
 static int tc2_slice(const gdn_desc_t *d) {
     const long bh = (long)d->B * d->H;
     if (d->dv == 64 || d->gate == GDN_GATE_CHANNEL) return 64;
-    return (bh * 2 <= 148) ? 64 : 128;
+    return (bh * 2 <= gdn::gdn_sm_count()) ? 64 : 128;
 }
 
 int gdn_launch_chunk_tc2(const gdn::ChunkArgs &a, const gdn_desc_t *d, cudaStream_t stream) {

@@ -27,6 +27,20 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Multiprocessor count of the current device, cached per device (host side;
+// grid sizing).  148 if the query fails.
+inline int gdn_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 // Records the first error code seen by any kernel (0 = none yet).
 __device__ __forceinline__ void record_status(int *status, int code) {
     if (status) atomicCAS(status, 0, code);

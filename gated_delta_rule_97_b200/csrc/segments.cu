@@ -145,7 +145,7 @@ int gdn_launch_eye(float *L, long BH, int dk, cudaStream_t stream) {
     const long n = BH * dk * dk;
     if (n <= 0) return 0;
     long blocks = (n + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > gdn::gdn_sm_count() * 16L) blocks = gdn::gdn_sm_count() * 16L;
     gdn::eye_kernel<<<(unsigned)blocks, 256, 0, stream>>>(L, n, dk);
     return (int)cudaGetLastError();
 }
