@@ -199,3 +199,96 @@ def chunk_backward(update, gate, q, k, v, g=None, beta=None, S0=None, dO=None, d
         out_g[sl] = np.cumsum(dG[::-1])[::-1]
         out_b[sl] = db
     return (out_q[:T], out_k[:T], out_v[:T], out_g[:T] if gated else None, out_b[:T] if delta else None, dS)
+
+
+def chunk_backward_channel(update, q, k, v, g, beta=None, S0=None, dO=None, dS_T=None, C=64):
+    """The chunkwise backward for a per-channel gate (KDA / GLA), float64, one
+    head: g [T, dk] (log alpha per key channel).  Returns (dq, dk, dv, dg,
+    dbeta, dS0) (dbeta None without the delta rule).
+
+    With G [C, dk] the in-chunk prefix, Qb = q (.) e^G, Kb = k (.) e^G,
+    Ki = k (.) e^{-G}, Kc = k (.) e^{G_C - G}, every Gamma factor sits inside a
+    product: A = lower-incl(Qb Ki^T), L = diag(beta) strict-lower(Kb Ki^T)
+    ("Kimi Delta Attention (KDA)": the channel-wise decay table; "Gated Linear
+    Attention (GLA)", Chunkwise form), and S' = S Diag(e^{G_C}) + Z^T Kc.  The
+    reverse pass is the scalar one with the gate gradient per channel:
+      dQb += tril(dA) Ki;  dKi = tril(dA)^T Qb + E^T Kb;  dKb += E Ki,
+      E = diag(beta) dL (strict lower);  dbeta_l += sum_m dL[l,m] (Kb Ki^T)[l,m]
+      dq = dQb e^G;  dk = dKb e^G + dKi e^{-G} + dKc e^{G_C - G}
+      dG += dQb Qb + dKb Kb - dKi Ki - dKc Kc  (elementwise), and in row C - 1
+      sum_l dKc_l Kc_l + e^{G_C} (.) sum_v dSn[v] (.) S[v]; dg = reverse prefix sums."""
+    T, dk = q.shape
+    dv_ = v.shape[1]
+    delta = update == "delta"
+    n = max(1, -(-T // C))
+    pad = lambda a: np.concatenate([a, np.zeros((n * C - T,) + a.shape[1:])])
+    qq, kk, vv, gg = pad(q), pad(k), pad(v), pad(g)
+    bb = pad(beta) if delta else np.zeros(n * C)
+    do = pad(dO) if dO is not None else np.zeros((n * C, dv_))
+    S = np.zeros((dv_, dk)) if S0 is None else np.array(S0, np.float64)
+    states, tiles = [], []
+    for r in range(n):
+        sl = slice(r * C, r * C + C)
+        qc, kc, vc, bc = qq[sl], kk[sl], vv[sl], bb[sl]
+        G = np.cumsum(gg[sl], axis=0)
+        GC = G[-1]
+        Qb, Kb, Ki, Kc = qc * np.exp(G), kc * np.exp(G), kc * np.exp(-G), kc * np.exp(GC - G)
+        A = np.tril(Qb @ Ki.T)
+        tl = dict(G=G, GC=GC, Qb=Qb, Kb=Kb, Ki=Ki, Kc=Kc, A=A)
+        if delta:
+            tl["P"] = np.tril(Kb @ Ki.T, -1)
+            tl["T"] = np.linalg.inv(np.eye(C) + bc[:, None] * tl["P"])
+            tl["W"] = tl["T"] @ (bc[:, None] * Kb)
+            Z = tl["T"] @ (bc[:, None] * vc) - tl["W"] @ S.T
+        else:
+            Z = vc
+        tl["Qt"] = Qb - (A @ tl["W"] if delta else 0.0)
+        states.append(S)
+        tiles.append(tl)
+        S = S * np.exp(GC)[None, :] + Z.T @ Kc
+    dS = np.zeros((dv_, dk)) if dS_T is None else np.array(dS_T, np.float64)
+    dSn = [None] * n
+    for r in range(n - 1, -1, -1):
+        tl, doc = tiles[r], do[r * C:(r + 1) * C]
+        dSn[r] = dS
+        nxt = dS * np.exp(tl["GC"])[None, :] + doc.T @ tl["Qt"]
+        if delta:
+            nxt = nxt - (dS @ tl["Kc"].T) @ tl["W"]
+        dS = nxt
+    out_q, out_k, out_v = np.zeros((n * C, dk)), np.zeros((n * C, dk)), np.zeros((n * C, dv_))
+    out_g, out_b = np.zeros((n * C, dk)), np.zeros(n * C)
+    for r in range(n):
+        tl, sl = tiles[r], slice(r * C, r * C + C)
+        vc, bc, doc = vv[sl], bb[sl], do[sl]
+        Sr, dSr = states[r], dSn[r]
+        G, GC, Qb, Kb, Ki, Kc, A = (tl[x] for x in ("G", "GC", "Qb", "Kb", "Ki", "Kc", "A"))
+        Z = (tl["T"] @ (bc[:, None] * vc) - tl["W"] @ Sr.T) if delta else vc
+        dZ = Kc @ dSr.T + A.T @ doc
+        dKc, dQb, dA = Z @ dSr, doc @ Sr, np.tril(doc @ Z.T)
+        dKb, db = np.zeros_like(Kb), np.zeros(C)
+        dQb = dQb + dA @ Ki
+        dKi = dA.T @ Qb
+        if delta:
+            Tm = tl["T"]
+            dW = -dZ @ Sr
+            tdz = Tm.T @ dZ
+            dvv = bc[:, None] * tdz
+            dT = (dZ @ (bc[:, None] * vc).T) + (dW @ (bc[:, None] * Kb).T)
+            dL = np.tril(-Tm.T @ dT @ Tm.T, -1)
+            kbw = Tm.T @ dW
+            dKb = dKb + bc[:, None] * kbw
+            db += np.sum(tdz * vc, axis=1) + np.sum(kbw * Kb, axis=1) + np.sum(dL * tl["P"], axis=1)
+            E = bc[:, None] * dL
+            dKb = dKb + E @ Ki
+            dKi = dKi + E.T @ Kb
+        else:
+            dvv = dZ
+        eG, emG, ec = np.exp(G), np.exp(-G), np.exp(GC - G)
+        out_q[sl] = dQb * eG
+        out_k[sl] = dKb * eG + dKi * emG + dKc * ec
+        out_v[sl] = dvv
+        dG = dQb * Qb + dKb * Kb - dKi * Ki - dKc * Kc
+        dG[-1] += np.sum(dKc * Kc, axis=0) + np.exp(GC) * np.sum(dSr * Sr, axis=0)
+        out_g[sl] = np.cumsum(dG[::-1], axis=0)[::-1]
+        out_b[sl] = db
+    return (out_q[:T], out_k[:T], out_v[:T], out_g[:T], out_b[:T] if delta else None, dS)

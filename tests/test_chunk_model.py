@@ -92,3 +92,26 @@ def test_chunk_backward_model_matches_oracle(update, gate, C, T, s0, grads):
                 assert a is None, name
                 continue
             assert rel_err(a, b[h]) < 1e-10, (name, rel_err(a, b[h]))
+
+
+@pytest.mark.parametrize("update", ["decay", "delta"])
+@pytest.mark.parametrize("C,T", [(64, 150), (16, 40), (64, 1)])
+def test_chunk_backward_channel_gate_model_matches_oracle(update, C, T):
+    """The per-channel gate (KDA / GLA) form of the chunkwise backward: every
+    decay factor inside the q / k products, the gate gradient per channel."""
+    from chunk_model import chunk_backward_channel
+
+    q, k, v, g, beta, S0 = rand_inputs(45, BH=2, T=T, dk=16, dv=12, gate="channel",
+                                       delta=(update == "delta"), s0=True, gmin=-0.5)
+    r = np.random.default_rng(46)
+    dO, dST = r.standard_normal((2, T, 12)), r.standard_normal((2, 12, 16))
+    ref = oracle.gdn_backward_np(update, "channel", q, k, v, g, beta, S0, dO, dST)
+    for h in range(2):
+        one = lambda a: None if a is None else a[h]
+        got = chunk_backward_channel(update, one(q), one(k), one(v), one(g), one(beta), one(S0), one(dO),
+                                     one(dST), C=C)
+        for name, a, b in zip(["dq", "dk", "dv", "dg", "dbeta", "dS0"], got, ref):
+            if b is None:
+                assert a is None, name
+                continue
+            assert rel_err(a, b[h]) < 1e-10, (name, rel_err(a, b[h]))
